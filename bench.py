@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark on B200: one step = one cfr_paged_decode call over
+every (sequence, query head) of the workload (schedule + decode + merge).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload cfr|tiny|gqa|tiered|alibi1m]
+
+Prints one JSON line (rank 0).  `value` is the effective KV-read bandwidth
+(algorithmic K/V bytes of all ranks / step time, GB/s) with every input resident
+in HBM; `ms_per_step` the device time of one step (CUDA events, max over ranks).
+The decode kernel's own launches are bracketed by CUDA events inside the timed
+steps for the roofline.  `e2e` repeats the measurement through the public call
+with the step's inputs (q, seq_lens, page table) copied from pinned host memory
+and (out, lse) read back, the KV cache staying resident.  `--impl reference`
+times the fp64 CPU oracle on the host cores instead.  With N > 1 (torchrun) each
+rank runs an independent replica of the workload (no collective on the path).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_long_context_b200 import accounting, binding, synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="cfr", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle work for the CPU baseline")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# --------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self, want: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        elif torch.cuda.is_available():
+            torch.cuda.set_device(0)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# --------------------------------------------------------------------------
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _reasons(self):
+        f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(f(self.h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self._reasons()
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# helpers
+# --------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_long_context_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, path: int):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary,
+    only when the kernel sources are unchanged since the capture."""
+    name = os.path.join(PROFILE_TRAFFIC, f"decode_kernel_{workload}.md")
+    if not os.path.exists(name):
+        return None
+    vals = {}
+    for line in open(name):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_digest") != kernel_source_digest():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def dtype_name(case) -> str:
+    fm = sorted({case.fmt_of_page(b, p) for b in range(case.batch)
+                 for p in range(-(-int(case.seq_lens[b]) // case.page_tokens))})
+    return "+".join(synth.FMT_NAMES[f] for f in fm)
+
+
+def config_of(case, name, world, l2note):
+    lens = [int(x) for x in case.seq_lens.cpu().tolist()]
+    return {"workload": case.name, "short_name": name, "batch": case.batch,
+            "q_heads": case.num_q_heads, "kv_heads": case.num_kv_heads,
+            "head_dim": case.head_dim, "page_tokens": case.page_tokens,
+            "context_tokens_total": sum(lens), "context_min": min(lens), "context_max": max(lens),
+            "kv_formats": dtype_name(case), "alibi": case.alibi_slopes is not None,
+            "l2": l2note, "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def cpu_baseline(case, budget_s: float, host=None):
+    """Time the fp64 oracle (as it stands) on the host cores over a bounded sample."""
+    import oracle
+    oracle.build()
+    hc = host if host is not None else case.to("cpu")
+    pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads)]
+    lens = [int(x) for x in case.seq_lens.cpu().tolist()]
+    # calibrate on one pair, then take as many pairs as fit the budget
+    t0 = time.perf_counter()
+    oracle.attend(hc, sel=[pairs[0]], nthreads=1)
+    t1 = time.perf_counter() - t0
+    threads = oracle.default_threads()
+    n = max(1, min(len(pairs), int(budget_s * threads / max(t1, 1e-6))))
+    # spread the sample over sequences and kv heads
+    step = max(1, len(pairs) // n)
+    sel = pairs[::step][:n]
+    t0 = time.perf_counter()
+    oracle.attend(hc, sel=sel, nthreads=threads)
+    dt = time.perf_counter() - t0
+    bytes_per_pair = {}
+    for b, n_b in enumerate(lens):
+        kv = 0
+        for p in range(-(-n_b // case.page_tokens)):
+            f = case.fmt_of_page(b, p)
+            kv += min(case.page_tokens, n_b - p * case.page_tokens) * accounting.kv_token_bytes(f, case.head_dim)
+        bytes_per_pair[b] = kv
+    sample_bytes = sum(bytes_per_pair[b] for b, _ in sel)
+    return {"value": sample_bytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(sel)} of {len(pairs)} (sequence, query head) pairs, "
+                      f"{sample_bytes} K/V bytes, {dt:.2f} s",
+            "seconds": dt}
+
+
+# --------------------------------------------------------------------------
+# our implementation
+# --------------------------------------------------------------------------
+
+def run_ours(args, dist):
+    dev = torch.device("cuda", dist.local)
+    case = synth.workload(args.workload, device=dev)
+    acct = accounting.step_bytes(case)
+    kv_bytes = acct["kv"] + acct["scales"]
+    bufs = binding.DecodeBuffers(case)
+    path = binding.decode_path(case)
+    stream = torch.cuda.current_stream(dev)
+    st = binding.paged_decode_raw(case, bufs, stream)
+    if st != 0:
+        raise binding.CfrError(st, "cfr_paged_decode")
+    torch.cuda.synchronize()
+    if int(bufs.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(bufs.err.item()):#x}")
+
+    flush = None
+    if acct["total"] < 2 * L2_BYTES:
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        l2note = "L2 flushed (512 MiB write) before every step, outside the timed events"
+    else:
+        l2note = f"inputs larger than L2 ({acct['total'] / 2**20:.0f} MiB > 126 MiB)"
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_SCHEDULE)
+        if evs:
+            evs[1].record(stream)
+        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_DECODE)
+        if evs:
+            evs[2].record(stream)
+        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_MERGE)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dist.local) as clk:
+        for k in range(K):
+            if flush is not None:
+                flush.fill_(1.0)
+            step(evs[k])
+        torch.cuda.synchronize()
+    dist.barrier()
+    step_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / K
+    kern_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    step_ms_max = dist.max(step_ms)
+    kern_ms_max = dist.max(kern_ms)
+    err = int(bufs.err.item())
+
+    # ---- end to end through the public call, host buffers ----
+    q_h = case.q.cpu().pin_memory()
+    sl_h = case.seq_lens.cpu().pin_memory()
+    pt_h = case.page_table.cpu().pin_memory()
+    pf_h = case.page_fmt.cpu().pin_memory() if case.page_fmt is not None else None
+    out_h = torch.empty_like(bufs.out, device="cpu").pin_memory()
+    lse_h = torch.empty_like(bufs.lse, device="cpu").pin_memory()
+    h2d = q_h.numel() * q_h.element_size() + sl_h.numel() * 4 + pt_h.numel() * 4 + \
+        (pf_h.numel() if pf_h is not None else 0)
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+
+    def e2e_step():
+        case.q.copy_(q_h, non_blocking=True)
+        case.seq_lens.copy_(sl_h, non_blocking=True)
+        case.page_table.copy_(pt_h, non_blocking=True)
+        if pf_h is not None:
+            case.page_fmt.copy_(pf_h, non_blocking=True)
+        binding.paged_decode_raw(case, bufs, stream)
+        out_h.copy_(bufs.out, non_blocking=True)
+        lse_h.copy_(bufs.lse, non_blocking=True)
+
+    for _ in range(min(args.warmup, 10)):
+        e2e_step()
+    torch.cuda.synchronize()
+    Ke = max(3, min(K, 500))
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ke)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(Ke):
+        if flush is not None:
+            flush.fill_(1.0)
+        ee[k][0].record(stream)
+        e2e_step()
+        ee[k][1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e2e_ms = dist.max(sum(a.elapsed_time(b) for a, b in ee) / Ke)
+    assert torch.equal(out_h, bufs.out.cpu())
+
+    peak, peak_kind = measured_peaks()
+    achieved = acct["total"] / (kern_ms_max * 1e-3) / 1e9
+    traffic = profiled_traffic(args.workload, path)
+    world = dist.world
+    value = world * kv_bytes / (step_ms_max * 1e-3) / 1e9
+    res = {
+        "metric": "decode-attn µs/step and KV-read GB/s as % of B200 HBM peak (1 GPU)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+        "us_per_step": round(step_ms_max * 1e3, 2),
+        "kv_read_gbs_per_gpu": round(kv_bytes / (step_ms_max * 1e-3) / 1e9, 2),
+        "hbm_frac_of_measured": round(kv_bytes / (step_ms_max * 1e-3) / 1e9 / peak, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": dtype_name(case), "data": "synthetic (seeded N(0,1) K/V/q, page-shaped workload)",
+        "config": config_of(case, args.workload, world, l2note),
+        "kernel_path": {1: "cuda-core", 2: "tcgen05"}.get(path, "?"),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_kind": peak_kind,
+                     "kernel_us": round(kern_ms_max * 1e3, 2),
+                     "algorithmic_bytes_per_launch": acct["total"]},
+        "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "us_per_step": round(e2e_ms * 1e3, 2)},
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+        "device_err_word": err,
+    }
+    return case, res
+
+
+def run_reference(args, dist):
+    """The fp64 CPU oracle, as it stands, timed on the host cores (rank 0 only)."""
+    import oracle
+    oracle.build()
+    case = synth.workload(args.workload, device="cpu")
+    pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads)]
+    lens = [int(x) for x in case.seq_lens.tolist()]
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.attend(case, sel=[pairs[0]], nthreads=1)
+    t1 = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = max(1, min(len(pairs), int(budget * threads / max(t1, 1e-6))))
+    sel = pairs[::max(1, len(pairs) // n)][:n]
+    sample_bytes = 0
+    for b, _ in sel:
+        for p in range(-(-lens[b] // case.page_tokens)):
+            f = case.fmt_of_page(b, p)
+            sample_bytes += min(case.page_tokens, lens[b] - p * case.page_tokens) * \
+                accounting.kv_token_bytes(f, case.head_dim)
+    for _ in range(args.warmup):
+        oracle.attend(case, sel=sel, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attend(case, sel=sel, nthreads=threads)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = sample_bytes / dt / 1e9
+    sample = (f"{len(sel)} of {len(pairs)} (sequence, query head) pairs per step, "
+              f"{sample_bytes} K/V bytes")
+    return {
+        "impl": "reference",
+        "metric": "decode-attn µs/step and KV-read GB/s as % of B200 HBM peak (1 GPU)",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) K/V/q, page-shaped workload)",
+        "config": config_of(case, args.workload, 1, "host memory"),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        class _D:
+            world = int(os.environ.get("WORLD_SIZE", "1"))
+        print(json.dumps(run_reference(args, _D())), flush=True)
+        return 0
+    dist = Dist(args.gpus)
+    try:
+        case, res = run_ours(args, dist)
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = {k: v for k, v in cpu_baseline(case, args.cpu_budget).items()
+                                   if k != "seconds"}
+        if dist.rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,248 @@
+/*
+ * cfr_paged.h -- C ABI of the B200 paged decode-attention library.
+ *
+ * One decode step of softmax attention for one query per head over a paged
+ * KV cache, computed on one GPU by hand-written sm_100a kernels:
+ *
+ *   out[b][h] = softmax(q[b][h] . K_b^T * sigma + bias_h) V_b
+ *
+ * over the n_b = seq_lens[b] cached tokens of sequence b (scaled dot-product
+ * attention as defined on the RustAttention page, "Mathematical Framework
+ * Covered"; the decode query attends to every cached token).  K and V live in
+ * fixed-size token pages reached through a page table (CFR-Atlas page, "page
+ * identity and token ranges": a page holds a token range of one layer/head,
+ * stored row-major [token][head_dim]).  Pages may be stored as fp32, bf16, or
+ * as int8 / int4 codes with a per-page, per-head scale (the INT8 and INT4
+ * tiers of the ARGUS page, "Visual Architecture"); quantised pages are
+ * expanded only in on-chip memory ("Transient FP16 Reconstruction ... in GPU
+ * SRAM").  Each page range's partial (running max, normaliser, weighted-V
+ * accumulator) is folded exactly (CFR-Atlas page, "exact folded
+ * online-softmax attention pass") and split partials are merged by their
+ * log-sum-exp (CMF page, "split-K flash-decoding").
+ *
+ * Conventions for every entry point:
+ *  - Ownership: every buffer belongs to the caller.  No entry point allocates
+ *    or frees memory.  "device" pointers must be CUDA device memory (or
+ *    managed memory) of the current device; "host" pointers host memory.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  All GPU work is enqueued on it; no entry point
+ *    synchronises with the host.
+ *  - Errors: arguments are checked on the host before anything is launched; a
+ *    rejected call returns a status and enqueues nothing.  Problems only the
+ *    device can see (a page id outside its pool, an unknown page format, a
+ *    sequence length outside [1, max_pages * page_tokens]) never fault: the
+ *    kernel skips the offending page or sequence and ORs a CFR_DEVERR_* bit
+ *    into *err_word (when err_word is not NULL).  The caller reads the word
+ *    after synchronising; a non-zero word means the outputs of the affected
+ *    sequences are not the attention result.
+ *  - No data-value checks: non-finite K/V/q values propagate.
+ */
+#ifndef CFR_PAGED_H
+#define CFR_PAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CFR_OK = 0,
+  CFR_ERR_INVALID_ARG = 1,  /* NULL where a buffer is required, negative size, misalignment */
+  CFR_ERR_UNSUPPORTED = 2,  /* valid but not implemented: head_dim, page_tokens, group size */
+  CFR_ERR_OVERFLOW = 3,     /* a byte size or index does not fit its type */
+  CFR_ERR_PAGE_INDEX = 4,   /* reserved for callers mapping a non-zero *err_word */
+  CFR_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute query) */
+  CFR_ERR_TIMEOUT = 6,      /* reserved for callers mapping CFR_DEVERR_TIMEOUT */
+  CFR_ERR_WORKSPACE = 7     /* workspace NULL, misaligned or smaller than required */
+} cfr_status;
+
+typedef enum {
+  CFR_FMT_F32 = 0,   /* IEEE binary32 rows: 4 * head_dim bytes */
+  CFR_FMT_BF16 = 1,  /* bfloat16 rows: 2 * head_dim bytes */
+  CFR_FMT_I8 = 2,    /* int8 two's-complement codes: head_dim bytes; value = code * scale */
+  CFR_FMT_I4 = 3,    /* int4 codes, 2 per byte: head_dim / 2 bytes; element 2i in the low
+                        nibble, 2i+1 in the high nibble of byte i; value = code * scale */
+  CFR_FMT_COUNT = 4
+} cfr_page_fmt;
+
+/* Bits of the device error word (OR-ed, never cleared by the library). */
+#define CFR_DEVERR_PAGE_ID 0x1u   /* page id < 0 or >= pool_pages[fmt]; page skipped */
+#define CFR_DEVERR_PAGE_FMT 0x2u  /* page format >= CFR_FMT_COUNT; page skipped */
+#define CFR_DEVERR_SEQ_LEN 0x4u   /* seq_lens[b] < 1 or > max_pages * page_tokens */
+#define CFR_DEVERR_POOL 0x8u      /* page refers to a format whose pool (or scales) is NULL */
+#define CFR_DEVERR_TIMEOUT 0x10u  /* a bounded on-device wait gave up; outputs undefined */
+
+/*
+ * The paged K/V pools of one layer.  One pool per storage format; a page's
+ * format selects its pool and the page table holds its slot inside that pool.
+ *
+ *   k_pool[f], v_pool[f]: device, uint8 [pool_pages[f]][num_kv_heads][page_tokens][row_bytes(f)]
+ *       row_bytes: F32 4*d, BF16 2*d, I8 d, I4 d/2.  Every (slot, kv head)
+ *       sub-page is a contiguous row-major [page_tokens][head_dim] block.
+ *       Base addresses must be 16-byte aligned.  NULL for unused formats.
+ *   scales[f]: device, float [pool_pages[f]][num_kv_heads][2] = (K scale, V scale)
+ *       for f = I8, I4; ignored (may be NULL) for F32, BF16.
+ *   pool_pages[f]: number of slots of pool f (0 when unused).
+ *   Tokens of a sequence's last page at or past its length are never read
+ *   as values (their bytes may hold anything, NaN included).
+ */
+typedef struct {
+  int32_t num_kv_heads;
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t page_tokens;  /* >= 8 */
+  const void *k_pool[CFR_FMT_COUNT];
+  const void *v_pool[CFR_FMT_COUNT];
+  const float *scales[CFR_FMT_COUNT];
+  int64_t pool_pages[CFR_FMT_COUNT];
+} cfr_kv_pool;
+
+/*
+ * Bytes of device workspace that cfr_paged_decode needs for these sizes on
+ * the current device (partials of every split plus the split schedule).
+ * Returns 0 when the sizes are invalid or the byte count overflows.
+ */
+size_t cfr_paged_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t max_pages, int32_t page_tokens);
+
+/*
+ * One decode-attention step for every (sequence, query head).
+ *
+ *  q           device, [batch][num_q_heads][head_dim], fp32 (q_fmt = CFR_FMT_F32) or
+ *              bf16 (CFR_FMT_BF16).  K is taken as already position-encoded
+ *              (RoPE applied by the caller); ALiBi is applied here.
+ *  kv          host pointer to the pool description above.
+ *  page_table  device, int32 [batch][max_pages]: slot of logical page p of sequence b
+ *              inside the pool of that page's format.  Entries past a
+ *              sequence's last page are never read.
+ *  seq_lens    device, int32 [batch]: n_b, 1 <= n_b <= max_pages * page_tokens.
+ *  page_fmt    device, uint8 [batch][max_pages] format of every page, or NULL:
+ *              every page has format uniform_fmt.
+ *  head_map    host, int32 [num_q_heads]: kv head of each query head, or NULL:
+ *              h -> h / (num_q_heads / num_kv_heads) (MHA, MQA, GQA; CFR-Atlas
+ *              page, "MHA/MQA/GQA head mapping").  At most 16 query heads may
+ *              share one kv head.
+ *  alibi_slopes device, float [num_q_heads] or NULL: bias -slope_h * (n_b - 1 - j) is
+ *              added to the score of token j (CFR-Atlas page, "RoPE/ALiBi
+ *              positional policy").
+ *  softmax_scale sigma; 0 selects 1/sqrt(head_dim).
+ *  out         device, float [batch][num_q_heads][head_dim], written.
+ *  lse         device, float [batch][num_q_heads] natural-log log-sum-exp of the
+ *              scores, written; or NULL.
+ *  workspace   device, >= cfr_paged_decode_workspace_size(...) bytes, 256-byte
+ *              aligned; contents on entry are ignored, on return undefined.
+ *              Calls that share a workspace must not overlap on the GPU.
+ *  err_word    device uint32 or NULL; CFR_DEVERR_* bits are OR-ed into it.
+ *
+ * A sequence with n_b <= 0 or n_b > max_pages * page_tokens gets out = 0 and
+ * lse = -inf and sets CFR_DEVERR_SEQ_LEN.
+ */
+cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                            const int32_t *page_table, int32_t max_pages,
+                            const int32_t *seq_lens, int32_t batch, const uint8_t *page_fmt,
+                            int32_t uniform_fmt, int32_t num_q_heads, const int32_t *head_map,
+                            const float *alibi_slopes, float softmax_scale, float *out,
+                            float *lse, void *workspace, size_t workspace_bytes,
+                            uint32_t *err_word, void *stream);
+
+/* Phase bits of cfr_paged_decode_phases. */
+#define CFR_PHASE_SCHEDULE 0x1u  /* split schedule from seq_lens into the workspace */
+#define CFR_PHASE_DECODE 0x2u    /* split partials into the workspace */
+#define CFR_PHASE_MERGE 0x4u     /* partials -> out, lse */
+#define CFR_PHASE_ALL 0x7u
+
+/*
+ * cfr_paged_decode split into its three stream-ordered launches, for timing
+ * one launch at a time (CUDA events between calls).  Same arguments and checks
+ * as cfr_paged_decode; `phases` selects which launches are enqueued.  A call
+ * without CFR_PHASE_SCHEDULE relies on the workspace still holding the schedule
+ * of an earlier call with the same seq_lens, batch and sizes; a call without
+ * CFR_PHASE_DECODE merges the partials already in the workspace.
+ * cfr_paged_decode(...) == cfr_paged_decode_phases(..., CFR_PHASE_ALL).
+ */
+cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                   const int32_t *page_table, int32_t max_pages,
+                                   const int32_t *seq_lens, int32_t batch,
+                                   const uint8_t *page_fmt, int32_t uniform_fmt,
+                                   int32_t num_q_heads, const int32_t *head_map,
+                                   const float *alibi_slopes, float softmax_scale, float *out,
+                                   float *lse, void *workspace, size_t workspace_bytes,
+                                   uint32_t *err_word, void *stream, uint32_t phases);
+
+/*
+ * Log-sum-exp merge of split partials into the attention output (the merge
+ * step of split-K decoding, CMF page, "split-K flash-decoding"; the combine
+ * rule of online softmax).  For each (b, h) over s in [split_off[b], split_off[b+1]):
+ *
+ *   M = max m_s over splits with l_s > 0,  w_s = 2^(m_s - M),
+ *   out[b][h] = sum_s w_s a_s / sum_s w_s l_s,  lse[b][h] = (M + log2 sum_s w_s l_s) ln 2.
+ *
+ * part_m are base-2 maxima (scores times log2 e).  Splits with l_s = 0 are
+ * skipped; with none left out = 0 and lse = -inf.  Summation runs over the
+ * splits in index order, so results are deterministic.
+ *
+ *  part_acc device float [S][num_q_heads][head_dim]; part_m, part_l device
+ *  float [S][num_q_heads]; split_off device int32 [batch + 1], non-decreasing,
+ *  split_off[0] = 0.  out device float [batch][num_q_heads][head_dim]; lse
+ *  device float [batch][num_q_heads] or NULL.  head_dim is 64 or 128.
+ */
+cfr_status cfr_merge_partials(const float *part_acc, const float *part_m, const float *part_l,
+                              const int32_t *split_off, int32_t batch, int32_t num_q_heads,
+                              int32_t head_dim, float *out, float *lse, void *stream);
+
+/*
+ * The ragged-batch split schedule that cfr_paged_decode uses, exposed for
+ * inspection.  From seq_lens alone (device), every sequence is cut into
+ * contiguous page ranges of `chunk` pages, where chunk = ceil(sum_b NP_b /
+ * target_splits) (at least 1) and NP_b = ceil(n_b / page_tokens); sequence b
+ * gets ceil(NP_b / chunk) splits.
+ *
+ *  split_off  device int32 [batch + 1]: first split index of each sequence.
+ *  splits     device int32 [max_splits][3]: (b, first page, end page) of each split.
+ *  num_splits device int32 [2]: (total splits, chunk pages), written.
+ *  max_splits capacity of `splits`; schedules needing more set CFR_DEVERR_SEQ_LEN
+ *             (cannot happen when max_splits >= target_splits + batch).
+ */
+cfr_status cfr_schedule_splits(const int32_t *seq_lens, int32_t batch, int32_t page_tokens,
+                               int32_t max_pages, int32_t target_splits, int32_t *split_off,
+                               int32_t *splits, int32_t max_splits, int32_t *num_splits,
+                               uint32_t *err_word, void *stream);
+
+/*
+ * Raw page gather (diagnostic): copies the stored bytes of tokens [0, n_tokens)
+ * of sequence b, kv head kv_head, in token order, through the same page-table
+ * resolution as the decode kernels.  Row j of K goes to
+ * k_raw_out + j * out_row_pitch (row_bytes of its page's format), likewise V.
+ * Bytes of a row past its row_bytes are left untouched; rows of skipped pages
+ * (bad id, bad format, NULL pool) are left untouched and set err_word bits.
+ *
+ *  page_table, page_fmt (or NULL + uniform_fmt): as for cfr_paged_decode, with
+ *  `batch` rows; 0 <= b < batch, 0 <= n_tokens <= max_pages * page_tokens.
+ *  k_raw_out, v_raw_out device, >= n_tokens * out_row_pitch bytes each;
+ *  out_row_pitch a multiple of 16, >= the largest row_bytes in use.
+ */
+cfr_status cfr_gather_pages(const cfr_kv_pool *kv, const int32_t *page_table,
+                            const uint8_t *page_fmt, int32_t uniform_fmt, int32_t batch,
+                            int32_t max_pages, int32_t b, int32_t kv_head, int32_t n_tokens,
+                            void *k_raw_out,
+                            void *v_raw_out, int64_t out_row_pitch, uint32_t *err_word,
+                            void *stream);
+
+/*
+ * Which decode kernel a call with these arguments would run (for tests and
+ * benchmarks): 1 = CUDA-core kernel, 2 = tensor-core (tcgen05) kernel, 0 if the
+ * arguments would be rejected.  Host only; launches nothing.
+ */
+int32_t cfr_paged_decode_path(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_pages,
+                              const uint8_t *page_fmt, int32_t uniform_fmt,
+                              int32_t num_q_heads, const int32_t *head_map);
+
+/* Static description of a status code. */
+const char *cfr_status_str(cfr_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CFR_PAGED_H */

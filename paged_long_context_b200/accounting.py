@@ -1,0 +1,48 @@
+"""Algorithmic byte and flop counts of one decode step (host logic for the roofline).
+
+Bytes that any implementation must move at least once per step:
+  K and V rows of every valid token of every (sequence, kv head), in their
+  storage format; the int8/int4 scales of the pages read (8 bytes per page and
+  kv head); the page-table entries (4 bytes per page of each sequence, plus 1
+  byte of page format when a format array is used); q; out (fp32) and lse.
+Flops: a q.k multiply-add and a p.v multiply-add per element per query head,
+4 * Hq * d per token.
+The per-head K+V byte count of an fp32 cache reproduces the CFR-Atlas page's
+benchmark accounting (65,536 tokens x head_dim 64 -> 33,554,432 bytes).
+"""
+from __future__ import annotations
+
+from . import synth
+
+
+def kv_token_bytes(fmt: int, head_dim: int) -> int:
+    """K+V bytes of one token of one kv head."""
+    return 2 * synth.row_bytes(fmt, head_dim)
+
+
+def step_bytes(case) -> dict:
+    lens = [int(x) for x in case.seq_lens.cpu().tolist()]
+    P, d, Hkv = case.page_tokens, case.head_dim, case.num_kv_heads
+    kv = 0
+    scales = 0
+    pages = 0
+    for b, n in enumerate(lens):
+        npg = -(-n // P)
+        pages += npg
+        for p in range(npg):
+            f = case.fmt_of_page(b, p)
+            valid = min(P, n - p * P)
+            kv += Hkv * valid * kv_token_bytes(f, d)
+            if f in (synth.I8, synth.I4):
+                scales += Hkv * 8
+    table = pages * (4 + (1 if case.page_fmt is not None else 0))
+    qb = case.batch * case.num_q_heads * d * (4 if case.q_fmt == synth.F32 else 2)
+    ob = case.batch * case.num_q_heads * (d + 1) * 4
+    total = kv + scales + table + qb + ob
+    return {"kv": kv, "scales": scales, "page_table": table, "q": qb, "out": ob, "total": total,
+            "tokens": sum(lens)}
+
+
+def step_flops(case) -> int:
+    tokens = sum(int(x) for x in case.seq_lens.cpu().tolist())
+    return 4 * case.num_q_heads * case.head_dim * tokens

@@ -1,0 +1,196 @@
+"""Thin Python binding of the C ABI in include/cfr_paged.h (ctypes).
+
+Argument marshalling only: every step of the attention computation runs in the
+CUDA kernels of libcfr_paged.so.  There is no fallback: if the library is not
+built, or a call is rejected, the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import synth
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcfr_paged.so")
+
+CFR_OK = 0
+STATUS = {0: "CFR_OK", 1: "CFR_ERR_INVALID_ARG", 2: "CFR_ERR_UNSUPPORTED", 3: "CFR_ERR_OVERFLOW",
+          4: "CFR_ERR_PAGE_INDEX", 5: "CFR_ERR_CUDA", 6: "CFR_ERR_TIMEOUT", 7: "CFR_ERR_WORKSPACE"}
+DEVERR_PAGE_ID, DEVERR_PAGE_FMT, DEVERR_SEQ_LEN, DEVERR_POOL, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+PATH_CUDA_CORE, PATH_TENSOR_CORE = 1, 2
+
+# every exported symbol the header declares
+EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_decode_phases",
+           "cfr_merge_partials",
+           "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str"]
+
+
+class CfrError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class KvPool(ctypes.Structure):
+    """Mirror of cfr_kv_pool."""
+    _fields_ = [
+        ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("page_tokens", ctypes.c_int32),
+        ("k_pool", ctypes.c_void_p * 4), ("v_pool", ctypes.c_void_p * 4),
+        ("scales", ctypes.c_void_p * 4), ("pool_pages", ctypes.c_int64 * 4),
+    ]
+
+
+_lib = None
+_VP, _I32, _I64, _SZ, _F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+
+
+def lib():
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m paged_long_context_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.cfr_paged_decode_workspace_size.restype = _SZ
+        L.cfr_paged_decode_workspace_size.argtypes = [_I32] * 6
+        L.cfr_paged_decode.restype = ctypes.c_int
+        L.cfr_paged_decode.argtypes = [_VP, _I32, ctypes.POINTER(KvPool), _VP, _I32, _VP, _I32, _VP,
+                                       _I32, _I32, _VP, _VP, _F32, _VP, _VP, _VP, _SZ, _VP, _VP]
+        L.cfr_paged_decode_phases.restype = ctypes.c_int
+        L.cfr_paged_decode_phases.argtypes = L.cfr_paged_decode.argtypes + [ctypes.c_uint32]
+        L.cfr_merge_partials.restype = ctypes.c_int
+        L.cfr_merge_partials.argtypes = [_VP, _VP, _VP, _VP, _I32, _I32, _I32, _VP, _VP, _VP]
+        L.cfr_schedule_splits.restype = ctypes.c_int
+        L.cfr_schedule_splits.argtypes = [_VP, _I32, _I32, _I32, _I32, _VP, _VP, _I32, _VP, _VP, _VP]
+        L.cfr_gather_pages.restype = ctypes.c_int
+        L.cfr_gather_pages.argtypes = [ctypes.POINTER(KvPool), _VP, _VP, _I32, _I32, _I32, _I32,
+                                       _I32, _I32, _VP, _VP, _I64, _VP, _VP]
+        L.cfr_paged_decode_path.restype = _I32
+        L.cfr_paged_decode_path.argtypes = [_I32, ctypes.POINTER(KvPool), _I32, _VP, _I32, _I32, _VP]
+        L.cfr_status_str.restype = ctypes.c_char_p
+        L.cfr_status_str.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> Optional[ctypes.c_void_p]:
+    if stream is None:
+        if torch.cuda.is_available():
+            return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        return None
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def status_str(status: int) -> str:
+    return lib().cfr_status_str(status).decode()
+
+
+def kv_pool_struct(case: "synth.DecodeCase") -> KvPool:
+    s = KvPool()
+    s.num_kv_heads, s.head_dim, s.page_tokens = case.num_kv_heads, case.head_dim, case.page_tokens
+    for f in range(4):
+        s.k_pool[f] = case.k_pool[f].data_ptr() if f in case.k_pool else None
+        s.v_pool[f] = case.v_pool[f].data_ptr() if f in case.v_pool else None
+        s.scales[f] = case.scales[f].data_ptr() if f in case.scales else None
+        s.pool_pages[f] = int(case.k_pool[f].shape[0]) if f in case.k_pool else 0
+    return s
+
+
+def workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_pages, page_tokens) -> int:
+    return int(lib().cfr_paged_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim,
+                                                     max_pages, page_tokens))
+
+
+def _head_map_host(case):
+    if case.head_map is None:
+        return None, None
+    hm = case.head_map.detach().to("cpu", torch.int32).contiguous()
+    return hm, ctypes.c_void_p(hm.data_ptr())
+
+
+def decode_path(case) -> int:
+    """1 = CUDA-core kernel, 2 = tcgen05 kernel, 0 = the call would be rejected."""
+    pool = kv_pool_struct(case)
+    hm, hmp = _head_map_host(case)
+    return int(lib().cfr_paged_decode_path(case.q_fmt, ctypes.byref(pool), case.max_pages,
+                                           _p(case.page_fmt), case.uniform_fmt, case.num_q_heads,
+                                           hmp))
+
+
+class DecodeBuffers:
+    """Caller-owned output and scratch buffers of one decode call (device)."""
+
+    def __init__(self, case, device=None, with_lse=True):
+        dev = device or case.device
+        self.out = torch.empty((case.batch, case.num_q_heads, case.head_dim), dtype=torch.float32,
+                               device=dev)
+        self.lse = torch.empty((case.batch, case.num_q_heads), dtype=torch.float32,
+                               device=dev) if with_lse else None
+        n = workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                           case.max_pages, case.page_tokens)
+        if n == 0:
+            raise CfrError(1, "cfr_paged_decode_workspace_size")
+        self.workspace = torch.empty((n,), dtype=torch.uint8, device=dev)
+        self.err = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+
+PHASE_SCHEDULE, PHASE_DECODE, PHASE_MERGE, PHASE_ALL = 0x1, 0x2, 0x4, 0x7
+
+
+def paged_decode_raw(case, bufs: DecodeBuffers, stream=None, workspace_bytes=None,
+                     phases: Optional[int] = None) -> int:
+    """Call cfr_paged_decode (or cfr_paged_decode_phases when ``phases`` is given) on a
+    case whose tensors live on the GPU; returns the status."""
+    pool = kv_pool_struct(case)
+    hm, hmp = _head_map_host(case)
+    nbytes = bufs.workspace.numel() if workspace_bytes is None else workspace_bytes
+    args = (_p(case.q), case.q_fmt, ctypes.byref(pool), _p(case.page_table), case.max_pages,
+            _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads,
+            hmp, _p(case.alibi_slopes), float(case.softmax_scale), _p(bufs.out), _p(bufs.lse),
+            _p(bufs.workspace), nbytes, _p(bufs.err), _stream(stream))
+    if phases is None:
+        return int(lib().cfr_paged_decode(*args))
+    return int(lib().cfr_paged_decode_phases(*args, phases))
+
+
+def paged_decode(case, bufs: Optional[DecodeBuffers] = None, stream=None) -> DecodeBuffers:
+    """Decode attention for every (sequence, query head); raises on a rejected call."""
+    bufs = bufs or DecodeBuffers(case)
+    st = paged_decode_raw(case, bufs, stream)
+    if st != CFR_OK:
+        raise CfrError(st, "cfr_paged_decode")
+    return bufs
+
+
+def merge_partials(part_acc, part_m, part_l, split_off, batch, num_q_heads, head_dim, out,
+                   lse=None, stream=None) -> int:
+    return int(lib().cfr_merge_partials(_p(part_acc), _p(part_m), _p(part_l), _p(split_off),
+                                        batch, num_q_heads, head_dim, _p(out), _p(lse),
+                                        _stream(stream)))
+
+
+def schedule_splits(seq_lens, batch, page_tokens, max_pages, target_splits, split_off, splits,
+                    max_splits, num_splits, err=None, stream=None) -> int:
+    return int(lib().cfr_schedule_splits(_p(seq_lens), batch, page_tokens, max_pages,
+                                         target_splits, _p(split_off), _p(splits), max_splits,
+                                         _p(num_splits), _p(err), _stream(stream)))
+
+
+def gather_pages(case, b, kv_head, n_tokens, k_out, v_out, pitch, err=None, stream=None) -> int:
+    pool = kv_pool_struct(case)
+    return int(lib().cfr_gather_pages(ctypes.byref(pool), _p(case.page_table), _p(case.page_fmt),
+                                      case.uniform_fmt, case.batch, case.max_pages, b, kv_head,
+                                      n_tokens,
+                                      _p(k_out), _p(v_out), pitch, _p(err), _stream(stream)))

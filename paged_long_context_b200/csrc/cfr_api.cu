@@ -1,0 +1,403 @@
+// cfr_api.cu -- the C ABI: host-side argument checks, workspace layout, kernel
+// selection and launches.  Nothing here allocates memory or synchronises.
+#include <climits>
+#include <cstring>
+
+#include "cfr_common.cuh"
+
+namespace cfr {
+
+void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
+                     int32_t *split_off, int32_t *splits, int max_splits, int32_t *num_splits,
+                     uint32_t *err, cudaStream_t stream);
+void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
+                  const int32_t *split_off, int batch, int Hq, int D, float *out, float *lse,
+                  cudaStream_t stream);
+void launch_gather(const DecodeParams &p, int b, int g, int n_tokens, void *k_out, void *v_out,
+                   long long pitch, cudaStream_t stream);
+cudaError_t launch_decode_cc(const DecodeParams &p, int grid, cudaStream_t stream);
+int cc_stages(int D, int gt, int pitch, size_t smem_limit);
+int cc_group_tile(int gmax);
+cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream);
+bool tc_supported(const DecodeParams &p, bool page_fmt_given);
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sms = 0;
+  size_t smem_optin = 0;
+};
+
+// SM count and opt-in shared memory of the current device (cached per device).
+bool device_info(DeviceInfo *out) {
+  static DeviceInfo cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+  if (dev < kMaxDevices && cache[dev].sms > 0) {
+    *out = cache[dev];
+    return true;
+  }
+  DeviceInfo di;
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  di.sms = v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return false;
+  di.smem_optin = static_cast<size_t>(v);
+  if (dev < kMaxDevices) cache[dev] = di;
+  *out = di;
+  return true;
+}
+
+bool mul_ok(size_t a, size_t b, size_t *r) {
+  if (a != 0 && b > SIZE_MAX / a) return false;
+  *r = a * b;
+  return true;
+}
+
+bool add_ok(size_t a, size_t b, size_t *r) {
+  if (b > SIZE_MAX - a) return false;
+  *r = a + b;
+  return true;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Target number of splits over the whole batch: about eight work items
+// (split x kv head) per SM, so that a persistent grid of one CTA per SM gets
+// an even share.
+int target_splits(int sms, int hkv) {
+  const long long items = 8LL * sms;
+  long long t = (items + hkv - 1) / hkv;
+  if (t < 1) t = 1;
+  if (t > (1 << 20)) t = 1 << 20;
+  return static_cast<int>(t);
+}
+
+struct WsLayout {
+  size_t header, split_off, splits, part_m, part_l, part_acc, total;
+  int max_splits;
+};
+
+bool ws_layout(int batch, int hq, int d, int max_pages, int target, WsLayout *w) {
+  long long ms = static_cast<long long>(target) + batch;
+  const long long cap = static_cast<long long>(batch) * max_pages;
+  if (cap < ms) ms = cap;
+  if (ms < 1) ms = 1;
+  if (ms > INT_MAX / 4) return false;
+  w->max_splits = static_cast<int>(ms);
+  size_t o = 0, t = 0;
+  w->header = 0;
+  o = 256;
+  w->split_off = o;
+  if (!mul_ok(static_cast<size_t>(batch) + 1, 4, &t) || !add_ok(o, t, &o)) return false;
+  o = align_up(o, 256);
+  w->splits = o;
+  if (!mul_ok(static_cast<size_t>(ms), 12, &t) || !add_ok(o, t, &o)) return false;
+  o = align_up(o, 256);
+  size_t mh = 0;
+  if (!mul_ok(static_cast<size_t>(ms), static_cast<size_t>(hq), &mh)) return false;
+  w->part_m = o;
+  if (!mul_ok(mh, 4, &t) || !add_ok(o, t, &o)) return false;
+  o = align_up(o, 256);
+  w->part_l = o;
+  if (!add_ok(o, t, &o)) return false;
+  o = align_up(o, 256);
+  w->part_acc = o;
+  if (!mul_ok(mh, static_cast<size_t>(d) * 4, &t) || !add_ok(o, t, &o)) return false;
+  w->total = align_up(o, 256);
+  return true;
+}
+
+bool valid_fmt(int f) { return f >= 0 && f < kFmtCount; }
+
+// Checks of the pool description shared by decode, gather and path queries.
+cfr_status check_pool(const cfr_kv_pool *kv) {
+  if (!kv) return CFR_ERR_INVALID_ARG;
+  if (kv->num_kv_heads <= 0 || kv->head_dim <= 0 || kv->page_tokens <= 0) return CFR_ERR_INVALID_ARG;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return CFR_ERR_UNSUPPORTED;
+  if (kv->page_tokens < 8) return CFR_ERR_UNSUPPORTED;
+  bool any = false;
+  for (int f = 0; f < kFmtCount; ++f) {
+    const bool has = kv->k_pool[f] || kv->v_pool[f];
+    if (!has) continue;
+    if (!kv->k_pool[f] || !kv->v_pool[f]) return CFR_ERR_INVALID_ARG;
+    if (!aligned(kv->k_pool[f], 16) || !aligned(kv->v_pool[f], 16)) return CFR_ERR_INVALID_ARG;
+    if (kv->pool_pages[f] < 0) return CFR_ERR_INVALID_ARG;
+    if ((f == CFR_FMT_I8 || f == CFR_FMT_I4) && kv->pool_pages[f] > 0) {
+      if (!kv->scales[f] || !aligned(kv->scales[f], 8)) return CFR_ERR_INVALID_ARG;
+    }
+    // byte offsets of the last row must fit in 64 bits
+    size_t t = 0;
+    if (!mul_ok(static_cast<size_t>(kv->pool_pages[f]), static_cast<size_t>(kv->num_kv_heads), &t) ||
+        !mul_ok(t, static_cast<size_t>(kv->page_tokens), &t) ||
+        !mul_ok(t, static_cast<size_t>(row_bytes(f, kv->head_dim)), &t) || t > (size_t)LLONG_MAX)
+      return CFR_ERR_OVERFLOW;
+    any = true;
+  }
+  if (!any) return CFR_ERR_INVALID_ARG;
+  return CFR_OK;
+}
+
+// Query-head groups per kv head, from a host head map (or the contiguous rule).
+cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *p) {
+  if (hq <= 0 || hq > kMaxQHeads || hkv <= 0 || hkv > kMaxQHeads) return CFR_ERR_UNSUPPORTED;
+  if (!head_map && hq % hkv != 0) return CFR_ERR_INVALID_ARG;
+  int count[kMaxQHeads + 1];
+  std::memset(count, 0, sizeof(count));
+  for (int h = 0; h < hq; ++h) {
+    const int g = head_map ? head_map[h] : h / (hq / hkv);
+    if (g < 0 || g >= hkv) return CFR_ERR_INVALID_ARG;
+    ++count[g];
+  }
+  int gmax = 0, off = 0;
+  for (int g = 0; g < hkv; ++g) {
+    p->grp_off[g] = static_cast<int16_t>(off);
+    off += count[g];
+    if (count[g] > gmax) gmax = count[g];
+  }
+  p->grp_off[hkv] = static_cast<int16_t>(off);
+  if (gmax > kMaxGroup) return CFR_ERR_UNSUPPORTED;
+  int fill[kMaxQHeads];
+  for (int g = 0; g < hkv; ++g) fill[g] = p->grp_off[g];
+  for (int h = 0; h < hq; ++h) {
+    const int g = head_map ? head_map[h] : h / (hq / hkv);
+    p->grp_heads[fill[g]++] = static_cast<int16_t>(h);
+  }
+  p->gmax = gmax < 1 ? 1 : gmax;
+  return CFR_OK;
+}
+
+void fill_pool(const cfr_kv_pool *kv, DecodeParams *p) {
+  for (int f = 0; f < kFmtCount; ++f) {
+    p->k_pool[f] = static_cast<const uint8_t *>(kv->k_pool[f]);
+    p->v_pool[f] = static_cast<const uint8_t *>(kv->v_pool[f]);
+    p->scales[f] = kv->scales[f];
+    p->pool_pages[f] = kv->k_pool[f] ? kv->pool_pages[f] : 0;
+  }
+  p->Hkv = kv->num_kv_heads;
+  p->D = kv->head_dim;
+  p->P = kv->page_tokens;
+}
+
+int widest_row(const cfr_kv_pool *kv, const uint8_t *page_fmt, int uniform_fmt) {
+  if (!page_fmt) return row_bytes(uniform_fmt, kv->head_dim);
+  int w = 0;
+  for (int f = 0; f < kFmtCount; ++f)
+    if (kv->k_pool[f] && row_bytes(f, kv->head_dim) > w) w = row_bytes(f, kv->head_dim);
+  return w;
+}
+
+cfr_status common_checks(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_pages,
+                         const uint8_t *page_fmt, int32_t uniform_fmt) {
+  cfr_status st = check_pool(kv);
+  if (st != CFR_OK) return st;
+  if (q_fmt != CFR_FMT_F32 && q_fmt != CFR_FMT_BF16) return CFR_ERR_INVALID_ARG;
+  if (max_pages <= 0) return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_pages) * kv->page_tokens > INT_MAX) return CFR_ERR_OVERFLOW;
+  if (!page_fmt) {
+    if (!valid_fmt(uniform_fmt)) return CFR_ERR_INVALID_ARG;
+    if (!kv->k_pool[uniform_fmt]) return CFR_ERR_INVALID_ARG;
+  }
+  return CFR_OK;
+}
+
+}  // namespace
+}  // namespace cfr
+
+using namespace cfr;
+
+extern "C" {
+
+size_t cfr_paged_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t max_pages, int32_t page_tokens) {
+  if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_pages <= 0 ||
+      page_tokens <= 0)
+    return 0;
+  DeviceInfo di;
+  if (!device_info(&di)) return 0;
+  WsLayout w;
+  if (!ws_layout(batch, num_q_heads, head_dim, max_pages, target_splits(di.sms, num_kv_heads), &w))
+    return 0;
+  return w.total;
+}
+
+int32_t cfr_paged_decode_path(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_pages,
+                              const uint8_t *page_fmt, int32_t uniform_fmt, int32_t num_q_heads,
+                              const int32_t *head_map) {
+  if (common_checks(q_fmt, kv, max_pages, page_fmt, uniform_fmt) != CFR_OK) return 0;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (build_groups(num_q_heads, kv->num_kv_heads, head_map, &p) != CFR_OK) return 0;
+  fill_pool(kv, &p);
+  p.q_fmt = q_fmt;
+  p.uniform_fmt = uniform_fmt;
+  p.Hq = num_q_heads;
+  p.max_pages = max_pages;
+  return tc_supported(p, page_fmt != nullptr) ? 2 : 1;
+}
+
+cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                            const int32_t *page_table, int32_t max_pages,
+                            const int32_t *seq_lens, int32_t batch, const uint8_t *page_fmt,
+                            int32_t uniform_fmt, int32_t num_q_heads, const int32_t *head_map,
+                            const float *alibi_slopes, float softmax_scale, float *out,
+                            float *lse, void *workspace, size_t workspace_bytes,
+                            uint32_t *err_word, void *stream) {
+  return cfr_paged_decode_phases(q, q_fmt, kv, page_table, max_pages, seq_lens, batch, page_fmt,
+                                 uniform_fmt, num_q_heads, head_map, alibi_slopes, softmax_scale,
+                                 out, lse, workspace, workspace_bytes, err_word, stream,
+                                 CFR_PHASE_ALL);
+}
+
+cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                   const int32_t *page_table, int32_t max_pages,
+                                   const int32_t *seq_lens, int32_t batch,
+                                   const uint8_t *page_fmt, int32_t uniform_fmt,
+                                   int32_t num_q_heads, const int32_t *head_map,
+                                   const float *alibi_slopes, float softmax_scale, float *out,
+                                   float *lse, void *workspace, size_t workspace_bytes,
+                                   uint32_t *err_word, void *stream, uint32_t phases) {
+  if (phases == 0 || (phases & ~CFR_PHASE_ALL)) return CFR_ERR_INVALID_ARG;
+  cfr_status st = common_checks(q_fmt, kv, max_pages, page_fmt, uniform_fmt);
+  if (st != CFR_OK) return st;
+  if (!q || !page_table || !seq_lens || !out || batch <= 0) return CFR_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return CFR_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || softmax_scale == INFINITY) return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * max_pages > INT_MAX) return CFR_ERR_OVERFLOW;
+
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  st = build_groups(num_q_heads, kv->num_kv_heads, head_map, &p);
+  if (st != CFR_OK) return st;
+  fill_pool(kv, &p);
+
+  DeviceInfo di;
+  if (!device_info(&di)) return CFR_ERR_CUDA;
+  const int target = target_splits(di.sms, kv->num_kv_heads);
+  WsLayout w;
+  if (!ws_layout(batch, num_q_heads, kv->head_dim, max_pages, target, &w)) return CFR_ERR_OVERFLOW;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return CFR_ERR_WORKSPACE;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *num_splits = reinterpret_cast<int32_t *>(ws + w.header);
+  int32_t *split_off = reinterpret_cast<int32_t *>(ws + w.split_off);
+  int32_t *splits = reinterpret_cast<int32_t *>(ws + w.splits);
+  p.q = q;
+  p.q_fmt = q_fmt;
+  p.page_table = page_table;
+  p.page_fmt = page_fmt;
+  p.uniform_fmt = uniform_fmt;
+  p.seq_lens = seq_lens;
+  p.slopes = alibi_slopes;
+  p.part_acc = reinterpret_cast<float *>(ws + w.part_acc);
+  p.part_m = reinterpret_cast<float *>(ws + w.part_m);
+  p.part_l = reinterpret_cast<float *>(ws + w.part_l);
+  p.splits = splits;
+  p.num_splits = num_splits;
+  p.err = err_word;
+  p.batch = batch;
+  p.max_pages = max_pages;
+  p.Hq = num_q_heads;
+  const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(kv->head_dim));
+  p.sigma_log2e = sigma * kLog2e;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool use_tc = tc_supported(p, page_fmt != nullptr);
+  if (!use_tc) {
+    p.pitch = widest_row(kv, page_fmt, uniform_fmt);
+    p.stages = cc_stages(p.D, cc_group_tile(p.gmax), p.pitch, di.smem_optin);
+    if (p.stages < 2) return CFR_ERR_UNSUPPORTED;
+  }
+  if (phases & CFR_PHASE_SCHEDULE) {
+    launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, split_off, splits,
+                    w.max_splits, num_splits, err_word, s);
+    if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
+  }
+  if (phases & CFR_PHASE_DECODE) {
+    const cudaError_t e = use_tc ? launch_decode_tc(p, di.sms, s) : launch_decode_cc(p, di.sms, s);
+    if (e != cudaSuccess) return CFR_ERR_CUDA;
+  }
+  if (phases & CFR_PHASE_MERGE) {
+    launch_merge(p.part_acc, p.part_m, p.part_l, split_off, batch, num_q_heads, kv->head_dim,
+                 out, lse, s);
+    if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
+  }
+  return CFR_OK;
+}
+
+cfr_status cfr_merge_partials(const float *part_acc, const float *part_m, const float *part_l,
+                              const int32_t *split_off, int32_t batch, int32_t num_q_heads,
+                              int32_t head_dim, float *out, float *lse, void *stream) {
+  if (!part_acc || !part_m || !part_l || !split_off || !out) return CFR_ERR_INVALID_ARG;
+  if (batch <= 0 || num_q_heads <= 0) return CFR_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return CFR_ERR_UNSUPPORTED;
+  if (!aligned(part_acc, 16) || !aligned(out, 16)) return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * num_q_heads > INT_MAX) return CFR_ERR_OVERFLOW;
+  launch_merge(part_acc, part_m, part_l, split_off, batch, num_q_heads, head_dim, out, lse,
+               static_cast<cudaStream_t>(stream));
+  return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
+}
+
+cfr_status cfr_schedule_splits(const int32_t *seq_lens, int32_t batch, int32_t page_tokens,
+                               int32_t max_pages, int32_t target_splits, int32_t *split_off,
+                               int32_t *splits, int32_t max_splits, int32_t *num_splits,
+                               uint32_t *err_word, void *stream) {
+  if (!seq_lens || !split_off || !splits || !num_splits) return CFR_ERR_INVALID_ARG;
+  if (batch <= 0 || page_tokens <= 0 || max_pages <= 0 || target_splits <= 0 || max_splits <= 0)
+    return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_pages) * page_tokens > INT_MAX) return CFR_ERR_OVERFLOW;
+  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, split_off, splits,
+                  max_splits, num_splits, err_word, static_cast<cudaStream_t>(stream));
+  return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
+}
+
+cfr_status cfr_gather_pages(const cfr_kv_pool *kv, const int32_t *page_table,
+                            const uint8_t *page_fmt, int32_t uniform_fmt, int32_t batch,
+                            int32_t max_pages, int32_t b, int32_t kv_head, int32_t n_tokens,
+                            void *k_raw_out,
+                            void *v_raw_out, int64_t out_row_pitch, uint32_t *err_word,
+                            void *stream) {
+  cfr_status st = common_checks(CFR_FMT_F32, kv, max_pages, page_fmt, uniform_fmt);
+  if (st != CFR_OK) return st;
+  if (!page_table || !k_raw_out || !v_raw_out) return CFR_ERR_INVALID_ARG;
+  if (batch <= 0 || b < 0 || b >= batch || kv_head < 0 || kv_head >= kv->num_kv_heads || n_tokens < 0) return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(n_tokens) > static_cast<long long>(max_pages) * kv->page_tokens)
+    return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * max_pages > INT_MAX) return CFR_ERR_OVERFLOW;
+  if (out_row_pitch % 16 != 0 || out_row_pitch < widest_row(kv, page_fmt, uniform_fmt))
+    return CFR_ERR_INVALID_ARG;
+  if (!aligned(k_raw_out, 16) || !aligned(v_raw_out, 16)) return CFR_ERR_INVALID_ARG;
+  if (n_tokens == 0) return CFR_OK;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  fill_pool(kv, &p);
+  p.page_table = page_table;
+  p.page_fmt = page_fmt;
+  p.uniform_fmt = uniform_fmt;
+  p.max_pages = max_pages;
+  p.err = err_word;
+  launch_gather(p, b, kv_head, n_tokens, k_raw_out, v_raw_out, out_row_pitch,
+                static_cast<cudaStream_t>(stream));
+  return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
+}
+
+const char *cfr_status_str(cfr_status status) {
+  switch (status) {
+    case CFR_OK: return "ok";
+    case CFR_ERR_INVALID_ARG: return "invalid argument";
+    case CFR_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CFR_ERR_OVERFLOW: return "size overflow";
+    case CFR_ERR_PAGE_INDEX: return "page index out of range";
+    case CFR_ERR_CUDA: return "CUDA error";
+    case CFR_ERR_TIMEOUT: return "device wait timed out";
+    case CFR_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

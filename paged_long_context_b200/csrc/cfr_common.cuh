@@ -1,0 +1,155 @@
+// cfr_common.cuh -- device helpers shared by the decode-attention kernels (sm_100a).
+//
+// mbarrier-based producer/consumer hand-off with bounded waits, the 1-D bulk
+// copy engine (TMA, no multicast), error-word reporting and small numeric
+// helpers.  Every spin on an mbarrier gives up after a wall-clock limit, sets
+// CFR_DEVERR_TIMEOUT in the error word and lets the kernel return.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "cfr_paged.h"
+
+namespace cfr {
+
+constexpr int kFmtCount = CFR_FMT_COUNT;
+constexpr int kMaxQHeads = 256;
+constexpr int kMaxGroup = 16;              // query heads per kv head
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+// Parameters of one decode call, shared by both decode kernels.
+struct DecodeParams {
+  const void *q;
+  const uint8_t *k_pool[kFmtCount];
+  const uint8_t *v_pool[kFmtCount];
+  const float *scales[kFmtCount];
+  long long pool_pages[kFmtCount];
+  const int32_t *page_table;
+  const uint8_t *page_fmt;
+  const int32_t *seq_lens;
+  const float *slopes;
+  float *part_acc;      // [S][Hq][D]
+  float *part_m;        // [S][Hq], base-2 maxima
+  float *part_l;        // [S][Hq]
+  const int32_t *splits;     // [S][3]: b, page begin, page end
+  const int32_t *num_splits; // [0] = S
+  uint32_t *err;
+  int q_fmt, uniform_fmt;
+  int batch, max_pages, Hq, Hkv, D, P;
+  int pitch;            // shared-memory row pitch (bytes) of the CUDA-core kernel's stages
+  int stages;
+  float sigma_log2e;    // softmax scale times log2(e)
+  int gmax;             // largest group size
+  int16_t grp_off[kMaxQHeads + 1];  // heads of kv head g: grp_heads[grp_off[g] .. grp_off[g+1])
+  int16_t grp_heads[kMaxQHeads];
+};
+
+__host__ __device__ inline int row_bytes(int fmt, int d) {
+  return fmt == CFR_FMT_F32 ? 4 * d : fmt == CFR_FMT_BF16 ? 2 * d : fmt == CFR_FMT_I8 ? d : d / 2;
+}
+
+__device__ __forceinline__ void set_err(uint32_t *err, uint32_t bits) {
+  if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier --------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile(
+      "{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(
+          smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase of `parity` to complete.  Returns false (and flags the
+// error word) when the wait exceeded kWaitLimitNs; `*timed_out` then stays set
+// so that callers stop waiting on anything else.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err,
+                                          bool *timed_out) {
+  if (*timed_out) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      set_err(err, CFR_DEVERR_TIMEOUT);
+      *timed_out = true;
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---- 1-D bulk copy global -> shared (TMA engine, no multicast) ---------------
+
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---- numerics ----------------------------------------------------------------
+
+// 2^x with the hardware approximation (PTX ex2.approx.ftz.f32); 2^-inf = 0.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float i8_at(uint32_t w, int k) {
+  return static_cast<float>(static_cast<int8_t>((w >> (8 * k)) & 0xFF));
+}
+
+// 4-bit two's complement nibble k (0..7) of w: element 2i is the low nibble of byte i
+__device__ __forceinline__ float i4_at(uint32_t w, int k) {
+  int v = static_cast<int>((w >> (4 * k)) & 0xF);
+  return static_cast<float>(v >= 8 ? v - 16 : v);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace cfr

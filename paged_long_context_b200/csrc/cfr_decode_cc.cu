@@ -1,0 +1,535 @@
+// cfr_decode_cc.cu -- split-KV paged decode attention on the CUDA cores.
+//
+// Persistent kernel, one CTA per SM.  Work item = (split of one sequence, kv
+// head): a contiguous range of pages of sequence b and the G query heads that
+// share kv head g (GQA: one K/V read serves the whole group; CFR-Atlas page,
+// "MHA/MQA/GQA head mapping").
+//
+// Warp roles:
+//  - warp 8 (one elected lane) is the producer: it resolves every page of the
+//    item through the page table, checks slot, format and pool, and streams
+//    each 64-token tile of K and V into a shared-memory ring with 1-D bulk
+//    copies (TMA engine, completion on an mbarrier).  Pages that do not
+//    resolve are skipped and reported in the error word, never dereferenced.
+//  - warps 0-7 consume tiles.  Per tile: (1) scores s = sigma*(q.k)*scale_k +
+//    ALiBi, in base 2, eight lanes per token row; (2) per head, the tile max,
+//    the rescale factor 2^(m_old - m_new), p = 2^(s - m_new) and the running
+//    normaliser -- the exact fold of online softmax (CFR-Atlas page, "exact
+//    folded online-softmax attention pass"; ARGUS page, "page-by-page online
+//    softmax"); (3) acc = acc*alpha + sum_t p_t*scale_v*v_t, one warp per eight
+//    tokens, lanes across head_dim.  Quantised rows are expanded to fp32 in
+//    registers only (ARGUS page, "Transient FP16 Reconstruction ... in GPU
+//    SRAM"); scales multiply the dot product and p, never the stored codes.
+//  - At the end of an item the eight warps' accumulators are summed in a fixed
+//    order and (m, l, acc) is written as the split's partial for the merge.
+//
+// Tokens past the sequence length and rows of skipped pages get p = 0 and are
+// never read, so stale or NaN shared-memory bytes cannot reach an FMA.
+#include "cfr_common.cuh"
+
+namespace cfr {
+
+constexpr int CC_T = 64;       // tokens per tile
+constexpr int CC_WARPS = 8;    // consumer warps
+constexpr int CC_THREADS = (CC_WARPS + 1) * 32;
+constexpr int CC_MAXF = 16;    // fragments (page pieces) per tile; page_tokens >= 8 gives <= 9
+
+struct CcFrag {
+  int fmt;
+  int ok;
+  float ks, vs;
+};
+
+struct CcStageMeta {
+  CcFrag frag[CC_MAXF];
+  int8_t row_frag[CC_T];
+  int rows;
+  int t0;
+};
+
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(CC_WARPS * 32) : "memory");
+}
+
+// N consecutive elements starting at element e0 of a stored row, widened to fp32
+// (codes for quantised formats; the scale is applied by the caller).
+template <int N>
+__device__ __forceinline__ void load_elems(int fmt, const uint8_t *row, int e0, float (&x)[N]) {
+  if (fmt == CFR_FMT_F32) {
+    const float4 *p = reinterpret_cast<const float4 *>(row + 4 * e0);
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 v = p[i];
+      x[4 * i] = v.x;
+      x[4 * i + 1] = v.y;
+      x[4 * i + 2] = v.z;
+      x[4 * i + 3] = v.w;
+    }
+    if constexpr (N % 4 == 2) {
+      const float2 v = *reinterpret_cast<const float2 *>(row + 4 * e0 + 4 * (N - 2));
+      x[N - 2] = v.x;
+      x[N - 1] = v.y;
+    }
+  } else if (fmt == CFR_FMT_BF16) {
+    const uint8_t *p = row + 2 * e0;
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 8; ++i) {
+        const uint4 w = reinterpret_cast<const uint4 *>(p)[i];
+        const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[8 * i + 2 * k] = bf16_lo(a[k]);
+          x[8 * i + 2 * k + 1] = bf16_hi(a[k]);
+        }
+      }
+    } else if constexpr (N == 4) {
+      const uint2 w = *reinterpret_cast<const uint2 *>(p);
+      x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+      x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+    }
+  } else if (fmt == CFR_FMT_I8) {
+    const uint8_t *p = row + e0;
+    if constexpr (N % 16 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 16; ++i) {
+        const uint4 w = reinterpret_cast<const uint4 *>(p)[i];
+        const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[16 * i + k] = i8_at(a[k / 4], k % 4);
+      }
+    } else if constexpr (N == 8) {
+      const uint2 w = *reinterpret_cast<const uint2 *>(p);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = i8_at(k < 4 ? w.x : w.y, k % 4);
+    } else if constexpr (N == 4) {
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = i8_at(w, k);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint16_t *>(p);
+      x[0] = i8_at(w, 0); x[1] = i8_at(w, 1);
+    }
+  } else {  // CFR_FMT_I4
+    const uint8_t *p = row + e0 / 2;
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 8; ++i) {
+        const uint32_t w = reinterpret_cast<const uint32_t *>(p)[i];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[8 * i + k] = i4_at(w, k);
+      }
+    } else if constexpr (N == 4) {
+      const uint32_t w = *reinterpret_cast<const uint16_t *>(p);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = i4_at(w, k);
+    } else {
+      const uint32_t w = *p;
+      x[0] = i4_at(w, 0); x[1] = i4_at(w, 1);
+    }
+  }
+}
+
+struct CcLayout {
+  uint64_t *full, *empty;
+  CcStageMeta *meta;
+  float *q_s;      // [GT][D]
+  float *sc;       // [2][GT][T]
+  float *alpha;    // [2][GT]
+  float *slope2;   // [GT] slope * log2(e)
+  float *red;      // [CC_WARPS][4][D]
+  int *flag;       // [1] wait outcome broadcast
+  uint8_t *ring;   // [stages][2][T][pitch]
+};
+
+template <int D, int GT>
+__host__ __device__ inline size_t cc_fixed_bytes(int stages) {
+  size_t o = 0;
+  o += 2 * stages * sizeof(uint64_t);
+  o = (o + 15) & ~size_t(15);
+  o += stages * sizeof(CcStageMeta);
+  o = (o + 15) & ~size_t(15);
+  o += GT * D * 4 + 2 * GT * CC_T * 4 + 2 * GT * 4 + GT * 4 + CC_WARPS * 4 * D * 4 + 16;
+  o = (o + 127) & ~size_t(127);
+  return o;
+}
+
+template <int D, int GT>
+__device__ inline CcLayout cc_layout(uint8_t *smem, int stages, int pitch) {
+  CcLayout L;
+  size_t o = 0;
+  L.full = reinterpret_cast<uint64_t *>(smem);
+  L.empty = L.full + stages;
+  o += 2 * stages * sizeof(uint64_t);
+  o = (o + 15) & ~size_t(15);
+  L.meta = reinterpret_cast<CcStageMeta *>(smem + o);
+  o += stages * sizeof(CcStageMeta);
+  o = (o + 15) & ~size_t(15);
+  L.q_s = reinterpret_cast<float *>(smem + o);
+  o += GT * D * 4;
+  L.sc = reinterpret_cast<float *>(smem + o);
+  o += 2 * GT * CC_T * 4;
+  L.alpha = reinterpret_cast<float *>(smem + o);
+  o += 2 * GT * 4;
+  L.slope2 = reinterpret_cast<float *>(smem + o);
+  o += GT * 4;
+  L.red = reinterpret_cast<float *>(smem + o);
+  o += CC_WARPS * 4 * D * 4;
+  L.flag = reinterpret_cast<int *>(smem + o);
+  o += 16;
+  o = (o + 127) & ~size_t(127);
+  L.ring = smem + o;
+  (void)pitch;
+  return L;
+}
+
+// Producer: one lane streams every tile of every item of this CTA.
+template <int D>
+__device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long nitems,
+                            bool *timed_out) {
+  int stage = 0;
+  uint32_t phase = 0;
+  const int P = p.P;
+  for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int slot = static_cast<int>(item / p.Hkv), g = static_cast<int>(item % p.Hkv);
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int n = p.seq_lens[b];
+    const int tok_end = min(n, pe * P);
+    for (int t0 = pb * P; t0 < tok_end; t0 += CC_T) {
+      if (!mbar_wait(&L.empty[stage], phase ^ 1u, p.err, timed_out)) return;
+      CcStageMeta &m = L.meta[stage];
+      uint8_t *kst = L.ring + static_cast<size_t>(stage) * 2 * CC_T * p.pitch;
+      uint8_t *vst = kst + CC_T * p.pitch;
+      const int rows = min(CC_T, tok_end - t0);
+      m.rows = rows;
+      m.t0 = t0;
+      // resolve the page pieces of this tile
+      int nf = 0;
+      uint32_t bytes = 0;
+      for (int r = 0; r < rows;) {
+        const int j = t0 + r, pg = j / P, tin = j - pg * P;
+        const int fr = min(rows - r, P - tin);
+        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
+        const int fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
+        const long long id = p.page_table[cell];
+        CcFrag f;
+        f.fmt = fmt;
+        f.ok = 0;
+        f.ks = f.vs = 1.f;
+        if (fmt < 0 || fmt >= kFmtCount) {
+          set_err(p.err, CFR_DEVERR_PAGE_FMT);
+        } else if (!p.k_pool[fmt] || !p.v_pool[fmt] ||
+                   ((fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) && !p.scales[fmt])) {
+          set_err(p.err, CFR_DEVERR_POOL);
+        } else if (id < 0 || id >= p.pool_pages[fmt]) {
+          set_err(p.err, CFR_DEVERR_PAGE_ID);
+        } else {
+          f.ok = 1;
+          if (fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) {
+            const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+            f.ks = s.x;
+            f.vs = s.y;
+          }
+          bytes += 2u * fr * row_bytes(fmt, D);
+        }
+        m.frag[nf] = f;
+        for (int rr = r; rr < r + fr; ++rr) m.row_frag[rr] = static_cast<int8_t>(nf);
+        ++nf;
+        r += fr;
+      }
+      mbar_arrive_expect_tx(&L.full[stage], bytes);
+      // issue the copies
+      int fi = 0;
+      for (int r = 0; r < rows; ++fi) {
+        const int j = t0 + r, pg = j / P, tin = j - pg * P;
+        const int fr = min(rows - r, P - tin);
+        const CcFrag &f = m.frag[fi];
+        if (f.ok) {
+          const long long cell = static_cast<long long>(b) * p.max_pages + pg;
+          const long long id = p.page_table[cell];
+          const int rb = row_bytes(f.fmt, D);
+          const long long off = ((id * p.Hkv + g) * P + tin) * rb;
+          const uint8_t *ks = p.k_pool[f.fmt] + off;
+          const uint8_t *vs = p.v_pool[f.fmt] + off;
+          if (rb == p.pitch) {
+            bulk_g2s(kst + r * p.pitch, ks, fr * rb, &L.full[stage]);
+            bulk_g2s(vst + r * p.pitch, vs, fr * rb, &L.full[stage]);
+          } else {
+            for (int rr = 0; rr < fr; ++rr) {
+              bulk_g2s(kst + (r + rr) * p.pitch, ks + rr * rb, rb, &L.full[stage]);
+              bulk_g2s(vst + (r + rr) * p.pitch, vs + rr * rb, rb, &L.full[stage]);
+            }
+          }
+        }
+        r += fr;
+      }
+      if (++stage == p.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+}
+
+template <int D, int GT>
+__device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long nitems,
+                            bool *timed_out) {
+  constexpr int EPT = D / 8;    // elements per thread in the score step (8 lanes per row)
+  constexpr int DPL = D / 32;   // dims per lane in the P.V step
+  constexpr int HC = GT < 4 ? GT : 4;  // heads per reduction round
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int P = p.P;
+  int stage = 0;
+  uint32_t phase = 0;
+  int tile_ctr = 0;
+
+  for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
+    const int slot = static_cast<int>(item / p.Hkv), g = static_cast<int>(item % p.Hkv);
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int n = p.seq_lens[b];
+    const int tok_end = min(n, pe * P);
+    const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
+
+    // the group's queries (fp32) and ALiBi slopes
+    for (int i = tid; i < GT * D; i += CC_WARPS * 32) {
+      const int hh = i / D, e = i - hh * D;
+      float v = 0.f;
+      if (hh < cnt) {
+        const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + hh]) * D + e;
+        v = p.q_fmt == CFR_FMT_F32 ? static_cast<const float *>(p.q)[qi]
+                                   : __uint_as_float(static_cast<uint32_t>(
+                                         static_cast<const uint16_t *>(p.q)[qi]) << 16);
+      }
+      L.q_s[i] = v;
+    }
+    if (tid < GT)
+      L.slope2[tid] = (p.slopes && tid < cnt) ? p.slopes[p.grp_heads[h0 + tid]] * kLog2e : 0.f;
+    consumers_sync();
+
+    float acc[GT][DPL];
+#pragma unroll
+    for (int h = 0; h < GT; ++h)
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[h][i] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+
+    for (int t0 = pb * P; t0 < tok_end; t0 += CC_T) {
+      // one thread waits (bounded); the outcome is broadcast so all warps agree
+      if (tid == 0) *L.flag = mbar_wait(&L.full[stage], phase, p.err, timed_out) ? 1 : 0;
+      consumers_sync();
+      if (*L.flag == 0) {
+        *timed_out = true;
+        return;
+      }
+      (void)mbar_try_wait(&L.full[stage], phase);  // acquire the copied bytes in every thread
+      const CcStageMeta &m = L.meta[stage];
+      const uint8_t *kst = L.ring + static_cast<size_t>(stage) * 2 * CC_T * p.pitch;
+      const uint8_t *vst = kst + CC_T * p.pitch;
+      float *sc = L.sc + (tile_ctr & 1) * GT * CC_T;
+      float *al = L.alpha + (tile_ctr & 1) * GT;
+      const int rows = m.rows;
+
+      // (1) scores, base 2
+#pragma unroll
+      for (int pass = 0; pass < CC_T / 32; ++pass) {
+        const int r = pass * 32 + warp * 4 + (lane >> 3), j8 = lane & 7;
+        float dot[GT];
+#pragma unroll
+        for (int h = 0; h < GT; ++h) dot[h] = 0.f;
+        bool valid = false;
+        float ks = 1.f;
+        if (r < rows) {
+          const CcFrag f = m.frag[m.row_frag[r]];
+          if (f.ok) {
+            valid = true;
+            ks = f.ks;
+            float x[EPT];
+            load_elems<EPT>(f.fmt, kst + r * p.pitch, j8 * EPT, x);
+#pragma unroll
+            for (int h = 0; h < GT; ++h) {
+              const float4 *qq = reinterpret_cast<const float4 *>(L.q_s + h * D + j8 * EPT);
+#pragma unroll
+              for (int i = 0; i < EPT / 4; ++i) {
+                const float4 q4 = qq[i];
+                dot[h] = fmaf(q4.x, x[4 * i], dot[h]);
+                dot[h] = fmaf(q4.y, x[4 * i + 1], dot[h]);
+                dot[h] = fmaf(q4.z, x[4 * i + 2], dot[h]);
+                dot[h] = fmaf(q4.w, x[4 * i + 3], dot[h]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < GT; ++h) {
+          dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 1);
+          dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 2);
+          dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 4);
+        }
+        if (r < CC_T) {
+          const float dist = static_cast<float>(n - 1 - (m.t0 + r));
+#pragma unroll
+          for (int h = 0; h < GT; ++h)
+            if ((h & 7) == j8)
+              sc[h * CC_T + r] =
+                  valid ? fmaf(dot[h] * ks, p.sigma_log2e, -L.slope2[h] * dist) : -INFINITY;
+        }
+      }
+      consumers_sync();
+
+      // (2) fold: tile max, rescale factor, probabilities, running normaliser
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int hh = warp + 8 * k;
+        if (hh < GT) {
+          const float v0 = sc[hh * CC_T + lane], v1 = sc[hh * CC_T + lane + 32];
+          float mt = fmaxf(v0, v1);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+          const float m_new = fmaxf(m_run[k], mt);
+          float alpha = 1.f, p0 = 0.f, p1 = 0.f;
+          if (m_new != -INFINITY) {
+            alpha = exp2_approx(m_run[k] - m_new);
+            p0 = exp2_approx(v0 - m_new);
+            p1 = exp2_approx(v1 - m_new);
+          }
+          sc[hh * CC_T + lane] = p0;
+          sc[hh * CC_T + lane + 32] = p1;
+          float ls = p0 + p1;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+          l_run[k] = fmaf(l_run[k], alpha, ls);
+          m_run[k] = m_new;
+          if (lane == 0) al[hh] = alpha;
+        }
+      }
+      consumers_sync();
+
+      // (3) acc = acc*alpha + sum_t p_t * scale_v * v_t over this warp's 8 tokens
+#pragma unroll
+      for (int h = 0; h < GT; ++h) {
+        const float a = al[h];
+        if (a != 1.f) {
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) acc[h][i] *= a;
+        }
+      }
+#pragma unroll 2
+      for (int rr = 0; rr < CC_T / CC_WARPS; ++rr) {
+        const int r = warp * (CC_T / CC_WARPS) + rr;
+        if (r >= rows) break;
+        const CcFrag f = m.frag[m.row_frag[r]];
+        if (!f.ok) continue;
+        float v[DPL];
+        load_elems<DPL>(f.fmt, vst + r * p.pitch, lane * DPL, v);
+#pragma unroll
+        for (int h = 0; h < GT; ++h) {
+          const float pw = sc[h * CC_T + r] * f.vs;
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) acc[h][i] = fmaf(pw, v[i], acc[h][i]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&L.empty[stage]);
+      if (++stage == p.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      ++tile_ctr;
+    }
+
+    // split partial: (m, l) from the fold warps, acc summed over the 8 warps
+    float *pa = p.part_acc + static_cast<long long>(slot) * p.Hq * D;
+#pragma unroll
+    for (int c0 = 0; c0 < GT; c0 += HC) {
+      consumers_sync();
+#pragma unroll
+      for (int hh = 0; hh < HC; ++hh)
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) L.red[(warp * HC + hh) * D + lane * DPL + i] = acc[c0 + hh][i];
+      consumers_sync();
+      for (int e = tid; e < HC * D; e += CC_WARPS * 32) {
+        const int hh = e / D, i = e - hh * D;
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < CC_WARPS; ++w) s += L.red[(w * HC + hh) * D + i];
+        if (c0 + hh < cnt) pa[static_cast<long long>(p.grp_heads[h0 + c0 + hh]) * D + i] = s;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int hh = warp + 8 * k;
+      if (hh < GT && hh < cnt && lane == 0) {
+        const long long c = static_cast<long long>(slot) * p.Hq + p.grp_heads[h0 + hh];
+        p.part_m[c] = m_run[k];
+        p.part_l[c] = l_run[k];
+      }
+    }
+    consumers_sync();
+  }
+}
+
+template <int D, int GT>
+__global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const CcLayout L = cc_layout<D, GT>(smem, p.stages, p.pitch);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&L.full[s], 1);
+      mbar_init(&L.empty[s], CC_WARPS);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const long long nitems = static_cast<long long>(p.num_splits[0]) * p.Hkv;
+  bool timed_out = false;
+  if (threadIdx.x >= CC_WARPS * 32) {
+    if (threadIdx.x == CC_WARPS * 32) cc_producer<D>(p, L, nitems, &timed_out);
+  } else {
+    cc_consumer<D, GT>(p, L, nitems, &timed_out);
+  }
+}
+
+template <int D, int GT>
+static cudaError_t cc_launch_t(const DecodeParams &p, int grid, cudaStream_t stream) {
+  const size_t smem = cc_fixed_bytes<D, GT>(p.stages) +
+                      static_cast<size_t>(p.stages) * 2 * CC_T * p.pitch;
+  cudaError_t e = cudaFuncSetAttribute(cc_decode_kernel<D, GT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cc_decode_kernel<D, GT><<<grid, CC_THREADS, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+// Number of ring stages that fit next to the fixed shared-memory part.
+int cc_stages(int D, int gt, int pitch, size_t smem_limit) {
+  size_t fixed = 0;
+  const size_t stage = static_cast<size_t>(2) * CC_T * pitch;
+  for (int s = 8; s >= 2; --s) {
+#define CFR_FIX(DD, GG) \
+  if (D == DD && gt == GG) fixed = cc_fixed_bytes<DD, GG>(s);
+    CFR_FIX(64, 1) CFR_FIX(64, 2) CFR_FIX(64, 4) CFR_FIX(64, 8) CFR_FIX(64, 16)
+    CFR_FIX(128, 1) CFR_FIX(128, 2) CFR_FIX(128, 4) CFR_FIX(128, 8) CFR_FIX(128, 16)
+#undef CFR_FIX
+    if (fixed + s * stage <= smem_limit) return s;
+  }
+  return 0;
+}
+
+int cc_group_tile(int gmax) {
+  return gmax <= 1 ? 1 : gmax <= 2 ? 2 : gmax <= 4 ? 4 : gmax <= 8 ? 8 : 16;
+}
+
+cudaError_t launch_decode_cc(const DecodeParams &p, int grid, cudaStream_t stream) {
+  const int gt = cc_group_tile(p.gmax);
+#define CFR_CASE(DD, GG) \
+  if (p.D == DD && gt == GG) return cc_launch_t<DD, GG>(p, grid, stream);
+  CFR_CASE(64, 1) CFR_CASE(64, 2) CFR_CASE(64, 4) CFR_CASE(64, 8) CFR_CASE(64, 16)
+  CFR_CASE(128, 1) CFR_CASE(128, 2) CFR_CASE(128, 4) CFR_CASE(128, 8) CFR_CASE(128, 16)
+#undef CFR_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cfr

@@ -1,0 +1,184 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, and
+rejects invalid arguments on the host before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from paged_long_context_b200 import binding, synth
+from paged_long_context_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cfr_paged.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return binding.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return sorted(set(re.findall(r"\b(cfr_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == sorted(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (cfr_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert binding.status_str(code) not in ("", "unknown status")
+    assert binding.status_str(99) == "unknown status"
+
+
+def _case(**kw):
+    spec = dict(name="abi", batch=2, num_q_heads=4, num_kv_heads=2, head_dim=64, page_tokens=16,
+                seq_lens=[40, 17], fmt="bf16", q_fmt="bf16")
+    spec.update(kw)
+    return synth.make_case(synth.CaseSpec(**spec), 3, "cpu")
+
+
+class FakeBufs:
+    """Host tensors standing in for device buffers: the calls below are all
+    rejected on the host before any pointer is dereferenced or any kernel runs."""
+
+    def __init__(self, case):
+        self.out = torch.empty((case.batch, case.num_q_heads, case.head_dim))
+        self.lse = torch.empty((case.batch, case.num_q_heads))
+        self.workspace = torch.empty((1 << 16,), dtype=torch.uint8)
+        self.err = torch.zeros((1,), dtype=torch.int32)
+
+
+def _decode(case, **over):
+    bufs = FakeBufs(case)
+    pool = binding.kv_pool_struct(case)
+    for k, v in over.pop("pool", {}).items():
+        if k in ("k_pool", "v_pool", "scales", "pool_pages"):
+            for f, val in v.items():
+                getattr(pool, k)[f] = val
+        else:
+            setattr(pool, k, v)
+    args = dict(q=binding._p(case.q), q_fmt=case.q_fmt, page_table=binding._p(case.page_table),
+                max_pages=case.max_pages, seq_lens=binding._p(case.seq_lens), batch=case.batch,
+                page_fmt=binding._p(case.page_fmt), uniform_fmt=case.uniform_fmt,
+                num_q_heads=case.num_q_heads, head_map=None, slopes=None, scale=0.0,
+                out=binding._p(bufs.out), lse=binding._p(bufs.lse),
+                ws=binding._p(bufs.workspace), ws_bytes=bufs.workspace.numel(),
+                err=binding._p(bufs.err))
+    args.update(over)
+    return binding.lib().cfr_paged_decode(
+        args["q"], args["q_fmt"], ctypes.byref(pool), args["page_table"], args["max_pages"],
+        args["seq_lens"], args["batch"], args["page_fmt"], args["uniform_fmt"],
+        args["num_q_heads"], args["head_map"], args["slopes"], args["scale"], args["out"],
+        args["lse"], args["ws"], args["ws_bytes"], args["err"], None)
+
+
+E = binding.STATUS
+INVALID, UNSUP, OVERFLOW = 1, 2, 3
+
+
+def _hm(vals):
+    t = torch.tensor(vals, dtype=torch.int32)
+    _hm.keep.append(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+_hm.keep = []
+
+
+@pytest.mark.parametrize("what,over,code", [
+    ("null q", dict(q=None), INVALID),
+    ("null page table", dict(page_table=None), INVALID),
+    ("null seq_lens", dict(seq_lens=None), INVALID),
+    ("null out", dict(out=None), INVALID),
+    ("batch 0", dict(batch=0), INVALID),
+    ("q format i8", dict(q_fmt=2), INVALID),
+    ("max_pages 0", dict(max_pages=0), INVALID),
+    ("uniform format out of range", dict(uniform_fmt=7), INVALID),
+    ("uniform format without pool", dict(uniform_fmt=0), INVALID),
+    ("negative scale", dict(scale=-1.0), INVALID),
+    ("nan scale", dict(scale=float("nan")), INVALID),
+    ("head_dim 96", dict(pool={"head_dim": 96}), UNSUP),
+    ("page_tokens 4", dict(pool={"page_tokens": 4}), UNSUP),
+    ("kv heads 0", dict(pool={"num_kv_heads": 0}), INVALID),
+    ("Hq not multiple of Hkv", dict(num_q_heads=3), INVALID),
+    ("Hq above 256", dict(num_q_heads=258, pool={"num_kv_heads": 258}), UNSUP),
+    ("head map out of range", dict(head_map=_hm([0, 1, 2, 0])), INVALID),
+    ("negative head map", dict(head_map=_hm([0, -1, 1, 0])), INVALID),
+    ("group of 17", dict(num_q_heads=17, pool={"num_kv_heads": 1}), UNSUP),
+    ("k pool without v pool", dict(pool={"k_pool": {1: None}}), INVALID),
+    ("negative pool pages", dict(pool={"pool_pages": {1: -5}}), INVALID),
+    ("pages x tokens overflow", dict(max_pages=1 << 28), OVERFLOW),
+    ("batch x pages overflow", dict(batch=1 << 20, max_pages=1 << 12), OVERFLOW),
+])
+def test_host_rejects(lib, what, over, code):
+    case = _case()
+    assert _decode(case, **over) == code, what
+
+
+def test_misaligned_pointers_rejected(lib):
+    case = _case()
+    k = case.k_pool[synth.BF16]
+    assert _decode(case, pool={"k_pool": {synth.BF16: k.data_ptr() + 4}}) == INVALID
+    qp = ctypes.c_void_p(case.q.data_ptr() + 2)
+    assert _decode(case, q=qp) == INVALID
+
+
+def test_quantised_pool_needs_scales(lib):
+    case = _case(fmt="i8")
+    assert _decode(case, pool={"scales": {synth.I8: None}}) == INVALID
+
+
+def test_pool_byte_size_overflow(lib):
+    case = _case()
+    assert _decode(case, pool={"pool_pages": {synth.BF16: 1 << 60}}) == OVERFLOW
+
+
+def test_merge_and_schedule_and_gather_rejects(lib):
+    L = binding.lib()
+    t = torch.zeros(64)
+    p = ctypes.c_void_p(t.data_ptr())
+    assert L.cfr_merge_partials(p, p, p, p, 1, 1, 96, p, None, None) == UNSUP
+    assert L.cfr_merge_partials(None, p, p, p, 1, 1, 64, p, None, None) == INVALID
+    assert L.cfr_merge_partials(p, p, p, p, 0, 1, 64, p, None, None) == INVALID
+    assert L.cfr_schedule_splits(p, 1, 16, 4, 0, p, p, 8, p, None, None) == INVALID
+    assert L.cfr_schedule_splits(None, 1, 16, 4, 4, p, p, 8, p, None, None) == INVALID
+    case = _case()
+    pool = binding.kv_pool_struct(case)
+    args = (ctypes.byref(pool), binding._p(case.page_table), None, case.uniform_fmt,
+            case.batch, case.max_pages)
+    assert L.cfr_gather_pages(*args, 0, 0, 16, p, p, 24, None, None) == INVALID   # pitch % 16
+    assert L.cfr_gather_pages(*args, 0, 0, 16, p, p, 64, None, None) == INVALID   # < row bytes
+    assert L.cfr_gather_pages(*args, 0, 5, 16, p, p, 128, None, None) == INVALID  # kv head
+    assert L.cfr_gather_pages(*args, 0, 0, 10_000, p, p, 128, None, None) == INVALID
+    assert L.cfr_gather_pages(*args, 2, 0, 16, p, p, 128, None, None) == INVALID    # b >= batch
+
+
+def test_workspace_size_rejects_bad_sizes(lib):
+    assert binding.workspace_size(0, 4, 2, 64, 4, 16) == 0
+    assert binding.workspace_size(1, 0, 2, 64, 4, 16) == 0
+    assert binding.workspace_size(1, 4, 2, 64, -1, 16) == 0
+
+
+def test_path_selection_is_host_only(lib):
+    # fp32 caches always take the CUDA-core kernel
+    assert binding.decode_path(_case(fmt="f32", q_fmt="f32")) == binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="f32", q_fmt="f32", head_dim=128)) == binding.PATH_CUDA_CORE
+    # rejected configurations report 0
+    assert binding.decode_path(_case(num_q_heads=3, num_kv_heads=2)) == 0
