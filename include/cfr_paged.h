@@ -171,6 +171,40 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
                                    uint32_t *err_word, void *stream, uint32_t phases);
 
 /*
+ * Bytes of the scratch array compiled into the library for
+ * cfr_paged_decode_static_workspace (one array per GPU that loads the library).
+ */
+#define CFR_STATIC_WORKSPACE_BYTES (8u << 20)
+
+/*
+ * cfr_paged_decode for callers that cannot allocate device memory: plugin or
+ * operator interfaces that hand over only inputs and outputs, and code that
+ * runs where another component owns every device allocation.  The pages this
+ * library follows describe no counterpart of this entry point; it exists only
+ * for such callers.
+ *
+ * Same arguments, checks and results as cfr_paged_decode, without `workspace`:
+ * the split schedule and partials live in a fixed array of
+ * CFR_STATIC_WORKSPACE_BYTES inside the library.  Nothing is allocated or
+ * freed.  A problem whose cfr_paged_decode_workspace_size exceeds
+ * CFR_STATIC_WORKSPACE_BYTES returns CFR_ERR_WORKSPACE and launches nothing.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it, so make that first call before any
+ * stream capture.  All calls share the array: calls whose GPU work overlaps
+ * race on it and must be serialised by the caller.  No part of the array needs
+ * to start at zero.
+ */
+cfr_status cfr_paged_decode_static_workspace(const void *q, int32_t q_fmt,
+                                             const cfr_kv_pool *kv,
+                                             const int32_t *page_table, int32_t max_pages,
+                                             const int32_t *seq_lens, int32_t batch,
+                                             const uint8_t *page_fmt, int32_t uniform_fmt,
+                                             int32_t num_q_heads, const int32_t *head_map,
+                                             const float *alibi_slopes, float softmax_scale,
+                                             float *out, float *lse, uint32_t *err_word,
+                                             void *stream);
+
+/*
  * Log-sum-exp merge of split partials into the attention output (the merge
  * step of split-K decoding, CMF page, "split-K flash-decoding"; the combine
  * rule of online softmax).  For each (b, h) over s in [split_off[b], split_off[b+1]):

@@ -26,7 +26,9 @@ PATH_CUDA_CORE, PATH_TENSOR_CORE = 1, 2
 # every exported symbol the header declares
 EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_decode_phases",
            "cfr_merge_partials",
-           "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str"]
+           "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str",
+           "cfr_paged_decode_static_workspace"]
+STATIC_WORKSPACE_BYTES = 8 << 20
 
 
 class CfrError(RuntimeError):
@@ -73,6 +75,10 @@ def lib():
                                        _I32, _I32, _VP, _VP, _I64, _VP, _VP]
         L.cfr_paged_decode_path.restype = _I32
         L.cfr_paged_decode_path.argtypes = [_I32, ctypes.POINTER(KvPool), _I32, _VP, _I32, _I32, _VP]
+        L.cfr_paged_decode_static_workspace.restype = ctypes.c_int
+        L.cfr_paged_decode_static_workspace.argtypes = [_VP, _I32, ctypes.POINTER(KvPool), _VP, _I32,
+                                                        _VP, _I32, _VP, _I32, _I32, _VP, _VP, _F32,
+                                                        _VP, _VP, _VP, _VP]
         L.cfr_status_str.restype = ctypes.c_char_p
         L.cfr_status_str.argtypes = [ctypes.c_int]
         _lib = L
@@ -194,3 +200,15 @@ def gather_pages(case, b, kv_head, n_tokens, k_out, v_out, pitch, err=None, stre
                                       case.uniform_fmt, case.batch, case.max_pages, b, kv_head,
                                       n_tokens,
                                       _p(k_out), _p(v_out), pitch, _p(err), _stream(stream)))
+
+
+def paged_decode_static_workspace(case, out, lse=None, err=None, stream=None) -> int:
+    """cfr_paged_decode_static_workspace: decode with the library's built-in scratch array
+    (for callers that cannot allocate device memory); returns the status."""
+    pool = kv_pool_struct(case)
+    hm, hmp = _head_map_host(case)
+    return int(lib().cfr_paged_decode_static_workspace(
+        _p(case.q), case.q_fmt, ctypes.byref(pool), _p(case.page_table), case.max_pages,
+        _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads, hmp,
+        _p(case.alibi_slopes), float(case.softmax_scale), _p(out), _p(lse), _p(err),
+        _stream(stream)))
