@@ -353,7 +353,7 @@ def run_ours(args, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": dtype_name(case), "data": "synthetic (seeded N(0,1) K/V/q, page-shaped workload)",
         "config": config_of(case, args.workload, world, l2note),
-        "kernel_path": {1: "cuda-core", 2: "tcgen05"}.get(path, "?"),
+        "kernel_path": {1: "cuda-core", 2: "tcgen05", 3: "cuda-core-f32-tma"}.get(path, "?"),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_kind": peak_kind,

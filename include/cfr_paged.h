@@ -265,8 +265,9 @@ cfr_status cfr_gather_pages(const cfr_kv_pool *kv, const int32_t *page_table,
 
 /*
  * Which decode kernel a call with these arguments would run (for tests and
- * benchmarks): 1 = CUDA-core kernel, 2 = tensor-core (tcgen05) kernel, 0 if the
- * arguments would be rejected.  Host only; launches nothing.
+ * benchmarks): 1 = general CUDA-core kernel (any format mix), 2 = tensor-core
+ * (tcgen05) kernel, 3 = fp32 CUDA-core kernel with TMA tensor-map tiles, 0 if
+ * the arguments would be rejected.  Host only; launches nothing.
  */
 int32_t cfr_paged_decode_path(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_pages,
                               const uint8_t *page_fmt, int32_t uniform_fmt,

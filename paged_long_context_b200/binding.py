@@ -21,7 +21,7 @@ CFR_OK = 0
 STATUS = {0: "CFR_OK", 1: "CFR_ERR_INVALID_ARG", 2: "CFR_ERR_UNSUPPORTED", 3: "CFR_ERR_OVERFLOW",
           4: "CFR_ERR_PAGE_INDEX", 5: "CFR_ERR_CUDA", 6: "CFR_ERR_TIMEOUT", 7: "CFR_ERR_WORKSPACE"}
 DEVERR_PAGE_ID, DEVERR_PAGE_FMT, DEVERR_SEQ_LEN, DEVERR_POOL, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
-PATH_CUDA_CORE, PATH_TENSOR_CORE = 1, 2
+PATH_CUDA_CORE, PATH_TENSOR_CORE, PATH_F32_TMA = 1, 2, 3
 
 # every exported symbol the header declares
 EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_decode_phases",
@@ -127,7 +127,8 @@ def _head_map_host(case):
 
 
 def decode_path(case) -> int:
-    """1 = CUDA-core kernel, 2 = tcgen05 kernel, 0 = the call would be rejected."""
+    """1 = general CUDA-core kernel, 2 = tcgen05 kernel, 3 = fp32 TMA kernel,
+    0 = the call would be rejected."""
     pool = kv_pool_struct(case)
     hm, hmp = _head_map_host(case)
     return int(lib().cfr_paged_decode_path(case.q_fmt, ctypes.byref(pool), case.max_pages,

@@ -20,6 +20,8 @@ int cc_stages(int D, int gt, int pitch, size_t smem_limit);
 int cc_group_tile(int gmax);
 cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream);
 bool tc_supported(const DecodeParams &p, bool page_fmt_given);
+cudaError_t launch_decode_f32(const DecodeParams &p, int grid, cudaStream_t stream);
+bool f32_supported(const DecodeParams &p, bool page_fmt_given);
 
 namespace {
 
@@ -238,7 +240,9 @@ int32_t cfr_paged_decode_path(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_
   p.uniform_fmt = uniform_fmt;
   p.Hq = num_q_heads;
   p.max_pages = max_pages;
-  return tc_supported(p, page_fmt != nullptr) ? 2 : 1;
+  if (tc_supported(p, page_fmt != nullptr)) return 2;
+  if (f32_supported(p, page_fmt != nullptr)) return 3;
+  return 1;
 }
 
 cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
@@ -308,7 +312,8 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool use_tc = tc_supported(p, page_fmt != nullptr);
-  if (!use_tc) {
+  const bool use_f32 = !use_tc && f32_supported(p, page_fmt != nullptr);
+  if (!use_tc && !use_f32) {
     p.pitch = widest_row(kv, page_fmt, uniform_fmt);
     p.stages = cc_stages(p.D, cc_group_tile(p.gmax), p.pitch, di.smem_optin);
     if (p.stages < 2) return CFR_ERR_UNSUPPORTED;
@@ -319,7 +324,9 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_DECODE) {
-    const cudaError_t e = use_tc ? launch_decode_tc(p, di.sms, s) : launch_decode_cc(p, di.sms, s);
+    const cudaError_t e = use_tc    ? launch_decode_tc(p, di.sms, s)
+                          : use_f32 ? launch_decode_f32(p, di.sms, s)
+                                    : launch_decode_cc(p, di.sms, s);
     if (e != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_MERGE) {

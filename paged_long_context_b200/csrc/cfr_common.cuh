@@ -152,4 +152,32 @@ __device__ __forceinline__ float i4_at(uint32_t w, int k) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Sets bits [lo, hi) of a 128-bit row mask held in four registers (every index
+// is a compile-time constant, so the mask never leaves registers).
+__device__ __forceinline__ void mask_set_range(uint32_t (&m)[4], int lo, int hi) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int a = max(lo, 32 * w), b = min(hi, 32 * w + 32);
+    if (a < b) {
+      const uint32_t n = static_cast<uint32_t>(b - a);
+      const uint32_t bits = n >= 32u ? 0xFFFFFFFFu : ((1u << n) - 1u);
+      m[w] |= bits << (a - 32 * w);
+    }
+  }
+}
+
+// Bit r (0..127) of a 128-bit row mask held in registers.
+__device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int r) {
+  const uint32_t w = r < 32 ? m[0] : r < 64 ? m[1] : r < 96 ? m[2] : m[3];
+  return (w >> (r & 31)) & 1u;
+}
+
+// Work item -> (split slot, kv head).  Items are numbered split-fastest, so the
+// CTAs that start together read different page slots of the pool rather than
+// the kv heads of one slot (those sit a fixed sub-page stride apart).
+__device__ __forceinline__ void item_coords(long long item, int nsplit, int &slot, int &g) {
+  slot = static_cast<int>(item % nsplit);
+  g = static_cast<int>(item / nsplit);
+}
+
 }  // namespace cfr

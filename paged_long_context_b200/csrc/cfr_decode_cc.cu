@@ -193,7 +193,8 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
   uint32_t phase = 0;
   const int P = p.P;
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int slot = static_cast<int>(item / p.Hkv), g = static_cast<int>(item % p.Hkv);
+    int slot, g;
+    item_coords(item, p.num_splits[0], slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
@@ -286,7 +287,8 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
   int tile_ctr = 0;
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
-    const int slot = static_cast<int>(item / p.Hkv), g = static_cast<int>(item % p.Hkv);
+    int slot, g;
+    item_coords(item, p.num_splits[0], slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);

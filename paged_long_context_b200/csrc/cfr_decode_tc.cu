@@ -1,19 +1,879 @@
-// cfr_decode_tc.cu -- tensor-core (tcgen05) paged decode attention.
-#include "cfr_common.cuh"
+// cfr_decode_tc.cu -- paged decode attention on the 5th-generation tensor cores
+// (tcgen05, accumulators in TMEM) for bf16, int8 and int4 K/V pages, head_dim 128.
+//
+// For a kv head serving G query heads, one 128-token tile is two small dense
+// contractions:
+//   S^T[128 tok x N] = K_tile[128 x 128] . Q^T           (M = tokens, K = head_dim)
+//   O^T[128 dim x N] = V_tile^T[128 x 128] . P^T          (M = head_dim, K = tokens)
+// N = 16 (G <= 8) or 32 (G <= 16) columns: G "hi" and G "lo" halves, so that q
+// (fp32 or bf16) and the probabilities p enter the 16-bit MMA as hi + lo pairs
+// (about 16 significant bits for bf16, 22 for fp16), accumulated in fp32.
+// bf16 pages run bf16 MMAs; int8 / int4 pages are expanded to fp16 codes in
+// shared memory (codes are exact in fp16) and run fp16 MMAs; their per-page
+// K scale multiplies the scores, their V scale multiplies the tile's P.V
+// result, both in fp32 (ARGUS page, "Transient FP16 Reconstruction ... in GPU
+// SRAM": pages are expanded on chip only, attention runs at 16-bit).
+//
+// Warp roles (320 threads, one CTA per SM, persistent over work items =
+// (split of a sequence, kv head)):
+//   warp 0      TMA producer: resolves pages, bf16 tiles by 2-D tensor-map
+//               boxes straight into the 128-byte-swizzled operand layout,
+//               int tiles by 1-D bulk copies of the raw rows.
+//   warp 1      TMEM allocation; lane 0 issues the MMAs (QK of tile i+1 ahead
+//               of PV of tile i) and commits them to mbarriers.
+//   warps 2-5   softmax / fold: thread t owns TMEM lane t = token t of S and
+//               dim t of O.  Per tile: scores (scale, ALiBi from the integer
+//               distance), tile max across the 128 tokens, p = 2^(s - m),
+//               running normaliser, hi/lo split of p into the MMA's B operand,
+//               and the exact fold acc = acc*2^(m_old-m_new) + O_tile of the
+//               previous tile (CFR-Atlas page, "exact folded online-softmax
+//               attention pass").
+//   warps 6-9   staging: int8/int4 rows -> fp16 operand rows; zeroes V rows of
+//               tokens that are not part of the input so stale or NaN bytes
+//               never meet a zero probability inside the MMA.
+// Every mbarrier wait is bounded; on a timeout the error word is set, every
+// role leaves its loop, the MMA pipe is drained and TMEM is freed.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstring>
+
+#include "cfr_tmap.cuh"
 
 namespace cfr {
 
+constexpr int TC_T = 128;            // tokens per tile
+constexpr int TC_D = 128;            // head_dim
+constexpr int TC_THREADS = 320;
+constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
+constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
+constexpr int TC_RAW_BYTES = 2 * TC_T * TC_D;  // raw int8 K + V rows (int4 uses half)
+constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2;
+
+struct TcMeta {
+  uint32_t valid[4];
+  int rows, t0, kind;
+  float ks, vs;
+};
+
+struct TcMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+};
+
+template <int NCOL, bool INTP>
+struct TcCfg {
+  static constexpr int STAGES = INTP ? 2 : 3;
+  static constexpr int Q_BYTES = NCOL * 256;       // [NCOL rows][128 cols] 16-bit, 2 halves
+  static constexpr int P_BYTES = NCOL * TC_T * 2;  // [128 tokens][NCOL] 16-bit
+  static constexpr int TMEM_COLS = 4 * NCOL;       // S x2, O x2
+};
+
+template <int NCOL, bool INTP>
+struct TcSmem {
+  uint64_t op_full[3], op_empty[3], raw_full[3];
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
+  uint64_t q_full, drain;
+  uint32_t tmem_base;
+  int flag_sm, flag_st;
+  TcMeta meta[3];
+  alignas(16) float red_max[2][4][16];
+  alignas(16) float red_l[4][16];
+};
+
+template <int NCOL, bool INTP>
+struct TcLayout {
+  static constexpr size_t head = (sizeof(TcSmem<NCOL, INTP>) + 1023) / 1024 * 1024;
+  static constexpr size_t op = head;
+  static constexpr size_t raw = op + TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_OP_BYTES);
+  static constexpr size_t q = raw + (INTP ? TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_RAW_BYTES) : 0);
+  static constexpr size_t pbuf = q + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::Q_BYTES);
+  static constexpr size_t total = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
+  static constexpr size_t launch_bytes = total + 1024;  // slack for 1024-byte alignment
+};
+
+// ---- tcgen05 / descriptor helpers -------------------------------------------
+
+// instruction descriptor, kind::f16, fp32 accumulator, M = 128
+__host__ __device__ constexpr uint32_t tc_idesc(int ab_bf16, int a_mn, int b_mn, int n) {
+  return (1u << 4) | (static_cast<uint32_t>(ab_bf16) << 7) | (static_cast<uint32_t>(ab_bf16) << 10) |
+         (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// shared-memory matrix descriptor (sm_100: version 1); layout 2 = 128-byte swizzle, 0 = none
+__device__ __forceinline__ uint64_t tc_sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                             uint32_t layout) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (static_cast<uint64_t>(layout) << 61);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15},"
+      " [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32]) {
+  float a[16], b[16];
+  tmem_ld<16>(taddr, a);
+  tmem_ld<16>(taddr + 16, b);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[i] = a[i];
+    v[16 + i] = b[i];
+  }
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// four int8 codes (one word) -> two half2 words holding the same integers
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t &a, uint32_t &b) {
+  const uint32_t u = w ^ 0x80808080u;                         // code + 128, unsigned
+  const __half2 bias = bits_h2(0x64806480u);                   // 1152 = 1024 + 128
+  a = h2_bits(__hsub2(bits_h2(prmt(u, 0x64646464u, 0x4140u)), bias));  // 1024 + u0, 1024 + u1
+  b = h2_bits(__hsub2(bits_h2(prmt(u, 0x64646464u, 0x4342u)), bias));
+}
+
+// one byte k (0..3) of a word of int4 codes (low nibble = even element) -> half2
+__device__ __forceinline__ uint32_t i4x2_to_h2(uint32_t u_biased, int k) {
+  const uint32_t t = prmt(u_biased, 0u, 0x4040u | static_cast<uint32_t>(k) | (static_cast<uint32_t>(k) << 8));
+  const uint32_t m = (t & 0x00F0000Fu) | 0x64006400u;  // 1024 + lo nibble, 1024 + 16 * hi nibble
+  const __half2 scale = __halves2half2(__float2half_rn(1.f), __float2half_rn(0.0625f));
+  const __half2 off = __halves2half2(__float2half_rn(-1032.f), __float2half_rn(-72.f));
+  return h2_bits(__hfma2(bits_h2(m), scale, off));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  const __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// ---- roles ------------------------------------------------------------------
+
+template <int NCOL, bool INTP>
+struct TcCtx {
+  const DecodeParams &p;
+  const TcMaps &maps;
+  TcSmem<NCOL, INTP> &S;
+  uint8_t *op, *raw, *qop, *pop;
+  long long nitems;
+  int nsplit;
+};
+
+template <int NCOL, bool INTP>
+__device__ void tc_producer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+  using Cfg = TcCfg<NCOL, INTP>;
+  const DecodeParams &p = c.p;
+  const int P = p.P;
+  const int box_rows = P < TC_T ? P : TC_T;
+  int stage = 0;
+  uint32_t phase = 0;
+  if (p.k_pool[CFR_FMT_BF16]) {
+    prefetch_map(&c.maps.k);
+    prefetch_map(&c.maps.v);
+  }
+  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int tok_end = min(p.seq_lens[b], pe * P);
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+      if (!mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out)) return;
+      TcMeta &m = c.S.meta[stage];
+      const int rows = min(TC_T, tok_end - t0);
+      uint32_t valid[4] = {0u, 0u, 0u, 0u};
+      uint32_t bytes = 0;
+      int kind = KIND_BF16;
+      float ks = 1.f, vs = 1.f;
+      // resolve every page piece of the tile (one piece when page_tokens >= 128)
+      for (int r = 0; r < rows; r += box_rows) {
+        const int j = t0 + r, pg = j / P;
+        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
+        const int fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
+        const long long id = p.page_table[cell];
+        bool ok = false;
+        if (fmt < 0 || fmt >= kFmtCount) {
+          set_err(p.err, CFR_DEVERR_PAGE_FMT);
+        } else if (fmt == CFR_FMT_F32 || !p.k_pool[fmt] ||
+                   ((fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) && !p.scales[fmt])) {
+          set_err(p.err, CFR_DEVERR_POOL);
+        } else if (id < 0 || id >= p.pool_pages[fmt]) {
+          set_err(p.err, CFR_DEVERR_PAGE_ID);
+        } else {
+          ok = true;
+        }
+        if (!ok) continue;
+        const int hi = min(rows, r + box_rows);
+        mask_set_range(valid, r, hi);
+        if (fmt == CFR_FMT_BF16) {
+          bytes += 4u * box_rows * 128u;
+        } else {
+          // quantised: page_tokens >= 128, so this is the tile's only piece
+          kind = fmt == CFR_FMT_I8 ? KIND_I8 : KIND_I4;
+          const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+          ks = s.x;
+          vs = s.y;
+          bytes += 2u * rows * static_cast<uint32_t>(row_bytes(fmt, TC_D));
+        }
+      }
+      for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
+      m.rows = rows;
+      m.t0 = t0;
+      m.kind = kind;
+      m.ks = ks;
+      m.vs = vs;
+      mbar_arrive_expect_tx(&c.S.raw_full[stage], bytes);
+      uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
+      for (int r = 0; r < rows; r += box_rows) {
+        if (!mask_bit(valid, r)) continue;
+        const int j = t0 + r, pg = j / P, tin = j - pg * P;
+        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
+        const long long id = p.page_table[cell];
+        if (kind == KIND_BF16) {
+          const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
+          tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, &c.S.raw_full[stage]);
+          tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, &c.S.raw_full[stage]);
+          tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, &c.S.raw_full[stage]);
+          tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, &c.S.raw_full[stage]);
+        } else if (INTP) {
+          const int fmt = kind == KIND_I8 ? CFR_FMT_I8 : CFR_FMT_I4;
+          const int rb = row_bytes(fmt, TC_D);
+          const long long off = ((id * p.Hkv + g) * P + tin) * rb;
+          uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
+          bulk_g2s(raw, p.k_pool[fmt] + off, rows * rb, &c.S.raw_full[stage]);
+          bulk_g2s(raw + TC_T * TC_D, p.v_pool[fmt] + off, rows * rb, &c.S.raw_full[stage]);
+        }
+      }
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+}
+
+// staging warpgroup: thread r (0..127) owns row r of every tile
+template <int NCOL, bool INTP>
+__device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+  using Cfg = TcCfg<NCOL, INTP>;
+  const DecodeParams &p = c.p;
+  const int r = threadIdx.x - 192;
+  const int P = p.P;
+  int stage = 0;
+  uint32_t phase = 0;
+  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    (void)g;
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int tok_end = min(p.seq_lens[b], pe * P);
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+      if (r == 0) c.S.flag_st = mbar_wait(&c.S.raw_full[stage], phase, p.err, timed_out) ? 1 : 0;
+      named_sync(3, 128);
+      if (c.S.flag_st == 0) {
+        *timed_out = true;
+        return;
+      }
+      (void)mbar_try_wait(&c.S.raw_full[stage], phase);
+      const TcMeta &m = c.S.meta[stage];
+      const bool valid = (m.valid[r >> 5] >> (r & 31)) & 1u;
+      uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
+      if (m.kind == KIND_BF16) {
+        if (!valid) {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            *reinterpret_cast<uint4 *>(op + 2 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+          }
+        }
+      } else if (INTP) {
+        const uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          uint8_t *dst = op + kv * 2 * TC_HALF;
+          if (!valid) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              *reinterpret_cast<uint4 *>(dst + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4 *>(dst + TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+            }
+            continue;
+          }
+          if (m.kind == KIND_I8) {
+            // 128 codes = 8 chunks of 16 bytes; start at a row-dependent chunk (no bank conflicts)
+            const uint8_t *src = raw + kv * TC_T * TC_D + r * TC_D;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int ci = (j + r) & 7;  // input chunk: codes 16ci .. 16ci+15
+              const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+              uint32_t o[8];
+              i8x4_to_h2x2(w.x, o[0], o[1]);
+              i8x4_to_h2x2(w.y, o[2], o[3]);
+              i8x4_to_h2x2(w.z, o[4], o[5]);
+              i8x4_to_h2x2(w.w, o[6], o[7]);
+              // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
+              uint8_t *hb = dst + (ci >> 2) * TC_HALF;
+              const int oc = (2 * ci) & 7;
+              *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+          } else {
+            // 128 codes = 64 bytes = 4 chunks of 16 bytes (32 codes each)
+            const uint8_t *src = raw + kv * TC_T * TC_D + r * (TC_D / 2);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int ci = (j + (r >> 1)) & 3;  // input chunk: codes 32ci .. 32ci+31
+              const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+              const uint32_t wv[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
+                                      w.w ^ 0x88888888u};
+              uint32_t o[16];
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) o[4 * q + k] = i4x2_to_h2(wv[q], k);
+              // output chunks 4ci .. 4ci+3 in half ci/2
+              uint8_t *hb = dst + (ci >> 1) * TC_HALF;
+              const int oc = (4 * ci) & 7;
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(hb + sw128(r, oc + q)) =
+                    make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            }
+          }
+        }
+      }
+      fence_async_smem();
+      named_sync(3, 128);
+      if (r == 0) mbar_arrive(&c.S.op_full[stage]);
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+}
+
+template <int NCOL, bool INTP>
+__device__ void tc_mma_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+  using Cfg = TcCfg<NCOL, INTP>;
+  const DecodeParams &p = c.p;
+  const int P = p.P;
+  const uint32_t tmem = c.S.tmem_base;
+  const uint32_t op0 = smem_u32(c.op), q0 = smem_u32(c.qop), p0 = smem_u32(c.pop);
+  int stage = 0;
+  uint32_t phase = 0;
+  long long tc = 0;
+  int item_k = 0;
+  bool pending = false;
+  int pend_stage = 0, pend_kind = 0;
+  long long pend_tc = 0;
+
+  auto issue_pv = [&](long long i, int st, int kind) -> bool {
+    const uint32_t par = static_cast<uint32_t>((i >> 1) & 1);
+    if (!mbar_wait(&c.S.p_full[i & 1], par, p.err, timed_out)) return false;
+    if (!mbar_wait(&c.S.o_empty[i & 1], par ^ 1u, p.err, timed_out)) return false;
+    tc_fence_after();
+    const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
+    const uint32_t vbase = op0 + st * TC_OP_BYTES + 2 * TC_HALF;
+    const uint32_t pbase = p0 + static_cast<uint32_t>(i & 1) * Cfg::P_BYTES;
+    const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(i & 1) * NCOL;
+#pragma unroll
+    for (int k = 0; k < TC_T / 16; ++k) {
+      const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
+      const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
+      tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+    }
+    tc_commit(&c.S.o_full[i & 1]);
+    tc_commit(&c.S.p_empty[i & 1]);
+    tc_commit(&c.S.op_empty[st]);
+    return true;
+  };
+
+  for (long long item = blockIdx.x; item < c.nitems && !*timed_out; item += gridDim.x, ++item_k) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    (void)g;
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int tok_end = min(p.seq_lens[b], pe * P);
+    if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(item_k & 1), p.err, timed_out)) break;
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+      if (!mbar_wait(&c.S.op_full[stage], phase, p.err, timed_out)) break;
+      const int kind = c.S.meta[stage].kind;
+      if (!mbar_wait(&c.S.s_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err,
+                     timed_out))
+        break;
+      tc_fence_after();
+      const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
+      const uint32_t kbase = op0 + stage * TC_OP_BYTES;
+      const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
+      const uint32_t d = tmem + static_cast<uint32_t>(tc & 1) * NCOL;
+#pragma unroll
+      for (int k = 0; k < TC_D / 16; ++k) {
+        const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
+        const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
+        tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+      }
+      tc_commit(&c.S.s_full[tc & 1]);
+      if (pending && !issue_pv(pend_tc, pend_stage, pend_kind)) break;
+      pending = true;
+      pend_tc = tc;
+      pend_stage = stage;
+      pend_kind = kind;
+      ++tc;
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  if (pending && !*timed_out) issue_pv(pend_tc, pend_stage, pend_kind);
+  // drain: every MMA issued so far has completed before TMEM is released
+  tc_commit(&c.S.drain);
+  bool t2 = false;
+  (void)mbar_wait(&c.S.drain, 0, p.err, &t2);
+}
+
+// elected bounded wait of the softmax warpgroup; the outcome is shared by all 128 threads
+template <int NCOL, bool INTP>
+__device__ __forceinline__ bool tc_group_wait(TcCtx<NCOL, INTP> &c, uint64_t *bar, uint32_t parity,
+                                              int tsm, bool *timed_out) {
+  if (tsm == 0) c.S.flag_sm = mbar_wait(bar, parity, c.p.err, timed_out) ? 1 : 0;
+  named_sync(2, 128);
+  const bool ok = c.S.flag_sm != 0;
+  named_sync(2, 128);
+  if (!ok) *timed_out = true;
+  return ok;
+}
+
+// folds the P.V product of tile i into the running accumulators (dim t of each head)
+template <int NCOL, bool INTP>
+__device__ __forceinline__ bool tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint32_t tmem, int lane,
+                                        int tsm, int cnt, float (&acc)[NCOL / 2],
+                                        const float (&alpha_prev)[NCOL / 2], float vscale_prev,
+                                        bool *timed_out) {
+  if (!tc_group_wait(c, &c.S.o_full[i & 1], static_cast<uint32_t>((i >> 1) & 1), tsm, timed_out))
+    return false;
+  tc_fence_after();
+  float o[NCOL];
+  tmem_ld<NCOL>(tmem + 2 * NCOL + static_cast<uint32_t>(i & 1) * NCOL, o);
+  tc_wait_ld();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&c.S.o_empty[i & 1]);
+#pragma unroll
+  for (int h = 0; h < NCOL / 2; ++h) {
+    float ohl = 0.f;
+#pragma unroll
+    for (int k = 0; k < NCOL; ++k)
+      if (k == cnt + h) ohl = o[k];
+    if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + ohl) * vscale_prev);
+  }
+  return true;
+}
+
+// softmax / fold warpgroup
+template <int NCOL, bool INTP>
+__device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+  using Cfg = TcCfg<NCOL, INTP>;
+  constexpr int GM = NCOL / 2;  // most query heads per tile
+  const DecodeParams &p = c.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int t = 32 * quarter + lane;  // TMEM lane: token t of S, dim t of O
+  const int tsm = threadIdx.x - 64;   // 0..127 within the warpgroup
+  const uint32_t tmem = c.S.tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
+  const int P = p.P;
+  int stage = 0;
+  uint32_t phase = 0;
+  long long tc = 0;
+  int item_k = 0;
+  bool q_ready = false;
+
+  // writes the hi/lo query operand of item `it` (both bf16 and fp16 copies)
+  auto write_q = [&](long long it) {
+    int slot, g;
+    item_coords(it, c.nsplit, slot, g);
+    const int b = p.splits[3 * slot];
+    const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
+    for (int idx = tsm; idx < NCOL * 16; idx += 128) {
+      const int n = idx >> 4, ch = idx & 15;  // row n, 8-element chunk ch of 16
+      const int head = n < cnt ? n : (n - cnt < cnt ? n - cnt : -1);
+      const bool lo_part = n >= cnt;
+      float x[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = 0.f;
+      if (head >= 0 && n < 2 * cnt) {
+        const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * TC_D + 8 * ch;
+        if (p.q_fmt == CFR_FMT_F32) {
+          const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi);
+          const float4 bb = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi + 4);
+          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = bb.x; x[5] = bb.y; x[6] = bb.z; x[7] = bb.w;
+        } else {
+          const uint4 w = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + qi);
+          const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            x[2 * k] = bf16_lo(a[k]);
+            x[2 * k + 1] = bf16_hi(a[k]);
+          }
+        }
+      }
+      uint32_t wb[4], wh[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float bl[2], fl[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float v = x[2 * k + e];
+          const float bh = __bfloat162float(__float2bfloat16_rn(v));
+          const float fh = __half2float(__float2half_rn(v));
+          bl[e] = lo_part ? v - bh : bh;
+          fl[e] = lo_part ? v - fh : fh;
+        }
+        wb[k] = pack_bf16(bl[0], bl[1]);
+        wh[k] = pack_f16(fl[0], fl[1]);
+      }
+      const int off = (ch >> 3) * (NCOL * 128) + sw128(n, ch & 7);
+      *reinterpret_cast<uint4 *>(c.qop + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      *reinterpret_cast<uint4 *>(c.qop + Cfg::Q_BYTES + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c.S.q_full);
+  };
+
+  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x, ++item_k) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int n = p.seq_lens[b];
+    const int tok_end = min(n, pe * P);
+    const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
+    if (!q_ready) write_q(item);
+    q_ready = false;
+
+    float slope2[GM], m_run[GM], l_part[GM], acc[GM], alpha_prev[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      slope2[h] = (p.slopes && h < cnt) ? p.slopes[p.grp_heads[h0 + h]] * kLog2e : 0.f;
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.f;
+      acc[h] = 0.f;
+      alpha_prev[h] = 1.f;
+    }
+    float vscale_prev = 1.f;
+    long long prev_tc = -1;
+
+    bool ok = true;
+    for (int t0 = pb * P; t0 < tok_end && ok; t0 += TC_T) {
+      // ---- scores of tile tc ----
+      if (!tc_group_wait(c, &c.S.s_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), tsm, timed_out)) { ok = false; break; }
+      tc_fence_after();
+      float sv[NCOL];
+      tmem_ld<NCOL>(tmem + static_cast<uint32_t>(tc & 1) * NCOL, sv);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.S.s_empty[tc & 1]);
+      // acquire the tile description published through the stage's op_full phase
+      // (that phase cannot move on before this tile's P.V has run)
+      (void)mbar_try_wait(&c.S.op_full[stage], phase);
+      const TcMeta &m = c.S.meta[stage];
+      const bool valid = (m.valid[t >> 5] >> (t & 31)) & 1u;
+      const float scale = m.ks * p.sigma_log2e;
+      const float dist = static_cast<float>(n - 1 - (m.t0 + t));
+      const int kind = m.kind;
+      const float vsc = kind == KIND_BF16 ? 1.f : m.vs * (1.f / 32768.f);
+      float s[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        float shl = 0.f;
+#pragma unroll
+        for (int k = 0; k < NCOL; ++k)
+          if (k == cnt + h) shl = sv[k];
+        s[h] = (valid && h < cnt) ? fmaf(sv[h] + shl, scale, -slope2[h] * dist) : -INFINITY;
+        float mx = s[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) c.S.red_max[tc & 1][quarter][h] = mx;
+      }
+      // the P buffer of this tile must be free (PV of tile tc-2 done)
+      if (!tc_group_wait(c, &c.S.p_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, tsm, timed_out)) { ok = false; break; }
+      float pr[GM], alpha[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        float mt = fmaxf(fmaxf(c.S.red_max[tc & 1][0][h], c.S.red_max[tc & 1][1][h]),
+                         fmaxf(c.S.red_max[tc & 1][2][h], c.S.red_max[tc & 1][3][h]));
+        const float m_new = fmaxf(m_run[h], mt);
+        if (m_new == -INFINITY) {
+          alpha[h] = 1.f;
+          pr[h] = 0.f;
+        } else {
+          alpha[h] = exp2_approx(m_run[h] - m_new);
+          pr[h] = exp2_approx(s[h] - m_new);
+        }
+        l_part[h] = fmaf(l_part[h], alpha[h], pr[h]);
+        m_run[h] = m_new;
+      }
+      // P^T row t: columns [hi(0..cnt) | lo(0..cnt) | 0]
+      {
+        float colv[NCOL];
+#pragma unroll
+        for (int k = 0; k < NCOL; ++k) colv[k] = 0.f;
+        const float pre = kind == KIND_BF16 ? 1.f : 32768.f;
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+          if (h < cnt) {
+            const float x = pr[h] * pre;
+            const float xh = kind == KIND_BF16 ? __bfloat162float(__float2bfloat16_rn(x))
+                                               : __half2float(__float2half_rn(x));
+            // place hi at column h and lo at column cnt + h
+#pragma unroll
+            for (int k = 0; k < NCOL; ++k) {
+              if (k == h) colv[k] = xh;
+              if (k == cnt + h) colv[k] = x - xh;
+            }
+          }
+        }
+        uint8_t *pb_ = c.pop + (tc & 1) * Cfg::P_BYTES;
+#pragma unroll
+        for (int grp = 0; grp < NCOL / 8; ++grp) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            w[k] = kind == KIND_BF16 ? pack_bf16(colv[8 * grp + 2 * k], colv[8 * grp + 2 * k + 1])
+                                     : pack_f16(colv[8 * grp + 2 * k], colv[8 * grp + 2 * k + 1]);
+          *reinterpret_cast<uint4 *>(pb_ + grp * 2048 + t * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.S.p_full[tc & 1]);
+
+      const bool last = t0 + TC_T >= tok_end;
+      if (last) {
+        // the next item's query operand can be written as soon as this item's
+        // last QK product has been read
+        const long long nx = item + gridDim.x;
+        if (nx < c.nitems) {
+          write_q(nx);
+          q_ready = true;
+        }
+      }
+      // fold the previous tile of this item
+      if (prev_tc >= 0 && !tc_fold(c, prev_tc, tmem, lane, tsm, cnt, acc, alpha_prev, vscale_prev, timed_out)) { ok = false; break; }
+#pragma unroll
+      for (int h = 0; h < GM; ++h) alpha_prev[h] = alpha[h];
+      vscale_prev = vsc;
+      prev_tc = tc;
+      ++tc;
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok || (prev_tc >= 0 && !tc_fold(c, prev_tc, tmem, lane, tsm, cnt, acc, alpha_prev, vscale_prev, timed_out))) {
+      *timed_out = true;
+      return;
+    }
+
+    // split partial: acc (dim t), m, and l summed over the 128 token slots
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      if (h < cnt) {
+        const int head = p.grp_heads[h0 + h];
+        p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * TC_D + t] = acc[h];
+        float l = l_part[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) c.S.red_l[quarter][h] = l;
+      }
+    }
+    named_sync(2, 128);
+    if (tsm < cnt) {
+      const long long cidx = static_cast<long long>(slot) * p.Hq + p.grp_heads[h0 + tsm];
+      float mrun = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < GM; ++h)
+        if (h == tsm) mrun = m_run[h];
+      p.part_m[cidx] = mrun;
+      p.part_l[cidx] = (c.S.red_l[0][tsm] + c.S.red_l[1][tsm]) + (c.S.red_l[2][tsm] + c.S.red_l[3][tsm]);
+    }
+    named_sync(2, 128);
+  }
+}
+
+template <int NCOL, bool INTP>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    tc_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ TcMaps maps) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t a0 = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + ((1024u - (a0 & 1023u)) & 1023u);
+  using L = TcLayout<NCOL, INTP>;
+  TcSmem<NCOL, INTP> &S = *reinterpret_cast<TcSmem<NCOL, INTP> *>(smem);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&S.op_full[s], 1);
+      mbar_init(&S.op_empty[s], 1);
+      mbar_init(&S.raw_full[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_empty[i], 4);
+      mbar_init(&S.p_full[i], 4);
+      mbar_init(&S.p_empty[i], 1);
+      mbar_init(&S.o_full[i], 1);
+      mbar_init(&S.o_empty[i], 4);
+    }
+    mbar_init(&S.q_full, 4);
+    mbar_init(&S.drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&S.tmem_base)),
+                 "r"(TcCfg<NCOL, INTP>::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  TcCtx<NCOL, INTP> c{p, maps, S, smem + L::op, smem + L::raw, smem + L::q, smem + L::pbuf,
+                      static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
+  bool timed_out = false;
+  if (warp == 0) {
+    if ((threadIdx.x & 31) == 0) tc_producer<NCOL, INTP>(c, &timed_out);
+  } else if (warp == 1) {
+    if ((threadIdx.x & 31) == 0) tc_mma_issuer<NCOL, INTP>(c, &timed_out);
+  } else if (warp < 6) {
+    tc_softmax<NCOL, INTP>(c, &timed_out);
+  } else {
+    tc_staging<NCOL, INTP>(c, &timed_out);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(S.tmem_base),
+                 "r"(TcCfg<NCOL, INTP>::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+static bool tc_int_pools(const DecodeParams &p, bool page_fmt_given) {
+  if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4];
+  return p.uniform_fmt == CFR_FMT_I8 || p.uniform_fmt == CFR_FMT_I4;
+}
+
 bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
-  (void)p;
-  (void)page_fmt_given;
-  return false;
+  if (p.D != TC_D || p.gmax > 16) return false;
+  if ((reinterpret_cast<uintptr_t>(p.q) & 15) != 0) return false;
+  if (page_fmt_given) {
+    if (p.k_pool[CFR_FMT_F32]) return false;
+    if (!p.k_pool[CFR_FMT_BF16] && !p.k_pool[CFR_FMT_I8] && !p.k_pool[CFR_FMT_I4]) return false;
+  } else if (p.uniform_fmt == CFR_FMT_F32) {
+    return false;
+  }
+  const bool ints = tc_int_pools(p, page_fmt_given);
+  if (ints) {
+    if (p.P % TC_T != 0) return false;
+  } else if (!((p.P <= TC_T && TC_T % p.P == 0) || p.P % TC_T == 0)) {
+    return false;
+  }
+  const long long rows = p.pool_pages[CFR_FMT_BF16] * p.Hkv * static_cast<long long>(p.P);
+  if (rows > 0x7fffffffLL) return false;
+  return true;
+}
+
+template <int NCOL, bool INTP>
+static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t stream) {
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (p.k_pool[CFR_FMT_BF16] && p.pool_pages[CFR_FMT_BF16] > 0) {
+    const long long rows = p.pool_pages[CFR_FMT_BF16] * p.Hkv * static_cast<long long>(p.P);
+    const int box_rows = p.P < TC_T ? p.P : TC_T;
+    if (!encode_pool_map(&maps.k, p.k_pool[CFR_FMT_BF16], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows,
+                         TC_D, box_rows) ||
+        !encode_pool_map(&maps.v, p.v_pool[CFR_FMT_BF16], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows,
+                         TC_D, box_rows))
+      return cudaErrorInvalidValue;
+  }
+  constexpr size_t smem = TcLayout<NCOL, INTP>::launch_bytes;
+  static_assert(smem <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<NCOL, INTP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  tc_decode_kernel<NCOL, INTP><<<grid, TC_THREADS, smem, stream>>>(p, maps);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream) {
-  (void)p;
-  (void)grid;
-  (void)stream;
-  return cudaErrorNotSupported;
+  const bool ints = tc_int_pools(p, p.page_fmt != nullptr);
+  if (p.gmax <= 8)
+    return ints ? tc_launch_t<16, true>(p, grid, stream) : tc_launch_t<16, false>(p, grid, stream);
+  return ints ? tc_launch_t<32, true>(p, grid, stream) : tc_launch_t<32, false>(p, grid, stream);
 }
 
 }  // namespace cfr

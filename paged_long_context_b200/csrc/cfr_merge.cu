@@ -41,24 +41,46 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(
   for (int i = 0; i < DPL; ++i) o_acc[i] = 0.f;
   float L = 0.f;
   if (M != -INFINITY) {
-    for (int s = s0; s < s1; ++s) {
+    // normaliser: lane-strided partial sums, then a fixed tree
+    for (int s = s0 + lane; s < s1; s += 32) {
       const long long c = static_cast<long long>(s) * Hq + h;
       const float l = part_l[c];
-      if (!(l > 0.f)) continue;
-      const float w = exp2_approx(part_m[c] - M);
-      L = fmaf(l, w, L);
-      const float *a = part_acc + c * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(a);
-        o_acc[0] = fmaf(w, v.x, o_acc[0]);
-        o_acc[1] = fmaf(w, v.y, o_acc[1]);
-        o_acc[2] = fmaf(w, v.z, o_acc[2]);
-        o_acc[3] = fmaf(w, v.w, o_acc[3]);
-      } else {
-        const float2 v = *reinterpret_cast<const float2 *>(a);
-        o_acc[0] = fmaf(w, v.x, o_acc[0]);
-        o_acc[1] = fmaf(w, v.y, o_acc[1]);
+      if (l > 0.f) L = fmaf(l, exp2_approx(part_m[c] - M), L);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    // accumulators: four splits per step with independent loads; empty splits
+    // contribute nothing whatever their accumulator holds
+    for (int s = s0; s < s1; s += 4) {
+      float w[4], a[4][DPL];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        w[u] = 0.f;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) a[u][i] = 0.f;
+        if (s + u < s1) {
+          const long long c = static_cast<long long>(s + u) * Hq + h;
+          const float l = part_l[c];
+          const float m = part_m[c];
+          const float *ap = part_acc + c * D + lane * DPL;
+          if constexpr (DPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(ap);
+            a[u][0] = v.x; a[u][1] = v.y; a[u][2] = v.z; a[u][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2 *>(ap);
+            a[u][0] = v.x; a[u][1] = v.y;
+          }
+          w[u] = l > 0.f ? exp2_approx(m - M) : 0.f;
+          if (!(l > 0.f)) {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) a[u][i] = 0.f;
+          }
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) o_acc[i] = fmaf(w[u], a[u][i], o_acc[i]);
     }
   }
   float *o = out + pair * D + lane * DPL;

@@ -177,8 +177,15 @@ def test_workspace_size_rejects_bad_sizes(lib):
 
 
 def test_path_selection_is_host_only(lib):
-    # fp32 caches always take the CUDA-core kernel
-    assert binding.decode_path(_case(fmt="f32", q_fmt="f32")) == binding.PATH_CUDA_CORE
-    assert binding.decode_path(_case(fmt="f32", q_fmt="f32", head_dim=128)) == binding.PATH_CUDA_CORE
+    # fp32 caches with at most two query heads per kv head take the fp32 TMA kernel
+    assert binding.decode_path(_case(fmt="f32", q_fmt="f32")) == binding.PATH_F32_TMA
+    assert binding.decode_path(_case(fmt="f32", q_fmt="f32", head_dim=128)) == binding.PATH_F32_TMA
+    assert binding.decode_path(_case(fmt="f32", q_fmt="bf16", num_q_heads=4, num_kv_heads=4)) == \
+        binding.PATH_F32_TMA
+    # wider groups, odd page sizes and format mixes with fp32 take the general kernel
+    assert binding.decode_path(_case(fmt="f32", num_q_heads=8, num_kv_heads=2)) == binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="f32", page_tokens=24)) == binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="tiered", tiers=[(0.5, "i8"), (0.5, "f32")])) == \
+        binding.PATH_CUDA_CORE
     # rejected configurations report 0
     assert binding.decode_path(_case(num_q_heads=3, num_kv_heads=2)) == 0
