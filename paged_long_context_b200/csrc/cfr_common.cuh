@@ -7,6 +7,8 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "cfr_paged.h"
@@ -128,6 +130,37 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+
+// Lets the next kernel of the stream start its prologue now (it still waits for
+// this grid's results before reading them).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the previous kernel of the stream has completed and its writes are
+// visible (returns at once when there is no such dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launches `kernel` so that it may overlap the tail of the previous kernel in the
+// stream (programmatic stream serialization); the kernel calls griddep_wait()
+// before touching that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after_previous(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---- numerics ----------------------------------------------------------------
 
 // 2^x with the hardware approximation (PTX ex2.approx.ftz.f32); 2^-inf = 0.
@@ -170,6 +203,47 @@ __device__ __forceinline__ void mask_set_range(uint32_t (&m)[4], int lo, int hi)
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int r) {
   const uint32_t w = r < 32 ? m[0] : r < 64 ? m[1] : r < 96 ? m[2] : m[3];
   return (w >> (r & 31)) & 1u;
+}
+
+// Page ids and formats of a run of pages of one sequence, staged in shared
+// memory by the producer warp so that resolving a tile reads no global memory.
+constexpr int kPageCache = 128;
+struct PageCache {
+  int32_t id[kPageCache];
+  uint8_t fmt[kPageCache];
+  int seq, base, count;
+};
+
+// Called by all 32 lanes of one warp: makes pages [pg, pg_last] of sequence b
+// available in the cache (pg_last - pg < kPageCache, pg_last < pg_end),
+// refilling it from pg with one coalesced read of the page table (up to pg_end)
+// when they are not all cached.
+__device__ __forceinline__ void page_cache_ensure(PageCache &pc, const DecodeParams &p, int b,
+                                                  int pg, int pg_last, int pg_end, int lane) {
+  __syncwarp();
+  if (b == pc.seq && pg >= pc.base && pg_last < pc.base + pc.count) return;
+  const int n = min(kPageCache, pg_end - pg);
+  const long long row = static_cast<long long>(b) * p.max_pages + pg;
+  for (int i = lane; i < n; i += 32) {
+    pc.id[i] = p.page_table[row + i];
+    pc.fmt[i] = p.page_fmt ? p.page_fmt[row + i] : static_cast<uint8_t>(p.uniform_fmt);
+  }
+  __syncwarp();
+  if (lane == 0) {
+    pc.seq = b;
+    pc.base = pg;
+    pc.count = n;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void page_cache_reset(PageCache &pc, int lane) {
+  if (lane == 0) {
+    pc.seq = -1;
+    pc.base = 0;
+    pc.count = 0;
+  }
+  __syncwarp();
 }
 
 // Work item -> (split slot, kv head).  Items are numbered split-fastest, so the

@@ -483,7 +483,9 @@ __global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_c
     }
     fence_mbar_init();
   }
+  griddep_launch_dependents();
   __syncthreads();
+  griddep_wait();  // the split schedule comes from the previous kernel
   const long long nitems = static_cast<long long>(p.num_splits[0]) * p.Hkv;
   bool timed_out = false;
   if (threadIdx.x >= CC_WARPS * 32) {
@@ -501,8 +503,8 @@ static cudaError_t cc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  cc_decode_kernel<D, GT><<<grid, CC_THREADS, smem, stream>>>(p);
-  return cudaGetLastError();
+  e = launch_after_previous(cc_decode_kernel<D, GT>, dim3(grid), dim3(CC_THREADS), smem, stream, p);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Number of ring stages that fit next to the fixed shared-memory part.

@@ -66,6 +66,7 @@ struct F32Smem {
   alignas(16) float alpha[2][GT];
   alignas(16) float red[F_WARPS][GT][D];
   int flag;
+  PageCache pc;
 };
 
 template <int D, int GT>
@@ -80,67 +81,89 @@ __host__ __device__ constexpr size_t f32_smem_bytes() {
   return f32_ring_offset<D, GT>() + static_cast<size_t>(F_STAGES) * 2 * F32Cfg<D>::TILE_BYTES + 1024;
 }
 
+// one tile of the producer warp: lane 0 waits for the stage; lane f resolves page
+// piece f of the tile and issues its boxes; lane 0 publishes which rows are valid
+// and the expected byte count.
 template <int D>
-__device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_t *full,
-                             uint64_t *empty, F32Meta *meta, uint8_t *ring, long long nitems,
-                             bool *timed_out) {
+__device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F32Maps &maps,
+                                                 uint64_t *full, uint64_t *empty, F32Meta *meta,
+                                                 uint8_t *ring, const PageCache &pc, int g, int t0,
+                                                 int tok_end, int box_rows, int stage,
+                                                 uint32_t phase, bool *timed_out, int lane) {
   using C = F32Cfg<D>;
   const int P = p.P;
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
+  if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+  const int rows = min(C::T, tok_end - t0);
+  const int npiece = (rows + box_rows - 1) / box_rows;  // <= 16
+  bool pvalid = false;
+  long long id = 0;
+  const int r = lane * box_rows;
+  if (lane < npiece) {
+    const int pg = (t0 + r) / P;
+    const int fmt = pc.fmt[pg - pc.base];
+    id = pc.id[pg - pc.base];
+    if (fmt != CFR_FMT_F32) {
+      set_err(p.err, fmt >= 0 && fmt < kFmtCount ? CFR_DEVERR_POOL : CFR_DEVERR_PAGE_FMT);
+    } else if (id < 0 || id >= p.pool_pages[CFR_FMT_F32]) {
+      set_err(p.err, CFR_DEVERR_PAGE_ID);
+    } else {
+      pvalid = true;
+    }
+  }
+  const uint32_t vb = __ballot_sync(0xffffffffu, pvalid);
+  if (lane == 0) {
+    F32Meta &m = meta[stage];
+    uint32_t valid[4] = {0u, 0u, 0u, 0u};
+    for (int f = 0; f < npiece; ++f)
+      if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
+    for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
+    m.rows = rows;
+    m.t0 = t0;
+    mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(__popc(vb)) * 2u * C::NB * box_rows * 128u);
+  }
+  if (pvalid) {
+    uint8_t *kst = ring + static_cast<size_t>(stage) * 2 * C::TILE_BYTES;
+    uint8_t *vst = kst + C::TILE_BYTES;
+    const int tin = (t0 + r) % P;
+    const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
+#pragma unroll
+    for (int blk = 0; blk < C::NB; ++blk) {
+      tma_load_2d(kst + blk * C::BLOCK_BYTES + r * 128, &maps.k, 32 * blk, y, &full[stage]);
+      tma_load_2d(vst + blk * C::BLOCK_BYTES + r * 128, &maps.v, 32 * blk, y, &full[stage]);
+    }
+  }
+  return true;
+}
+
+// Producer warp: all 32 lanes keep the page-table cache filled and issue the
+// boxes of each tile together.
+template <int D>
+__device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_t *full,
+                             uint64_t *empty, F32Meta *meta, uint8_t *ring, PageCache &pc,
+                             long long nitems, bool *timed_out) {
+  using C = F32Cfg<D>;
+  const int P = p.P;
+  const int lane = threadIdx.x & 31;
   const int box_rows = P < C::T ? P : C::T;
   int stage = 0;
   uint32_t phase = 0;
-  prefetch_map(&maps.k);
-  prefetch_map(&maps.v);
+  if (lane == 0) {
+    prefetch_map(&maps.k);
+    prefetch_map(&maps.v);
+  }
+  page_cache_reset(pc, lane);
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
     item_coords(item, p.num_splits[0], slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int tok_end = min(p.seq_lens[b], pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += C::T) {
-      if (!mbar_wait(&empty[stage], phase ^ 1u, p.err, timed_out)) return;
-      F32Meta &m = meta[stage];
-      const int rows = min(C::T, tok_end - t0);
-      uint32_t valid[4] = {0u, 0u, 0u, 0u};
-      uint32_t bytes = 0;
-      // pass 1: resolve the pages of the tile
-      for (int r = 0; r < rows; r += box_rows) {
-        const int j = t0 + r, pg = j / P;
-        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
-        const int fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
-        const long long id = p.page_table[cell];
-        bool ok = false;
-        if (fmt != CFR_FMT_F32) {
-          set_err(p.err, fmt >= 0 && fmt < kFmtCount ? CFR_DEVERR_POOL : CFR_DEVERR_PAGE_FMT);
-        } else if (id < 0 || id >= p.pool_pages[CFR_FMT_F32]) {
-          set_err(p.err, CFR_DEVERR_PAGE_ID);
-        } else {
-          ok = true;
-        }
-        if (ok) {
-          const int hi = min(rows, r + box_rows);
-          mask_set_range(valid, r, hi);
-          bytes += 2u * C::NB * box_rows * 128u;
-        }
-      }
-      for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
-      m.rows = rows;
-      m.t0 = t0;
-      mbar_arrive_expect_tx(&full[stage], bytes);
-      // pass 2: issue the boxes of the resolved pages
-      uint8_t *kst = ring + static_cast<size_t>(stage) * 2 * C::TILE_BYTES;
-      uint8_t *vst = kst + C::TILE_BYTES;
-      for (int r = 0; r < rows; r += box_rows) {
-        if (!mask_bit(valid, r)) continue;
-        const int j = t0 + r, pg = j / P, tin = j - pg * P;
-        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
-        const long long id = p.page_table[cell];
-        const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
-#pragma unroll
-        for (int blk = 0; blk < C::NB; ++blk) {
-          tma_load_2d(kst + blk * C::BLOCK_BYTES + r * 128, &maps.k, 32 * blk, y, &full[stage]);
-          tma_load_2d(vst + blk * C::BLOCK_BYTES + r * 128, &maps.v, 32 * blk, y, &full[stage]);
-        }
-      }
+      page_cache_ensure(pc, p, b, t0 / P, (min(t0 + C::T, tok_end) - 1) / P, pe, lane);
+      if (!f32_produce_tile<D>(p, maps, full, empty, meta, ring, pc, g, t0, tok_end, box_rows, stage,
+                               phase, timed_out, lane))
+        return;
       if (++stage == F_STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -386,12 +409,13 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     }
     fence_mbar_init();
   }
+  griddep_launch_dependents();
   __syncthreads();
+  griddep_wait();  // the split schedule comes from the previous kernel
   const long long nitems = static_cast<long long>(p.num_splits[0]) * p.Hkv;
   bool timed_out = false;
   if (threadIdx.x >= F_WARPS * 32) {
-    if (threadIdx.x == F_WARPS * 32)
-      f32_producer<D>(p, maps, S.full, S.empty, S.meta, ring, nitems, &timed_out);
+    f32_producer<D>(p, maps, S.full, S.empty, S.meta, ring, S.pc, nitems, &timed_out);
   } else {
     f32_consumer<D, GT>(p, S, ring, nitems, &timed_out);
   }
@@ -430,8 +454,9 @@ static cudaError_t f32_launch_t(const DecodeParams &p, int grid, cudaStream_t st
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  f32_decode_kernel<D, GT><<<grid, F_THREADS, smem, stream>>>(p, maps);
-  return cudaGetLastError();
+  e = launch_after_previous(f32_decode_kernel<D, GT>, dim3(grid), dim3(F_THREADS), smem, stream, p,
+                            maps);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode_f32(const DecodeParams &p, int grid, cudaStream_t stream) {

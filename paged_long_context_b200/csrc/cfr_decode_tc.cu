@@ -5,7 +5,7 @@
 // contractions:
 //   S^T[128 tok x N] = K_tile[128 x 128] . Q^T           (M = tokens, K = head_dim)
 //   O^T[128 dim x N] = V_tile^T[128 x 128] . P^T          (M = head_dim, K = tokens)
-// N = 16 (G <= 8) or 32 (G <= 16) columns: G "hi" and G "lo" halves, so that q
+// N = 16 (G <= 8) or 32 (G <= 16) columns: N/2 "hi" and N/2 "lo" columns, so that q
 // (fp32 or bf16) and the probabilities p enter the 16-bit MMA as hi + lo pairs
 // (about 16 significant bits for bf16, 22 for fp16), accumulated in fp32.
 // bf16 pages run bf16 MMAs; int8 / int4 pages are expanded to fp16 codes in
@@ -52,7 +52,7 @@ constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2;
 
 struct TcMeta {
   uint32_t valid[4];
-  int rows, t0, kind;
+  int rows, t0, kind, direct;
   float ks, vs;
 };
 
@@ -75,10 +75,11 @@ struct TcSmem {
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
   uint64_t q_full, drain;
   uint32_t tmem_base;
-  int flag_sm, flag_st;
+  int flag_st[3];
   TcMeta meta[3];
   alignas(16) float red_max[2][4][16];
   alignas(16) float red_l[4][16];
+  PageCache pc;
 };
 
 template <int NCOL, bool INTP>
@@ -217,90 +218,135 @@ struct TcCtx {
   int nsplit;
 };
 
+// non-blocking probe of an mbarrier phase
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// one tile of the producer warp: lane 0 waits for the stage; lane f resolves
+// page piece f of the tile and issues its copies, so a tile made of many small
+// pages is issued in parallel; lane 0 publishes the tile description and the
+// expected byte count.
+template <int NCOL, bool INTP>
+__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int g, int t0,
+                                                int tok_end, int stage, uint32_t phase,
+                                                bool *timed_out, int lane) {
+  const DecodeParams &p = c.p;
+  const PageCache &pc = c.S.pc;
+  const int P = p.P;
+  const int box_rows = P < TC_T ? P : TC_T;
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
+  if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+  const int rows = min(TC_T, tok_end - t0);
+  const int npiece = (rows + box_rows - 1) / box_rows;  // <= 16
+  // ---- resolve piece `lane` ----
+  bool pvalid = false;
+  int fmt = -1;
+  long long id = 0;
+  const int r = lane * box_rows;
+  if (lane < npiece) {
+    const int pg = (t0 + r) / P;
+    fmt = pc.fmt[pg - pc.base];
+    id = pc.id[pg - pc.base];
+    if (fmt < 0 || fmt >= kFmtCount) {
+      set_err(p.err, CFR_DEVERR_PAGE_FMT);
+    } else if (fmt == CFR_FMT_F32 || !p.k_pool[fmt] ||
+               ((fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) && !p.scales[fmt])) {
+      set_err(p.err, CFR_DEVERR_POOL);
+    } else if (id < 0 || id >= p.pool_pages[fmt]) {
+      set_err(p.err, CFR_DEVERR_PAGE_ID);
+    } else {
+      pvalid = true;
+    }
+  }
+  const uint32_t vb = __ballot_sync(0xffffffffu, pvalid);
+  // quantised pages need page_tokens >= 128: the tile is then one piece (lane 0)
+  const int kind0 = (fmt == CFR_FMT_I8 && pvalid) ? KIND_I8 : (fmt == CFR_FMT_I4 && pvalid) ? KIND_I4 : KIND_BF16;
+  const int kind = __shfl_sync(0xffffffffu, kind0, 0);
+  uint64_t *done = nullptr;
+  if (lane == 0) {
+    TcMeta &m = c.S.meta[stage];
+    uint32_t valid[4] = {0u, 0u, 0u, 0u};
+    for (int f = 0; f < npiece; ++f)
+      if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
+    float ks = 1.f, vs = 1.f;
+    uint32_t bytes;
+    if (kind == KIND_BF16) {
+      bytes = static_cast<uint32_t>(__popc(vb)) * 4u * box_rows * 128u;
+    } else {
+      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+      ks = sc.x;
+      vs = sc.y;
+      bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, TC_D));
+    }
+    // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA; every
+    // other tile passes through the staging warps
+    const bool direct = kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu;
+    for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
+    m.rows = rows;
+    m.t0 = t0;
+    m.kind = kind;
+    m.direct = direct ? 1 : 0;
+    m.ks = ks;
+    m.vs = vs;
+    done = direct ? &c.S.op_full[stage] : &c.S.raw_full[stage];
+    if (direct) mbar_arrive(&c.S.raw_full[stage]);  // lets the staging warps skip this tile
+    mbar_arrive_expect_tx(done, bytes);
+  }
+  // every lane learns where its copies complete
+  const int dsel = __shfl_sync(0xffffffffu, (lane == 0 && done == &c.S.op_full[stage]) ? 1 : 0, 0);
+  done = dsel ? &c.S.op_full[stage] : &c.S.raw_full[stage];
+  if (pvalid) {
+    const int tin = (t0 + r) % P;
+    uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
+    if (kind == KIND_BF16) {
+      const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
+      tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, done);
+      tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
+      tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, done);
+      tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
+    } else if (INTP) {
+      const int rb = row_bytes(fmt, TC_D);
+      const long long off = ((id * p.Hkv + g) * P + tin) * rb;
+      uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
+      bulk_g2s(raw, p.k_pool[fmt] + off, rows * rb, done);
+      bulk_g2s(raw + TC_T * TC_D, p.v_pool[fmt] + off, rows * rb, done);
+    }
+  }
+  return true;
+}
+
+// Producer warp: all 32 lanes keep the page-table cache filled and issue the
+// copies of each tile together.
 template <int NCOL, bool INTP>
 __device__ void tc_producer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
-  const int box_rows = P < TC_T ? P : TC_T;
+  const int lane = threadIdx.x & 31;
   int stage = 0;
   uint32_t phase = 0;
-  if (p.k_pool[CFR_FMT_BF16]) {
+  if (lane == 0 && p.k_pool[CFR_FMT_BF16]) {
     prefetch_map(&c.maps.k);
     prefetch_map(&c.maps.v);
   }
+  page_cache_reset(c.S.pc, lane);
   for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int tok_end = min(p.seq_lens[b], pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
-      if (!mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out)) return;
-      TcMeta &m = c.S.meta[stage];
-      const int rows = min(TC_T, tok_end - t0);
-      uint32_t valid[4] = {0u, 0u, 0u, 0u};
-      uint32_t bytes = 0;
-      int kind = KIND_BF16;
-      float ks = 1.f, vs = 1.f;
-      // resolve every page piece of the tile (one piece when page_tokens >= 128)
-      for (int r = 0; r < rows; r += box_rows) {
-        const int j = t0 + r, pg = j / P;
-        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
-        const int fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
-        const long long id = p.page_table[cell];
-        bool ok = false;
-        if (fmt < 0 || fmt >= kFmtCount) {
-          set_err(p.err, CFR_DEVERR_PAGE_FMT);
-        } else if (fmt == CFR_FMT_F32 || !p.k_pool[fmt] ||
-                   ((fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) && !p.scales[fmt])) {
-          set_err(p.err, CFR_DEVERR_POOL);
-        } else if (id < 0 || id >= p.pool_pages[fmt]) {
-          set_err(p.err, CFR_DEVERR_PAGE_ID);
-        } else {
-          ok = true;
-        }
-        if (!ok) continue;
-        const int hi = min(rows, r + box_rows);
-        mask_set_range(valid, r, hi);
-        if (fmt == CFR_FMT_BF16) {
-          bytes += 4u * box_rows * 128u;
-        } else {
-          // quantised: page_tokens >= 128, so this is the tile's only piece
-          kind = fmt == CFR_FMT_I8 ? KIND_I8 : KIND_I4;
-          const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
-          ks = s.x;
-          vs = s.y;
-          bytes += 2u * rows * static_cast<uint32_t>(row_bytes(fmt, TC_D));
-        }
-      }
-      for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
-      m.rows = rows;
-      m.t0 = t0;
-      m.kind = kind;
-      m.ks = ks;
-      m.vs = vs;
-      mbar_arrive_expect_tx(&c.S.raw_full[stage], bytes);
-      uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
-      for (int r = 0; r < rows; r += box_rows) {
-        if (!mask_bit(valid, r)) continue;
-        const int j = t0 + r, pg = j / P, tin = j - pg * P;
-        const long long cell = static_cast<long long>(b) * p.max_pages + pg;
-        const long long id = p.page_table[cell];
-        if (kind == KIND_BF16) {
-          const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
-          tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, &c.S.raw_full[stage]);
-          tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, &c.S.raw_full[stage]);
-          tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, &c.S.raw_full[stage]);
-          tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, &c.S.raw_full[stage]);
-        } else if (INTP) {
-          const int fmt = kind == KIND_I8 ? CFR_FMT_I8 : CFR_FMT_I4;
-          const int rb = row_bytes(fmt, TC_D);
-          const long long off = ((id * p.Hkv + g) * P + tin) * rb;
-          uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
-          bulk_g2s(raw, p.k_pool[fmt] + off, rows * rb, &c.S.raw_full[stage]);
-          bulk_g2s(raw + TC_T * TC_D, p.v_pool[fmt] + off, rows * rb, &c.S.raw_full[stage]);
-        }
-      }
+      page_cache_ensure(c.S.pc, p, b, t0 / P, (min(t0 + TC_T, tok_end) - 1) / P, pe, lane);
+      if (!tc_produce_tile(c, b, g, t0, tok_end, stage, phase, timed_out, lane)) return;
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -309,7 +355,7 @@ __device__ void tc_producer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   }
 }
 
-// staging warpgroup: thread r (0..127) owns row r of every tile
+// staging warpgroup: thread r (0..127) owns row r of every tile that is not direct
 template <int NCOL, bool INTP>
 __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
@@ -325,83 +371,87 @@ __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int tok_end = min(p.seq_lens[b], pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
-      if (r == 0) c.S.flag_st = mbar_wait(&c.S.raw_full[stage], phase, p.err, timed_out) ? 1 : 0;
+      // elected bounded wait; the outcome slot is per stage, so a slow reader can
+      // never see the next use of the slot (that needs every thread's barrier)
+      if (r == 0) c.S.flag_st[stage] = mbar_wait(&c.S.raw_full[stage], phase, p.err, timed_out) ? 1 : 0;
       named_sync(3, 128);
-      if (c.S.flag_st == 0) {
+      if (c.S.flag_st[stage] == 0) {
         *timed_out = true;
         return;
       }
       (void)mbar_try_wait(&c.S.raw_full[stage], phase);
       const TcMeta &m = c.S.meta[stage];
-      const bool valid = (m.valid[r >> 5] >> (r & 31)) & 1u;
-      uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
-      if (m.kind == KIND_BF16) {
-        if (!valid) {
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            *reinterpret_cast<uint4 *>(op + 2 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-          }
-        }
-      } else if (INTP) {
-        const uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
-#pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
-          uint8_t *dst = op + kv * 2 * TC_HALF;
+      if (!m.direct) {
+        const bool valid = (m.valid[r >> 5] >> (r & 31)) & 1u;
+        uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
+        if (m.kind == KIND_BF16) {
           if (!valid) {
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-              *reinterpret_cast<uint4 *>(dst + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4 *>(dst + TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4 *>(op + 2 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
             }
-            continue;
           }
-          if (m.kind == KIND_I8) {
-            // 128 codes = 8 chunks of 16 bytes; start at a row-dependent chunk (no bank conflicts)
-            const uint8_t *src = raw + kv * TC_T * TC_D + r * TC_D;
+        } else if (INTP) {
+          const uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int ci = (j + r) & 7;  // input chunk: codes 16ci .. 16ci+15
-              const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
-              uint32_t o[8];
-              i8x4_to_h2x2(w.x, o[0], o[1]);
-              i8x4_to_h2x2(w.y, o[2], o[3]);
-              i8x4_to_h2x2(w.z, o[4], o[5]);
-              i8x4_to_h2x2(w.w, o[6], o[7]);
-              // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
-              uint8_t *hb = dst + (ci >> 2) * TC_HALF;
-              const int oc = (2 * ci) & 7;
-              *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
-              *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+          for (int kv = 0; kv < 2; ++kv) {
+            uint8_t *dst = op + kv * 2 * TC_HALF;
+            if (!valid) {
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) {
+                *reinterpret_cast<uint4 *>(dst + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(dst + TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+              }
+              continue;
             }
-          } else {
-            // 128 codes = 64 bytes = 4 chunks of 16 bytes (32 codes each)
-            const uint8_t *src = raw + kv * TC_T * TC_D + r * (TC_D / 2);
+            if (m.kind == KIND_I8) {
+              // 128 codes = 8 chunks of 16 bytes; start at a row-dependent chunk (no bank conflicts)
+              const uint8_t *src = raw + kv * TC_T * TC_D + r * TC_D;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int ci = (j + (r >> 1)) & 3;  // input chunk: codes 32ci .. 32ci+31
-              const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
-              const uint32_t wv[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
-                                      w.w ^ 0x88888888u};
-              uint32_t o[16];
+              for (int j = 0; j < 8; ++j) {
+                const int ci = (j + r) & 7;  // input chunk: codes 16ci .. 16ci+15
+                const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+                uint32_t o[8];
+                i8x4_to_h2x2(w.x, o[0], o[1]);
+                i8x4_to_h2x2(w.y, o[2], o[3]);
+                i8x4_to_h2x2(w.z, o[4], o[5]);
+                i8x4_to_h2x2(w.w, o[6], o[7]);
+                // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
+                uint8_t *hb = dst + (ci >> 2) * TC_HALF;
+                const int oc = (2 * ci) & 7;
+                *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+              }
+            } else {
+              // 128 codes = 64 bytes = 4 chunks of 16 bytes (32 codes each)
+              const uint8_t *src = raw + kv * TC_T * TC_D + r * (TC_D / 2);
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
+              for (int j = 0; j < 4; ++j) {
+                const int ci = (j + (r >> 1)) & 3;  // input chunk: codes 32ci .. 32ci+31
+                const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+                const uint32_t wv[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
+                                        w.w ^ 0x88888888u};
+                uint32_t o[16];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) o[4 * q + k] = i4x2_to_h2(wv[q], k);
-              // output chunks 4ci .. 4ci+3 in half ci/2
-              uint8_t *hb = dst + (ci >> 1) * TC_HALF;
-              const int oc = (4 * ci) & 7;
+                for (int q = 0; q < 4; ++q)
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(hb + sw128(r, oc + q)) =
-                    make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                  for (int k = 0; k < 4; ++k) o[4 * q + k] = i4x2_to_h2(wv[q], k);
+                // output chunks 4ci .. 4ci+3 in half ci/2
+                uint8_t *hb = dst + (ci >> 1) * TC_HALF;
+                const int oc = (4 * ci) & 7;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  *reinterpret_cast<uint4 *>(hb + sw128(r, oc + q)) =
+                      make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+              }
             }
           }
         }
+        fence_async_smem();
+        named_sync(3, 128);
+        if (r == 0) mbar_arrive(&c.S.op_full[stage]);
       }
-      fence_async_smem();
-      named_sync(3, 128);
-      if (r == 0) mbar_arrive(&c.S.op_full[stage]);
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -410,6 +460,24 @@ __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   }
 }
 
+// token range of work item `item` (no-op past the last item)
+template <int NCOL, bool INTP>
+__device__ __forceinline__ void tc_item_range(TcCtx<NCOL, INTP> &c, long long item, int &t0, int &end,
+                                              bool &need_q) {
+  if (item < c.nitems) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    (void)g;
+    const int b = c.p.splits[3 * slot];
+    t0 = c.p.splits[3 * slot + 1] * c.p.P;
+    end = min(c.p.seq_lens[b], c.p.splits[3 * slot + 2] * c.p.P);
+    need_q = true;
+  }
+}
+
+// MMA issuer (one thread).  QK of a tile is issued as soon as its operands and
+// an S buffer are ready; P.V of a tile as soon as its probabilities and an O
+// buffer are ready -- polled without blocking, so neither waits on the other.
 template <int NCOL, bool INTP>
 __device__ void tc_mma_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
@@ -417,99 +485,105 @@ __device__ void tc_mma_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   const int P = p.P;
   const uint32_t tmem = c.S.tmem_base;
   const uint32_t op0 = smem_u32(c.op), q0 = smem_u32(c.qop), p0 = smem_u32(c.pop);
-  int stage = 0;
-  uint32_t phase = 0;
-  long long tc = 0;
-  int item_k = 0;
-  bool pending = false;
-  int pend_stage = 0, pend_kind = 0;
-  long long pend_tc = 0;
-
-  auto issue_pv = [&](long long i, int st, int kind) -> bool {
-    const uint32_t par = static_cast<uint32_t>((i >> 1) & 1);
-    if (!mbar_wait(&c.S.p_full[i & 1], par, p.err, timed_out)) return false;
-    if (!mbar_wait(&c.S.o_empty[i & 1], par ^ 1u, p.err, timed_out)) return false;
-    tc_fence_after();
-    const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
-    const uint32_t vbase = op0 + st * TC_OP_BYTES + 2 * TC_HALF;
-    const uint32_t pbase = p0 + static_cast<uint32_t>(i & 1) * Cfg::P_BYTES;
-    const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(i & 1) * NCOL;
+  // QK cursor over the flattened (item, tile) sequence
+  long long q_item = blockIdx.x;
+  int q_item_k = 0, q_t0 = 0, q_end = 0, q_stage = 0;
+  uint32_t q_phase = 0;
+  bool q_need_q = false;
+  tc_item_range(c, q_item, q_t0, q_end, q_need_q);
+  long long qk_tc = 0, pv_tc = 0;
+  // stage and kind of the tiles between the two cursors (at most four), four bits
+  // each, kept in registers
+  uint32_t stage_bits = 0, kind_bits = 0;
+  uint64_t idle_since = 0;
+  while (!*timed_out) {
+    bool progress = false;
+    // ---- QK of the next tile ----
+    if (q_item < c.nitems) {
+      if (q_need_q && mbar_test(&c.S.q_full, static_cast<uint32_t>(q_item_k & 1))) q_need_q = false;
+      if (!q_need_q && mbar_test(&c.S.op_full[q_stage], q_phase) &&
+          mbar_test(&c.S.s_empty[qk_tc & 1], static_cast<uint32_t>((qk_tc >> 1) & 1) ^ 1u)) {
+        tc_fence_after();
+        const int kind = c.S.meta[q_stage].kind;
+        const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
+        const uint32_t kbase = op0 + q_stage * TC_OP_BYTES;
+        const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
+        const uint32_t d = tmem + static_cast<uint32_t>(qk_tc & 1) * NCOL;
 #pragma unroll
-    for (int k = 0; k < TC_T / 16; ++k) {
-      const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
-      const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
-      tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
-    }
-    tc_commit(&c.S.o_full[i & 1]);
-    tc_commit(&c.S.p_empty[i & 1]);
-    tc_commit(&c.S.op_empty[st]);
-    return true;
-  };
-
-  for (long long item = blockIdx.x; item < c.nitems && !*timed_out; item += gridDim.x, ++item_k) {
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    (void)g;
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
-    const int tok_end = min(p.seq_lens[b], pe * P);
-    if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(item_k & 1), p.err, timed_out)) break;
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
-      if (!mbar_wait(&c.S.op_full[stage], phase, p.err, timed_out)) break;
-      const int kind = c.S.meta[stage].kind;
-      if (!mbar_wait(&c.S.s_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err,
-                     timed_out))
-        break;
-      tc_fence_after();
-      const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
-      const uint32_t kbase = op0 + stage * TC_OP_BYTES;
-      const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
-      const uint32_t d = tmem + static_cast<uint32_t>(tc & 1) * NCOL;
-#pragma unroll
-      for (int k = 0; k < TC_D / 16; ++k) {
-        const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
-        const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
-        tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        for (int k = 0; k < TC_D / 16; ++k) {
+          const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
+          const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
+          tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        tc_commit(&c.S.s_full[qk_tc & 1]);
+        const uint32_t sh = 4u * static_cast<uint32_t>(qk_tc & 7);
+        stage_bits = (stage_bits & ~(0xFu << sh)) | (static_cast<uint32_t>(q_stage) << sh);
+        kind_bits = (kind_bits & ~(0xFu << sh)) | (static_cast<uint32_t>(kind) << sh);
+        ++qk_tc;
+        if (++q_stage == Cfg::STAGES) {
+          q_stage = 0;
+          q_phase ^= 1u;
+        }
+        q_t0 += TC_T;
+        if (q_t0 >= q_end) {
+          q_item += gridDim.x;
+          ++q_item_k;
+          tc_item_range(c, q_item, q_t0, q_end, q_need_q);
+        }
+        progress = true;
       }
-      tc_commit(&c.S.s_full[tc & 1]);
-      if (pending && !issue_pv(pend_tc, pend_stage, pend_kind)) break;
-      pending = true;
-      pend_tc = tc;
-      pend_stage = stage;
-      pend_kind = kind;
-      ++tc;
-      if (++stage == Cfg::STAGES) {
-        stage = 0;
-        phase ^= 1u;
+    }
+    // ---- P.V of the oldest tile whose probabilities are ready ----
+    if (pv_tc < qk_tc) {
+      const uint32_t par = static_cast<uint32_t>((pv_tc >> 1) & 1);
+      if (mbar_test(&c.S.p_full[pv_tc & 1], par) && mbar_test(&c.S.o_empty[pv_tc & 1], par ^ 1u)) {
+        tc_fence_after();
+        const uint32_t sh = 4u * static_cast<uint32_t>(pv_tc & 7);
+        const int st = static_cast<int>((stage_bits >> sh) & 0xFu);
+        const int kind = static_cast<int>((kind_bits >> sh) & 0xFu);
+        const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
+        const uint32_t vbase = op0 + st * TC_OP_BYTES + 2 * TC_HALF;
+        const uint32_t pbase = p0 + static_cast<uint32_t>(pv_tc & 1) * Cfg::P_BYTES;
+        const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(pv_tc & 1) * NCOL;
+#pragma unroll
+        for (int k = 0; k < TC_T / 16; ++k) {
+          const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
+          const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
+          tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        tc_commit(&c.S.o_full[pv_tc & 1]);
+        tc_commit(&c.S.p_empty[pv_tc & 1]);
+        tc_commit(&c.S.op_empty[st]);
+        ++pv_tc;
+        progress = true;
+      }
+    }
+    if (q_item >= c.nitems && pv_tc == qk_tc) break;
+    if (progress) {
+      idle_since = 0;
+    } else {
+      const uint64_t now = global_ns();
+      if (idle_since == 0) {
+        idle_since = now;
+      } else if (now - idle_since > kWaitLimitNs) {
+        set_err(p.err, CFR_DEVERR_TIMEOUT);
+        *timed_out = true;
       }
     }
   }
-  if (pending && !*timed_out) issue_pv(pend_tc, pend_stage, pend_kind);
   // drain: every MMA issued so far has completed before TMEM is released
   tc_commit(&c.S.drain);
   bool t2 = false;
   (void)mbar_wait(&c.S.drain, 0, p.err, &t2);
 }
 
-// elected bounded wait of the softmax warpgroup; the outcome is shared by all 128 threads
-template <int NCOL, bool INTP>
-__device__ __forceinline__ bool tc_group_wait(TcCtx<NCOL, INTP> &c, uint64_t *bar, uint32_t parity,
-                                              int tsm, bool *timed_out) {
-  if (tsm == 0) c.S.flag_sm = mbar_wait(bar, parity, c.p.err, timed_out) ? 1 : 0;
-  named_sync(2, 128);
-  const bool ok = c.S.flag_sm != 0;
-  named_sync(2, 128);
-  if (!ok) *timed_out = true;
-  return ok;
-}
-
 // folds the P.V product of tile i into the running accumulators (dim t of each head)
 template <int NCOL, bool INTP>
-__device__ __forceinline__ bool tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint32_t tmem, int lane,
-                                        int tsm, int cnt, float (&acc)[NCOL / 2],
+__device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint32_t tmem, int lane,
+                                        int cnt, float (&acc)[NCOL / 2],
                                         const float (&alpha_prev)[NCOL / 2], float vscale_prev,
                                         bool *timed_out) {
-  if (!tc_group_wait(c, &c.S.o_full[i & 1], static_cast<uint32_t>((i >> 1) & 1), tsm, timed_out))
-    return false;
+  (void)mbar_wait(&c.S.o_full[i & 1], static_cast<uint32_t>((i >> 1) & 1), c.p.err, timed_out);
   tc_fence_after();
   float o[NCOL];
   tmem_ld<NCOL>(tmem + 2 * NCOL + static_cast<uint32_t>(i & 1) * NCOL, o);
@@ -518,48 +592,30 @@ __device__ __forceinline__ bool tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint3
   __syncwarp();
   if (lane == 0) mbar_arrive(&c.S.o_empty[i & 1]);
 #pragma unroll
-  for (int h = 0; h < NCOL / 2; ++h) {
-    float ohl = 0.f;
-#pragma unroll
-    for (int k = 0; k < NCOL; ++k)
-      if (k == cnt + h) ohl = o[k];
-    if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + ohl) * vscale_prev);
-  }
-  return true;
+  for (int h = 0; h < NCOL / 2; ++h)
+    if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
 }
 
-// softmax / fold warpgroup
+// writes the hi/lo query operand of item `it` (both bf16 and fp16 copies); the
+// warpgroup's 128 threads (index tsm) share the work, each warp then arrives on q_full
 template <int NCOL, bool INTP>
-__device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP> &c, long long it, int tsm, int lane) {
   using Cfg = TcCfg<NCOL, INTP>;
-  constexpr int GM = NCOL / 2;  // most query heads per tile
   const DecodeParams &p = c.p;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int quarter = warp & 3;
-  const int t = 32 * quarter + lane;  // TMEM lane: token t of S, dim t of O
-  const int tsm = threadIdx.x - 64;   // 0..127 within the warpgroup
-  const uint32_t tmem = c.S.tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
-  const int P = p.P;
-  int stage = 0;
-  uint32_t phase = 0;
-  long long tc = 0;
-  int item_k = 0;
-  bool q_ready = false;
-
-  // writes the hi/lo query operand of item `it` (both bf16 and fp16 copies)
-  auto write_q = [&](long long it) {
+  {
     int slot, g;
     item_coords(it, c.nsplit, slot, g);
     const int b = p.splits[3 * slot];
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
     for (int idx = tsm; idx < NCOL * 16; idx += 128) {
       const int n = idx >> 4, ch = idx & 15;  // row n, 8-element chunk ch of 16
-      const int head = n < cnt ? n : (n - cnt < cnt ? n - cnt : -1);
-      const bool lo_part = n >= cnt;
+      constexpr int GM = NCOL / 2;            // rows [0, GM): hi parts, [GM, NCOL): lo parts
+      const bool lo_part = n >= GM;
+      const int head = lo_part ? n - GM : n;
       float x[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = 0.f;
-      if (head >= 0 && n < 2 * cnt) {
+      if (head < cnt) {
         const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * TC_D + 8 * ch;
         if (p.q_fmt == CFR_FMT_F32) {
           const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi);
@@ -597,16 +653,36 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&c.S.q_full);
-  };
+  }
+}
 
-  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x, ++item_k) {
+// softmax / fold warpgroup.  Every thread waits on the mbarriers itself; a
+// thread whose wait gives up keeps the same control flow (later waits return at
+// once), so the one named barrier per tile is always reached by all 128 threads.
+template <int NCOL, bool INTP>
+__device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+  using Cfg = TcCfg<NCOL, INTP>;
+  constexpr int GM = NCOL / 2;  // most query heads per tile
+  const DecodeParams &p = c.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int t = 32 * quarter + lane;  // TMEM lane: token t of S, dim t of O
+  const int tsm = threadIdx.x - 64;   // 0..127 within the warpgroup
+  const uint32_t tmem = c.S.tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
+  const int P = p.P;
+  int stage = 0;
+  uint32_t phase = 0;
+  long long tc = 0;
+  bool q_ready = false;
+
+  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
-    if (!q_ready) write_q(item);
+    if (!q_ready) tc_write_q(c, item, tsm, lane);
     q_ready = false;
 
     float slope2[GM], m_run[GM], l_part[GM], acc[GM], alpha_prev[GM];
@@ -621,10 +697,9 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
     float vscale_prev = 1.f;
     long long prev_tc = -1;
 
-    bool ok = true;
-    for (int t0 = pb * P; t0 < tok_end && ok; t0 += TC_T) {
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       // ---- scores of tile tc ----
-      if (!tc_group_wait(c, &c.S.s_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), tsm, timed_out)) { ok = false; break; }
+      (void)mbar_wait(&c.S.s_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), p.err, timed_out);
       tc_fence_after();
       float sv[NCOL];
       tmem_ld<NCOL>(tmem + static_cast<uint32_t>(tc & 1) * NCOL, sv);
@@ -644,18 +719,15 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
       float s[GM];
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
-        float shl = 0.f;
-#pragma unroll
-        for (int k = 0; k < NCOL; ++k)
-          if (k == cnt + h) shl = sv[k];
-        s[h] = (valid && h < cnt) ? fmaf(sv[h] + shl, scale, -slope2[h] * dist) : -INFINITY;
+        s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
         float mx = s[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         if (lane == 0) c.S.red_max[tc & 1][quarter][h] = mx;
       }
-      // the P buffer of this tile must be free (PV of tile tc-2 done)
-      if (!tc_group_wait(c, &c.S.p_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, tsm, timed_out)) { ok = false; break; }
+      // the P buffer of this tile must be free (P.V of tile tc-2 done)
+      (void)mbar_wait(&c.S.p_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err, timed_out);
+      named_sync(2, 128);
       float pr[GM], alpha[GM];
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
@@ -672,7 +744,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
         l_part[h] = fmaf(l_part[h], alpha[h], pr[h]);
         m_run[h] = m_new;
       }
-      // P^T row t: columns [hi(0..cnt) | lo(0..cnt) | 0]
+      // P^T row t: columns [hi(0..GM) | lo(0..GM)]
       {
         float colv[NCOL];
 #pragma unroll
@@ -680,17 +752,11 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
         const float pre = kind == KIND_BF16 ? 1.f : 32768.f;
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
-          if (h < cnt) {
-            const float x = pr[h] * pre;
-            const float xh = kind == KIND_BF16 ? __bfloat162float(__float2bfloat16_rn(x))
-                                               : __half2float(__float2half_rn(x));
-            // place hi at column h and lo at column cnt + h
-#pragma unroll
-            for (int k = 0; k < NCOL; ++k) {
-              if (k == h) colv[k] = xh;
-              if (k == cnt + h) colv[k] = x - xh;
-            }
-          }
+          const float x = pr[h] * pre;  // 0 for the padding heads h >= cnt
+          const float xh = kind == KIND_BF16 ? __bfloat162float(__float2bfloat16_rn(x))
+                                             : __half2float(__float2half_rn(x));
+          colv[h] = xh;
+          colv[GM + h] = x - xh;
         }
         uint8_t *pb_ = c.pop + (tc & 1) * Cfg::P_BYTES;
 #pragma unroll
@@ -707,18 +773,17 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.S.p_full[tc & 1]);
 
-      const bool last = t0 + TC_T >= tok_end;
-      if (last) {
+      if (t0 + TC_T >= tok_end) {
         // the next item's query operand can be written as soon as this item's
         // last QK product has been read
         const long long nx = item + gridDim.x;
         if (nx < c.nitems) {
-          write_q(nx);
+          tc_write_q(c, nx, tsm, lane);
           q_ready = true;
         }
       }
       // fold the previous tile of this item
-      if (prev_tc >= 0 && !tc_fold(c, prev_tc, tmem, lane, tsm, cnt, acc, alpha_prev, vscale_prev, timed_out)) { ok = false; break; }
+      if (prev_tc >= 0) tc_fold(c, prev_tc, tmem, lane, cnt, acc, alpha_prev, vscale_prev, timed_out);
 #pragma unroll
       for (int h = 0; h < GM; ++h) alpha_prev[h] = alpha[h];
       vscale_prev = vsc;
@@ -729,10 +794,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
         phase ^= 1u;
       }
     }
-    if (!ok || (prev_tc >= 0 && !tc_fold(c, prev_tc, tmem, lane, tsm, cnt, acc, alpha_prev, vscale_prev, timed_out))) {
-      *timed_out = true;
-      return;
-    }
+    if (prev_tc >= 0) tc_fold(c, prev_tc, tmem, lane, cnt, acc, alpha_prev, vscale_prev, timed_out);
 
     // split partial: acc (dim t), m, and l summed over the 128 token slots
 #pragma unroll
@@ -794,15 +856,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the split schedule comes from the previous kernel
 
   TcCtx<NCOL, INTP> c{p, maps, S, smem + L::op, smem + L::raw, smem + L::q, smem + L::pbuf,
                       static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
   bool timed_out = false;
   if (warp == 0) {
-    if ((threadIdx.x & 31) == 0) tc_producer<NCOL, INTP>(c, &timed_out);
+    tc_producer<NCOL, INTP>(c, &timed_out);
   } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0) tc_mma_issuer<NCOL, INTP>(c, &timed_out);
   } else if (warp < 6) {
@@ -865,8 +929,9 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  tc_decode_kernel<NCOL, INTP><<<grid, TC_THREADS, smem, stream>>>(p, maps);
-  return cudaGetLastError();
+  e = launch_after_previous(tc_decode_kernel<NCOL, INTP>, dim3(grid), dim3(TC_THREADS), smem, stream,
+                            p, maps);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream) {

@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     const int32_t *__restrict__ seq_lens, int batch, int P, int max_pages, int target,
     int32_t *__restrict__ split_off, int32_t *__restrict__ splits, int max_splits,
     int32_t *__restrict__ num_splits, uint32_t *err) {
+  griddep_launch_dependents();
   __shared__ long long red_ll[33];
   __shared__ int red_i[33];
   long long local = 0;
