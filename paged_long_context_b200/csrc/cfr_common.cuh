@@ -2,8 +2,9 @@
 //
 // mbarrier-based producer/consumer hand-off with bounded waits, the 1-D bulk
 // copy engine (TMA, no multicast), error-word reporting and small numeric
-// helpers.  Every spin on an mbarrier gives up after a wall-clock limit, sets
-// CFR_DEVERR_TIMEOUT in the error word and lets the kernel return.
+// helpers.  Every spin on an mbarrier gives up after a clock-cycle limit (about
+// two seconds), sets CFR_DEVERR_TIMEOUT in the error word and lets the kernel
+// return.
 #pragma once
 
 #include <cstdint>
@@ -18,7 +19,6 @@ namespace cfr {
 constexpr int kFmtCount = CFR_FMT_COUNT;
 constexpr int kMaxQHeads = 256;
 constexpr int kMaxGroup = 16;              // query heads per kv head
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 // Parameters of one decode call, shared by both decode kernels.
 struct DecodeParams {
@@ -53,12 +53,6 @@ __host__ __device__ inline int row_bytes(int fmt, int d) {
 
 __device__ __forceinline__ void set_err(uint32_t *err, uint32_t bits) {
   if (err) atomicOr(err, bits);
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -100,22 +94,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Spin limit of every wait, in SM clock cycles: 4e9 cycles is about 2 s at the
+// B200's top SM clock (more at lower clocks).  The cycle counter is read only
+// every 64 polls, so the limit check costs nothing on the fast path.
+constexpr long long kWaitLimitCycles = 4000000000LL;
+
 // Waits for the phase of `parity` to complete.  Returns false (and flags the
-// error word) when the wait exceeded kWaitLimitNs; `*timed_out` then stays set
-// so that callers stop waiting on anything else.
+// error word) when the wait exceeded kWaitLimitCycles; `*timed_out` then stays
+// set so that callers stop waiting on anything else.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err,
                                           bool *timed_out) {
   if (*timed_out) return false;
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
+  const long long t0 = clock64();
+  for (uint32_t spins = 1;; ++spins) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((spins & 63u) == 0 && clock64() - t0 > kWaitLimitCycles) {
       set_err(err, CFR_DEVERR_TIMEOUT);
       *timed_out = true;
       return false;
     }
   }
-  return true;
 }
 
 // ---- 1-D bulk copy global -> shared (TMA engine, no multicast) ---------------

@@ -14,13 +14,14 @@
 // result, both in fp32 (ARGUS page, "Transient FP16 Reconstruction ... in GPU
 // SRAM": pages are expanded on chip only, attention runs at 16-bit).
 //
-// Warp roles (320 threads, one CTA per SM, persistent over work items =
+// Warp roles (352 threads, one CTA per SM, persistent over work items =
 // (split of a sequence, kv head)):
 //   warp 0      TMA producer: resolves pages, bf16 tiles by 2-D tensor-map
 //               boxes straight into the 128-byte-swizzled operand layout,
 //               int tiles by 1-D bulk copies of the raw rows.
-//   warp 1      TMEM allocation; lane 0 issues the MMAs (QK of tile i+1 ahead
-//               of PV of tile i) and commits them to mbarriers.
+//   warp 1      TMEM allocation; lane 0 issues the QK products.
+//   warp 10     lane 0 issues the P.V products (a thread of its own, so the two
+//               kinds of MMA never wait for each other's issue).
 //   warps 2-5   softmax / fold: thread t owns TMEM lane t = token t of S and
 //               dim t of O.  Per tile: scores (scale, ALiBi from the integer
 //               distance), tile max across the 128 tokens, p = 2^(s - m),
@@ -44,7 +45,7 @@ namespace cfr {
 
 constexpr int TC_T = 128;            // tokens per tile
 constexpr int TC_D = 128;            // head_dim
-constexpr int TC_THREADS = 320;
+constexpr int TC_THREADS = 352;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
 constexpr int TC_RAW_BYTES = 2 * TC_T * TC_D;  // raw int8 K + V rows (int4 uses half)
@@ -66,13 +67,14 @@ struct TcCfg {
   static constexpr int STAGES = INTP ? 2 : 3;
   static constexpr int Q_BYTES = NCOL * 256;       // [NCOL rows][128 cols] 16-bit, 2 halves
   static constexpr int P_BYTES = NCOL * TC_T * 2;  // [128 tokens][NCOL] 16-bit
-  static constexpr int TMEM_COLS = 4 * NCOL;       // S x2, O x2
+  static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
+  static constexpr int TMEM_COLS = NCOL == 16 ? 128 : 256;  // S x2 + O x3 columns, power of two
 };
 
 template <int NCOL, bool INTP>
 struct TcSmem {
   uint64_t op_full[3], op_empty[3], raw_full[3];
-  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[3], o_empty[3];
   uint64_t q_full, drain;
   uint32_t tmem_base;
   int flag_st[3];
@@ -217,6 +219,39 @@ struct TcCtx {
   long long nitems;
   int nsplit;
 };
+
+
+// Maximum over the 32 lanes of each of NV values per lane (NV a power of two,
+// NV <= 16), by a transposing reduction: each exchange step halves the values a
+// lane keeps, so the warp spends NV-1 + log2(32/NV) shuffles instead of 5*NV.
+// Returns the maximum of value `head` (written to *head); lanes whose low bits
+// below the last halving offset are zero hold distinct heads.
+template <int NV>
+__device__ __forceinline__ float warp_multi_max(const float (&v)[NV], int lane, int *head) {
+  float cur[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) cur[i] = v[i];
+  int h = 0;
+  int off = 16;
+#pragma unroll
+  for (int n = NV; n > 1; n >>= 1) {
+    const int half = n >> 1;
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? cur[i] : cur[half + i];
+      const float keep = upper ? cur[half + i] : cur[i];
+      cur[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+    }
+    h = 2 * h + (upper ? 1 : 0);
+    off >>= 1;
+  }
+  float r = cur[0];
+#pragma unroll
+  for (int o = off; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
+  *head = h;
+  return r;
+}
 
 // non-blocking probe of an mbarrier phase
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
@@ -460,121 +495,101 @@ __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   }
 }
 
-// token range of work item `item` (no-op past the last item)
+// QK issuer (warp 1, one thread): for every tile in order, once its operands
+// are staged and an S buffer is free, S^T = K . [q_hi | q_lo]^T into TMEM.
 template <int NCOL, bool INTP>
-__device__ __forceinline__ void tc_item_range(TcCtx<NCOL, INTP> &c, long long item, int &t0, int &end,
-                                              bool &need_q) {
-  if (item < c.nitems) {
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    (void)g;
-    const int b = c.p.splits[3 * slot];
-    t0 = c.p.splits[3 * slot + 1] * c.p.P;
-    end = min(c.p.seq_lens[b], c.p.splits[3 * slot + 2] * c.p.P);
-    need_q = true;
-  }
-}
-
-// MMA issuer (one thread).  QK of a tile is issued as soon as its operands and
-// an S buffer are ready; P.V of a tile as soon as its probabilities and an O
-// buffer are ready -- polled without blocking, so neither waits on the other.
-template <int NCOL, bool INTP>
-__device__ void tc_mma_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+__device__ void tc_qk_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
   const uint32_t tmem = c.S.tmem_base;
-  const uint32_t op0 = smem_u32(c.op), q0 = smem_u32(c.qop), p0 = smem_u32(c.pop);
-  // QK cursor over the flattened (item, tile) sequence
-  long long q_item = blockIdx.x;
-  int q_item_k = 0, q_t0 = 0, q_end = 0, q_stage = 0;
-  uint32_t q_phase = 0;
-  bool q_need_q = false;
-  tc_item_range(c, q_item, q_t0, q_end, q_need_q);
-  long long qk_tc = 0, pv_tc = 0;
-  // stage and kind of the tiles between the two cursors (at most four), four bits
-  // each, kept in registers
-  uint32_t stage_bits = 0, kind_bits = 0;
-  uint64_t idle_since = 0;
-  while (!*timed_out) {
-    bool progress = false;
-    // ---- QK of the next tile ----
-    if (q_item < c.nitems) {
-      if (q_need_q && mbar_test(&c.S.q_full, static_cast<uint32_t>(q_item_k & 1))) q_need_q = false;
-      if (!q_need_q && mbar_test(&c.S.op_full[q_stage], q_phase) &&
-          mbar_test(&c.S.s_empty[qk_tc & 1], static_cast<uint32_t>((qk_tc >> 1) & 1) ^ 1u)) {
-        tc_fence_after();
-        const int kind = c.S.meta[q_stage].kind;
-        const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
-        const uint32_t kbase = op0 + q_stage * TC_OP_BYTES;
-        const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
-        const uint32_t d = tmem + static_cast<uint32_t>(qk_tc & 1) * NCOL;
+  const uint32_t op0 = smem_u32(c.op), q0 = smem_u32(c.qop);
+  int stage = 0;
+  uint32_t phase = 0;
+  long long tc = 0;
+  int item_k = 0;
+  for (long long item = blockIdx.x; item < c.nitems && !*timed_out; item += gridDim.x, ++item_k) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    (void)g;
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int tok_end = min(p.seq_lens[b], pe * P);
+    if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(item_k & 1), p.err, timed_out)) break;
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+      if (!mbar_wait(&c.S.op_full[stage], phase, p.err, timed_out)) break;
+      if (!mbar_wait(&c.S.s_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err,
+                     timed_out))
+        break;
+      tc_fence_after();
+      const int kind = c.S.meta[stage].kind;
+      const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
+      const uint32_t kbase = op0 + stage * TC_OP_BYTES;
+      const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
+      const uint32_t d = tmem + static_cast<uint32_t>(tc & 1) * NCOL;
 #pragma unroll
-        for (int k = 0; k < TC_D / 16; ++k) {
-          const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
-          const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
-          tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
-        }
-        tc_commit(&c.S.s_full[qk_tc & 1]);
-        const uint32_t sh = 4u * static_cast<uint32_t>(qk_tc & 7);
-        stage_bits = (stage_bits & ~(0xFu << sh)) | (static_cast<uint32_t>(q_stage) << sh);
-        kind_bits = (kind_bits & ~(0xFu << sh)) | (static_cast<uint32_t>(kind) << sh);
-        ++qk_tc;
-        if (++q_stage == Cfg::STAGES) {
-          q_stage = 0;
-          q_phase ^= 1u;
-        }
-        q_t0 += TC_T;
-        if (q_t0 >= q_end) {
-          q_item += gridDim.x;
-          ++q_item_k;
-          tc_item_range(c, q_item, q_t0, q_end, q_need_q);
-        }
-        progress = true;
+      for (int k = 0; k < TC_D / 16; ++k) {
+        const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
+        const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
+        tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
       }
-    }
-    // ---- P.V of the oldest tile whose probabilities are ready ----
-    if (pv_tc < qk_tc) {
-      const uint32_t par = static_cast<uint32_t>((pv_tc >> 1) & 1);
-      if (mbar_test(&c.S.p_full[pv_tc & 1], par) && mbar_test(&c.S.o_empty[pv_tc & 1], par ^ 1u)) {
-        tc_fence_after();
-        const uint32_t sh = 4u * static_cast<uint32_t>(pv_tc & 7);
-        const int st = static_cast<int>((stage_bits >> sh) & 0xFu);
-        const int kind = static_cast<int>((kind_bits >> sh) & 0xFu);
-        const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
-        const uint32_t vbase = op0 + st * TC_OP_BYTES + 2 * TC_HALF;
-        const uint32_t pbase = p0 + static_cast<uint32_t>(pv_tc & 1) * Cfg::P_BYTES;
-        const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(pv_tc & 1) * NCOL;
-#pragma unroll
-        for (int k = 0; k < TC_T / 16; ++k) {
-          const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
-          const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
-          tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
-        }
-        tc_commit(&c.S.o_full[pv_tc & 1]);
-        tc_commit(&c.S.p_empty[pv_tc & 1]);
-        tc_commit(&c.S.op_empty[st]);
-        ++pv_tc;
-        progress = true;
-      }
-    }
-    if (q_item >= c.nitems && pv_tc == qk_tc) break;
-    if (progress) {
-      idle_since = 0;
-    } else {
-      const uint64_t now = global_ns();
-      if (idle_since == 0) {
-        idle_since = now;
-      } else if (now - idle_since > kWaitLimitNs) {
-        set_err(p.err, CFR_DEVERR_TIMEOUT);
-        *timed_out = true;
+      tc_commit(&c.S.s_full[tc & 1]);
+      ++tc;
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
       }
     }
   }
-  // drain: every MMA issued so far has completed before TMEM is released
+  // drain: every MMA this thread issued has completed before TMEM is released
   tc_commit(&c.S.drain);
-  bool t2 = false;
-  (void)mbar_wait(&c.S.drain, 0, p.err, &t2);
+}
+
+// P.V issuer (warp 10, one thread): for every tile in order, once its
+// probabilities are written and an O buffer is free, O^T = V^T . [p_hi | p_lo]^T
+// into TMEM; the commit then frees the stage, the P buffer and signals the fold.
+template <int NCOL, bool INTP>
+__device__ void tc_pv_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+  using Cfg = TcCfg<NCOL, INTP>;
+  const DecodeParams &p = c.p;
+  const int P = p.P;
+  const uint32_t tmem = c.S.tmem_base;
+  const uint32_t op0 = smem_u32(c.op), p0 = smem_u32(c.pop);
+  int stage = 0;
+  long long tc = 0;
+  for (long long item = blockIdx.x; item < c.nitems && !*timed_out; item += gridDim.x) {
+    int slot, g;
+    item_coords(item, c.nsplit, slot, g);
+    (void)g;
+    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const int tok_end = min(p.seq_lens[b], pe * P);
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+      const int ob = static_cast<int>(tc % Cfg::O_BUFS);
+      if (!mbar_wait(&c.S.p_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), p.err, timed_out))
+        break;
+      if (!mbar_wait(&c.S.o_empty[ob], static_cast<uint32_t>((tc / Cfg::O_BUFS) & 1) ^ 1u, p.err,
+                     timed_out))
+        break;
+      tc_fence_after();
+      // the tile description stays valid until this P.V has freed the stage
+      const int kind = c.S.meta[stage].kind;
+      const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
+      const uint32_t vbase = op0 + stage * TC_OP_BYTES + 2 * TC_HALF;
+      const uint32_t pbase = p0 + static_cast<uint32_t>(tc & 1) * Cfg::P_BYTES;
+      const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(ob) * NCOL;
+#pragma unroll
+      for (int k = 0; k < TC_T / 16; ++k) {
+        const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
+        const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
+        tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+      }
+      tc_commit(&c.S.o_full[ob]);
+      tc_commit(&c.S.p_empty[tc & 1]);
+      tc_commit(&c.S.op_empty[stage]);
+      ++tc;
+      if (++stage == Cfg::STAGES) stage = 0;
+    }
+  }
+  tc_commit(&c.S.drain);
 }
 
 // folds the P.V product of tile i into the running accumulators (dim t of each head)
@@ -583,14 +598,16 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint3
                                         int cnt, float (&acc)[NCOL / 2],
                                         const float (&alpha_prev)[NCOL / 2], float vscale_prev,
                                         bool *timed_out) {
-  (void)mbar_wait(&c.S.o_full[i & 1], static_cast<uint32_t>((i >> 1) & 1), c.p.err, timed_out);
+  const int ob = static_cast<int>(i % TcCfg<NCOL, INTP>::O_BUFS);
+  (void)mbar_wait(&c.S.o_full[ob], static_cast<uint32_t>((i / TcCfg<NCOL, INTP>::O_BUFS) & 1),
+                  c.p.err, timed_out);
   tc_fence_after();
   float o[NCOL];
-  tmem_ld<NCOL>(tmem + 2 * NCOL + static_cast<uint32_t>(i & 1) * NCOL, o);
+  tmem_ld<NCOL>(tmem + 2 * NCOL + static_cast<uint32_t>(ob) * NCOL, o);
   tc_wait_ld();
   tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive(&c.S.o_empty[i & 1]);
+  if (lane == 0) mbar_arrive(&c.S.o_empty[ob]);
 #pragma unroll
   for (int h = 0; h < NCOL / 2; ++h)
     if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
@@ -685,17 +702,20 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
     if (!q_ready) tc_write_q(c, item, tsm, lane);
     q_ready = false;
 
-    float slope2[GM], m_run[GM], l_part[GM], acc[GM], alpha_prev[GM];
+    // folds lag two tiles behind the scores: tiles prev2 (older) and prev1 wait,
+    // each with its rescale factors and V scale
+    float slope2[GM], m_run[GM], l_part[GM], acc[GM], alpha1[GM], alpha2[GM];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       slope2[h] = (p.slopes && h < cnt) ? p.slopes[p.grp_heads[h0 + h]] * kLog2e : 0.f;
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
       acc[h] = 0.f;
-      alpha_prev[h] = 1.f;
+      alpha1[h] = 1.f;
+      alpha2[h] = 1.f;
     }
-    float vscale_prev = 1.f;
-    long long prev_tc = -1;
+    float vs1 = 1.f, vs2 = 1.f;
+    long long prev1 = -1, prev2 = -1;
 
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       // ---- scores of tile tc ----
@@ -718,22 +738,31 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
       const float vsc = kind == KIND_BF16 ? 1.f : m.vs * (1.f / 32768.f);
       float s[GM];
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
+      for (int h = 0; h < GM; ++h)
         s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
-        float mx = s[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) c.S.red_max[tc & 1][quarter][h] = mx;
+      {
+        int hm;
+        const float mx = warp_multi_max<GM>(s, lane, &hm);
+        // lanes whose bits below the last halving offset are zero hold head hm's max
+        if ((lane & ((32 / GM) - 1)) == 0) c.S.red_max[tc & 1][quarter][hm] = mx;
       }
       // the P buffer of this tile must be free (P.V of tile tc-2 done)
       (void)mbar_wait(&c.S.p_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err, timed_out);
       named_sync(2, 128);
-      float pr[GM], alpha[GM];
+      float pr[GM], alpha[GM], mt[GM];
+#pragma unroll
+      for (int h4 = 0; h4 < GM; h4 += 4) {
+        float4 a[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[q] = *reinterpret_cast<const float4 *>(&c.S.red_max[tc & 1][q][h4]);
+        mt[h4 + 0] = fmaxf(fmaxf(a[0].x, a[1].x), fmaxf(a[2].x, a[3].x));
+        mt[h4 + 1] = fmaxf(fmaxf(a[0].y, a[1].y), fmaxf(a[2].y, a[3].y));
+        mt[h4 + 2] = fmaxf(fmaxf(a[0].z, a[1].z), fmaxf(a[2].z, a[3].z));
+        mt[h4 + 3] = fmaxf(fmaxf(a[0].w, a[1].w), fmaxf(a[2].w, a[3].w));
+      }
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
-        float mt = fmaxf(fmaxf(c.S.red_max[tc & 1][0][h], c.S.red_max[tc & 1][1][h]),
-                         fmaxf(c.S.red_max[tc & 1][2][h], c.S.red_max[tc & 1][3][h]));
-        const float m_new = fmaxf(m_run[h], mt);
+        const float m_new = fmaxf(m_run[h], mt[h]);
         if (m_new == -INFINITY) {
           alpha[h] = 1.f;
           pr[h] = 0.f;
@@ -782,19 +811,25 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
           q_ready = true;
         }
       }
-      // fold the previous tile of this item
-      if (prev_tc >= 0) tc_fold(c, prev_tc, tmem, lane, cnt, acc, alpha_prev, vscale_prev, timed_out);
+      // fold the tile two behind (its P.V has long been issued)
+      if (prev2 >= 0) tc_fold(c, prev2, tmem, lane, cnt, acc, alpha2, vs2, timed_out);
+      prev2 = prev1;
+      vs2 = vs1;
 #pragma unroll
-      for (int h = 0; h < GM; ++h) alpha_prev[h] = alpha[h];
-      vscale_prev = vsc;
-      prev_tc = tc;
+      for (int h = 0; h < GM; ++h) {
+        alpha2[h] = alpha1[h];
+        alpha1[h] = alpha[h];
+      }
+      prev1 = tc;
+      vs1 = vsc;
       ++tc;
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
       }
     }
-    if (prev_tc >= 0) tc_fold(c, prev_tc, tmem, lane, cnt, acc, alpha_prev, vscale_prev, timed_out);
+    if (prev2 >= 0) tc_fold(c, prev2, tmem, lane, cnt, acc, alpha2, vs2, timed_out);
+    if (prev1 >= 0) tc_fold(c, prev1, tmem, lane, cnt, acc, alpha1, vs1, timed_out);
 
     // split partial: acc (dim t), m, and l summed over the 128 token slots
 #pragma unroll
@@ -842,11 +877,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&S.s_empty[i], 4);
       mbar_init(&S.p_full[i], 4);
       mbar_init(&S.p_empty[i], 1);
+    }
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&S.o_full[i], 1);
       mbar_init(&S.o_empty[i], 4);
     }
     mbar_init(&S.q_full, 4);
-    mbar_init(&S.drain, 1);
+    mbar_init(&S.drain, 2);  // one commit from each MMA issuer
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -868,7 +905,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 0) {
     tc_producer<NCOL, INTP>(c, &timed_out);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) tc_mma_issuer<NCOL, INTP>(c, &timed_out);
+    if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP>(c, &timed_out);
+  } else if (warp == 10) {
+    if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP>(c, &timed_out);
   } else if (warp < 6) {
     tc_softmax<NCOL, INTP>(c, &timed_out);
   } else {
@@ -877,6 +916,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    if ((threadIdx.x & 31) == 0) {
+      bool t2 = false;
+      (void)mbar_wait(&S.drain, 0, p.err, &t2);  // every MMA of both issuers has completed
+    }
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(S.tmem_base),
