@@ -13,6 +13,13 @@ Parity status of each oracle function (what pins it is listed in the tests):
   attend(mode=2)  pinned against mode 0 (split + merge invariant).
   merge           pinned: closed forms and against attend(mode=2).
   kv_bytes        pinned: the CFR-Atlas page's printed byte counts.
+  demote          pinned: hand-derived byte patterns (rounding, clamping,
+                  nibble order), the E4M3 table of the format definition and
+                  the library's float8 conversion, reconstruction-error bounds,
+                  scaling invariances, the all-zero block.
+  append          pinned: byte layout (a token appended to an empty page is
+                  what a decode over one token returns), the library's bf16
+                  rounding, fault cases.
 """
 
 from __future__ import annotations
@@ -30,6 +37,9 @@ _SRC = os.path.join(_HERE, "cfr_oracle.c")
 _LIB = os.path.join(_HERE, "libcfr_oracle.so")
 
 OK, BAD_ARG, BAD_PAGE, NO_MEMORY, EMPTY = 0, 1, 2, 3, 4
+NFMT = 5  # F32, BF16, I8, I4, FP8 (E4M3)
+# bits the oracle reports for skipped pages or tokens
+DEV_PAGE_ID, DEV_PAGE_FMT, DEV_SEQ_LEN = 0x1, 0x2, 0x4
 
 
 def build(force: bool = False) -> str:
@@ -49,8 +59,8 @@ class _Problem(ctypes.Structure):
         ("page_tokens", ctypes.c_int32), ("max_pages", ctypes.c_int32),
         ("q_fmt", ctypes.c_int32), ("uniform_fmt", ctypes.c_int32),
         ("q", ctypes.c_void_p),
-        ("k_pool", ctypes.c_void_p * 4), ("v_pool", ctypes.c_void_p * 4),
-        ("scales", ctypes.c_void_p * 4), ("pool_pages", ctypes.c_int64 * 4),
+        ("k_pool", ctypes.c_void_p * 5), ("v_pool", ctypes.c_void_p * 5),
+        ("scales", ctypes.c_void_p * 5), ("pool_pages", ctypes.c_int64 * 5),
         ("page_table", ctypes.c_void_p), ("page_fmt", ctypes.c_void_p),
         ("seq_lens", ctypes.c_void_p), ("head_map", ctypes.c_void_p),
         ("alibi_slopes", ctypes.c_void_p), ("softmax_scale", ctypes.c_double),
@@ -75,6 +85,24 @@ def _load():
             ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
         lib.cfr_oracle_kv_bytes.restype = ctypes.c_int64
         lib.cfr_oracle_kv_bytes.argtypes = [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32]
+        vp = ctypes.c_void_p
+        lib.cfr_oracle_demote.restype = ctypes.c_int
+        lib.cfr_oracle_demote.argtypes = [
+            ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+            ctypes.c_int32, vp, vp, vp, ctypes.c_int64,
+            ctypes.c_int32, vp, vp, vp, ctypes.c_int64,
+            vp, vp, vp, ctypes.c_int32, vp]
+        lib.cfr_oracle_append.restype = ctypes.c_int
+        lib.cfr_oracle_append.argtypes = [
+            ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, vp, vp, vp,
+            vp, ctypes.c_int32, vp, ctypes.c_int32, vp, ctypes.c_int32,
+            ctypes.c_int32, vp, vp, vp]
+        lib.cfr_oracle_e4m3_code.restype = ctypes.c_int32
+        lib.cfr_oracle_e4m3_code.argtypes = [ctypes.c_float]
+        lib.cfr_oracle_e4m3_value.restype = ctypes.c_double
+        lib.cfr_oracle_e4m3_value.argtypes = [ctypes.c_int32]
+        lib.cfr_oracle_bf16_bits.restype = ctypes.c_int32
+        lib.cfr_oracle_bf16_bits.argtypes = [ctypes.c_float]
         _lib = lib
     return _lib
 
@@ -134,7 +162,7 @@ def attend(case, sel: Optional[Sequence[tuple]] = None, mode: int = 0, arg: int 
     pr.q_fmt, pr.uniform_fmt = case.q_fmt, case.uniform_fmt
     q = h(case.q)
     pr.q = q.data_ptr()
-    for f in range(4):
+    for f in range(NFMT):
         pr.k_pool[f] = kp[f].data_ptr() if f in kp else None
         pr.v_pool[f] = vp[f].data_ptr() if f in vp else None
         pr.scales[f] = sc[f].data_ptr() if f in sc else None
@@ -190,3 +218,73 @@ def merge(part_acc, part_m, part_l, split_off, batch: int, num_q_heads: int, hea
 def kv_bytes(fmt: int, tokens: int, head_dim: int) -> int:
     """K+V bytes of `tokens` tokens of one head stored in format ``fmt``."""
     return int(_load().cfr_oracle_kv_bytes(fmt, tokens, head_dim))
+
+
+def demote(num_kv_heads: int, head_dim: int, page_tokens: int, src_fmt: int, src_k, src_v,
+           src_scales, dst_fmt: int, dst_k, dst_v, dst_scales, src_slots, dst_slots,
+           valid_tokens=None) -> int:
+    """Oracle page demotion on host tensors; writes dst_k/dst_v/dst_scales in place.
+
+    Pools are contiguous uint8 CPU tensors [slots][Hkv][P][row_bytes], scales
+    float32 [slots][Hkv][2] (None for float formats).  Returns the OR of the
+    DEV_* bits of skipped pages.
+    """
+    lib = _load()
+    for t in (src_k, src_v, dst_k, dst_v, src_scales, dst_scales):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise ValueError("oracle.demote needs contiguous CPU tensors")
+    ss = _host(torch.as_tensor(src_slots, dtype=torch.int32))
+    ds = _host(torch.as_tensor(dst_slots, dtype=torch.int32))
+    vt = None if valid_tokens is None else _host(torch.as_tensor(valid_tokens, dtype=torch.int32))
+    err = ctypes.c_uint32(0)
+    rc = lib.cfr_oracle_demote(num_kv_heads, head_dim, page_tokens,
+                               src_fmt, _ptr(src_k), _ptr(src_v), _ptr(src_scales),
+                               int(src_k.shape[0]),
+                               dst_fmt, _ptr(dst_k), _ptr(dst_v), _ptr(dst_scales),
+                               int(dst_k.shape[0]),
+                               _ptr(ss), _ptr(ds), _ptr(vt), int(ss.numel()), ctypes.byref(err))
+    if rc != OK:
+        raise OracleError(rc)
+    return int(err.value)
+
+
+def append(num_kv_heads: int, head_dim: int, page_tokens: int, k_pool: dict, v_pool: dict,
+           page_table, page_fmt, uniform_fmt: int, positions, new_fmt: int, k_new, v_new) -> int:
+    """Oracle KV append on host tensors (pools dict fmt -> uint8 CPU tensor, written in place).
+
+    Returns the OR of the DEV_* bits of skipped sequences.
+    """
+    lib = _load()
+    kp = (ctypes.c_void_p * NFMT)(*[k_pool[f].data_ptr() if f in k_pool else None
+                                     for f in range(NFMT)])
+    vpp = (ctypes.c_void_p * NFMT)(*[v_pool[f].data_ptr() if f in v_pool else None
+                                      for f in range(NFMT)])
+    pages = (ctypes.c_int64 * NFMT)(*[int(k_pool[f].shape[0]) if f in k_pool else 0
+                                       for f in range(NFMT)])
+    pt = _host(page_table.to(torch.int32))
+    pf = _host(page_fmt)
+    pos = _host(torch.as_tensor(positions, dtype=torch.int32))
+    kn, vn = _host(k_new), _host(v_new)
+    err = ctypes.c_uint32(0)
+    rc = lib.cfr_oracle_append(num_kv_heads, head_dim, page_tokens, kp, vpp, pages,
+                               _ptr(pt), int(pt.shape[1]), _ptr(pf), uniform_fmt,
+                               _ptr(pos), int(pos.numel()), new_fmt, _ptr(kn), _ptr(vn),
+                               ctypes.byref(err))
+    if rc != OK:
+        raise OracleError(rc)
+    return int(err.value)
+
+
+def e4m3_code(x: float) -> int:
+    """The oracle's E4M3 code for fp32 x (nearest, ties to even, saturating)."""
+    return int(_load().cfr_oracle_e4m3_code(float(x)))
+
+
+def e4m3_value(code: int) -> float:
+    """The value of E4M3 code ``code`` by the format definition."""
+    return float(_load().cfr_oracle_e4m3_value(int(code)))
+
+
+def bf16_bits(x: float) -> int:
+    """The oracle's bfloat16 bits for fp32 x (nearest, ties to even)."""
+    return int(_load().cfr_oracle_bf16_bits(float(x))) & 0xFFFF

@@ -25,9 +25,11 @@
  *     page_fmt[b][p] (uniform_fmt when page_fmt is NULL);
  *   - the row of kv head g is at byte ((slot * Hkv + g) * P + t) * row_bytes;
  *   - values: F32 as stored, BF16 widened from its 16 bits, I8 code * scale,
- *     I4 nibble code * scale, with scale = scales[fmt][slot][g][0 for K, 1 for V]
- *     (ARGUS page, "Why It Works: Storage vs. Computation": pages are stored
- *     compressed and restored to full precision before attention);
+ *     I4 nibble code * scale, FP8 E4M3 value * scale, with
+ *     scale = scales[fmt][slot][g][0 for K, 1 for V]
+ *     (ARGUS page, "Visual Architecture": the FP8, INT8 and INT4 tiers of the
+ *     compression cascade; "Why It Works: Storage vs. Computation": pages are
+ *     stored compressed and restored to full precision before attention);
  *   - sigma = softmax_scale, or 1/sqrt(d) when softmax_scale is 0;
  *   - bias_j = -slope_h * (n - 1 - j) with ALiBi slopes, else 0
  *     (CFR-Atlas page, "RoPE/ALiBi positional policy");
@@ -52,7 +54,8 @@
 #define ORC_BF16 1
 #define ORC_I8 2
 #define ORC_I4 3
-#define ORC_NFMT 4
+#define ORC_FP8 4
+#define ORC_NFMT 5
 
 #define ORC_OK 0
 #define ORC_BAD_ARG 1
@@ -66,7 +69,7 @@ typedef struct {
   const void *q;                       /* [B][Hq][d] f32 or bf16 bits */
   const void *k_pool[ORC_NFMT];
   const void *v_pool[ORC_NFMT];
-  const float *scales[ORC_NFMT];       /* [slots][Hkv][2] for I8/I4 */
+  const float *scales[ORC_NFMT];       /* [slots][Hkv][2] for I8/I4/FP8 */
   int64_t pool_pages[ORC_NFMT];
   const int32_t *page_table;           /* [B][max_pages] */
   const uint8_t *page_fmt;             /* [B][max_pages] or NULL */
@@ -103,12 +106,30 @@ static int orc_i4_code(unsigned char byte, int high) {
   return nib < 8 ? nib : nib - 16;
 }
 
+/*
+ * FP8 E4M3 (the OCP 8-bit floating-point format without infinities): sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits.  Exponent field 0 holds the
+ * subnormals m * 2^-9; fields 1..15 hold (1 + m/8) * 2^(e-7), except e = 15,
+ * m = 7, which is NaN.  Largest finite magnitude: 448.
+ */
+static double orc_e4m3_value(unsigned char byte) {
+  const int e = (byte >> 3) & 15, m = byte & 7;
+  double mag;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) mag = ldexp((double)m, -9);
+  else mag = ldexp(1.0 + m / 8.0, e - 7);
+  return (byte & 0x80) ? -mag : mag;
+}
+
+static int orc_quantised(int fmt) { return fmt == ORC_I8 || fmt == ORC_I4 || fmt == ORC_FP8; }
+
 static long orc_row_bytes(int fmt, int d) {
   switch (fmt) {
     case ORC_F32: return 4L * d;
     case ORC_BF16: return 2L * d;
     case ORC_I8: return (long)d;
     case ORC_I4: return (long)d / 2;
+    case ORC_FP8: return (long)d;
   }
   return -1;
 }
@@ -120,6 +141,7 @@ static double orc_element(int fmt, const unsigned char *row, int i, double scale
     case ORC_BF16: return orc_from_bf16(row + 2L * i);
     case ORC_I8: return (double)orc_i8_code(row[i]) * scale;
     case ORC_I4: return (double)orc_i4_code(row[i / 2], i % 2) * scale;
+    case ORC_FP8: return orc_e4m3_value(row[i]) * scale;
   }
   return NAN;
 }
@@ -154,7 +176,7 @@ static int orc_materialise(const orc_problem *pr, int b, int g, int n, int skip_
     const long slot = pr->page_table[cell];
     int ok = fmt >= 0 && fmt < ORC_NFMT && pr->k_pool[fmt] && pr->v_pool[fmt] &&
              slot >= 0 && slot < pr->pool_pages[fmt] &&
-             ((fmt != ORC_I8 && fmt != ORC_I4) || pr->scales[fmt]);
+             (!orc_quantised(fmt) || pr->scales[fmt]);
     if (!ok) {
       if (!skip_invalid) return ORC_BAD_PAGE;
       keep[j] = 0;
@@ -167,7 +189,7 @@ static int orc_materialise(const orc_problem *pr, int b, int g, int n, int skip_
     const unsigned char *krow = (const unsigned char *)pr->k_pool[fmt] + off;
     const unsigned char *vrow = (const unsigned char *)pr->v_pool[fmt] + off;
     double ks = 1.0, vs = 1.0;
-    if (fmt == ORC_I8 || fmt == ORC_I4) {
+    if (orc_quantised(fmt)) {
       const float *sc = pr->scales[fmt] + (slot * Hkv + g) * 2;
       ks = (double)sc[0];
       vs = (double)sc[1];
@@ -482,3 +504,247 @@ int64_t cfr_oracle_kv_bytes(int32_t fmt, int64_t tokens, int32_t head_dim) {
   if (rb < 0 || tokens < 0) return -1;
   return 2 * tokens * rb;
 }
+
+/* ---- page demotion and KV append ----------------------------------------
+ *
+ * The compression cascade of the ARGUS page ("Visual Architecture": hot pages
+ * in full precision, cold pages re-encoded FP8 -> INT8 -> INT4) re-encodes a
+ * whole page of one storage format into another.  The reading followed here,
+ * per (page, kv head, K-or-V) block of P rows x d, over its `valid` first rows:
+ *
+ *   x      = the stored value as fp32 (F32 as is, BF16 widened, quantised
+ *            formats code * scale rounded to fp32);
+ *   amax   = max |x| over the valid rows (fp32);
+ *   scale  = amax / Q in fp32, Q = 127 (I8), 7 (I4), 448 (FP8);
+ *   I8/I4  code = clamp(round_half_even(x / scale), -Q, Q), the division in fp32;
+ *   FP8    code = E4M3 nearest to x / scale (ties to even, saturating at 448);
+ *   BF16   x rounded to bfloat16 (nearest, ties to even);
+ *   F32    x.
+ * With amax = 0 the scale is 0 and every code is 0; a NaN value gets integer
+ * code 0 and the FP8 NaN code 0x7F.  Rows at or past `valid`
+ * are written as zero bytes.  Every decision that turns a float into a code is
+ * taken in fp32, the precision in which the values are stored.
+ */
+
+#define ORC_DEV_PAGE_ID 0x1u
+#define ORC_DEV_PAGE_FMT 0x2u
+#define ORC_DEV_SEQ_LEN 0x4u
+
+static float orc_value_f32(int fmt, const unsigned char *row, int i, float scale) {
+  switch (fmt) {
+    case ORC_F32: {
+      float f;
+      memcpy(&f, row + 4L * i, sizeof f);
+      return f;
+    }
+    case ORC_BF16: return (float)orc_from_bf16(row + 2L * i);
+    case ORC_I8: return (float)orc_i8_code(row[i]) * scale;
+    case ORC_I4: return (float)orc_i4_code(row[i / 2], i % 2) * scale;
+    case ORC_FP8: return (float)orc_e4m3_value(row[i]) * scale;
+  }
+  return NAN;
+}
+
+/* bfloat16 nearest to x (ties to even); NaN becomes the quiet NaN 0x7FC0 */
+static uint16_t orc_bf16_bits(float x) {
+  uint32_t w;
+  memcpy(&w, &x, sizeof w);
+  if (isnan(x)) return 0x7FC0;
+  /* keep the upper 16 bits, adding half an ulp of bf16 minus one unless the kept part is odd */
+  uint32_t lsb = (w >> 16) & 1u;
+  w += 0x7FFFu + lsb;
+  return (uint16_t)(w >> 16);
+}
+
+/* E4M3 code nearest to x (ties to even mantissa), magnitudes above 448 saturate to 448 */
+static unsigned char orc_e4m3_code(float x) {
+  if (isnan(x)) return 0x7F;
+  const unsigned char sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range: multiples of 2^-9; 8 * 2^-9 is the smallest normal, code 0x08 */
+    int m = (int)rint(ldexp(a, 9));
+    return sign | (unsigned char)m;
+  }
+  int k;
+  (void)frexp(a, &k);            /* a = f * 2^k, f in [0.5, 1) */
+  int e = k - 1;                 /* a in [2^e, 2^(e+1)) */
+  int r = (int)rint(ldexp(a, 3 - e));  /* in [8, 16] */
+  if (r == 16) {
+    r = 8;
+    ++e;
+  }
+  int code = ((e + 7) << 3) | (r - 8);
+  if (code > 0x7E) code = 0x7E;
+  return sign | (unsigned char)code;
+}
+
+static int orc_qmax(int fmt) { return fmt == ORC_I8 ? 127 : fmt == ORC_I4 ? 7 : 448; }
+
+/* re-encodes one block: src rows [P][rb_src] -> dst rows [P][rb_dst] */
+static void orc_demote_block(int src_fmt, const unsigned char *src, float src_scale, int dst_fmt,
+                             unsigned char *dst, float *dst_scale, int P, int d, int valid) {
+  const long rs = orc_row_bytes(src_fmt, d), rd = orc_row_bytes(dst_fmt, d);
+  memset(dst, 0, (size_t)(rd * P));
+  float scale = 0.0f;
+  if (orc_quantised(dst_fmt)) {
+    float amax = 0.0f;
+    for (int t = 0; t < valid; ++t)
+      for (int i = 0; i < d; ++i) {
+        float a = fabsf(orc_value_f32(src_fmt, src + t * rs, i, src_scale));
+        if (a > amax) amax = a;
+      }
+    scale = amax / (float)orc_qmax(dst_fmt);
+    *dst_scale = scale;
+  }
+  for (int t = 0; t < valid; ++t) {
+    unsigned char *row = dst + t * rd;
+    for (int i = 0; i < d; ++i) {
+      const float x = orc_value_f32(src_fmt, src + t * rs, i, src_scale);
+      if (dst_fmt == ORC_F32) {
+        memcpy(row + 4L * i, &x, sizeof x);
+      } else if (dst_fmt == ORC_BF16) {
+        uint16_t hbits = orc_bf16_bits(x);
+        memcpy(row + 2L * i, &hbits, sizeof hbits);
+      } else if (dst_fmt == ORC_FP8) {
+        row[i] = scale > 0.0f ? orc_e4m3_code(x / scale) : 0;
+      } else {
+        const int q = orc_qmax(dst_fmt);
+        int c = 0;
+        if (scale > 0.0f) {
+          float r = rintf(x / scale);
+          c = isnan(r) ? 0 : r > (float)q ? q : r < (float)-q ? -q : (int)r;
+        }
+        if (dst_fmt == ORC_I8) {
+          row[i] = (unsigned char)(c & 0xFF);
+        } else {
+          const unsigned char nib = (unsigned char)(c & 15);
+          row[i / 2] |= (i % 2) ? (unsigned char)(nib << 4) : nib;
+        }
+      }
+    }
+  }
+}
+
+/*
+ * Demotes num_pages pages: page k is read from slot src_slots[k] of the source
+ * pool (format src_fmt) and written to slot dst_slots[k] of the destination
+ * pool (format dst_fmt), every kv head, K and V, over its valid_tokens[k] first
+ * rows (all P when valid_tokens is NULL).  Pools are
+ * [slots][Hkv][P][row_bytes]; scales [slots][Hkv][2] (K, V).  A page whose
+ * slot is out of range (ORC_DEV_PAGE_ID) or whose valid count is outside
+ * [1, P] (ORC_DEV_SEQ_LEN) is skipped and the bit is OR-ed into *err.
+ */
+int cfr_oracle_demote(int32_t num_kv_heads, int32_t head_dim, int32_t page_tokens,
+                      int32_t src_fmt, const uint8_t *src_k, const uint8_t *src_v,
+                      const float *src_scales, int64_t src_pages, int32_t dst_fmt,
+                      uint8_t *dst_k, uint8_t *dst_v, float *dst_scales, int64_t dst_pages,
+                      const int32_t *src_slots, const int32_t *dst_slots,
+                      const int32_t *valid_tokens, int32_t num_pages, uint32_t *err) {
+  if (num_kv_heads <= 0 || head_dim <= 0 || head_dim % 2 || page_tokens <= 0 || num_pages < 0 ||
+      src_fmt < 0 || src_fmt >= ORC_NFMT || dst_fmt < 0 || dst_fmt >= ORC_NFMT ||
+      !src_k || !src_v || !dst_k || !dst_v || !src_slots || !dst_slots || !err ||
+      (orc_quantised(src_fmt) && !src_scales) || (orc_quantised(dst_fmt) && !dst_scales))
+    return ORC_BAD_ARG;
+  const int d = head_dim, P = page_tokens, H = num_kv_heads;
+  const long rs = orc_row_bytes(src_fmt, d), rd = orc_row_bytes(dst_fmt, d);
+  for (int k = 0; k < num_pages; ++k) {
+    const int64_t s = src_slots[k], t = dst_slots[k];
+    const int valid = valid_tokens ? valid_tokens[k] : P;
+    if (s < 0 || s >= src_pages || t < 0 || t >= dst_pages) {
+      *err |= ORC_DEV_PAGE_ID;
+      continue;
+    }
+    if (valid < 1 || valid > P) {
+      *err |= ORC_DEV_SEQ_LEN;
+      continue;
+    }
+    for (int g = 0; g < H; ++g) {
+      const long src_off = (s * H + g) * (long)P * rs, dst_off = (t * H + g) * (long)P * rd;
+      const float ks = orc_quantised(src_fmt) ? src_scales[(s * H + g) * 2 + 0] : 1.0f;
+      const float vs = orc_quantised(src_fmt) ? src_scales[(s * H + g) * 2 + 1] : 1.0f;
+      float kd = 0.0f, vd = 0.0f;
+      orc_demote_block(src_fmt, src_k + src_off, ks, dst_fmt, dst_k + dst_off, &kd, P, d, valid);
+      orc_demote_block(src_fmt, src_v + src_off, vs, dst_fmt, dst_v + dst_off, &vd, P, d, valid);
+      if (orc_quantised(dst_fmt)) {
+        dst_scales[(t * H + g) * 2 + 0] = kd;
+        dst_scales[(t * H + g) * 2 + 1] = vd;
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/*
+ * Appends one token to every sequence b with positions[b] >= 0: the new K and
+ * V rows k_new[b][g][:], v_new[b][g][:] (fp32 or bf16 by new_fmt) become token
+ * j = positions[b] of the sequence, i.e. row j % P of logical page j / P,
+ * whose slot and format come from the page table as in the decode.  The page
+ * must be an F32 or BF16 page (new tokens enter the full-precision hot tier,
+ * ARGUS page, "The One-Minute Explanation": recent tokens stay in high
+ * precision); values are widened to F32 or rounded to BF16 (nearest, ties to
+ * even).  Faults are skipped and reported in *err: j beyond max_pages * P
+ * (ORC_DEV_SEQ_LEN), a quantised or unknown page format or a missing pool
+ * (ORC_DEV_PAGE_FMT), a slot outside its pool (ORC_DEV_PAGE_ID).
+ */
+int cfr_oracle_append(int32_t num_kv_heads, int32_t head_dim, int32_t page_tokens,
+                      uint8_t *const *k_pool, uint8_t *const *v_pool, const int64_t *pool_pages,
+                      const int32_t *page_table, int32_t max_pages, const uint8_t *page_fmt,
+                      int32_t uniform_fmt, const int32_t *positions, int32_t batch,
+                      int32_t new_fmt, const void *k_new, const void *v_new, uint32_t *err) {
+  if (num_kv_heads <= 0 || head_dim <= 0 || page_tokens <= 0 || max_pages < 0 || batch < 0 ||
+      !k_pool || !v_pool || !pool_pages || !page_table || !positions || !k_new || !v_new ||
+      !err || (new_fmt != ORC_F32 && new_fmt != ORC_BF16))
+    return ORC_BAD_ARG;
+  const int d = head_dim, P = page_tokens, H = num_kv_heads;
+  for (int b = 0; b < batch; ++b) {
+    const long j = positions[b];
+    if (j < 0) continue;
+    if (j >= (long)max_pages * P) {
+      *err |= ORC_DEV_SEQ_LEN;
+      continue;
+    }
+    const long cell = (long)b * max_pages + j / P;
+    const int fmt = page_fmt ? (int)page_fmt[cell] : uniform_fmt;
+    if ((fmt != ORC_F32 && fmt != ORC_BF16) || !k_pool[fmt] || !v_pool[fmt]) {
+      *err |= ORC_DEV_PAGE_FMT;
+      continue;
+    }
+    const long slot = page_table[cell];
+    if (slot < 0 || slot >= pool_pages[fmt]) {
+      *err |= ORC_DEV_PAGE_ID;
+      continue;
+    }
+    const long rb = orc_row_bytes(fmt, d);
+    for (int g = 0; g < H; ++g) {
+      unsigned char *kr = k_pool[fmt] + ((slot * H + g) * (long)P + j % P) * rb;
+      unsigned char *vr = v_pool[fmt] + ((slot * H + g) * (long)P + j % P) * rb;
+      for (int i = 0; i < d; ++i) {
+        const long e = ((long)b * H + g) * d + i;
+        float kx, vx;
+        if (new_fmt == ORC_F32) {
+          kx = ((const float *)k_new)[e];
+          vx = ((const float *)v_new)[e];
+        } else {
+          kx = (float)orc_from_bf16((const unsigned char *)k_new + 2 * e);
+          vx = (float)orc_from_bf16((const unsigned char *)v_new + 2 * e);
+        }
+        if (fmt == ORC_F32) {
+          memcpy(kr + 4L * i, &kx, sizeof kx);
+          memcpy(vr + 4L * i, &vx, sizeof vx);
+        } else {
+          uint16_t kb = orc_bf16_bits(kx), vb = orc_bf16_bits(vx);
+          memcpy(kr + 2L * i, &kb, sizeof kb);
+          memcpy(vr + 2L * i, &vb, sizeof vb);
+        }
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/* the E4M3 code of x and the decoded value of a code, exposed for pinning */
+int32_t cfr_oracle_e4m3_code(float x) { return orc_e4m3_code(x); }
+double cfr_oracle_e4m3_value(int32_t code) { return orc_e4m3_value((unsigned char)code); }
+int32_t cfr_oracle_bf16_bits(float x) { return orc_bf16_bits(x); }

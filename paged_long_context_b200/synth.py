@@ -13,15 +13,16 @@ Storage layout (one pool per storage format, caller-owned):
 Each (physical page, kv head) sub-page is a contiguous row-major
 [token][head_dim] block, the page content described on the CFR-Atlas page
 (section "KvRegenerator": K and V written row-major [token][head_dim]).
-row_bytes: F32 4*d, BF16 2*d, I8 d, I4 d/2.
+row_bytes: F32 4*d, BF16 2*d, I8 d, I4 d/2, FP8 d.
 
-Quantised pages (ARGUS page, "Visual Architecture": INT8, INT4 "2-way
+Quantised pages (ARGUS page, "Visual Architecture": FP8, INT8, INT4 "2-way
 bit-packed") carry one fp32 scale per (page, kv head, K-or-V):
-scale = max|x| / 127 (int8) or max|x| / 7 (int4) over the valid tokens of that
-block, code = clamp(round_half_even(x / scale)).  int4 codes are 4-bit two's
-complement; element 2i sits in the low nibble and element 2i+1 in the high
-nibble of byte i of a row.  The quantiser is input generation: the attention
-result depends only on the stored codes and scales.
+scale = max|x| / 127 (int8), max|x| / 7 (int4) or max|x| / 448 (FP8 E4M3) over
+the valid tokens of that block; integer codes = clamp(round_half_even(x /
+scale)), FP8 codes = the E4M3 value nearest to x / scale.  int4 codes are 4-bit
+two's complement; element 2i sits in the low nibble and element 2i+1 in the
+high nibble of byte i of a row.  The quantiser is input generation: the
+attention result depends only on the stored codes and scales.
 
 Tokens past a sequence's length inside its last page are not part of the
 input; float pools hold NaN there (and in unused pool slots) so that any stray
@@ -42,13 +43,16 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 import torch
 
-F32, BF16, I8, I4 = 0, 1, 2, 3
-FMT_COUNT = 4
-FMT_NAMES = {F32: "f32", BF16: "bf16", I8: "i8", I4: "i4"}
+F32, BF16, I8, I4, FP8 = 0, 1, 2, 3, 4
+FMT_COUNT = 5
+FMT_NAMES = {F32: "f32", BF16: "bf16", I8: "i8", I4: "i4", FP8: "fp8"}
+QUANTISED = (I8, I4, FP8)
 FMT_BY_NAME = {v: k for k, v in FMT_NAMES.items()}
 
 BF16_NAN_BITS = 0x7FC0
 I8_FILL = 0x80  # code -128: never written by the quantiser
+FP8_FILL = 0x7F  # E4M3 NaN: never written by the quantiser
+FP8_MAX = 448.0  # largest finite E4M3 magnitude
 
 
 def row_bytes(fmt: int, head_dim: int) -> int:
@@ -61,6 +65,8 @@ def row_bytes(fmt: int, head_dim: int) -> int:
         return head_dim
     if fmt == I4:
         return head_dim // 2
+    if fmt == FP8:
+        return head_dim
     raise ValueError(f"unknown page format {fmt}")
 
 
@@ -157,6 +163,22 @@ def _quant_int(x: torch.Tensor, valid: int, qmax: int):
     return codes.to(torch.int16), scale
 
 
+def _quant_fp8(x: torch.Tensor, valid: int):
+    """E4M3 encoding of one page block x: f32 [Hkv][P][d] with scale max|x| / 448.
+
+    Returns (uint8 codes [Hkv][P][d], scale f32 [Hkv]); an all-zero block gets
+    scale 0 and zero codes.
+    """
+    xv = x[:, :valid, :]
+    amax = xv.abs().amax(dim=(1, 2))
+    scale = amax / FP8_MAX
+    safe = torch.where(scale > 0, scale, torch.ones_like(scale))
+    y = (x / safe[:, None, None]).clamp_(-FP8_MAX, FP8_MAX)
+    codes = y.to(torch.float8_e4m3fn).view(torch.uint8).clone()
+    codes = torch.where(scale[:, None, None] > 0, codes, torch.zeros_like(codes))
+    return codes, scale
+
+
 def _pack_int4(codes: torch.Tensor) -> torch.Tensor:
     """codes int16 [..., d] in [-8, 7] -> uint8 [..., d/2]; even element in the low nibble."""
     nib = (codes & 0xF).to(torch.uint8)
@@ -166,8 +188,8 @@ def _pack_int4(codes: torch.Tensor) -> torch.Tensor:
 def _encode_page(x: torch.Tensor, fmt: int, valid: int):
     """Encode one page block x f32 [Hkv][P][d] into pool bytes uint8 [Hkv][P][row_bytes].
 
-    Rows at or past ``valid`` are filled with NaN (float formats) or code -128
-    (int8) / nibble 8 (int4).  Returns (bytes, scale or None).
+    Rows at or past ``valid`` are filled with NaN (float formats and FP8) or
+    code -128 (int8) / nibble 8 (int4).  Returns (bytes, scale or None).
     """
     hkv, ptok, d = x.shape
     if fmt == F32:
@@ -187,6 +209,10 @@ def _encode_page(x: torch.Tensor, fmt: int, valid: int):
         codes, scale = _quant_int(x, valid, 7)
         codes[:, valid:, :] = -8
         return _pack_int4(codes), scale
+    if fmt == FP8:
+        codes, scale = _quant_fp8(x, valid)
+        codes[:, valid:, :] = FP8_FILL
+        return codes, scale
     raise ValueError(fmt)
 
 
@@ -275,7 +301,7 @@ def make_case(spec: CaseSpec, seed: int, device="cpu") -> DecodeCase:
             k_pool[f] = torch.full((total[f], Hkv, P, d), BF16_NAN_BITS, dtype=torch.int16, device=device).view(torch.uint8).reshape(shape)
             v_pool[f] = torch.full((total[f], Hkv, P, d), BF16_NAN_BITS, dtype=torch.int16, device=device).view(torch.uint8).reshape(shape)
         else:
-            fill = I8_FILL if f == I8 else 0x88
+            fill = I8_FILL if f == I8 else FP8_FILL if f == FP8 else 0x88
             k_pool[f] = torch.full(shape, fill, dtype=torch.uint8, device=device)
             v_pool[f] = torch.full(shape, fill, dtype=torch.uint8, device=device)
             scales[f] = torch.zeros((total[f], Hkv, 2), dtype=torch.float32, device=device)

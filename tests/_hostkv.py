@@ -7,7 +7,8 @@ byte decoding or index arithmetic shows up as a disagreement.
 import numpy as np
 import torch
 
-F32, BF16, I8, I4 = 0, 1, 2, 3
+F32, BF16, I8, I4, FP8 = 0, 1, 2, 3, 4
+QUANTISED = (I8, I4, FP8)
 
 
 def decode_rows(raw: np.ndarray, fmt: int, d: int) -> np.ndarray:
@@ -28,6 +29,10 @@ def decode_rows(raw: np.ndarray, fmt: int, d: int) -> np.ndarray:
         out[..., 0::2] = lo
         out[..., 1::2] = hi
         return out
+    if fmt == FP8:
+        # E4M3 through torch's float8 dtype (a library decoder, not the oracle's)
+        t = torch.from_numpy(np.ascontiguousarray(raw)).view(torch.float8_e4m3fn)
+        return t.to(torch.float64).numpy()
     raise ValueError(fmt)
 
 
@@ -45,7 +50,7 @@ def host_kv(case, b: int, g: int):
         vb = case.v_pool[f][slot, g].cpu().numpy()
         k = decode_rows(kb, f, d)
         v = decode_rows(vb, f, d)
-        if f in (I8, I4):
+        if f in QUANTISED:
             s = case.scales[f][slot, g].cpu().numpy().astype(np.float64)
             k = k * s[0]
             v = v * s[1]

@@ -20,7 +20,8 @@ from paged_long_context_b200 import synth
 from tests._hostkv import host_kv, host_q, kv_head_of, sigma_of, decode_rows
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
-F32, BF16, I8, I4 = synth.F32, synth.BF16, synth.I8, synth.I4
+F32, BF16, I8, I4, FP8 = synth.F32, synth.BF16, synth.I8, synth.I4, synth.FP8
+QUANTISED = synth.QUANTISED
 
 
 def small(name="s", B=2, Hq=4, Hkv=2, d=16, P=8, lens=(37, 20), fmt="f32", q_fmt="f32",
@@ -100,13 +101,13 @@ def test_byte_patterns_decode(oracle_mod, pat):
     slot = int(case.page_table[0, 0])
     row = torch.tensor(list(raw), dtype=torch.uint8)
     case.v_pool[fmt][slot, 0, 0] = row
-    if fmt in (I8, I4):
+    if fmt in QUANTISED:
         case.scales[fmt][slot, 0, 1] = scale
     out, lse = oracle_mod.attend(case)
     # a single token has weight exactly 1: the output is its V row
     np.testing.assert_array_equal(out[0], np.array(expect, dtype=np.float64))
     # the independent numpy decoder agrees with the golden values too
-    dec = decode_rows(row.numpy(), fmt, d) * (scale if fmt in (I8, I4) else 1.0)
+    dec = decode_rows(row.numpy(), fmt, d) * (scale if fmt in QUANTISED else 1.0)
     np.testing.assert_array_equal(dec, np.array(expect))
 
 
@@ -134,11 +135,24 @@ def test_all_int8_and_int4_codes(oracle_mod):
     np.testing.assert_array_equal(out[0], np.array(expect, dtype=np.float64))
 
 
+def test_all_fp8_codes(oracle_mod):
+    # every E4M3 byte through the n = 1 closed form, against torch's float8 decoding
+    d = 256
+    case = small(B=1, Hq=1, Hkv=1, d=d, P=4, lens=(1,), fmt="fp8")
+    slot = int(case.page_table[0, 0])
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    case.v_pool[FP8][slot, 0, 0] = codes
+    case.scales[FP8][slot, 0, 1] = 0.5
+    out, _ = oracle_mod.attend(case)
+    want = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy() * 0.5
+    np.testing.assert_array_equal(out[0], want)
+
+
 # --------------------------------------------------------------------------
 # 3. Closed forms of softmax attention
 # --------------------------------------------------------------------------
 
-FMTS = ["f32", "bf16", "i8", "i4"]
+FMTS = ["f32", "bf16", "i8", "i4", "fp8"]
 
 
 @pytest.mark.parametrize("fmt", FMTS)
