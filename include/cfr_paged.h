@@ -12,8 +12,8 @@
  * fixed-size token pages reached through a page table (CFR-Atlas page, "page
  * identity and token ranges": a page holds a token range of one layer/head,
  * stored row-major [token][head_dim]).  Pages may be stored as fp32, bf16, or
- * as int8 / int4 codes with a per-page, per-head scale (the INT8 and INT4
- * tiers of the ARGUS page, "Visual Architecture"); quantised pages are
+ * as FP8 (E4M3) / int8 / int4 codes with a per-page, per-head scale (the FP8,
+ * INT8 and INT4 tiers of the ARGUS page, "Visual Architecture"); quantised pages are
  * expanded only in on-chip memory ("Transient FP16 Reconstruction ... in GPU
  * SRAM").  Each page range's partial (running max, normaliser, weighted-V
  * accumulator) is folded exactly (CFR-Atlas page, "exact folded
@@ -64,7 +64,10 @@ typedef enum {
   CFR_FMT_I8 = 2,    /* int8 two's-complement codes: head_dim bytes; value = code * scale */
   CFR_FMT_I4 = 3,    /* int4 codes, 2 per byte: head_dim / 2 bytes; element 2i in the low
                         nibble, 2i+1 in the high nibble of byte i; value = code * scale */
-  CFR_FMT_COUNT = 4
+  CFR_FMT_FP8 = 4,   /* FP8 E4M3 codes (sign, 4 exponent bits with bias 7, 3 mantissa bits,
+                        no infinities, 0x7F/0xFF NaN, largest 448): head_dim bytes;
+                        value = e4m3(code) * scale */
+  CFR_FMT_COUNT = 5
 } cfr_page_fmt;
 
 /* Bits of the device error word (OR-ed, never cleared by the library). */
@@ -79,11 +82,11 @@ typedef enum {
  * format selects its pool and the page table holds its slot inside that pool.
  *
  *   k_pool[f], v_pool[f]: device, uint8 [pool_pages[f]][num_kv_heads][page_tokens][row_bytes(f)]
- *       row_bytes: F32 4*d, BF16 2*d, I8 d, I4 d/2.  Every (slot, kv head)
+ *       row_bytes: F32 4*d, BF16 2*d, I8 d, I4 d/2, FP8 d.  Every (slot, kv head)
  *       sub-page is a contiguous row-major [page_tokens][head_dim] block.
  *       Base addresses must be 16-byte aligned.  NULL for unused formats.
  *   scales[f]: device, float [pool_pages[f]][num_kv_heads][2] = (K scale, V scale)
- *       for f = I8, I4; ignored (may be NULL) for F32, BF16.
+ *       for f = I8, I4, FP8; ignored (may be NULL) for F32, BF16.
  *   pool_pages[f]: number of slots of pool f (0 when unused).
  *   Tokens of a sequence's last page at or past its length are never read
  *   as values (their bytes may hold anything, NaN included).
@@ -262,6 +265,73 @@ cfr_status cfr_gather_pages(const cfr_kv_pool *kv, const int32_t *page_table,
                             void *k_raw_out,
                             void *v_raw_out, int64_t out_row_pitch, uint32_t *err_word,
                             void *stream);
+
+/*
+ * Page demotion: re-encodes whole pages from one storage format into another,
+ * the compression cascade of the ARGUS page ("Visual Architecture": full
+ * precision hot pages, then FP8, INT8 and INT4 tiers).  Page k is read from
+ * slot src_slots[k] of the src_fmt pool described by `kv` and written, every
+ * kv head, K and V, to slot dst_slots[k] of the destination pool.  Per
+ * (page, kv head, K-or-V) block, over its first valid_tokens[k] rows (all
+ * page_tokens rows when valid_tokens is NULL):
+ *   x     = the stored value as fp32 (quantised sources: code * scale, fp32 product);
+ *   scale = max|x| / Q in fp32 with Q = 127 (I8), 7 (I4), 448 (FP8);
+ *   I8/I4 code = clamp(round_half_even(x / scale), -Q, Q) (IEEE fp32 division);
+ *   FP8   code = the E4M3 value nearest to x / scale, ties to even, saturating at 448;
+ *   BF16  nearest bfloat16 (ties to even);  F32  x.
+ * A block of zeros gets scale 0 and zero codes.  Rows at or past the valid
+ * count are written as zero bytes.  Codes and scales are bit-exact functions
+ * of the stored source bytes (no data-value checks: NaN sources give
+ * unspecified codes).
+ *
+ *  kv           host; geometry (num_kv_heads, head_dim 64 or 128, page_tokens >= 8)
+ *               and the source pool k_pool/v_pool/scales/pool_pages[src_fmt].
+ *  src_fmt, dst_fmt  any two different formats.
+ *  dst_k_pool, dst_v_pool  device, uint8 [dst_pool_pages][num_kv_heads][page_tokens]
+ *               [row_bytes(dst_fmt)], 16-byte aligned, written; must not overlap
+ *               the source pages.
+ *  dst_scales   device float [dst_pool_pages][num_kv_heads][2], written for
+ *               quantised dst_fmt (may be NULL otherwise).
+ *  src_slots, dst_slots  device int32 [num_pages]; destination slots must be
+ *               distinct.  A slot outside its pool skips the page and sets
+ *               CFR_DEVERR_PAGE_ID.
+ *  valid_tokens device int32 [num_pages] or NULL; a count outside [1, page_tokens]
+ *               skips the page and sets CFR_DEVERR_SEQ_LEN.
+ * The page table is the caller's: point page_table/page_fmt at the new slot
+ * and format once the demotion has completed on the stream.
+ */
+cfr_status cfr_demote_pages(const cfr_kv_pool *kv, int32_t src_fmt, int32_t dst_fmt,
+                            void *dst_k_pool, void *dst_v_pool, float *dst_scales,
+                            int64_t dst_pool_pages, const int32_t *src_slots,
+                            const int32_t *dst_slots, const int32_t *valid_tokens,
+                            int32_t num_pages, uint32_t *err_word, void *stream);
+
+/*
+ * KV append: writes one new token per sequence into the full-precision tier
+ * (recent tokens stay in high fidelity; ARGUS page, "The One-Minute
+ * Explanation").  For every b with positions[b] >= 0, the rows
+ * k_new[b][g][:], v_new[b][g][:] (every kv head g) become token
+ * j = positions[b] of sequence b: row j % page_tokens of logical page
+ * j / page_tokens, resolved through page_table / page_fmt exactly as the
+ * decode resolves it.  Values are stored as fp32 (F32 pages) or rounded to
+ * the nearest bfloat16 (BF16 pages).  positions[b] < 0 appends nothing.
+ *
+ *  kv          host; the F32 and BF16 pools in it are WRITTEN (their pointers
+ *              must be writable device memory); other pools are ignored.
+ *  page_table, page_fmt (or NULL + uniform_fmt F32/BF16), max_pages: as for
+ *              cfr_paged_decode, `batch` rows.
+ *  positions   device int32 [batch].
+ *  k_new, v_new device [batch][num_kv_heads][head_dim], fp32 (new_fmt = CFR_FMT_F32)
+ *              or bf16 (CFR_FMT_BF16).
+ * Device-side faults skip the sequence and set err_word bits: a position at or
+ * past max_pages * page_tokens (CFR_DEVERR_SEQ_LEN), a page that is not F32 or
+ * BF16 or whose pool is NULL (CFR_DEVERR_PAGE_FMT), a slot outside its pool
+ * (CFR_DEVERR_PAGE_ID).  Sequences must not share the written page row.
+ */
+cfr_status cfr_append_kv(const cfr_kv_pool *kv, const int32_t *page_table, int32_t max_pages,
+                         const uint8_t *page_fmt, int32_t uniform_fmt, const int32_t *positions,
+                         int32_t batch, const void *k_new, const void *v_new, int32_t new_fmt,
+                         uint32_t *err_word, void *stream);
 
 /*
  * Which decode kernel a call with these arguments would run (for tests and

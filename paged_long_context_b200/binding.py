@@ -27,7 +27,8 @@ PATH_CUDA_CORE, PATH_TENSOR_CORE, PATH_F32_TMA = 1, 2, 3
 EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_decode_phases",
            "cfr_merge_partials",
            "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str",
-           "cfr_paged_decode_static_workspace"]
+           "cfr_paged_decode_static_workspace", "cfr_demote_pages", "cfr_append_kv"]
+FMT_COUNT = 5
 STATIC_WORKSPACE_BYTES = 8 << 20
 
 
@@ -42,8 +43,8 @@ class KvPool(ctypes.Structure):
     _fields_ = [
         ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("page_tokens", ctypes.c_int32),
-        ("k_pool", ctypes.c_void_p * 4), ("v_pool", ctypes.c_void_p * 4),
-        ("scales", ctypes.c_void_p * 4), ("pool_pages", ctypes.c_int64 * 4),
+        ("k_pool", ctypes.c_void_p * FMT_COUNT), ("v_pool", ctypes.c_void_p * FMT_COUNT),
+        ("scales", ctypes.c_void_p * FMT_COUNT), ("pool_pages", ctypes.c_int64 * FMT_COUNT),
     ]
 
 
@@ -79,6 +80,12 @@ def lib():
         L.cfr_paged_decode_static_workspace.argtypes = [_VP, _I32, ctypes.POINTER(KvPool), _VP, _I32,
                                                         _VP, _I32, _VP, _I32, _I32, _VP, _VP, _F32,
                                                         _VP, _VP, _VP, _VP]
+        L.cfr_demote_pages.restype = ctypes.c_int
+        L.cfr_demote_pages.argtypes = [ctypes.POINTER(KvPool), _I32, _I32, _VP, _VP, _VP, _I64,
+                                       _VP, _VP, _VP, _I32, _VP, _VP]
+        L.cfr_append_kv.restype = ctypes.c_int
+        L.cfr_append_kv.argtypes = [ctypes.POINTER(KvPool), _VP, _I32, _VP, _I32, _VP, _I32,
+                                    _VP, _VP, _I32, _VP, _VP]
         L.cfr_status_str.restype = ctypes.c_char_p
         L.cfr_status_str.argtypes = [ctypes.c_int]
         _lib = L
@@ -103,15 +110,23 @@ def status_str(status: int) -> str:
     return lib().cfr_status_str(status).decode()
 
 
-def kv_pool_struct(case: "synth.DecodeCase") -> KvPool:
+def pool_struct(num_kv_heads: int, head_dim: int, page_tokens: int, k_pool: dict, v_pool: dict,
+                scales: Optional[dict] = None) -> KvPool:
+    """cfr_kv_pool from dicts format -> device tensor."""
     s = KvPool()
-    s.num_kv_heads, s.head_dim, s.page_tokens = case.num_kv_heads, case.head_dim, case.page_tokens
-    for f in range(4):
-        s.k_pool[f] = case.k_pool[f].data_ptr() if f in case.k_pool else None
-        s.v_pool[f] = case.v_pool[f].data_ptr() if f in case.v_pool else None
-        s.scales[f] = case.scales[f].data_ptr() if f in case.scales else None
-        s.pool_pages[f] = int(case.k_pool[f].shape[0]) if f in case.k_pool else 0
+    s.num_kv_heads, s.head_dim, s.page_tokens = num_kv_heads, head_dim, page_tokens
+    scales = scales or {}
+    for f in range(FMT_COUNT):
+        s.k_pool[f] = k_pool[f].data_ptr() if f in k_pool else None
+        s.v_pool[f] = v_pool[f].data_ptr() if f in v_pool else None
+        s.scales[f] = scales[f].data_ptr() if f in scales else None
+        s.pool_pages[f] = int(k_pool[f].shape[0]) if f in k_pool else 0
     return s
+
+
+def kv_pool_struct(case: "synth.DecodeCase") -> KvPool:
+    return pool_struct(case.num_kv_heads, case.head_dim, case.page_tokens, case.k_pool,
+                       case.v_pool, case.scales)
 
 
 def workspace_size(batch, num_q_heads, num_kv_heads, head_dim, max_pages, page_tokens) -> int:
@@ -213,3 +228,24 @@ def paged_decode_static_workspace(case, out, lse=None, err=None, stream=None) ->
         _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads, hmp,
         _p(case.alibi_slopes), float(case.softmax_scale), _p(out), _p(lse), _p(err),
         _stream(stream)))
+
+
+def demote_pages(pool: KvPool, src_fmt: int, dst_fmt: int, dst_k, dst_v, dst_scales,
+                 src_slots, dst_slots, valid_tokens=None, err=None, stream=None) -> int:
+    """cfr_demote_pages: re-encode pages of the src_fmt pool described by ``pool`` into
+    the destination pool tensors (device uint8 [slots][Hkv][P][row_bytes]); returns the status."""
+    n = int(src_slots.numel())
+    return int(lib().cfr_demote_pages(ctypes.byref(pool), src_fmt, dst_fmt, _p(dst_k), _p(dst_v),
+                                      _p(dst_scales), int(dst_k.shape[0]), _p(src_slots),
+                                      _p(dst_slots), _p(valid_tokens), n, _p(err),
+                                      _stream(stream)))
+
+
+def append_kv(pool: KvPool, page_table, page_fmt, uniform_fmt: int, positions, k_new, v_new,
+              err=None, stream=None) -> int:
+    """cfr_append_kv: write one token per sequence into its F32/BF16 page; returns the status."""
+    new_fmt = synth.F32 if k_new.dtype == torch.float32 else synth.BF16
+    return int(lib().cfr_append_kv(ctypes.byref(pool), _p(page_table), int(page_table.shape[1]),
+                                   _p(page_fmt), uniform_fmt, _p(positions),
+                                   int(positions.numel()), _p(k_new), _p(v_new), new_fmt, _p(err),
+                                   _stream(stream)))

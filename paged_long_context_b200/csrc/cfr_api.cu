@@ -130,7 +130,7 @@ cfr_status check_pool(const cfr_kv_pool *kv) {
     if (!kv->k_pool[f] || !kv->v_pool[f]) return CFR_ERR_INVALID_ARG;
     if (!aligned(kv->k_pool[f], 16) || !aligned(kv->v_pool[f], 16)) return CFR_ERR_INVALID_ARG;
     if (kv->pool_pages[f] < 0) return CFR_ERR_INVALID_ARG;
-    if ((f == CFR_FMT_I8 || f == CFR_FMT_I4) && kv->pool_pages[f] > 0) {
+    if (is_quantised(f) && kv->pool_pages[f] > 0) {
       if (!kv->scales[f] || !aligned(kv->scales[f], 8)) return CFR_ERR_INVALID_ARG;
     }
     // byte offsets of the last row must fit in 64 bits

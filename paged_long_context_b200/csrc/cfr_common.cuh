@@ -10,6 +10,8 @@
 #include <cstdint>
 #include <utility>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "cfr_paged.h"
@@ -48,7 +50,12 @@ struct DecodeParams {
 };
 
 __host__ __device__ inline int row_bytes(int fmt, int d) {
-  return fmt == CFR_FMT_F32 ? 4 * d : fmt == CFR_FMT_BF16 ? 2 * d : fmt == CFR_FMT_I8 ? d : d / 2;
+  return fmt == CFR_FMT_F32 ? 4 * d : fmt == CFR_FMT_BF16 ? 2 * d : fmt == CFR_FMT_I4 ? d / 2 : d;
+}
+
+// formats whose values are codes times a per-(page, kv head) scale
+__host__ __device__ inline bool is_quantised(int fmt) {
+  return fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4 || fmt == CFR_FMT_FP8;
 }
 
 __device__ __forceinline__ void set_err(uint32_t *err, uint32_t bits) {
@@ -180,6 +187,21 @@ __device__ __forceinline__ float i8_at(uint32_t w, int k) {
 __device__ __forceinline__ float i4_at(uint32_t w, int k) {
   int v = static_cast<int>((w >> (4 * k)) & 0xF);
   return static_cast<float>(v >= 8 ? v - 16 : v);
+}
+
+// bytes 2i and 2i+1 of w (E4M3 codes) as an fp16 pair, element 2i in the low
+// half (every E4M3 value, NaN included, is exact in fp16)
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t w, int i) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+      static_cast<__nv_fp8x2_storage_t>((w >> (16 * i)) & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// E4M3 code k (0..3) of w as fp32
+__device__ __forceinline__ float e4m3_at(uint32_t w, int k) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>((w >> (8 * k)) & 0xFFu),
+                                               __NV_E4M3);
+  return __half2float(__half(h));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -112,6 +112,28 @@ __device__ __forceinline__ void load_elems(int fmt, const uint8_t *row, int e0, 
       const uint32_t w = *reinterpret_cast<const uint16_t *>(p);
       x[0] = i8_at(w, 0); x[1] = i8_at(w, 1);
     }
+  } else if (fmt == CFR_FMT_FP8) {
+    const uint8_t *p = row + e0;
+    if constexpr (N % 16 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 16; ++i) {
+        const uint4 w = reinterpret_cast<const uint4 *>(p)[i];
+        const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[16 * i + k] = e4m3_at(a[k / 4], k % 4);
+      }
+    } else if constexpr (N == 8) {
+      const uint2 w = *reinterpret_cast<const uint2 *>(p);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = e4m3_at(k < 4 ? w.x : w.y, k % 4);
+    } else if constexpr (N == 4) {
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = e4m3_at(w, k);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint16_t *>(p);
+      x[0] = e4m3_at(w, 0); x[1] = e4m3_at(w, 1);
+    }
   } else {  // CFR_FMT_I4
     const uint8_t *p = row + e0 / 2;
     if constexpr (N % 8 == 0) {
@@ -221,14 +243,13 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
         f.ks = f.vs = 1.f;
         if (fmt < 0 || fmt >= kFmtCount) {
           set_err(p.err, CFR_DEVERR_PAGE_FMT);
-        } else if (!p.k_pool[fmt] || !p.v_pool[fmt] ||
-                   ((fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) && !p.scales[fmt])) {
+        } else if (!p.k_pool[fmt] || !p.v_pool[fmt] || (is_quantised(fmt) && !p.scales[fmt])) {
           set_err(p.err, CFR_DEVERR_POOL);
         } else if (id < 0 || id >= p.pool_pages[fmt]) {
           set_err(p.err, CFR_DEVERR_PAGE_ID);
         } else {
           f.ok = 1;
-          if (fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) {
+          if (is_quantised(fmt)) {
             const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
             f.ks = s.x;
             f.vs = s.y;

@@ -1,5 +1,6 @@
 // cfr_decode_tc.cu -- paged decode attention on the 5th-generation tensor cores
-// (tcgen05, accumulators in TMEM) for bf16, int8 and int4 K/V pages, head_dim 128.
+// (tcgen05, accumulators in TMEM) for bf16, FP8 (E4M3), int8 and int4 K/V pages,
+// head_dim 128.
 //
 // For a kv head serving G query heads, one 128-token tile is two small dense
 // contractions:
@@ -8,8 +9,8 @@
 // N = 16 (G <= 8) or 32 (G <= 16) columns: N/2 "hi" and N/2 "lo" columns, so that q
 // (fp32 or bf16) and the probabilities p enter the 16-bit MMA as hi + lo pairs
 // (about 16 significant bits for bf16, 22 for fp16), accumulated in fp32.
-// bf16 pages run bf16 MMAs; int8 / int4 pages are expanded to fp16 codes in
-// shared memory (codes are exact in fp16) and run fp16 MMAs; their per-page
+// bf16 pages run bf16 MMAs; FP8 / int8 / int4 pages are expanded to fp16 codes
+// in shared memory (their codes are exact in fp16) and run fp16 MMAs; their per-page
 // K scale multiplies the scores, their V scale multiplies the tile's P.V
 // result, both in fp32 (ARGUS page, "Transient FP16 Reconstruction ... in GPU
 // SRAM": pages are expanded on chip only, attention runs at 16-bit).
@@ -29,7 +30,7 @@
 //               and the exact fold acc = acc*2^(m_old-m_new) + O_tile of the
 //               previous tile (CFR-Atlas page, "exact folded online-softmax
 //               attention pass").
-//   warps 6-9   staging: int8/int4 rows -> fp16 operand rows; zeroes V rows of
+//   warps 6-9   staging: FP8/int8/int4 rows -> fp16 operand rows; zeroes V rows of
 //               tokens that are not part of the input so stale or NaN bytes
 //               never meet a zero probability inside the MMA.
 // Every mbarrier wait is bounded; on a timeout the error word is set, every
@@ -48,8 +49,8 @@ constexpr int TC_D = 128;            // head_dim
 constexpr int TC_THREADS = 352;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
-constexpr int TC_RAW_BYTES = 2 * TC_T * TC_D;  // raw int8 K + V rows (int4 uses half)
-constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2;
+constexpr int TC_RAW_BYTES = 2 * TC_T * TC_D;  // raw int8 / FP8 K + V rows (int4 uses half)
+constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2, KIND_FP8 = 3;
 
 struct TcMeta {
   uint32_t valid[4];
@@ -293,8 +294,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
     id = pc.id[pg - pc.base];
     if (fmt < 0 || fmt >= kFmtCount) {
       set_err(p.err, CFR_DEVERR_PAGE_FMT);
-    } else if (fmt == CFR_FMT_F32 || !p.k_pool[fmt] ||
-               ((fmt == CFR_FMT_I8 || fmt == CFR_FMT_I4) && !p.scales[fmt])) {
+    } else if (fmt == CFR_FMT_F32 || !p.k_pool[fmt] || (is_quantised(fmt) && !p.scales[fmt])) {
       set_err(p.err, CFR_DEVERR_POOL);
     } else if (id < 0 || id >= p.pool_pages[fmt]) {
       set_err(p.err, CFR_DEVERR_PAGE_ID);
@@ -304,7 +304,11 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
   }
   const uint32_t vb = __ballot_sync(0xffffffffu, pvalid);
   // quantised pages need page_tokens >= 128: the tile is then one piece (lane 0)
-  const int kind0 = (fmt == CFR_FMT_I8 && pvalid) ? KIND_I8 : (fmt == CFR_FMT_I4 && pvalid) ? KIND_I4 : KIND_BF16;
+  const int kind0 = !pvalid                ? KIND_BF16
+                    : fmt == CFR_FMT_I8    ? KIND_I8
+                    : fmt == CFR_FMT_I4    ? KIND_I4
+                    : fmt == CFR_FMT_FP8   ? KIND_FP8
+                                           : KIND_BF16;
   const int kind = __shfl_sync(0xffffffffu, kind0, 0);
   uint64_t *done = nullptr;
   if (lane == 0) {
@@ -453,6 +457,25 @@ __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
                 i8x4_to_h2x2(w.z, o[4], o[5]);
                 i8x4_to_h2x2(w.w, o[6], o[7]);
                 // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
+                uint8_t *hb = dst + (ci >> 2) * TC_HALF;
+                const int oc = (2 * ci) & 7;
+                *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+              }
+            } else if (m.kind == KIND_FP8) {
+              // 128 E4M3 codes = 8 chunks of 16 bytes, each to two fp16 output chunks
+              const uint8_t *src = raw + kv * TC_T * TC_D + r * TC_D;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int ci = (j + r) & 7;
+                const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                uint32_t o[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  o[2 * q] = e4m3x2_to_h2(wv[q], 0);
+                  o[2 * q + 1] = e4m3x2_to_h2(wv[q], 1);
+                }
                 uint8_t *hb = dst + (ci >> 2) * TC_HALF;
                 const int oc = (2 * ci) & 7;
                 *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -928,9 +951,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
+// quantised pools present: tiles pass through the raw staging buffers
 static bool tc_int_pools(const DecodeParams &p, bool page_fmt_given) {
-  if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4];
-  return p.uniform_fmt == CFR_FMT_I8 || p.uniform_fmt == CFR_FMT_I4;
+  if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4] || p.k_pool[CFR_FMT_FP8];
+  return is_quantised(p.uniform_fmt);
 }
 
 bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
@@ -938,7 +962,9 @@ bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
   if ((reinterpret_cast<uintptr_t>(p.q) & 15) != 0) return false;
   if (page_fmt_given) {
     if (p.k_pool[CFR_FMT_F32]) return false;
-    if (!p.k_pool[CFR_FMT_BF16] && !p.k_pool[CFR_FMT_I8] && !p.k_pool[CFR_FMT_I4]) return false;
+    if (!p.k_pool[CFR_FMT_BF16] && !p.k_pool[CFR_FMT_I8] && !p.k_pool[CFR_FMT_I4] &&
+        !p.k_pool[CFR_FMT_FP8])
+      return false;
   } else if (p.uniform_fmt == CFR_FMT_F32) {
     return false;
   }

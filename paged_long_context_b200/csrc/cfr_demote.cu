@@ -1,0 +1,365 @@
+// cfr_demote.cu -- page demotion down the compression cascade, and KV append.
+//
+// Demotion re-encodes whole pages from one storage format into another: the
+// compression cascade of the ARGUS page ("Visual Architecture": hot pages in
+// full precision, cold pages FP8 -> INT8 -> INT4).  Per (page, kv head,
+// K-or-V) block of P rows x d, over its first `valid` rows:
+//   x      = stored value as fp32 (quantised sources: code * scale in fp32);
+//   scale  = max|x| / Q in fp32 (Q = 127 int8, 7 int4, 448 FP8 E4M3);
+//   int    code = clamp(round_half_even(x / scale), -Q, Q), IEEE fp32 division;
+//   FP8    code = E4M3 nearest to x / scale, saturating at 448;
+//   BF16   x rounded to nearest even; F32: x.
+// An all-zero block gets scale 0 and zero codes; rows past `valid` are
+// written as zero bytes.  One CTA per block: pass 1 reduces max|x| over the
+// valid rows, pass 2 re-reads the block (from L2: a block is at most a few
+// hundred KiB and is re-read right away) and writes the codes with coalesced
+// vector stores.  The kernel is bound by HBM: it reads the source block once
+// from DRAM and writes the destination block once.
+//
+// Append writes the new K and V rows of one decode step into the hot tier:
+// token j = positions[b] of sequence b goes to row j % P of logical page j / P
+// (ARGUS page, "The One-Minute Explanation": recent tokens stay in
+// high-fidelity memory), widened to fp32 or rounded to bf16.
+#include <climits>
+
+#include <cuda_bf16.h>
+
+#include "cfr_common.cuh"
+
+namespace cfr {
+
+namespace {
+
+constexpr int kDemoteThreads = 512;
+constexpr int kVec = 8;  // elements per vector access
+
+struct DemoteParams {
+  const uint8_t *src_k, *src_v;
+  const float *src_scales;
+  long long src_pages;
+  uint8_t *dst_k, *dst_v;
+  float *dst_scales;
+  long long dst_pages;
+  const int32_t *src_slots, *dst_slots, *valid_tokens;
+  uint32_t *err;
+  int src_fmt, dst_fmt, Hkv, D, P;
+};
+
+// eight consecutive stored elements starting at element e of a block, as fp32
+__device__ __forceinline__ void load8(int fmt, const uint8_t *blk, long long e, float scale,
+                                      float (&x)[kVec]) {
+  if (fmt == CFR_FMT_F32) {
+    const float4 *p = reinterpret_cast<const float4 *>(blk + 4 * e);
+    const float4 a = p[0], b = p[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else if (fmt == CFR_FMT_BF16) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(blk + 2 * e);
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[2 * k] = bf16_lo(a[k]);
+      x[2 * k + 1] = bf16_hi(a[k]);
+    }
+  } else if (fmt == CFR_FMT_I8) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(blk + e);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(i8_at(k < 4 ? w.x : w.y, k & 3), scale);
+  } else if (fmt == CFR_FMT_FP8) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(blk + e);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(e4m3_at(k < 4 ? w.x : w.y, k & 3), scale);
+  } else {  // CFR_FMT_I4
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(blk + e / 2);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(i4_at(w, k), scale);
+  }
+}
+
+__device__ __forceinline__ int int_code(float x, float scale, int q) {
+  if (!(scale > 0.f)) return 0;
+  const int c = __float2int_rn(__fdiv_rn(x, scale));  // NaN -> 0
+  return min(max(c, -q), q);
+}
+
+__device__ __forceinline__ uint32_t fp8_code(float x, float scale) {
+  if (!(scale > 0.f)) return 0u;
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(x, scale), __NV_SATFINITE, __NV_E4M3));
+}
+
+// encodes eight values and stores them at element e of the destination block
+__device__ __forceinline__ void store8(int fmt, uint8_t *blk, long long e, float scale,
+                                       const float (&x)[kVec]) {
+  if (fmt == CFR_FMT_F32) {
+    float4 *p = reinterpret_cast<float4 *>(blk + 4 * e);
+    p[0] = make_float4(x[0], x[1], x[2], x[3]);
+    p[1] = make_float4(x[4], x[5], x[6], x[7]);
+  } else if (fmt == CFR_FMT_BF16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(x[2 * k]));
+      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(x[2 * k + 1]));
+      w[k] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(blk + 2 * e) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if (fmt == CFR_FMT_I8) {
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      w[k >> 2] |= (static_cast<uint32_t>(int_code(x[k], scale, 127)) & 0xFFu) << (8 * (k & 3));
+    *reinterpret_cast<uint2 *>(blk + e) = make_uint2(w[0], w[1]);
+  } else if (fmt == CFR_FMT_FP8) {
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w[k >> 2] |= fp8_code(x[k], scale) << (8 * (k & 3));
+    *reinterpret_cast<uint2 *>(blk + e) = make_uint2(w[0], w[1]);
+  } else {  // CFR_FMT_I4: element 2i in the low nibble of byte i
+    uint32_t w = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w |= (static_cast<uint32_t>(int_code(x[k], scale, 7)) & 0xFu) << (4 * k);
+    *reinterpret_cast<uint32_t *>(blk + e / 2) = w;
+  }
+}
+
+__device__ __forceinline__ void store_zero8(int fmt, uint8_t *blk, long long e) {
+  if (fmt == CFR_FMT_F32) {
+    float4 *p = reinterpret_cast<float4 *>(blk + 4 * e);
+    p[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    p[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else if (fmt == CFR_FMT_BF16) {
+    *reinterpret_cast<uint4 *>(blk + 2 * e) = make_uint4(0u, 0u, 0u, 0u);
+  } else if (fmt == CFR_FMT_I4) {
+    *reinterpret_cast<uint32_t *>(blk + e / 2) = 0u;
+  } else {
+    *reinterpret_cast<uint2 *>(blk + e) = make_uint2(0u, 0u);
+  }
+}
+
+__device__ __forceinline__ float qmax_of(int fmt) {
+  return fmt == CFR_FMT_I8 ? 127.f : fmt == CFR_FMT_I4 ? 7.f : 448.f;
+}
+
+// block (page k, kv head g, K or V) = blockIdx.x
+__global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) {
+  __shared__ float red[kDemoteThreads / 32];
+  const long long blk_id = blockIdx.x;
+  const int kv = static_cast<int>(blk_id & 1);
+  const int g = static_cast<int>((blk_id >> 1) % p.Hkv);
+  const long long k = (blk_id >> 1) / p.Hkv;
+  const long long s = p.src_slots[k], t = p.dst_slots[k];
+  const int valid = p.valid_tokens ? p.valid_tokens[k] : p.P;
+  if (s < 0 || s >= p.src_pages || t < 0 || t >= p.dst_pages) {
+    if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_PAGE_ID);
+    return;
+  }
+  if (valid < 1 || valid > p.P) {
+    if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_SEQ_LEN);
+    return;
+  }
+  const long long blk_elems = static_cast<long long>(p.P) * p.D;
+  const uint8_t *src = (kv ? p.src_v : p.src_k) + (s * p.Hkv + g) * p.P * row_bytes(p.src_fmt, p.D);
+  uint8_t *dst = (kv ? p.dst_v : p.dst_k) + (t * p.Hkv + g) * p.P * row_bytes(p.dst_fmt, p.D);
+  const float src_scale = is_quantised(p.src_fmt) ? p.src_scales[(s * p.Hkv + g) * 2 + kv] : 1.f;
+  const long long nvec_valid = static_cast<long long>(valid) * p.D / kVec;
+  const long long nvec = blk_elems / kVec;
+
+  float scale = 1.f;
+  if (is_quantised(p.dst_fmt)) {
+    float amax = 0.f;
+    for (long long v = threadIdx.x; v < nvec_valid; v += kDemoteThreads) {
+      float x[kVec];
+      load8(p.src_fmt, src, v * kVec, src_scale, x);
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < kDemoteThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+    scale = __fdiv_rn(amax, qmax_of(p.dst_fmt));
+    if (threadIdx.x == 0) p.dst_scales[(t * p.Hkv + g) * 2 + kv] = scale;
+  }
+  for (long long v = threadIdx.x; v < nvec; v += kDemoteThreads) {
+    if (v < nvec_valid) {
+      float x[kVec];
+      load8(p.src_fmt, src, v * kVec, src_scale, x);
+      store8(p.dst_fmt, dst, v * kVec, scale, x);
+    } else {
+      store_zero8(p.dst_fmt, dst, v * kVec);
+    }
+  }
+}
+
+struct AppendParams {
+  uint8_t *k_pool[kFmtCount];
+  uint8_t *v_pool[kFmtCount];
+  long long pool_pages[kFmtCount];
+  const int32_t *page_table;
+  const uint8_t *page_fmt;
+  const int32_t *positions;
+  const void *k_new, *v_new;
+  uint32_t *err;
+  int uniform_fmt, new_fmt, max_pages, Hkv, D, P;
+};
+
+// sequence b = blockIdx.x; threads cover Hkv x D elements of K and V
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+  const int b = blockIdx.x;
+  const long long j = p.positions[b];
+  if (j < 0) return;
+  if (j >= static_cast<long long>(p.max_pages) * p.P) {
+    if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_SEQ_LEN);
+    return;
+  }
+  const long long cell = static_cast<long long>(b) * p.max_pages + j / p.P;
+  const int fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
+  if ((fmt != CFR_FMT_F32 && fmt != CFR_FMT_BF16) || !p.k_pool[fmt] || !p.v_pool[fmt]) {
+    if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_PAGE_FMT);
+    return;
+  }
+  const long long slot = p.page_table[cell];
+  if (slot < 0 || slot >= p.pool_pages[fmt]) {
+    if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_PAGE_ID);
+    return;
+  }
+  const int rb = row_bytes(fmt, p.D);
+  const int tin = static_cast<int>(j % p.P);
+  const int n = p.Hkv * p.D;
+  for (int i = threadIdx.x; i < 2 * n; i += blockDim.x) {
+    const int kv = i >= n;
+    const int e = kv ? i - n : i;
+    const int g = e / p.D, c = e - g * p.D;
+    const long long src_i = static_cast<long long>(b) * n + e;
+    const void *srcv = kv ? p.v_new : p.k_new;
+    const float x = p.new_fmt == CFR_FMT_F32
+                        ? static_cast<const float *>(srcv)[src_i]
+                        : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(srcv)[src_i]) << 16);
+    uint8_t *row = (kv ? p.v_pool[fmt] : p.k_pool[fmt]) + ((slot * p.Hkv + g) * p.P + tin) * rb;
+    if (fmt == CFR_FMT_F32)
+      reinterpret_cast<float *>(row)[c] = x;
+    else
+      reinterpret_cast<uint16_t *>(row)[c] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+  }
+}
+
+bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// pool geometry shared by demotion and append
+cfr_status check_geometry(const cfr_kv_pool *kv) {
+  if (!kv) return CFR_ERR_INVALID_ARG;
+  if (kv->num_kv_heads <= 0 || kv->head_dim <= 0 || kv->page_tokens <= 0) return CFR_ERR_INVALID_ARG;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return CFR_ERR_UNSUPPORTED;
+  if (kv->page_tokens < 8) return CFR_ERR_UNSUPPORTED;
+  return CFR_OK;
+}
+
+bool pool_bytes_fit(long long pages, const cfr_kv_pool *kv, int fmt) {
+  if (pages < 0) return false;
+  const long long per = static_cast<long long>(kv->num_kv_heads) * kv->page_tokens *
+                        row_bytes(fmt, kv->head_dim);
+  return pages == 0 || per <= LLONG_MAX / pages;
+}
+
+}  // namespace
+}  // namespace cfr
+
+using namespace cfr;
+
+extern "C" {
+
+cfr_status cfr_demote_pages(const cfr_kv_pool *kv, int32_t src_fmt, int32_t dst_fmt,
+                            void *dst_k_pool, void *dst_v_pool, float *dst_scales,
+                            int64_t dst_pool_pages, const int32_t *src_slots,
+                            const int32_t *dst_slots, const int32_t *valid_tokens,
+                            int32_t num_pages, uint32_t *err_word, void *stream) {
+  cfr_status st = check_geometry(kv);
+  if (st != CFR_OK) return st;
+  if (src_fmt < 0 || src_fmt >= kFmtCount || dst_fmt < 0 || dst_fmt >= kFmtCount ||
+      src_fmt == dst_fmt)
+    return CFR_ERR_INVALID_ARG;
+  if (num_pages < 0) return CFR_ERR_INVALID_ARG;
+  if (!kv->k_pool[src_fmt] || !kv->v_pool[src_fmt] || !dst_k_pool || !dst_v_pool)
+    return CFR_ERR_INVALID_ARG;
+  if (!aligned_to(kv->k_pool[src_fmt], 16) || !aligned_to(kv->v_pool[src_fmt], 16) ||
+      !aligned_to(dst_k_pool, 16) || !aligned_to(dst_v_pool, 16))
+    return CFR_ERR_INVALID_ARG;
+  if (is_quantised(src_fmt) && (!kv->scales[src_fmt] || !aligned_to(kv->scales[src_fmt], 8)))
+    return CFR_ERR_INVALID_ARG;
+  if (is_quantised(dst_fmt) && (!dst_scales || !aligned_to(dst_scales, 8))) return CFR_ERR_INVALID_ARG;
+  if (!pool_bytes_fit(kv->pool_pages[src_fmt], kv, src_fmt) || !pool_bytes_fit(dst_pool_pages, kv, dst_fmt))
+    return CFR_ERR_OVERFLOW;
+  if (static_cast<long long>(num_pages) * kv->num_kv_heads * 2 > INT_MAX) return CFR_ERR_OVERFLOW;
+  if (num_pages == 0) return CFR_OK;
+  if (!src_slots || !dst_slots) return CFR_ERR_INVALID_ARG;
+  DemoteParams p;
+  p.src_k = static_cast<const uint8_t *>(kv->k_pool[src_fmt]);
+  p.src_v = static_cast<const uint8_t *>(kv->v_pool[src_fmt]);
+  p.src_scales = kv->scales[src_fmt];
+  p.src_pages = kv->pool_pages[src_fmt];
+  p.dst_k = static_cast<uint8_t *>(dst_k_pool);
+  p.dst_v = static_cast<uint8_t *>(dst_v_pool);
+  p.dst_scales = dst_scales;
+  p.dst_pages = dst_pool_pages;
+  p.src_slots = src_slots;
+  p.dst_slots = dst_slots;
+  p.valid_tokens = valid_tokens;
+  p.err = err_word;
+  p.src_fmt = src_fmt;
+  p.dst_fmt = dst_fmt;
+  p.Hkv = kv->num_kv_heads;
+  p.D = kv->head_dim;
+  p.P = kv->page_tokens;
+  const unsigned blocks = static_cast<unsigned>(num_pages) * kv->num_kv_heads * 2u;
+  demote_kernel<<<blocks, kDemoteThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
+}
+
+cfr_status cfr_append_kv(const cfr_kv_pool *kv, const int32_t *page_table, int32_t max_pages,
+                         const uint8_t *page_fmt, int32_t uniform_fmt, const int32_t *positions,
+                         int32_t batch, const void *k_new, const void *v_new, int32_t new_fmt,
+                         uint32_t *err_word, void *stream) {
+  cfr_status st = check_geometry(kv);
+  if (st != CFR_OK) return st;
+  if (!page_table || !positions || !k_new || !v_new) return CFR_ERR_INVALID_ARG;
+  if (batch <= 0 || max_pages <= 0) return CFR_ERR_INVALID_ARG;
+  if (new_fmt != CFR_FMT_F32 && new_fmt != CFR_FMT_BF16) return CFR_ERR_INVALID_ARG;
+  if (!page_fmt && uniform_fmt != CFR_FMT_F32 && uniform_fmt != CFR_FMT_BF16) return CFR_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_pages) * kv->page_tokens > INT_MAX ||
+      static_cast<long long>(batch) * max_pages > INT_MAX)
+    return CFR_ERR_OVERFLOW;
+  AppendParams p;
+  bool any = false;
+  for (int f = 0; f < kFmtCount; ++f) {
+    const bool hot = f == CFR_FMT_F32 || f == CFR_FMT_BF16;
+    p.k_pool[f] = hot ? static_cast<uint8_t *>(const_cast<void *>(kv->k_pool[f])) : nullptr;
+    p.v_pool[f] = hot ? static_cast<uint8_t *>(const_cast<void *>(kv->v_pool[f])) : nullptr;
+    p.pool_pages[f] = p.k_pool[f] ? kv->pool_pages[f] : 0;
+    if (!p.k_pool[f] != !p.v_pool[f]) return CFR_ERR_INVALID_ARG;
+    if (p.k_pool[f]) {
+      if (!aligned_to(p.k_pool[f], 16) || !aligned_to(p.v_pool[f], 16)) return CFR_ERR_INVALID_ARG;
+      if (!pool_bytes_fit(kv->pool_pages[f], kv, f)) return CFR_ERR_OVERFLOW;
+      any = true;
+    }
+  }
+  if (!any) return CFR_ERR_INVALID_ARG;
+  p.page_table = page_table;
+  p.page_fmt = page_fmt;
+  p.positions = positions;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.err = err_word;
+  p.uniform_fmt = uniform_fmt;
+  p.new_fmt = new_fmt;
+  p.max_pages = max_pages;
+  p.Hkv = kv->num_kv_heads;
+  p.D = kv->head_dim;
+  p.P = kv->page_tokens;
+  append_kernel<<<batch, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -189,3 +189,74 @@ def test_path_selection_is_host_only(lib):
         binding.PATH_CUDA_CORE
     # rejected configurations report 0
     assert binding.decode_path(_case(num_q_heads=3, num_kv_heads=2)) == 0
+
+
+def test_path_selection_fp8(lib):
+    # FP8 pages: head_dim 128 with 128-token pages take the tensor-core kernel
+    assert binding.decode_path(_case(fmt="fp8", head_dim=128, page_tokens=128)) == \
+        binding.PATH_TENSOR_CORE
+    # other shapes take the general kernel
+    assert binding.decode_path(_case(fmt="fp8")) == binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="fp8", head_dim=128, page_tokens=64)) == \
+        binding.PATH_CUDA_CORE
+
+
+def test_fp8_pool_needs_scales(lib):
+    case = _case(fmt="fp8")
+    assert _decode(case, pool={"scales": {synth.FP8: None}}) == INVALID
+
+
+def _demote(pool, src, dst, dk, dv, dsc, n=1, dst_pages=None, slots=True):
+    t = torch.zeros(8, dtype=torch.int32)
+    sp = ctypes.c_void_p(t.data_ptr()) if slots else None
+    return binding.lib().cfr_demote_pages(
+        ctypes.byref(pool), src, dst, dk, dv, dsc,
+        dst_pages if dst_pages is not None else 4, sp, sp, None, n, None, None)
+
+
+def test_demote_rejects(lib):
+    case = _case()                          # bf16 pool, d 64, P 16
+    pool = binding.kv_pool_struct(case)
+    buf = torch.zeros(1 << 16, dtype=torch.uint8)
+    sc = torch.zeros(64)
+    p = ctypes.c_void_p(buf.data_ptr())
+    ps = ctypes.c_void_p(sc.data_ptr())
+    BF, I8, F32 = synth.BF16, synth.I8, synth.F32
+    assert _demote(pool, BF, BF, p, p, ps) == INVALID                  # same format
+    assert _demote(pool, BF, 9, p, p, ps) == INVALID                   # unknown format
+    assert _demote(pool, F32, I8, p, p, ps) == INVALID                 # no source pool
+    assert _demote(pool, BF, I8, None, p, ps) == INVALID               # no destination
+    assert _demote(pool, BF, I8, p, p, None) == INVALID                # quantised without scales
+    assert _demote(pool, BF, I8, ctypes.c_void_p(buf.data_ptr() + 8), p, ps) == INVALID
+    assert _demote(pool, BF, I8, p, p, ps, n=-1) == INVALID
+    assert _demote(pool, BF, I8, p, p, ps, slots=False) == INVALID     # slots missing
+    assert _demote(pool, BF, I8, p, p, ps, dst_pages=-1) == OVERFLOW
+    assert _demote(pool, BF, I8, p, p, ps, n=0) == 0                   # nothing to do
+    pool.head_dim = 96
+    assert _demote(pool, BF, I8, p, p, ps) == UNSUP
+    case8 = _case(fmt="i8")
+    pool8 = binding.kv_pool_struct(case8)
+    pool8.scales[I8] = None
+    assert _demote(pool8, I8, synth.I4, p, p, ps) == INVALID           # quantised source, no scales
+
+
+def test_append_rejects(lib):
+    case = _case()
+    pool = binding.kv_pool_struct(case)
+    t = torch.zeros(4096)
+    p = ctypes.c_void_p(t.data_ptr())
+    L = binding.lib()
+    pt = binding._p(case.page_table)
+    BF = synth.BF16
+    args = lambda **o: (ctypes.byref(o.get("pool", pool)), o.get("pt", pt), o.get("mp", case.max_pages),
+                        None, o.get("uf", BF), o.get("pos", p), o.get("b", case.batch),
+                        o.get("kn", p), p, o.get("nf", synth.F32), None, None)
+    assert L.cfr_append_kv(*args(pt=None)) == INVALID
+    assert L.cfr_append_kv(*args(pos=None)) == INVALID
+    assert L.cfr_append_kv(*args(kn=None)) == INVALID
+    assert L.cfr_append_kv(*args(b=0)) == INVALID
+    assert L.cfr_append_kv(*args(nf=synth.I8)) == INVALID
+    assert L.cfr_append_kv(*args(uf=synth.I8)) == INVALID             # new tokens go to F32/BF16
+    assert L.cfr_append_kv(*args(mp=1 << 28)) == OVERFLOW
+    case8 = _case(fmt="i8")
+    assert L.cfr_append_kv(*args(pool=binding.kv_pool_struct(case8))) == INVALID  # no hot pool

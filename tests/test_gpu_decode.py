@@ -17,7 +17,7 @@ from tests._hostkv import decode_rows
 
 pytestmark = pytest.mark.gpu
 
-F32, BF16, I8, I4 = synth.F32, synth.BF16, synth.I8, synth.I4
+F32, BF16, I8, I4, FP8 = synth.F32, synth.BF16, synth.I8, synth.I4, synth.FP8
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -36,7 +36,7 @@ def _cuda():
 HEADS = [(4, 4), (6, 3), (8, 2), (8, 1), (16, 1)]
 
 
-@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4"])
+@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4", "fp8"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("heads", HEADS, ids=lambda h: f"{h[0]}q{h[1]}kv")
 def test_parity_formats_heads(fmt, d, heads):
@@ -49,7 +49,7 @@ def test_parity_formats_heads(fmt, d, heads):
 
 
 @pytest.mark.parametrize("P", [8, 16, 32, 64, 128, 256, 512])
-@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8"])
+@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "fp8"])
 def test_parity_page_sizes(P, fmt):
     lens = (1, P - 1 if P > 1 else 1, P, P + 1, 3 * P + 5, 1000)
     case = small_case(B=6, Hq=8, Hkv=2, d=128, P=P, lens=lens, fmt=fmt,
@@ -70,6 +70,18 @@ def test_parity_tiered_pages(P, d):
     check(case, out, lse)
 
 
+@pytest.mark.parametrize("P", [16, 128, 256])
+def test_parity_tiered_with_fp8_pages(P):
+    # the whole cascade: int4, int8, FP8, bf16 pages in one sequence
+    case = small_case(B=3, Hq=8, Hkv=2, d=128, P=P, lens=(20 * P + 3, 9 * P, 2 * P + 1),
+                      fmt="tiered", tiers=[(0.2, "i4"), (0.3, "i8"), (0.2, "fp8"), (0.3, "bf16")])
+    out, lse, err = run(case)
+    assert err == 0
+    assert binding.decode_path(case) == (binding.PATH_TENSOR_CORE if P >= 128
+                                         else binding.PATH_CUDA_CORE)
+    check(case, out, lse)
+
+
 def test_parity_tiered_with_fp32_hot_pages():
     case = small_case(B=2, Hq=4, Hkv=2, d=64, P=32, lens=(700, 130), fmt="tiered",
                       tiers=[(0.3, "i4"), (0.3, "i8"), (0.2, "bf16"), (0.2, "f32")], q_fmt="f32")
@@ -78,7 +90,7 @@ def test_parity_tiered_with_fp32_hot_pages():
     check(case, out, lse)
 
 
-@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4"])
+@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4", "fp8"])
 def test_parity_alibi(fmt):
     case = small_case(B=2, Hq=8, Hkv=2, d=128, P=64, lens=(3000, 129), fmt=fmt,
                       q_fmt="f32" if fmt == "f32" else "bf16", alibi=True)
@@ -142,7 +154,7 @@ def test_parity_many_sequences_ragged():
 # edge cases and device-side error reporting (host-made faults; nothing faults)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4"])
+@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4", "fp8"])
 def test_single_token_is_v0(fmt):
     case = small_case(B=2, Hq=4, Hkv=2, d=128, P=16, lens=(1, 1), fmt=fmt,
                       q_fmt="f32" if fmt == "f32" else "bf16")
@@ -203,7 +215,7 @@ def pool_vmax(case):
     m = 0.0
     for f, t in case.v_pool.items():
         x = decode_rows(t.cpu().numpy(), f, case.head_dim)
-        if f in (I8, I4):
+        if f in synth.QUANTISED:
             x = x * case.scales[f].cpu().numpy()[:, :, None, 1:2].astype(np.float64)
         x = x[np.isfinite(x)]
         if x.size:
@@ -259,9 +271,10 @@ def test_runs_on_a_side_stream():
 # the boundary's other entry points
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4", "tiered"])
+@pytest.mark.parametrize("fmt", ["f32", "bf16", "i8", "i4", "fp8", "tiered"])
 def test_gather_is_bit_exact(fmt):
-    kw = dict(tiers=[(0.25, "i4"), (0.5, "i8"), (0.25, "bf16")]) if fmt == "tiered" else {}
+    kw = dict(tiers=[(0.25, "i4"), (0.25, "i8"), (0.25, "fp8"), (0.25, "bf16")]) \
+        if fmt == "tiered" else {}
     case = small_case(B=2, Hq=4, Hkv=2, d=128, P=16, lens=(150, 77), fmt=fmt, **kw)
     pitch = 512
     n = 150

@@ -1,0 +1,251 @@
+"""GPU parity of page demotion and KV append against the oracle, through the C ABI.
+
+Demotion codes and scales are integer / byte decisions taken in fp32 on both
+sides, so the bar is bit-exact.  Append is a byte copy (with bf16 rounding),
+also bit-exact.  A demoted or appended cache then decodes to the oracle's
+attention result within the decode tolerances.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_long_context_b200 import binding, synth
+from tests._gpu import check, run, small_case
+
+pytestmark = pytest.mark.gpu
+
+F32, BF16, I8, I4, FP8 = synth.F32, synth.BF16, synth.I8, synth.I4, synth.FP8
+FMTS = [F32, BF16, I8, I4, FP8]
+QUANTISED = synth.QUANTISED
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from paged_long_context_b200 import build
+    build.build()
+    oracle.build()
+
+
+def _src_case(fmt, d, P, lens, seed=5):
+    return small_case(B=len(lens), Hq=4, Hkv=2, d=d, P=P, lens=lens, fmt=synth.FMT_NAMES[fmt],
+                      q_fmt="bf16", seed=seed)
+
+
+def _pages_of(case):
+    """(slot, valid tokens) of every page of every sequence."""
+    out = []
+    P = case.page_tokens
+    for b in range(case.batch):
+        n = int(case.seq_lens[b])
+        for p in range(-(-n // P)):
+            out.append((int(case.page_table[b, p]), min(P, n - p * P)))
+    return out
+
+
+def _demote_both(case, src, dst, src_slots, dst_slots, valid, n_dst):
+    """Demote on the GPU and in the oracle; returns both results on the host."""
+    Hkv, d, P = case.num_kv_heads, case.head_dim, case.page_tokens
+    rb = synth.row_bytes(dst, d)
+    dk = torch.full((n_dst, Hkv, P, rb), 0xAB, dtype=torch.uint8, device="cuda")
+    dv = torch.full_like(dk, 0xAB)
+    dsc = torch.full((n_dst, Hkv, 2), -1.0, device="cuda") if dst in QUANTISED else None
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool = binding.kv_pool_struct(case)
+    st = binding.demote_pages(pool, src, dst, dk, dv, dsc,
+                              torch.tensor(src_slots, dtype=torch.int32, device="cuda"),
+                              torch.tensor(dst_slots, dtype=torch.int32, device="cuda"),
+                              torch.tensor(valid, dtype=torch.int32, device="cuda"), err)
+    assert st == 0
+    torch.cuda.synchronize()
+    hk, hv = dk.cpu(), dv.cpu()
+    hsc = None if dsc is None else dsc.cpu()
+    ok = torch.full((n_dst, Hkv, P, rb), 0xAB, dtype=torch.uint8)
+    ov = ok.clone()
+    osc = torch.full((n_dst, Hkv, 2), -1.0) if dst in QUANTISED else None
+    sc = case.scales[src].cpu().contiguous() if src in QUANTISED else None
+    oerr = oracle.demote(Hkv, d, P, src, case.k_pool[src].cpu().contiguous(),
+                         case.v_pool[src].cpu().contiguous(), sc, dst, ok, ov, osc,
+                         src_slots, dst_slots, valid)
+    return (hk, hv, hsc, int(err.item())), (ok, ov, osc, oerr)
+
+
+@pytest.mark.parametrize("src", FMTS, ids=lambda f: synth.FMT_NAMES[f])
+@pytest.mark.parametrize("dst", FMTS, ids=lambda f: synth.FMT_NAMES[f])
+@pytest.mark.parametrize("d,P", [(64, 16), (128, 256)])
+def test_demote_bit_exact(src, dst, d, P):
+    if src == dst:
+        pytest.skip("same format")
+    case = _src_case(src, d, P, lens=(5 * P + 3, P, 2 * P - 1))
+    pages = _pages_of(case)
+    n = len(pages)
+    g = torch.Generator().manual_seed(n)
+    dst_slots = torch.randperm(n + 3, generator=g)[:n].tolist()
+    (hk, hv, hsc, err), (ok, ov, osc, oerr) = _demote_both(
+        case, src, dst, [s for s, _ in pages], dst_slots, [v for _, v in pages], n + 3)
+    assert err == 0 and oerr == 0
+    assert torch.equal(hk, ok) and torch.equal(hv, ov)
+    if hsc is not None:
+        assert torch.equal(hsc, osc)
+
+
+def test_demote_reports_and_skips_bad_pages():
+    case = _src_case(BF16, 128, 16, lens=(64,))
+    pages = _pages_of(case)
+    src = [s for s, _ in pages] + [10_000, pages[0][0], pages[1][0]]
+    dst = list(range(len(pages))) + [len(pages), 99, len(pages) + 1]
+    valid = [v for _, v in pages] + [16, 16, 0]
+    (hk, hv, hsc, err), (ok, ov, osc, oerr) = _demote_both(case, BF16, I8, src, dst, valid,
+                                                           len(pages) + 2)
+    assert err == binding.DEVERR_PAGE_ID | binding.DEVERR_SEQ_LEN
+    assert oerr == oracle.DEV_PAGE_ID | oracle.DEV_SEQ_LEN
+    assert torch.equal(hk, ok) and torch.equal(hsc, osc)
+    assert int((hk[len(pages):] != 0xAB).sum()) == 0            # skipped pages untouched
+
+
+@pytest.mark.parametrize("P", [16, 256])
+def test_demoted_cache_decodes(P):
+    # a bf16 cache whose oldest pages are demoted on the GPU to int4 / int8 / FP8
+    # (the compression cascade), then decoded: parity with the oracle on the
+    # demoted cache
+    case = small_case(B=3, Hq=8, Hkv=2, d=128, P=P, lens=(12 * P + 5, 6 * P, 3 * P + 1),
+                      fmt="bf16", alibi=True, seed=21)
+    Hkv, d = case.num_kv_heads, case.head_dim
+    plan = {I4: [], I8: [], FP8: []}
+    for b in range(case.batch):
+        n = int(case.seq_lens[b])
+        np_ = -(-n // P)
+        for p in range(np_ - 1):                        # the last (hot) page stays bf16
+            tier = I4 if p < np_ // 4 else I8 if p < np_ // 2 else FP8 if p < 3 * np_ // 4 else None
+            if tier is not None:
+                plan[tier].append((b, p, min(P, n - p * P)))
+    pools_k, pools_v, scales = {BF16: case.k_pool[BF16]}, {BF16: case.v_pool[BF16]}, {}
+    page_fmt = torch.full((case.batch, case.max_pages), BF16, dtype=torch.uint8)
+    page_table = case.page_table.clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    src_pool = binding.kv_pool_struct(case)
+    for f, items in plan.items():
+        rb = synth.row_bytes(f, d)
+        k = torch.zeros((len(items), Hkv, P, rb), dtype=torch.uint8, device="cuda")
+        v = torch.zeros_like(k)
+        s = torch.zeros((len(items), Hkv, 2), device="cuda")
+        src_slots = torch.tensor([int(case.page_table[b, p]) for b, p, _ in items],
+                                 dtype=torch.int32, device="cuda")
+        valid = torch.tensor([n for _, _, n in items], dtype=torch.int32, device="cuda")
+        dst_slots = torch.arange(len(items), dtype=torch.int32, device="cuda")
+        assert binding.demote_pages(src_pool, BF16, f, k, v, s, src_slots, dst_slots, valid,
+                                    err) == 0
+        pools_k[f], pools_v[f], scales[f] = k, v, s
+        for i, (b, p, _) in enumerate(items):
+            page_table[b, p] = i
+            page_fmt[b, p] = f
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    case.k_pool, case.v_pool, case.scales = pools_k, pools_v, scales
+    case.page_table = page_table.to("cuda")
+    case.page_fmt = page_fmt.to("cuda")
+    out, lse, err2 = run(case)
+    assert err2 == 0
+    check(case, out, lse)
+
+
+@pytest.mark.parametrize("page_fmt", [F32, BF16])
+@pytest.mark.parametrize("new_fmt", [F32, BF16])
+def test_append_bit_exact_and_decodes(page_fmt, new_fmt):
+    P, d, Hkv = 16, 128, 2
+    lens = (37, 16, 5)
+    case = small_case(B=3, Hq=4, Hkv=Hkv, d=d, P=P, lens=lens, fmt=synth.FMT_NAMES[page_fmt],
+                      q_fmt="bf16", spare_pages=2, seed=8)
+    # sequence 1 fills its page exactly: give it the next page from the spare slots
+    pt = case.page_table.clone()
+    if pt.shape[1] < 3:
+        pt = torch.cat([pt, torch.full((3, 3 - pt.shape[1]), -1, dtype=torch.int32,
+                                       device=pt.device)], 1)
+    used = set(int(x) for x in pt[pt >= 0].tolist())
+    spare = [i for i in range(case.k_pool[page_fmt].shape[0]) if i not in used]
+    pt[1, 1] = spare[0]
+    case.page_table, case.max_pages = pt, pt.shape[1]
+    g = torch.Generator().manual_seed(4)
+    kn = torch.randn((3, Hkv, d), generator=g)
+    vn = torch.randn((3, Hkv, d), generator=g)
+    if new_fmt == BF16:
+        kn, vn = kn.to(torch.bfloat16), vn.to(torch.bfloat16)
+    positions = torch.tensor(lens, dtype=torch.int32)
+    host_k = {page_fmt: case.k_pool[page_fmt].cpu().contiguous()}
+    host_v = {page_fmt: case.v_pool[page_fmt].cpu().contiguous()}
+    oerr = oracle.append(Hkv, d, P, host_k, host_v, pt.cpu(), None, page_fmt, positions, new_fmt,
+                         kn, vn)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool = binding.kv_pool_struct(case)
+    st = binding.append_kv(pool, case.page_table, None, page_fmt, positions.cuda(), kn.cuda(),
+                           vn.cuda(), err)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and oerr == 0
+    assert torch.equal(case.k_pool[page_fmt].cpu(), host_k[page_fmt])
+    assert torch.equal(case.v_pool[page_fmt].cpu(), host_v[page_fmt])
+    # the extended sequences decode like the oracle says
+    case.seq_lens = (positions + 1).cuda()
+    out, lse, err2 = run(case)
+    assert err2 == 0
+    check(case, out, lse)
+
+
+def test_append_faults_reported():
+    case = small_case(B=2, Hq=4, Hkv=2, d=64, P=16, lens=(20, 20), fmt="tiered",
+                      tiers=[(0.5, "i8"), (0.5, "bf16")])
+    kn = torch.zeros((2, 2, 64), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pool = binding.kv_pool_struct(case)
+    before = case.k_pool[BF16].clone()
+    # sequence 0 appends into its int8 page 0 (not a hot page); sequence 1 past the table
+    pos = torch.tensor([3, 16 * case.max_pages], dtype=torch.int32, device="cuda")
+    assert binding.append_kv(pool, case.page_table, case.page_fmt, BF16, pos, kn, kn, err) == 0
+    torch.cuda.synchronize()
+    assert int(err.item()) == binding.DEVERR_PAGE_FMT | binding.DEVERR_SEQ_LEN
+    assert torch.equal(case.k_pool[BF16], before)
+
+
+# ---------------------------------------------------------------------------
+# full size, in the launch configuration the benchmark times
+# ---------------------------------------------------------------------------
+
+def test_demote_full_size_workload():
+    from paged_long_context_b200 import demote_workload
+    w = demote_workload.build("cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    demote_workload.run(w, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    src = w.src
+    Hkv, d, P = src.num_kv_heads, src.head_dim, src.page_tokens
+    for f, job in w.jobs.items():
+        # every (page, kv head) block of random values is non-zero: its largest
+        # code has magnitude Q (127, 7, or 448 = E4M3 0x7E)
+        k = job.dst_k[: job.n]
+        if f == I8:
+            mag = k.view(torch.int8).to(torch.int32).abs()
+            assert int(mag.amax(dim=(2, 3)).min()) == 127
+        elif f == I4:
+            lo = (k & 0xF).to(torch.int32)
+            hi = (k >> 4).to(torch.int32)
+            mag = torch.maximum(torch.where(lo >= 8, 16 - lo, lo), torch.where(hi >= 8, 16 - hi, hi))
+            assert int(mag.amax(dim=(2, 3)).min()) == 7
+        elif f == FP8:
+            assert int((k & 0x7F).amax(dim=(2, 3)).min()) == 0x7E
+        # sampled pages bit-exact against the oracle
+        idx = list(range(0, job.n, max(1, job.n // 6)))[:6]
+        s_slots = [int(job.src_slots[i]) for i in idx]
+        dk = torch.full((len(idx), Hkv, P, synth.row_bytes(f, d)), 0xAB, dtype=torch.uint8)
+        dv = dk.clone()
+        dsc = torch.zeros((len(idx), Hkv, 2))
+        src_k = src.k_pool[BF16][s_slots].cpu().contiguous()
+        src_v = src.v_pool[BF16][s_slots].cpu().contiguous()
+        assert oracle.demote(Hkv, d, P, BF16, src_k, src_v, None, f, dk, dv, dsc,
+                             list(range(len(idx))), list(range(len(idx)))) == 0
+        d_slots = [int(job.dst_slots[i]) for i in idx]
+        assert torch.equal(job.dst_k[d_slots].cpu(), dk)
+        assert torch.equal(job.dst_v[d_slots].cpu(), dv)
+        assert torch.equal(job.dst_scales[d_slots].cpu(), dsc)
