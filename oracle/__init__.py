@@ -17,6 +17,10 @@ Parity status of each oracle function (what pins it is listed in the tests):
                   nibble order), the E4M3 table of the format definition and
                   the library's float8 conversion, reconstruction-error bounds,
                   scaling invariances, the all-zero block.
+  attend(sink, window)  pinned: full window equals full attention, a window of
+                  one token returns its V row, without ALiBi equals attention
+                  over a sequence holding only the chosen tokens, decimal brute
+                  force with ALiBi.
   append          pinned: byte layout (a token appended to an empty page is
                   what a decode over one token returns), the library's bf16
                   rounding, fault cases.
@@ -64,6 +68,7 @@ class _Problem(ctypes.Structure):
         ("page_table", ctypes.c_void_p), ("page_fmt", ctypes.c_void_p),
         ("seq_lens", ctypes.c_void_p), ("head_map", ctypes.c_void_p),
         ("alibi_slopes", ctypes.c_void_p), ("softmax_scale", ctypes.c_double),
+        ("sink_tokens", ctypes.c_int32), ("window_tokens", ctypes.c_int32),
     ]
 
 
@@ -132,10 +137,13 @@ def default_threads() -> int:
 
 def attend(case, sel: Optional[Sequence[tuple]] = None, mode: int = 0, arg: int = 0,
            skip_invalid: bool = False, nthreads: Optional[int] = None,
-           mem_limit: int = 16 << 30, allow_empty: bool = False, host_pools=None):
+           mem_limit: int = 16 << 30, allow_empty: bool = False, host_pools=None,
+           sink_tokens: int = 0, window_tokens: int = 0):
     """Oracle output for a ``synth.DecodeCase``.
 
     sel: list of (b, h) pairs (default: every pair, b-major).
+    window_tokens > 0 restricts every softmax to the first ``sink_tokens`` and the
+    last ``window_tokens`` tokens of its sequence.
     mode 0 direct definition, 1 fold with block ``arg`` tokens, 2 ``arg`` splits + merge.
     Returns (out float64 [n_sel][d], lse float64 [n_sel]).  ``host_pools`` may
     pass pre-copied host tensors (dict with keys k_pool, v_pool, scales) so a
@@ -178,6 +186,7 @@ def attend(case, sel: Optional[Sequence[tuple]] = None, mode: int = 0, arg: int 
     al = h(case.alibi_slopes)
     pr.alibi_slopes = al.data_ptr() if al is not None else None
     pr.softmax_scale = float(case.softmax_scale)
+    pr.sink_tokens, pr.window_tokens = int(sink_tokens), int(window_tokens)
 
     if sel is None:
         n_sel = case.batch * case.num_q_heads

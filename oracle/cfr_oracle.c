@@ -36,6 +36,12 @@
  *   - kv head g = head_map[h], or h / (Hq / Hkv) when head_map is NULL
  *     (CFR-Atlas page, "MHA/MQA/GQA head mapping").
  *
+ * Token subsets: with window_tokens > 0 the softmax runs over the tokens
+ * j < sink_tokens and j >= n - window_tokens only (the attention sinks kept by
+ * the ARGUS page, "sink_tokens: keep initial attention sinks", and the recent
+ * window of the CFR-Atlas page's KeepRecent policy; exactness holds on the
+ * chosen set); ALiBi distances stay n - 1 - j.
+ *
  * Modes: 0 evaluates the definition directly.  1 folds blocks of `arg` tokens
  * one at a time into a running (max, normaliser, accumulator) -- the folded
  * online-softmax pass of the CFR-Atlas page ("exact folded online-softmax
@@ -77,6 +83,7 @@ typedef struct {
   const int32_t *head_map;             /* [Hq] or NULL */
   const float *alibi_slopes;           /* [Hq] or NULL */
   double softmax_scale;                /* 0 => 1/sqrt(d) */
+  int32_t sink_tokens, window_tokens;  /* window_tokens > 0: attend to [0, sink) and [n-window, n) only */
 } orc_problem;
 
 /* ---- decoding of one stored element ------------------------------------ */
@@ -340,6 +347,7 @@ static int orc_check(const orc_problem *pr) {
     return ORC_BAD_ARG;
   if (!pr->head_map && pr->num_q_heads % pr->num_kv_heads) return ORC_BAD_ARG;
   if (pr->head_dim % 2) return ORC_BAD_ARG;
+  if (pr->sink_tokens < 0 || pr->window_tokens < 0) return ORC_BAD_ARG;
   return ORC_OK;
 }
 
@@ -361,6 +369,11 @@ static int orc_run(const orc_problem *pr, const int32_t *sel_h, int64_t k0, int6
   unsigned char *keep = (unsigned char *)malloc((size_t)n);
   int rc = (!K || !V || !keep) ? ORC_NO_MEMORY
                                : orc_materialise(pr, b, g, n, skip_invalid, K, V, keep);
+  if (!rc && pr->window_tokens > 0) {
+    /* only the sink tokens and the recent window take part */
+    for (int j = 0; j < n; ++j)
+      if (!(j < pr->sink_tokens || j >= n - pr->window_tokens)) keep[j] = 0;
+  }
   int err = ORC_OK;
   if (!rc) {
 #pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(dynamic, 1)
