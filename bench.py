@@ -50,6 +50,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="cfr", choices=sorted(synth.WORKLOADS) + ["demote"])
+    ap.add_argument("--sink", type=int, default=0,
+                    help="with --window: attend to the first SINK tokens of each sequence too")
+    ap.add_argument("--window", type=int, default=0,
+                    help="attend only to the last WINDOW tokens (and the sinks); 0 = every token")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the CPU baseline")
@@ -209,16 +213,28 @@ def config_of(case, name, world, l2note):
             "l2": l2note, "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
-def cpu_baseline(case, budget_s: float, host=None):
+def _pair_bytes(case, b: int, sink: int, window: int) -> int:
+    """K/V bytes one (sequence b, query head) pair's softmax reads (its subset's tokens)."""
+    n_b = int(case.seq_lens[b])
+    P = case.page_tokens
+    kv = 0
+    for p in range(-(-n_b // P)):
+        f = case.fmt_of_page(b, p)
+        kv += accounting._tokens_in_page(n_b, p, P, sink, window) * \
+            accounting.kv_token_bytes(f, case.head_dim)
+    return kv
+
+
+def cpu_baseline(case, budget_s: float, host=None, sink: int = 0, window: int = 0):
     """Time the fp64 oracle (as it stands) on the host cores over a bounded sample."""
     import oracle
     oracle.build()
     hc = host if host is not None else case.to("cpu")
     pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads)]
-    lens = [int(x) for x in case.seq_lens.cpu().tolist()]
+    sub = dict(sink_tokens=sink, window_tokens=window)
     # calibrate on one pair, then take as many pairs as fit the budget
     t0 = time.perf_counter()
-    oracle.attend(hc, sel=[pairs[0]], nthreads=1)
+    oracle.attend(hc, sel=[pairs[0]], nthreads=1, **sub)
     t1 = time.perf_counter() - t0
     threads = oracle.default_threads()
     n = max(1, min(len(pairs), int(budget_s * threads / max(t1, 1e-6))))
@@ -227,19 +243,12 @@ def cpu_baseline(case, budget_s: float, host=None):
     sel = pairs[::step][:n]
     reps, t0 = 0, time.perf_counter()
     while True:                      # repeat a small sample until the timing is stable
-        oracle.attend(hc, sel=sel, nthreads=threads)
+        oracle.attend(hc, sel=sel, nthreads=threads, **sub)
         reps += 1
         if time.perf_counter() - t0 >= min(2.0, budget_s) or reps >= 1000:
             break
     dt = (time.perf_counter() - t0) / reps
-    bytes_per_pair = {}
-    for b, n_b in enumerate(lens):
-        kv = 0
-        for p in range(-(-n_b // case.page_tokens)):
-            f = case.fmt_of_page(b, p)
-            kv += min(case.page_tokens, n_b - p * case.page_tokens) * accounting.kv_token_bytes(f, case.head_dim)
-        bytes_per_pair[b] = kv
-    sample_bytes = sum(bytes_per_pair[b] for b, _ in sel)
+    sample_bytes = sum(_pair_bytes(case, b, sink, window) for b, _ in sel)
     return {"value": sample_bytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"{len(sel)} of {len(pairs)} (sequence, query head) pairs, "
                       f"{sample_bytes} K/V bytes, {dt:.3f} s per pass, {reps} passes",
@@ -253,12 +262,13 @@ def cpu_baseline(case, budget_s: float, host=None):
 def run_ours(args, dist):
     dev = torch.device("cuda", dist.local)
     case = synth.workload(args.workload, device=dev)
-    acct = accounting.step_bytes(case)
+    sw = (args.sink, args.window) if args.window > 0 else None
+    acct = accounting.step_bytes(case, args.sink, args.window)
     kv_bytes = acct["kv"] + acct["scales"]
     bufs = binding.DecodeBuffers(case)
     path = binding.decode_path(case)
     stream = torch.cuda.current_stream(dev)
-    st = binding.paged_decode_raw(case, bufs, stream)
+    st = binding.paged_decode_raw(case, bufs, stream, sink_window=sw)
     if st != 0:
         raise binding.CfrError(st, "cfr_paged_decode")
     torch.cuda.synchronize()
@@ -273,14 +283,14 @@ def run_ours(args, dist):
         l2note = f"inputs larger than L2 ({acct['total'] / 2**20:.0f} MiB > 126 MiB)"
 
     def full_step():
-        binding.paged_decode_raw(case, bufs, stream)
+        binding.paged_decode_raw(case, bufs, stream, sink_window=sw)
 
     def phased_step(evs):
-        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_SCHEDULE)
+        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_SCHEDULE, sink_window=sw)
         evs[0].record(stream)
-        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_DECODE)
+        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_DECODE, sink_window=sw)
         evs[1].record(stream)
-        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_MERGE)
+        binding.paged_decode_raw(case, bufs, stream, phases=binding.PHASE_MERGE, sink_window=sw)
 
     for _ in range(args.warmup):
         if flush is not None:
@@ -335,7 +345,7 @@ def run_ours(args, dist):
         case.page_table.copy_(pt_h, non_blocking=True)
         if pf_h is not None:
             case.page_fmt.copy_(pf_h, non_blocking=True)
-        binding.paged_decode_raw(case, bufs, stream)
+        binding.paged_decode_raw(case, bufs, stream, sink_window=sw)
         out_h.copy_(bufs.out, non_blocking=True)
         lse_h.copy_(bufs.lse, non_blocking=True)
 
@@ -371,7 +381,8 @@ def run_ours(args, dist):
         "hbm_frac_of_measured": round(kv_bytes / (step_ms_max * 1e-3) / 1e9 / peak, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": dtype_name(case), "data": "synthetic (seeded N(0,1) K/V/q, page-shaped workload)",
-        "config": config_of(case, args.workload, world, l2note),
+        "config": dict(config_of(case, args.workload, world, l2note),
+                       **({"sink_tokens": args.sink, "window_tokens": args.window} if sw else {})),
         "kernel_path": {1: "cuda-core", 2: "tcgen05", 3: "cuda-core-f32-tma"}.get(path, "?"),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -395,29 +406,27 @@ def run_reference(args, dist):
     oracle.build()
     case = synth.workload(args.workload, device="cpu")
     pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads)]
-    lens = [int(x) for x in case.seq_lens.tolist()]
+    sub = dict(sink_tokens=args.sink, window_tokens=args.window)
     threads = oracle.default_threads()
     t0 = time.perf_counter()
-    oracle.attend(case, sel=[pairs[0]], nthreads=1)
+    oracle.attend(case, sel=[pairs[0]], nthreads=1, **sub)
     t1 = time.perf_counter() - t0
     budget = 150.0 / max(1, args.steps + args.warmup)
     n = max(1, min(len(pairs), int(budget * threads / max(t1, 1e-6))))
     sel = pairs[::max(1, len(pairs) // n)][:n]
-    sample_bytes = 0
-    for b, _ in sel:
-        for p in range(-(-lens[b] // case.page_tokens)):
-            f = case.fmt_of_page(b, p)
-            sample_bytes += min(case.page_tokens, lens[b] - p * case.page_tokens) * \
-                accounting.kv_token_bytes(f, case.head_dim)
+    sample_bytes = sum(_pair_bytes(case, b, args.sink, args.window) for b, _ in sel)
     for _ in range(args.warmup):
-        oracle.attend(case, sel=sel, nthreads=threads)
+        oracle.attend(case, sel=sel, nthreads=threads, **sub)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.attend(case, sel=sel, nthreads=threads)
+        oracle.attend(case, sel=sel, nthreads=threads, **sub)
     dt = (time.perf_counter() - t0) / args.steps
     value = sample_bytes / dt / 1e9
     sample = (f"{len(sel)} of {len(pairs)} (sequence, query head) pairs per step, "
               f"{sample_bytes} K/V bytes")
+    cfg = config_of(case, args.workload, 1, "host memory")
+    if args.window > 0:
+        cfg.update(sink_tokens=args.sink, window_tokens=args.window)
     return {
         "impl": "reference",
         "metric": "decode-attn µs/step and KV-read GB/s as % of B200 HBM peak (1 GPU)",
@@ -425,7 +434,7 @@ def run_reference(args, dist):
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) K/V/q, page-shaped workload)",
-        "config": config_of(case, args.workload, 1, "host memory"),
+        "config": cfg,
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -609,8 +618,9 @@ def main():
         else:
             case, res = run_ours(args, dist)
             if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = {k: v for k, v in cpu_baseline(case, args.cpu_budget).items()
-                                       if k != "seconds"}
+                res["cpu_baseline"] = {k: v for k, v in cpu_baseline(
+                    case, args.cpu_budget, sink=args.sink, window=args.window).items()
+                    if k != "seconds"}
         if dist.rank == 0:
             print(json.dumps(res), flush=True)
     finally:

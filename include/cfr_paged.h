@@ -174,6 +174,36 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
                                    uint32_t *err_word, void *stream, uint32_t phases);
 
 /*
+ * cfr_paged_decode restricted to a sink + recent-window token subset: each
+ * softmax runs over the first sink_tokens tokens (attention sinks; ARGUS page,
+ * "sink_tokens: keep initial attention sinks") and the last window_tokens
+ * tokens (the recent window of the CFR-Atlas page's KeepRecent policy) of its
+ * sequence, and over nothing else:
+ *
+ *   S_b = { j : j < sink_tokens or j >= n_b - window_tokens },
+ *   out[b][h] = sum_{j in S_b} softmax_j(...) V_j,  ALiBi distance n_b - 1 - j as usual.
+ *
+ * The result is exact on the chosen set (no approximation of the skipped
+ * tokens); pages holding no token of S_b are never read.  Same arguments,
+ * workspace and errors as cfr_paged_decode, plus sink_tokens >= 0 and
+ * window_tokens >= 1 (CFR_ERR_INVALID_ARG otherwise).  With
+ * sink_tokens + window_tokens >= n_b the sequence is attended in full.
+ * `phases` selects launches as for cfr_paged_decode_phases (CFR_PHASE_ALL for
+ * one whole step); a call without CFR_PHASE_SCHEDULE needs the schedule of an
+ * earlier call with the same seq_lens, sizes, sink_tokens and window_tokens.
+ */
+cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                        const int32_t *page_table, int32_t max_pages,
+                                        const int32_t *seq_lens, int32_t batch,
+                                        const uint8_t *page_fmt, int32_t uniform_fmt,
+                                        int32_t num_q_heads, const int32_t *head_map,
+                                        const float *alibi_slopes, float softmax_scale,
+                                        float *out, float *lse, void *workspace,
+                                        size_t workspace_bytes, uint32_t *err_word, void *stream,
+                                        int32_t sink_tokens, int32_t window_tokens,
+                                        uint32_t phases);
+
+/*
  * Bytes of the scratch array compiled into the library for
  * cfr_paged_decode_static_workspace (one array per GPU that loads the library).
  */

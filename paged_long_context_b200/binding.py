@@ -27,7 +27,8 @@ PATH_CUDA_CORE, PATH_TENSOR_CORE, PATH_F32_TMA = 1, 2, 3
 EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_decode_phases",
            "cfr_merge_partials",
            "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str",
-           "cfr_paged_decode_static_workspace", "cfr_demote_pages", "cfr_append_kv"]
+           "cfr_paged_decode_static_workspace", "cfr_demote_pages", "cfr_append_kv",
+           "cfr_paged_decode_sink_window"]
 FMT_COUNT = 5
 STATIC_WORKSPACE_BYTES = 8 << 20
 
@@ -80,6 +81,9 @@ def lib():
         L.cfr_paged_decode_static_workspace.argtypes = [_VP, _I32, ctypes.POINTER(KvPool), _VP, _I32,
                                                         _VP, _I32, _VP, _I32, _I32, _VP, _VP, _F32,
                                                         _VP, _VP, _VP, _VP]
+        L.cfr_paged_decode_sink_window.restype = ctypes.c_int
+        L.cfr_paged_decode_sink_window.argtypes = L.cfr_paged_decode.argtypes + [_I32, _I32,
+                                                                                  ctypes.c_uint32]
         L.cfr_demote_pages.restype = ctypes.c_int
         L.cfr_demote_pages.argtypes = [ctypes.POINTER(KvPool), _I32, _I32, _VP, _VP, _VP, _I64,
                                        _VP, _VP, _VP, _I32, _VP, _VP]
@@ -172,9 +176,10 @@ PHASE_SCHEDULE, PHASE_DECODE, PHASE_MERGE, PHASE_ALL = 0x1, 0x2, 0x4, 0x7
 
 
 def paged_decode_raw(case, bufs: DecodeBuffers, stream=None, workspace_bytes=None,
-                     phases: Optional[int] = None) -> int:
-    """Call cfr_paged_decode (or cfr_paged_decode_phases when ``phases`` is given) on a
-    case whose tensors live on the GPU; returns the status."""
+                     phases: Optional[int] = None, sink_window: Optional[tuple] = None) -> int:
+    """Call cfr_paged_decode (cfr_paged_decode_phases when ``phases`` is given,
+    cfr_paged_decode_sink_window when ``sink_window`` = (sink_tokens, window_tokens)
+    is given) on a case whose tensors live on the GPU; returns the status."""
     pool = kv_pool_struct(case)
     hm, hmp = _head_map_host(case)
     nbytes = bufs.workspace.numel() if workspace_bytes is None else workspace_bytes
@@ -182,15 +187,21 @@ def paged_decode_raw(case, bufs: DecodeBuffers, stream=None, workspace_bytes=Non
             _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads,
             hmp, _p(case.alibi_slopes), float(case.softmax_scale), _p(bufs.out), _p(bufs.lse),
             _p(bufs.workspace), nbytes, _p(bufs.err), _stream(stream))
+    if sink_window is not None:
+        return int(lib().cfr_paged_decode_sink_window(*args, int(sink_window[0]),
+                                                      int(sink_window[1]),
+                                                      PHASE_ALL if phases is None else phases))
     if phases is None:
         return int(lib().cfr_paged_decode(*args))
     return int(lib().cfr_paged_decode_phases(*args, phases))
 
 
-def paged_decode(case, bufs: Optional[DecodeBuffers] = None, stream=None) -> DecodeBuffers:
-    """Decode attention for every (sequence, query head); raises on a rejected call."""
+def paged_decode(case, bufs: Optional[DecodeBuffers] = None, stream=None,
+                 sink_window: Optional[tuple] = None) -> DecodeBuffers:
+    """Decode attention for every (sequence, query head), over all tokens or a
+    (sink_tokens, window_tokens) subset; raises on a rejected call."""
     bufs = bufs or DecodeBuffers(case)
-    st = paged_decode_raw(case, bufs, stream)
+    st = paged_decode_raw(case, bufs, stream, sink_window=sink_window)
     if st != CFR_OK:
         raise CfrError(st, "cfr_paged_decode")
     return bufs

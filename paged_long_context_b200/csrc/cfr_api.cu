@@ -8,8 +8,8 @@
 namespace cfr {
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
-                     int32_t *split_off, int32_t *splits, int max_splits, int32_t *num_splits,
-                     uint32_t *err, cudaStream_t stream);
+                     int sink, int window, int32_t *split_off, int32_t *splits, int max_splits,
+                     int32_t *num_splits, uint32_t *err, cudaStream_t stream);
 void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
                   const int32_t *split_off, int batch, int Hq, int D, float *out, float *lse,
                   cudaStream_t stream);
@@ -86,7 +86,8 @@ struct WsLayout {
 };
 
 bool ws_layout(int batch, int hq, int d, int max_pages, int target, WsLayout *w) {
-  long long ms = static_cast<long long>(target) + batch;
+  // ceil(len / chunk) summed over at most two page ranges per sequence
+  long long ms = static_cast<long long>(target) + 2LL * batch;
   const long long cap = static_cast<long long>(batch) * max_pages;
   if (cap < ms) ms = cap;
   if (ms < 1) ms = 1;
@@ -258,14 +259,20 @@ cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
                                  CFR_PHASE_ALL);
 }
 
-cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
-                                   const int32_t *page_table, int32_t max_pages,
-                                   const int32_t *seq_lens, int32_t batch,
-                                   const uint8_t *page_fmt, int32_t uniform_fmt,
-                                   int32_t num_q_heads, const int32_t *head_map,
-                                   const float *alibi_slopes, float softmax_scale, float *out,
-                                   float *lse, void *workspace, size_t workspace_bytes,
-                                   uint32_t *err_word, void *stream, uint32_t phases) {
+}  // extern "C"
+
+namespace cfr {
+namespace {
+
+// Every decode entry point: checks, schedule, decode and merge launches.
+// window > 0 restricts each softmax to the first `sink` and last `window` tokens.
+cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                       const int32_t *page_table, int32_t max_pages, const int32_t *seq_lens,
+                       int32_t batch, const uint8_t *page_fmt, int32_t uniform_fmt,
+                       int32_t num_q_heads, const int32_t *head_map, const float *alibi_slopes,
+                       float softmax_scale, float *out, float *lse, void *workspace,
+                       size_t workspace_bytes, uint32_t *err_word, void *stream, uint32_t phases,
+                       int32_t sink, int32_t window) {
   if (phases == 0 || (phases & ~CFR_PHASE_ALL)) return CFR_ERR_INVALID_ARG;
   cfr_status st = common_checks(q_fmt, kv, max_pages, page_fmt, uniform_fmt);
   if (st != CFR_OK) return st;
@@ -309,6 +316,8 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
   p.Hq = num_q_heads;
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(kv->head_dim));
   p.sigma_log2e = sigma * kLog2e;
+  p.sink = sink;
+  p.window = window;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool use_tc = tc_supported(p, page_fmt != nullptr);
@@ -319,8 +328,8 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
     if (p.stages < 2) return CFR_ERR_UNSUPPORTED;
   }
   if (phases & CFR_PHASE_SCHEDULE) {
-    launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, split_off, splits,
-                    w.max_splits, num_splits, err_word, s);
+    launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, split_off,
+                    splits, w.max_splits, num_splits, err_word, s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_DECODE) {
@@ -335,6 +344,40 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   return CFR_OK;
+}
+
+}  // namespace
+}  // namespace cfr
+
+extern "C" {
+
+cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                   const int32_t *page_table, int32_t max_pages,
+                                   const int32_t *seq_lens, int32_t batch,
+                                   const uint8_t *page_fmt, int32_t uniform_fmt,
+                                   int32_t num_q_heads, const int32_t *head_map,
+                                   const float *alibi_slopes, float softmax_scale, float *out,
+                                   float *lse, void *workspace, size_t workspace_bytes,
+                                   uint32_t *err_word, void *stream, uint32_t phases) {
+  return decode_impl(q, q_fmt, kv, page_table, max_pages, seq_lens, batch, page_fmt, uniform_fmt,
+                     num_q_heads, head_map, alibi_slopes, softmax_scale, out, lse, workspace,
+                     workspace_bytes, err_word, stream, phases, 0, 0);
+}
+
+cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                        const int32_t *page_table, int32_t max_pages,
+                                        const int32_t *seq_lens, int32_t batch,
+                                        const uint8_t *page_fmt, int32_t uniform_fmt,
+                                        int32_t num_q_heads, const int32_t *head_map,
+                                        const float *alibi_slopes, float softmax_scale,
+                                        float *out, float *lse, void *workspace,
+                                        size_t workspace_bytes, uint32_t *err_word, void *stream,
+                                        int32_t sink_tokens, int32_t window_tokens,
+                                        uint32_t phases) {
+  if (sink_tokens < 0 || window_tokens < 1) return CFR_ERR_INVALID_ARG;
+  return decode_impl(q, q_fmt, kv, page_table, max_pages, seq_lens, batch, page_fmt, uniform_fmt,
+                     num_q_heads, head_map, alibi_slopes, softmax_scale, out, lse, workspace,
+                     workspace_bytes, err_word, stream, phases, sink_tokens, window_tokens);
 }
 
 cfr_status cfr_merge_partials(const float *part_acc, const float *part_m, const float *part_l,
@@ -358,7 +401,7 @@ cfr_status cfr_schedule_splits(const int32_t *seq_lens, int32_t batch, int32_t p
   if (batch <= 0 || page_tokens <= 0 || max_pages <= 0 || target_splits <= 0 || max_splits <= 0)
     return CFR_ERR_INVALID_ARG;
   if (static_cast<long long>(max_pages) * page_tokens > INT_MAX) return CFR_ERR_OVERFLOW;
-  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, split_off, splits,
+  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, 0, 0, split_off, splits,
                   max_splits, num_splits, err_word, static_cast<cudaStream_t>(stream));
   return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
 }

@@ -45,6 +45,7 @@ struct DecodeParams {
   int stages;
   float sigma_log2e;    // softmax scale times log2(e)
   int gmax;             // largest group size
+  int sink, window;     // window > 0: only tokens j < sink or j >= n - window take part
   int16_t grp_off[kMaxQHeads + 1];  // heads of kv head g: grp_heads[grp_off[g] .. grp_off[g+1])
   int16_t grp_heads[kMaxQHeads];
 };
@@ -224,6 +225,26 @@ __device__ __forceinline__ void mask_set_range(uint32_t (&m)[4], int lo, int hi)
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int r) {
   const uint32_t w = r < 32 ? m[0] : r < 64 ? m[1] : r < 96 ? m[2] : m[3];
   return (w >> (r & 31)) & 1u;
+}
+
+// Token j of a sequence of n tokens takes part in the softmax: every token, or
+// with a window only the first `sink` tokens (attention sinks) and the last
+// `window` tokens (the recent window).
+__device__ __forceinline__ bool in_token_set(const DecodeParams &p, int n, int j) {
+  return p.window <= 0 || j < p.sink || j >= n - p.window;
+}
+
+// Clears the rows of a tile (tokens t0 .. t0 + rows - 1) that fall between the
+// sink tokens and the recent window.
+__device__ __forceinline__ void mask_clear_gap(uint32_t (&m)[4], const DecodeParams &p, int n,
+                                               int t0, int rows) {
+  if (p.window <= 0) return;
+  const int lo = max(p.sink - t0, 0), hi = min(n - p.window - t0, rows);
+  if (lo >= hi) return;
+  uint32_t gap[4] = {0u, 0u, 0u, 0u};
+  mask_set_range(gap, lo, hi);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) m[w] &= ~gap[w];
 }
 
 // Page ids and formats of a run of pages of one sequence, staged in shared

@@ -23,8 +23,9 @@
 //  - At the end of an item the eight warps' accumulators are summed in a fixed
 //    order and (m, l, acc) is written as the split's partial for the merge.
 //
-// Tokens past the sequence length and rows of skipped pages get p = 0 and are
-// never read, so stale or NaN shared-memory bytes cannot reach an FMA.
+// Tokens past the sequence length, tokens outside a sink + recent-window subset
+// and rows of skipped pages get p = 0 and are never read, so stale or NaN
+// shared-memory bytes cannot reach an FMA.
 #include "cfr_common.cuh"
 
 namespace cfr {
@@ -365,7 +366,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
         float ks = 1.f;
         if (r < rows) {
           const CcFrag f = m.frag[m.row_frag[r]];
-          if (f.ok) {
+          if (f.ok && in_token_set(p, n, m.t0 + r)) {
             valid = true;
             ks = f.ks;
             float x[EPT];
@@ -443,7 +444,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
         const int r = warp * (CC_T / CC_WARPS) + rr;
         if (r >= rows) break;
         const CcFrag f = m.frag[m.row_frag[r]];
-        if (!f.ok) continue;
+        if (!f.ok || !in_token_set(p, n, m.t0 + r)) continue;
         float v[DPL];
         load_elems<DPL>(f.fmt, vst + r * p.pitch, lane * DPL, v);
 #pragma unroll

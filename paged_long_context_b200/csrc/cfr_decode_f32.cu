@@ -87,8 +87,8 @@ __host__ __device__ constexpr size_t f32_smem_bytes() {
 template <int D>
 __device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F32Maps &maps,
                                                  uint64_t *full, uint64_t *empty, F32Meta *meta,
-                                                 uint8_t *ring, const PageCache &pc, int g, int t0,
-                                                 int tok_end, int box_rows, int stage,
+                                                 uint8_t *ring, const PageCache &pc, int g, int n,
+                                                 int t0, int tok_end, int box_rows, int stage,
                                                  uint32_t phase, bool *timed_out, int lane) {
   using C = F32Cfg<D>;
   const int P = p.P;
@@ -118,6 +118,7 @@ __device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F3
     uint32_t valid[4] = {0u, 0u, 0u, 0u};
     for (int f = 0; f < npiece; ++f)
       if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
+    mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
     for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
     m.rows = rows;
     m.t0 = t0;
@@ -158,11 +159,12 @@ __device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_
     int slot, g;
     item_coords(item, p.num_splits[0], slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
-    const int tok_end = min(p.seq_lens[b], pe * P);
+    const int n = p.seq_lens[b];
+    const int tok_end = min(n, pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += C::T) {
       page_cache_ensure(pc, p, b, t0 / P, (min(t0 + C::T, tok_end) - 1) / P, pe, lane);
-      if (!f32_produce_tile<D>(p, maps, full, empty, meta, ring, pc, g, t0, tok_end, box_rows, stage,
-                               phase, timed_out, lane))
+      if (!f32_produce_tile<D>(p, maps, full, empty, meta, ring, pc, g, n, t0, tok_end, box_rows,
+                               stage, phase, timed_out, lane))
         return;
       if (++stage == F_STAGES) {
         stage = 0;

@@ -271,7 +271,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 // pages is issued in parallel; lane 0 publishes the tile description and the
 // expected byte count.
 template <int NCOL, bool INTP>
-__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int g, int t0,
+__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int g, int n, int t0,
                                                 int tok_end, int stage, uint32_t phase,
                                                 bool *timed_out, int lane) {
   const DecodeParams &p = c.p;
@@ -316,6 +316,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
     uint32_t valid[4] = {0u, 0u, 0u, 0u};
     for (int f = 0; f < npiece; ++f)
       if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
+    mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
     float ks = 1.f, vs = 1.f;
     uint32_t bytes;
     if (kind == KIND_BF16) {
@@ -382,10 +383,11 @@ __device__ void tc_producer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
-    const int tok_end = min(p.seq_lens[b], pe * P);
+    const int n = p.seq_lens[b];
+    const int tok_end = min(n, pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       page_cache_ensure(c.S.pc, p, b, t0 / P, (min(t0 + TC_T, tok_end) - 1) / P, pe, lane);
-      if (!tc_produce_tile(c, b, g, t0, tok_end, stage, phase, timed_out, lane)) return;
+      if (!tc_produce_tile(c, b, g, n, t0, tok_end, stage, phase, timed_out, lane)) return;
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;

@@ -11,10 +11,12 @@
 //   BF16   x rounded to nearest even; F32: x.
 // An all-zero block gets scale 0 and zero codes; rows past `valid` are
 // written as zero bytes.  One CTA per block: pass 1 reduces max|x| over the
-// valid rows, pass 2 re-reads the block (from L2: a block is at most a few
-// hundred KiB and is re-read right away) and writes the codes with coalesced
-// vector stores.  The kernel is bound by HBM: it reads the source block once
-// from DRAM and writes the destination block once.
+// valid rows with every load of a thread in flight at once, pass 2 encodes and
+// writes the codes with coalesced vector stores.  A block of up to 4096
+// vectors of 8 elements (bf16 / int / FP8 sources; 2048 for fp32, e.g. 256
+// tokens x 128 dims) stays in registers between the passes; a larger one is
+// read again in pass 2, from L2.  The kernel is bound by HBM: it reads the
+// source block once from DRAM and writes the destination block once.
 //
 // Append writes the new K and V rows of one decode step into the hot tier:
 // token j = positions[b] of sequence b goes to row j % P of logical page j / P
@@ -45,35 +47,74 @@ struct DemoteParams {
   int src_fmt, dst_fmt, Hkv, D, P;
 };
 
-// eight consecutive stored elements starting at element e of a block, as fp32
-__device__ __forceinline__ void load8(int fmt, const uint8_t *blk, long long e, float scale,
-                                      float (&x)[kVec]) {
-  if (fmt == CFR_FMT_F32) {
-    const float4 *p = reinterpret_cast<const float4 *>(blk + 4 * e);
-    const float4 a = p[0], b = p[1];
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  } else if (fmt == CFR_FMT_BF16) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(blk + 2 * e);
-    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+// Raw stored bytes of kVec consecutive elements of a source format, loaded with
+// one or two vector accesses and decoded later (so that every load of a thread
+// is in flight before the first one is used).
+template <int SRC>
+struct RawVec {
+  uint2 w;  // CFR_FMT_I8 and CFR_FMT_FP8: 8 one-byte codes
+};
+template <>
+struct RawVec<CFR_FMT_F32> {
+  uint4 a, b;
+};
+template <>
+struct RawVec<CFR_FMT_BF16> {
+  uint4 a;
+};
+template <>
+struct RawVec<CFR_FMT_I4> {
+  uint32_t w;
+};
+
+template <int SRC>
+__device__ __forceinline__ RawVec<SRC> load_raw(const uint8_t *blk, long long v) {
+  RawVec<SRC> r;
+  if constexpr (SRC == CFR_FMT_F32) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(blk + 32 * v);
+    r.a = p[0];
+    r.b = p[1];
+  } else if constexpr (SRC == CFR_FMT_BF16) {
+    r.a = *reinterpret_cast<const uint4 *>(blk + 16 * v);
+  } else if constexpr (SRC == CFR_FMT_I4) {
+    r.w = *reinterpret_cast<const uint32_t *>(blk + 4 * v);
+  } else {
+    r.w = *reinterpret_cast<const uint2 *>(blk + 8 * v);
+  }
+  return r;
+}
+
+// the eight values of a raw vector as fp32 (quantised: code * scale, fp32 product)
+template <int SRC>
+__device__ __forceinline__ void decode_raw(const RawVec<SRC> &r, float scale, float (&x)[kVec]) {
+  if constexpr (SRC == CFR_FMT_F32) {
+    const uint32_t a[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = __uint_as_float(a[k]);
+  } else if constexpr (SRC == CFR_FMT_BF16) {
+    const uint32_t a[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       x[2 * k] = bf16_lo(a[k]);
       x[2 * k + 1] = bf16_hi(a[k]);
     }
-  } else if (fmt == CFR_FMT_I8) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(blk + e);
+  } else if constexpr (SRC == CFR_FMT_I8) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(i8_at(k < 4 ? w.x : w.y, k & 3), scale);
-  } else if (fmt == CFR_FMT_FP8) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(blk + e);
+    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(i8_at(k < 4 ? r.w.x : r.w.y, k & 3), scale);
+  } else if constexpr (SRC == CFR_FMT_FP8) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(e4m3_at(k < 4 ? w.x : w.y, k & 3), scale);
+    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(e4m3_at(k < 4 ? r.w.x : r.w.y, k & 3), scale);
   } else {  // CFR_FMT_I4
-    const uint32_t w = *reinterpret_cast<const uint32_t *>(blk + e / 2);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(i4_at(w, k), scale);
+    for (int k = 0; k < 8; ++k) x[k] = __fmul_rn(i4_at(r.w, k), scale);
   }
+}
+
+// vectors a thread holds in registers: a block of up to kDemoteThreads * R
+// vectors is read from DRAM once and encoded from registers
+template <int SRC>
+constexpr int resident_vectors() {
+  return SRC == CFR_FMT_F32 ? 4 : 8;
 }
 
 __device__ __forceinline__ int int_code(float x, float scale, int q) {
@@ -141,8 +182,11 @@ __device__ __forceinline__ float qmax_of(int fmt) {
 }
 
 // block (page k, kv head g, K or V) = blockIdx.x
+template <int SRC>
 __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) {
-  __shared__ float red[kDemoteThreads / 32];
+  constexpr int R = resident_vectors<SRC>();
+  constexpr int T = kDemoteThreads;
+  __shared__ float red[T / 32];
   const long long blk_id = blockIdx.x;
   const int kv = static_cast<int>(blk_id & 1);
   const int g = static_cast<int>((blk_id >> 1) % p.Hkv);
@@ -157,41 +201,84 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
     if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_SEQ_LEN);
     return;
   }
-  const long long blk_elems = static_cast<long long>(p.P) * p.D;
-  const uint8_t *src = (kv ? p.src_v : p.src_k) + (s * p.Hkv + g) * p.P * row_bytes(p.src_fmt, p.D);
+  const uint8_t *src = (kv ? p.src_v : p.src_k) + (s * p.Hkv + g) * p.P * row_bytes(SRC, p.D);
   uint8_t *dst = (kv ? p.dst_v : p.dst_k) + (t * p.Hkv + g) * p.P * row_bytes(p.dst_fmt, p.D);
-  const float src_scale = is_quantised(p.src_fmt) ? p.src_scales[(s * p.Hkv + g) * 2 + kv] : 1.f;
+  const float src_scale = is_quantised(SRC) ? p.src_scales[(s * p.Hkv + g) * 2 + kv] : 1.f;
   const long long nvec_valid = static_cast<long long>(valid) * p.D / kVec;
-  const long long nvec = blk_elems / kVec;
+  const long long nvec = static_cast<long long>(p.P) * p.D / kVec;
+  const int tid = threadIdx.x;
+  // the whole valid part of the block fits the registers of the CTA
+  const bool resident = nvec_valid <= static_cast<long long>(R) * T;
+  RawVec<SRC> buf[R];
 
   float scale = 1.f;
   if (is_quantised(p.dst_fmt)) {
+    // pass 1: max |x| over the valid rows, R independent loads in flight per thread
     float amax = 0.f;
-    for (long long v = threadIdx.x; v < nvec_valid; v += kDemoteThreads) {
-      float x[kVec];
-      load8(p.src_fmt, src, v * kVec, src_scale, x);
+    for (long long c0 = 0; c0 < nvec_valid; c0 += static_cast<long long>(R) * T) {
 #pragma unroll
-      for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(x[i]));
+      for (int r = 0; r < R; ++r) {
+        const long long v = c0 + static_cast<long long>(r) * T + tid;
+        if (v < nvec_valid) buf[r] = load_raw<SRC>(src, v);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const long long v = c0 + static_cast<long long>(r) * T + tid;
+        if (v < nvec_valid) {
+          float x[kVec];
+          decode_raw<SRC>(buf[r], src_scale, x);
+#pragma unroll
+          for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(x[i]));
+        }
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
     __syncthreads();
     amax = red[0];
 #pragma unroll
-    for (int w = 1; w < kDemoteThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+    for (int w = 1; w < T / 32; ++w) amax = fmaxf(amax, red[w]);
     scale = __fdiv_rn(amax, qmax_of(p.dst_fmt));
-    if (threadIdx.x == 0) p.dst_scales[(t * p.Hkv + g) * 2 + kv] = scale;
-  }
-  for (long long v = threadIdx.x; v < nvec; v += kDemoteThreads) {
-    if (v < nvec_valid) {
-      float x[kVec];
-      load8(p.src_fmt, src, v * kVec, src_scale, x);
-      store8(p.dst_fmt, dst, v * kVec, scale, x);
-    } else {
-      store_zero8(p.dst_fmt, dst, v * kVec);
+    if (tid == 0) p.dst_scales[(t * p.Hkv + g) * 2 + kv] = scale;
+  } else if (resident) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const long long v = static_cast<long long>(r) * T + tid;
+      if (v < nvec_valid) buf[r] = load_raw<SRC>(src, v);
     }
   }
+  // pass 2: encode and store (from registers when resident, else chunk by chunk
+  // again, the re-read hitting L2)
+  if (resident) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const long long v = static_cast<long long>(r) * T + tid;
+      if (v < nvec_valid) {
+        float x[kVec];
+        decode_raw<SRC>(buf[r], src_scale, x);
+        store8(p.dst_fmt, dst, v * kVec, scale, x);
+      }
+    }
+  } else {
+    for (long long c0 = 0; c0 < nvec_valid; c0 += static_cast<long long>(R) * T) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const long long v = c0 + static_cast<long long>(r) * T + tid;
+        if (v < nvec_valid) buf[r] = load_raw<SRC>(src, v);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const long long v = c0 + static_cast<long long>(r) * T + tid;
+        if (v < nvec_valid) {
+          float x[kVec];
+          decode_raw<SRC>(buf[r], src_scale, x);
+          store8(p.dst_fmt, dst, v * kVec, scale, x);
+        }
+      }
+    }
+  }
+  for (long long v = nvec_valid + tid; v < nvec; v += T) store_zero8(p.dst_fmt, dst, v * kVec);
 }
 
 struct AppendParams {
@@ -314,7 +401,14 @@ cfr_status cfr_demote_pages(const cfr_kv_pool *kv, int32_t src_fmt, int32_t dst_
   p.D = kv->head_dim;
   p.P = kv->page_tokens;
   const unsigned blocks = static_cast<unsigned>(num_pages) * kv->num_kv_heads * 2u;
-  demote_kernel<<<blocks, kDemoteThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (src_fmt) {
+    case CFR_FMT_F32: demote_kernel<CFR_FMT_F32><<<blocks, kDemoteThreads, 0, s>>>(p); break;
+    case CFR_FMT_BF16: demote_kernel<CFR_FMT_BF16><<<blocks, kDemoteThreads, 0, s>>>(p); break;
+    case CFR_FMT_I8: demote_kernel<CFR_FMT_I8><<<blocks, kDemoteThreads, 0, s>>>(p); break;
+    case CFR_FMT_I4: demote_kernel<CFR_FMT_I4><<<blocks, kDemoteThreads, 0, s>>>(p); break;
+    default: demote_kernel<CFR_FMT_FP8><<<blocks, kDemoteThreads, 0, s>>>(p); break;
+  }
   return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
 }
 

@@ -4,7 +4,10 @@
 // pages, chunk = ceil(total pages / target_splits), so that splits carry about
 // equal numbers of tokens whatever the length mix (the split-K decoding of the
 // CMF page, "split-K flash-decoding so throughput holds at depth", sized here by
-// the sequence lengths).  Writes split_off[B+1], the (b, first page, end page)
+// the sequence lengths).  With a sink + recent window subset (window > 0) only
+// the pages holding tokens of the subset are scheduled: the pages of the first
+// `sink` tokens and those of the last `window` tokens, two page ranges when a
+// gap separates them.  Writes split_off[B+1], the (b, first page, end page)
 // triple of every split, and (total splits, chunk).  Deterministic.
 #include "cfr_common.cuh"
 
@@ -65,18 +68,39 @@ __device__ __forceinline__ int valid_pages(int n, int P, int max_pages) {
   return (n + P - 1) / P;
 }
 
+// Page ranges [0, *a_end) and [*b_begin, np) of a sequence of n tokens and np
+// pages that hold the tokens taking part (the second range is empty when the
+// first covers everything).
+__device__ __forceinline__ void page_ranges(int n, int np, int P, int sink, int window, int *a_end,
+                                            int *b_begin) {
+  *a_end = np;
+  *b_begin = np;
+  if (window <= 0 || np <= 0 || static_cast<long long>(sink) + window >= n) return;
+  const int ps = (sink + P - 1) / P;       // pages of the sink tokens
+  const int pw = (n - window) / P;         // first page of the window
+  if (pw <= ps) return;
+  *a_end = ps;
+  *b_begin = pw;
+}
+
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
-    const int32_t *__restrict__ seq_lens, int batch, int P, int max_pages, int target,
-    int32_t *__restrict__ split_off, int32_t *__restrict__ splits, int max_splits,
+    const int32_t *__restrict__ seq_lens, int batch, int P, int max_pages, int target, int sink,
+    int window, int32_t *__restrict__ split_off, int32_t *__restrict__ splits, int max_splits,
     int32_t *__restrict__ num_splits, uint32_t *err) {
   griddep_launch_dependents();
   __shared__ long long red_ll[33];
   __shared__ int red_i[33];
   long long local = 0;
   for (int b = threadIdx.x; b < batch; b += blockDim.x) {
-    const int np = valid_pages(seq_lens[b], P, max_pages);
-    if (np < 0) set_err(err, CFR_DEVERR_SEQ_LEN);
-    else local += np;
+    const int n = seq_lens[b];
+    const int np = valid_pages(n, P, max_pages);
+    if (np < 0) {
+      set_err(err, CFR_DEVERR_SEQ_LEN);
+    } else {
+      int a_end, b_begin;
+      page_ranges(n, np, P, sink, window, &a_end, &b_begin);
+      local += a_end + (np - b_begin);
+    }
   }
   const long long total = block_sum_ll(local, red_ll);
   const long long tgt = target > 0 ? target : 1;
@@ -87,9 +111,13 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
   bool overflow = false;
   for (int base = 0; base < batch; base += blockDim.x) {
     const int b = base + threadIdx.x;
-    int np = b < batch ? valid_pages(seq_lens[b], P, max_pages) : -1;
+    const int n = b < batch ? seq_lens[b] : 0;
+    int np = b < batch ? valid_pages(n, P, max_pages) : -1;
     if (np < 0) np = 0;
-    const int cnt = (np + chunk - 1) / chunk;
+    int a_end, b_begin;
+    page_ranges(n, np, P, sink, window, &a_end, &b_begin);
+    const int cnt_a = (a_end + chunk - 1) / chunk;
+    const int cnt = cnt_a + (np - b_begin + chunk - 1) / chunk;
     int tot = 0;
     const int excl = block_exclusive_scan(cnt, red_i, &tot) + running;
     if (b < batch) {
@@ -100,8 +128,10 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
           overflow = true;
           break;
         }
-        const int pb = s * chunk;
-        const int pe = pb + chunk < np ? pb + chunk : np;
+        // splits of the first range, then of the second
+        const int r0 = s < cnt_a ? 0 : b_begin, r1 = s < cnt_a ? a_end : np;
+        const int pb = r0 + (s < cnt_a ? s : s - cnt_a) * chunk;
+        const int pe = pb + chunk < r1 ? pb + chunk : r1;
         splits[3 * idx + 0] = b;
         splits[3 * idx + 1] = pb;
         splits[3 * idx + 2] = pe;
@@ -119,10 +149,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
 }
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
-                     int32_t *split_off, int32_t *splits, int max_splits, int32_t *num_splits,
-                     uint32_t *err, cudaStream_t stream) {
-  schedule_kernel<<<1, kSchedThreads, 0, stream>>>(seq_lens, batch, P, max_pages, target,
-                                                   split_off, splits, max_splits, num_splits, err);
+                     int sink, int window, int32_t *split_off, int32_t *splits, int max_splits,
+                     int32_t *num_splits, uint32_t *err, cudaStream_t stream) {
+  schedule_kernel<<<1, kSchedThreads, 0, stream>>>(seq_lens, batch, P, max_pages, target, sink,
+                                                   window, split_off, splits, max_splits,
+                                                   num_splits, err);
 }
 
 }  // namespace cfr

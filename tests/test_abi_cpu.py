@@ -260,3 +260,19 @@ def test_append_rejects(lib):
     assert L.cfr_append_kv(*args(mp=1 << 28)) == OVERFLOW
     case8 = _case(fmt="i8")
     assert L.cfr_append_kv(*args(pool=binding.kv_pool_struct(case8))) == INVALID  # no hot pool
+
+
+def test_sink_window_rejects(lib):
+    case = _case()
+    bufs = FakeBufs(case)
+    pool = binding.kv_pool_struct(case)
+    args = (binding._p(case.q), case.q_fmt, ctypes.byref(pool), binding._p(case.page_table),
+            case.max_pages, binding._p(case.seq_lens), case.batch, binding._p(case.page_fmt),
+            case.uniform_fmt, case.num_q_heads, None, None, 0.0, binding._p(bufs.out),
+            binding._p(bufs.lse), binding._p(bufs.workspace), bufs.workspace.numel(),
+            binding._p(bufs.err), None)
+    L = binding.lib()
+    assert L.cfr_paged_decode_sink_window(*args, -1, 16, binding.PHASE_ALL) == INVALID
+    assert L.cfr_paged_decode_sink_window(*args, 4, 0, binding.PHASE_ALL) == INVALID
+    assert L.cfr_paged_decode_sink_window(*args, 4, 16, 0) == INVALID
+    assert L.cfr_paged_decode_sink_window(*args, 4, 16, 0x10) == INVALID
