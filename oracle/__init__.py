@@ -17,6 +17,9 @@ Parity status of each oracle function (what pins it is listed in the tests):
                   nibble order), the E4M3 table of the format definition and
                   the library's float8 conversion, reconstruction-error bounds,
                   scaling invariances, the all-zero block.
+  attend(num_queries > 1)  pinned: one query row equals the single-query
+                  definition over its prefix, torch SDPA in fp64 with the causal
+                  mask of the last Q positions, decimal brute force.
   attend(sink, window)  pinned: full window equals full attention, a window of
                   one token returns its V row, without ALiBi equals attention
                   over a sequence holding only the chosen tokens, decimal brute
@@ -69,6 +72,7 @@ class _Problem(ctypes.Structure):
         ("seq_lens", ctypes.c_void_p), ("head_map", ctypes.c_void_p),
         ("alibi_slopes", ctypes.c_void_p), ("softmax_scale", ctypes.c_double),
         ("sink_tokens", ctypes.c_int32), ("window_tokens", ctypes.c_int32),
+        ("num_queries", ctypes.c_int32),
     ]
 
 
@@ -141,7 +145,9 @@ def attend(case, sel: Optional[Sequence[tuple]] = None, mode: int = 0, arg: int 
            sink_tokens: int = 0, window_tokens: int = 0):
     """Oracle output for a ``synth.DecodeCase``.
 
-    sel: list of (b, h) pairs (default: every pair, b-major).
+    sel: list of (b, h) pairs (default: every pair, b-major).  With Q =
+    case.num_queries > 1, h is a query row qi * Hq + head: query qi of the last Q
+    positions, attending causally.
     window_tokens > 0 restricts every softmax to the first ``sink_tokens`` and the
     last ``window_tokens`` tokens of its sequence.
     mode 0 direct definition, 1 fold with block ``arg`` tokens, 2 ``arg`` splits + merge.
@@ -187,9 +193,10 @@ def attend(case, sel: Optional[Sequence[tuple]] = None, mode: int = 0, arg: int 
     pr.alibi_slopes = al.data_ptr() if al is not None else None
     pr.softmax_scale = float(case.softmax_scale)
     pr.sink_tokens, pr.window_tokens = int(sink_tokens), int(window_tokens)
+    pr.num_queries = int(getattr(case, "num_queries", 1))
 
     if sel is None:
-        n_sel = case.batch * case.num_q_heads
+        n_sel = case.batch * case.num_q_heads * int(getattr(case, "num_queries", 1))
         sb = sh = None
     else:
         n_sel = len(sel)

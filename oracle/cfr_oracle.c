@@ -42,6 +42,15 @@
  * window of the CFR-Atlas page's KeepRecent policy; exactness holds on the
  * chosen set); ALiBi distances stay n - 1 - j.
  *
+ * Several queries per sequence (num_queries = Q > 1): the queries are the
+ * last Q tokens of the sequence, at positions n - Q + i (i = 0..Q-1), with q
+ * laid out [B][Q][Hq][d]; query i attends causally to the tokens j <= n - Q + i
+ * (the causal mask of the RustAttention page, "Mathematical Framework
+ * Covered", applied to the query rows of a speculative or chunked-prefill
+ * step over the paged cache), with ALiBi distance n - Q + i - j.  Query i of
+ * sequence b is therefore the single-query definition over the first
+ * n - Q + i + 1 tokens.  Outputs are [B][Q][Hq][d] and [B][Q][Hq].
+ *
  * Modes: 0 evaluates the definition directly.  1 folds blocks of `arg` tokens
  * one at a time into a running (max, normaliser, accumulator) -- the folded
  * online-softmax pass of the CFR-Atlas page ("exact folded online-softmax
@@ -84,6 +93,7 @@ typedef struct {
   const float *alibi_slopes;           /* [Hq] or NULL */
   double softmax_scale;                /* 0 => 1/sqrt(d) */
   int32_t sink_tokens, window_tokens;  /* window_tokens > 0: attend to [0, sink) and [n-window, n) only */
+  int32_t num_queries;                 /* Q >= 1 query tokens per sequence (0 is read as 1) */
 } orc_problem;
 
 /* ---- decoding of one stored element ------------------------------------ */
@@ -153,8 +163,11 @@ static double orc_element(int fmt, const unsigned char *row, int i, double scale
   return NAN;
 }
 
-static double orc_query(const orc_problem *pr, int b, int h, int i) {
-  long idx = ((long)b * pr->num_q_heads + h) * pr->head_dim + i;
+static int orc_nq(const orc_problem *pr) { return pr->num_queries > 1 ? pr->num_queries : 1; }
+
+/* element i of query row (b, query qi, head h) */
+static double orc_query(const orc_problem *pr, int b, int qi, int h, int i) {
+  long idx = (((long)b * orc_nq(pr) + qi) * pr->num_q_heads + h) * pr->head_dim + i;
   const unsigned char *base = (const unsigned char *)pr->q;
   if (pr->q_fmt == ORC_F32) return orc_from_f32(base + 4L * idx);
   return orc_from_bf16(base + 2L * idx);
@@ -271,10 +284,22 @@ static void orc_combine(int d, double *m, double *l, double *a, double m2, doubl
   *m = mn;
 }
 
-/* one (b, h): out[d] and lse; K/V/keep already materialised for kv head of h */
-static int orc_one(const orc_problem *pr, int b, int h, int n, const double *K, const double *V,
-                   const unsigned char *keep, int mode, long arg, double *out, double *lse) {
+/*
+ * one (b, query row vh): out[d] and lse.  vh = qi * Hq + h selects query qi of
+ * head h; that query sees the first n - Q + qi + 1 of the n materialised tokens
+ * (all n with one query).  K/V/keep are materialised for the kv head of h.
+ */
+static int orc_one(const orc_problem *pr, int b, int vh, int n_all, const double *K,
+                   const double *V, const unsigned char *keep, int mode, long arg, double *out,
+                   double *lse) {
   const int d = pr->head_dim, P = pr->page_tokens;
+  const int h = vh % pr->num_q_heads, qi = vh / pr->num_q_heads;
+  const int n = n_all - orc_nq(pr) + qi + 1;
+  if (n <= 0) {
+    for (int i = 0; i < d; ++i) out[i] = 0.0;
+    *lse = -INFINITY;
+    return ORC_EMPTY;
+  }
   double *qv = (double *)malloc(sizeof(double) * d);
   double *a = (double *)malloc(sizeof(double) * d);
   double *a2 = (double *)malloc(sizeof(double) * d);
@@ -282,7 +307,7 @@ static int orc_one(const orc_problem *pr, int b, int h, int n, const double *K, 
     free(qv); free(a); free(a2);
     return ORC_NO_MEMORY;
   }
-  for (int i = 0; i < d; ++i) qv[i] = orc_query(pr, b, h, i);
+  for (int i = 0; i < d; ++i) qv[i] = orc_query(pr, b, qi, h, i);
   double m = -INFINITY, l = 0.0;
   for (int i = 0; i < d; ++i) a[i] = 0.0;
   if (mode == 0) {
@@ -348,6 +373,7 @@ static int orc_check(const orc_problem *pr) {
   if (!pr->head_map && pr->num_q_heads % pr->num_kv_heads) return ORC_BAD_ARG;
   if (pr->head_dim % 2) return ORC_BAD_ARG;
   if (pr->sink_tokens < 0 || pr->window_tokens < 0) return ORC_BAD_ARG;
+  if (pr->num_queries < 0 || (orc_nq(pr) > 1 && pr->window_tokens > 0)) return ORC_BAD_ARG;
   return ORC_OK;
 }
 
@@ -378,11 +404,12 @@ static int orc_run(const orc_problem *pr, const int32_t *sel_h, int64_t k0, int6
   if (!rc) {
 #pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(dynamic, 1)
     for (int64_t kk = k0; kk < k1; ++kk) {
-      const int h = sel_h ? sel_h[kk] : (int)(kk % pr->num_q_heads);
-      int r = orc_one(pr, b, h, n, K, V, keep, mode, arg, out + kk * d, lse + kk);
+      const int64_t rows = (int64_t)orc_nq(pr) * pr->num_q_heads;
+      const int vh = sel_h ? sel_h[kk] : (int)(kk % rows);
+      int r = orc_one(pr, b, vh, n, K, V, keep, mode, arg, out + kk * d, lse + kk);
       if (r) {
 #pragma omp critical
-        err = r;
+        err = (err == ORC_OK || err == ORC_EMPTY) ? r : err;
       }
     }
   }
@@ -392,7 +419,8 @@ static int orc_run(const orc_problem *pr, const int32_t *sel_h, int64_t k0, int6
 
 /*
  * Attention output for the selected (sel_b[k], sel_h[k]) pairs, k < n_sel, in
- * that order (all pairs b-major when sel_b is NULL: n_sel must be B*Hq).
+ * that order (all pairs b-major when sel_b is NULL: n_sel must be B*Q*Hq).
+ * sel_h is a query row vh = qi * Hq + h (just h with one query).
  * out: [n_sel][d], lse: [n_sel] natural-log log-sum-exp of the scores.
  * Consecutive selections with the same (b, kv head) form a run that shares one
  * materialisation of K and V.  Runs execute concurrently on `nthreads` OpenMP
@@ -407,7 +435,8 @@ int cfr_oracle_attend(const orc_problem *pr, const int32_t *sel_b, const int32_t
                       int64_t mem_limit, double *out, double *lse) {
   int rc = orc_check(pr);
   if (rc) return rc;
-  if (!sel_b && n_sel != (int64_t)pr->batch * pr->num_q_heads) return ORC_BAD_ARG;
+  const int64_t rows = (int64_t)orc_nq(pr) * pr->num_q_heads;  /* query rows per sequence */
+  if (!sel_b && n_sel != (int64_t)pr->batch * rows) return ORC_BAD_ARG;
   /* split the selection into runs */
   int64_t *run_start = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n_sel + 1));
   int *run_b = (int *)malloc(sizeof(int) * (size_t)(n_sel + 1));
@@ -418,10 +447,10 @@ int cfr_oracle_attend(const orc_problem *pr, const int32_t *sel_b, const int32_t
   }
   int64_t nrun = 0, biggest = 0;
   for (int64_t k = 0; k < n_sel; ++k) {
-    const int b = sel_b ? sel_b[k] : (int)(k / pr->num_q_heads);
-    const int h = sel_h ? sel_h[k] : (int)(k % pr->num_q_heads);
-    if (b < 0 || b >= pr->batch || h < 0 || h >= pr->num_q_heads) { rc = ORC_BAD_ARG; break; }
-    const int g = orc_kv_head(pr, h);
+    const int b = sel_b ? sel_b[k] : (int)(k / rows);
+    const int vh = sel_h ? sel_h[k] : (int)(k % rows);
+    if (b < 0 || b >= pr->batch || vh < 0 || vh >= rows) { rc = ORC_BAD_ARG; break; }
+    const int g = orc_kv_head(pr, vh % pr->num_q_heads);
     if (g < 0 || g >= pr->num_kv_heads) { rc = ORC_BAD_ARG; break; }
     if (pr->seq_lens[b] > (long)pr->max_pages * pr->page_tokens) { rc = ORC_BAD_ARG; break; }
     if (nrun == 0 || run_b[nrun - 1] != b || run_g[nrun - 1] != g) {

@@ -83,7 +83,7 @@ class DecodeCase:
     max_pages: int
     seq_lens: torch.Tensor            # int32 [B]
     q_fmt: int                        # F32 or BF16
-    q: torch.Tensor                   # f32 [B][Hq][d] or uint16 bf16 bits [B][Hq][d]
+    q: torch.Tensor                   # f32 or bf16 bits [B][Q * Hq][d] = [B][Q][Hq][d]
     k_pool: Dict[int, torch.Tensor]   # fmt -> uint8 [pages][Hkv][P][row_bytes]
     v_pool: Dict[int, torch.Tensor]
     scales: Dict[int, torch.Tensor]   # I8/I4 -> f32 [pages][Hkv][2] (K scale, V scale)
@@ -95,6 +95,7 @@ class DecodeCase:
     softmax_scale: float              # 0.0 => 1/sqrt(head_dim)
     seed: int
     spec: dict
+    num_queries: int = 1              # Q query tokens per sequence (the last Q positions)
 
     @property
     def device(self) -> torch.device:
@@ -237,6 +238,7 @@ class CaseSpec:
     softmax_scale: float = 0.0
     spare_pages: int = 0                  # extra unused pool slots (NaN / fill bytes)
     use_page_fmt: Optional[bool] = None   # force passing a page_fmt array
+    num_queries: int = 1                  # query tokens per sequence (speculative / chunked)
 
 
 def tier_of_page(spec: CaseSpec, p: int, num_pages: int) -> int:
@@ -325,7 +327,8 @@ def make_case(spec: CaseSpec, seed: int, device="cpu") -> DecodeCase:
     use_pf = spec.use_page_fmt if spec.use_page_fmt is not None else mixed
 
     gq = _gen(device, _mix(seed, 0x0A11))
-    qf = torch.randn((B, Hq, d), generator=gq, device=device, dtype=torch.float32)
+    Q = max(1, int(spec.num_queries))
+    qf = torch.randn((B, Q * Hq, d), generator=gq, device=device, dtype=torch.float32)
     if spec.q_fmt == "f32":
         q, q_fmt = qf, F32
     else:
@@ -340,7 +343,7 @@ def make_case(spec: CaseSpec, seed: int, device="cpu") -> DecodeCase:
         page_table=page_table.to(device), page_fmt=page_fmt.to(device) if use_pf else None,
         uniform_fmt=uniform, head_map=None if head_map is None else head_map.to(device),
         alibi_slopes=None if slopes is None else slopes.to(device),
-        softmax_scale=float(spec.softmax_scale), seed=seed, spec=dataclasses.asdict(spec))
+        softmax_scale=float(spec.softmax_scale), seed=seed, spec=dataclasses.asdict(spec), num_queries=Q)
 
 
 def page_values(seed: int, b: int, p: int, hkv: int, P: int, d: int, device):
