@@ -54,6 +54,8 @@ def parse():
                     help="with --window: attend to the first SINK tokens of each sequence too")
     ap.add_argument("--window", type=int, default=0,
                     help="attend only to the last WINDOW tokens (and the sinks); 0 = every token")
+    ap.add_argument("--queries", type=int, default=1,
+                    help="query tokens per sequence (multi-query decode, causal over the last Q)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the CPU baseline")
@@ -230,7 +232,7 @@ def cpu_baseline(case, budget_s: float, host=None, sink: int = 0, window: int = 
     import oracle
     oracle.build()
     hc = host if host is not None else case.to("cpu")
-    pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads)]
+    pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads * case.num_queries)]
     sub = dict(sink_tokens=sink, window_tokens=window)
     # calibrate on one pair, then take as many pairs as fit the budget
     t0 = time.perf_counter()
@@ -261,7 +263,7 @@ def cpu_baseline(case, budget_s: float, host=None, sink: int = 0, window: int = 
 
 def run_ours(args, dist):
     dev = torch.device("cuda", dist.local)
-    case = synth.workload(args.workload, device=dev)
+    case = synth.workload(args.workload, device=dev, num_queries=args.queries)
     sw = (args.sink, args.window) if args.window > 0 else None
     acct = accounting.step_bytes(case, args.sink, args.window)
     kv_bytes = acct["kv"] + acct["scales"]
@@ -382,7 +384,8 @@ def run_ours(args, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": dtype_name(case), "data": "synthetic (seeded N(0,1) K/V/q, page-shaped workload)",
         "config": dict(config_of(case, args.workload, world, l2note),
-                       **({"sink_tokens": args.sink, "window_tokens": args.window} if sw else {})),
+                       **({"sink_tokens": args.sink, "window_tokens": args.window} if sw else {}),
+                       **({"queries_per_sequence": args.queries} if args.queries > 1 else {})),
         "kernel_path": {1: "cuda-core", 2: "tcgen05", 3: "cuda-core-f32-tma"}.get(path, "?"),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -404,8 +407,8 @@ def run_reference(args, dist):
     """The fp64 CPU oracle, as it stands, timed on the host cores (rank 0 only)."""
     import oracle
     oracle.build()
-    case = synth.workload(args.workload, device="cpu")
-    pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads)]
+    case = synth.workload(args.workload, device="cpu", num_queries=args.queries)
+    pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads * case.num_queries)]
     sub = dict(sink_tokens=args.sink, window_tokens=args.window)
     threads = oracle.default_threads()
     t0 = time.perf_counter()
@@ -427,6 +430,8 @@ def run_reference(args, dist):
     cfg = config_of(case, args.workload, 1, "host memory")
     if args.window > 0:
         cfg.update(sink_tokens=args.sink, window_tokens=args.window)
+    if args.queries > 1:
+        cfg.update(queries_per_sequence=args.queries)
     return {
         "impl": "reference",
         "metric": "decode-attn µs/step and KV-read GB/s as % of B200 HBM peak (1 GPU)",

@@ -204,6 +204,37 @@ cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_
                                         uint32_t phases);
 
 /*
+ * Multi-query decode over the paged cache: every sequence carries Q =
+ * num_queries query tokens, its last Q positions (a speculative-decoding
+ * verification step or a chunk of prefill over the cached prefix).  Query qi
+ * (0 <= qi < Q) of sequence b sits at position n_b - Q + qi and attends
+ * causally to the tokens j <= n_b - Q + qi (the causal mask of the
+ * scaled dot-product definition, RustAttention page, "Mathematical Framework
+ * Covered"); its ALiBi distance is n_b - Q + qi - j.  K/V of every query token
+ * are already in the cache (as for cfr_paged_decode, whose num_queries = 1
+ * case this is).
+ *
+ *  q    device [batch][num_queries][num_q_heads][head_dim] (fp32 or bf16 by q_fmt).
+ *  out  device float [batch][num_queries][num_q_heads][head_dim];
+ *  lse  device float [batch][num_queries][num_q_heads] or NULL.
+ *  workspace  >= cfr_paged_decode_workspace_size(batch, num_q_heads * num_queries, ...).
+ * Every K/V page is read once for all Q queries of the kv head's group: the
+ * query rows (qi, h) of one kv head form its group, at most 16 rows
+ * (num_queries * query heads per kv head <= 16, CFR_ERR_UNSUPPORTED otherwise;
+ * num_queries in [1, 16], CFR_ERR_INVALID_ARG below 1).  A sequence with
+ * n_b < num_queries gets out = 0 and lse = -inf for every row and sets
+ * CFR_DEVERR_SEQ_LEN.  `phases` as for cfr_paged_decode_phases.
+ */
+cfr_status cfr_paged_decode_multi(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                  const int32_t *page_table, int32_t max_pages,
+                                  const int32_t *seq_lens, int32_t batch, const uint8_t *page_fmt,
+                                  int32_t uniform_fmt, int32_t num_q_heads, int32_t num_queries,
+                                  const int32_t *head_map, const float *alibi_slopes,
+                                  float softmax_scale, float *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, uint32_t *err_word, void *stream,
+                                  uint32_t phases);
+
+/*
  * Bytes of the scratch array compiled into the library for
  * cfr_paged_decode_static_workspace (one array per GPU that loads the library).
  */

@@ -51,8 +51,9 @@ def step_bytes(case, sink: int = 0, window: int = 0) -> dict:
             if f in synth.QUANTISED:
                 scales += Hkv * 8
     table = pages * (4 + (1 if case.page_fmt is not None else 0))
-    qb = case.batch * case.num_q_heads * d * (4 if case.q_fmt == synth.F32 else 2)
-    ob = case.batch * case.num_q_heads * (d + 1) * 4
+    rows = case.batch * case.num_q_heads * getattr(case, "num_queries", 1)   # query rows
+    qb = rows * d * (4 if case.q_fmt == synth.F32 else 2)
+    ob = rows * (d + 1) * 4
     total = kv + scales + table + qb + ob
     return {"kv": kv, "scales": scales, "page_table": table, "q": qb, "out": ob, "total": total,
             "tokens": tokens}

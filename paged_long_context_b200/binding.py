@@ -28,7 +28,7 @@ EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_dec
            "cfr_merge_partials",
            "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str",
            "cfr_paged_decode_static_workspace", "cfr_demote_pages", "cfr_append_kv",
-           "cfr_paged_decode_sink_window"]
+           "cfr_paged_decode_sink_window", "cfr_paged_decode_multi"]
 FMT_COUNT = 5
 STATIC_WORKSPACE_BYTES = 8 << 20
 
@@ -84,6 +84,10 @@ def lib():
         L.cfr_paged_decode_sink_window.restype = ctypes.c_int
         L.cfr_paged_decode_sink_window.argtypes = L.cfr_paged_decode.argtypes + [_I32, _I32,
                                                                                   ctypes.c_uint32]
+        L.cfr_paged_decode_multi.restype = ctypes.c_int
+        L.cfr_paged_decode_multi.argtypes = [_VP, _I32, ctypes.POINTER(KvPool), _VP, _I32, _VP, _I32,
+                                             _VP, _I32, _I32, _I32, _VP, _VP, _F32, _VP, _VP, _VP,
+                                             _SZ, _VP, _VP, ctypes.c_uint32]
         L.cfr_demote_pages.restype = ctypes.c_int
         L.cfr_demote_pages.argtypes = [ctypes.POINTER(KvPool), _I32, _I32, _VP, _VP, _VP, _I64,
                                        _VP, _VP, _VP, _I32, _VP, _VP]
@@ -160,11 +164,11 @@ class DecodeBuffers:
 
     def __init__(self, case, device=None, with_lse=True):
         dev = device or case.device
-        self.out = torch.empty((case.batch, case.num_q_heads, case.head_dim), dtype=torch.float32,
-                               device=dev)
-        self.lse = torch.empty((case.batch, case.num_q_heads), dtype=torch.float32,
+        rows = case.num_q_heads * getattr(case, "num_queries", 1)   # [Q][Hq] query rows
+        self.out = torch.empty((case.batch, rows, case.head_dim), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((case.batch, rows), dtype=torch.float32,
                                device=dev) if with_lse else None
-        n = workspace_size(case.batch, case.num_q_heads, case.num_kv_heads, case.head_dim,
+        n = workspace_size(case.batch, rows, case.num_kv_heads, case.head_dim,
                            case.max_pages, case.page_tokens)
         if n == 0:
             raise CfrError(1, "cfr_paged_decode_workspace_size")
@@ -179,7 +183,8 @@ def paged_decode_raw(case, bufs: DecodeBuffers, stream=None, workspace_bytes=Non
                      phases: Optional[int] = None, sink_window: Optional[tuple] = None) -> int:
     """Call cfr_paged_decode (cfr_paged_decode_phases when ``phases`` is given,
     cfr_paged_decode_sink_window when ``sink_window`` = (sink_tokens, window_tokens)
-    is given) on a case whose tensors live on the GPU; returns the status."""
+    is given, cfr_paged_decode_multi when the case has several queries per
+    sequence) on a case whose tensors live on the GPU; returns the status."""
     pool = kv_pool_struct(case)
     hm, hmp = _head_map_host(case)
     nbytes = bufs.workspace.numel() if workspace_bytes is None else workspace_bytes
@@ -187,6 +192,15 @@ def paged_decode_raw(case, bufs: DecodeBuffers, stream=None, workspace_bytes=Non
             _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads,
             hmp, _p(case.alibi_slopes), float(case.softmax_scale), _p(bufs.out), _p(bufs.lse),
             _p(bufs.workspace), nbytes, _p(bufs.err), _stream(stream))
+    if getattr(case, "num_queries", 1) > 1:
+        if sink_window is not None:
+            raise ValueError("sink/window subsets take one query per sequence")
+        return int(lib().cfr_paged_decode_multi(
+            _p(case.q), case.q_fmt, ctypes.byref(pool), _p(case.page_table), case.max_pages,
+            _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads,
+            case.num_queries, hmp, _p(case.alibi_slopes), float(case.softmax_scale), _p(bufs.out),
+            _p(bufs.lse), _p(bufs.workspace), nbytes, _p(bufs.err), _stream(stream),
+            PHASE_ALL if phases is None else phases))
     if sink_window is not None:
         return int(lib().cfr_paged_decode_sink_window(*args, int(sink_window[0]),
                                                       int(sink_window[1]),

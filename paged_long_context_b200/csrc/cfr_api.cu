@@ -8,8 +8,8 @@
 namespace cfr {
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
-                     int sink, int window, int32_t *split_off, int32_t *splits, int max_splits,
-                     int32_t *num_splits, uint32_t *err, cudaStream_t stream);
+                     int sink, int window, int nq, int32_t *split_off, int32_t *splits,
+                     int max_splits, int32_t *num_splits, uint32_t *err, cudaStream_t stream);
 void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
                   const int32_t *split_off, int batch, int Hq, int D, float *out, float *lse,
                   cudaStream_t stream);
@@ -146,16 +146,20 @@ cfr_status check_pool(const cfr_kv_pool *kv) {
   return CFR_OK;
 }
 
-// Query-head groups per kv head, from a host head map (or the contiguous rule).
-cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *p) {
-  if (hq <= 0 || hq > kMaxQHeads || hkv <= 0 || hkv > kMaxQHeads) return CFR_ERR_UNSUPPORTED;
+// Query-row groups per kv head, from a host head map (or the contiguous rule).
+// With nq queries per sequence the rows are vh = qi * hq + h (qi < nq); row vh
+// belongs to the kv head of query head h.
+cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *p, int nq = 1) {
+  if (hq <= 0 || hkv <= 0 || hkv > kMaxQHeads || nq <= 0) return CFR_ERR_UNSUPPORTED;
+  if (static_cast<long long>(hq) * nq > kMaxQHeads) return CFR_ERR_UNSUPPORTED;
   if (!head_map && hq % hkv != 0) return CFR_ERR_INVALID_ARG;
+  const int rows = hq * nq;
   int count[kMaxQHeads + 1];
   std::memset(count, 0, sizeof(count));
   for (int h = 0; h < hq; ++h) {
     const int g = head_map ? head_map[h] : h / (hq / hkv);
     if (g < 0 || g >= hkv) return CFR_ERR_INVALID_ARG;
-    ++count[g];
+    count[g] += nq;
   }
   int gmax = 0, off = 0;
   for (int g = 0; g < hkv; ++g) {
@@ -167,11 +171,14 @@ cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *
   if (gmax > kMaxGroup) return CFR_ERR_UNSUPPORTED;
   int fill[kMaxQHeads];
   for (int g = 0; g < hkv; ++g) fill[g] = p->grp_off[g];
-  for (int h = 0; h < hq; ++h) {
+  for (int vh = 0; vh < rows; ++vh) {
+    const int h = vh % hq;
     const int g = head_map ? head_map[h] : h / (hq / hkv);
-    p->grp_heads[fill[g]++] = static_cast<int16_t>(h);
+    p->grp_heads[fill[g]++] = static_cast<int16_t>(vh);
   }
   p->gmax = gmax < 1 ? 1 : gmax;
+  p->nq = nq;
+  p->hq_real = hq;
   return CFR_OK;
 }
 
@@ -272,7 +279,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
                        int32_t num_q_heads, const int32_t *head_map, const float *alibi_slopes,
                        float softmax_scale, float *out, float *lse, void *workspace,
                        size_t workspace_bytes, uint32_t *err_word, void *stream, uint32_t phases,
-                       int32_t sink, int32_t window) {
+                       int32_t sink, int32_t window, int32_t nq) {
   if (phases == 0 || (phases & ~CFR_PHASE_ALL)) return CFR_ERR_INVALID_ARG;
   cfr_status st = common_checks(q_fmt, kv, max_pages, page_fmt, uniform_fmt);
   if (st != CFR_OK) return st;
@@ -283,15 +290,16 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
 
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
-  st = build_groups(num_q_heads, kv->num_kv_heads, head_map, &p);
+  st = build_groups(num_q_heads, kv->num_kv_heads, head_map, &p, nq);
   if (st != CFR_OK) return st;
   fill_pool(kv, &p);
+  const int rows = num_q_heads * nq;  // query rows per sequence
 
   DeviceInfo di;
   if (!device_info(&di)) return CFR_ERR_CUDA;
   const int target = target_splits(di.sms, kv->num_kv_heads);
   WsLayout w;
-  if (!ws_layout(batch, num_q_heads, kv->head_dim, max_pages, target, &w)) return CFR_ERR_OVERFLOW;
+  if (!ws_layout(batch, rows, kv->head_dim, max_pages, target, &w)) return CFR_ERR_OVERFLOW;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return CFR_ERR_WORKSPACE;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -313,7 +321,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.err = err_word;
   p.batch = batch;
   p.max_pages = max_pages;
-  p.Hq = num_q_heads;
+  p.Hq = rows;
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(kv->head_dim));
   p.sigma_log2e = sigma * kLog2e;
   p.sink = sink;
@@ -328,8 +336,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
     if (p.stages < 2) return CFR_ERR_UNSUPPORTED;
   }
   if (phases & CFR_PHASE_SCHEDULE) {
-    launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, split_off,
-                    splits, w.max_splits, num_splits, err_word, s);
+    launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, nq,
+                    split_off, splits, w.max_splits, num_splits, err_word, s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_DECODE) {
@@ -339,8 +347,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
     if (e != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_MERGE) {
-    launch_merge(p.part_acc, p.part_m, p.part_l, split_off, batch, num_q_heads, kv->head_dim,
-                 out, lse, s);
+    launch_merge(p.part_acc, p.part_m, p.part_l, split_off, batch, rows, kv->head_dim, out, lse,
+                 s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   return CFR_OK;
@@ -361,7 +369,7 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
                                    uint32_t *err_word, void *stream, uint32_t phases) {
   return decode_impl(q, q_fmt, kv, page_table, max_pages, seq_lens, batch, page_fmt, uniform_fmt,
                      num_q_heads, head_map, alibi_slopes, softmax_scale, out, lse, workspace,
-                     workspace_bytes, err_word, stream, phases, 0, 0);
+                     workspace_bytes, err_word, stream, phases, 0, 0, 1);
 }
 
 cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
@@ -377,7 +385,22 @@ cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_
   if (sink_tokens < 0 || window_tokens < 1) return CFR_ERR_INVALID_ARG;
   return decode_impl(q, q_fmt, kv, page_table, max_pages, seq_lens, batch, page_fmt, uniform_fmt,
                      num_q_heads, head_map, alibi_slopes, softmax_scale, out, lse, workspace,
-                     workspace_bytes, err_word, stream, phases, sink_tokens, window_tokens);
+                     workspace_bytes, err_word, stream, phases, sink_tokens, window_tokens, 1);
+}
+
+cfr_status cfr_paged_decode_multi(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
+                                  const int32_t *page_table, int32_t max_pages,
+                                  const int32_t *seq_lens, int32_t batch, const uint8_t *page_fmt,
+                                  int32_t uniform_fmt, int32_t num_q_heads, int32_t num_queries,
+                                  const int32_t *head_map, const float *alibi_slopes,
+                                  float softmax_scale, float *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, uint32_t *err_word, void *stream,
+                                  uint32_t phases) {
+  if (num_queries < 1 || num_queries > 16) return num_queries < 1 ? CFR_ERR_INVALID_ARG
+                                                                 : CFR_ERR_UNSUPPORTED;
+  return decode_impl(q, q_fmt, kv, page_table, max_pages, seq_lens, batch, page_fmt, uniform_fmt,
+                     num_q_heads, head_map, alibi_slopes, softmax_scale, out, lse, workspace,
+                     workspace_bytes, err_word, stream, phases, 0, 0, num_queries);
 }
 
 cfr_status cfr_merge_partials(const float *part_acc, const float *part_m, const float *part_l,
@@ -401,8 +424,8 @@ cfr_status cfr_schedule_splits(const int32_t *seq_lens, int32_t batch, int32_t p
   if (batch <= 0 || page_tokens <= 0 || max_pages <= 0 || target_splits <= 0 || max_splits <= 0)
     return CFR_ERR_INVALID_ARG;
   if (static_cast<long long>(max_pages) * page_tokens > INT_MAX) return CFR_ERR_OVERFLOW;
-  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, 0, 0, split_off, splits,
-                  max_splits, num_splits, err_word, static_cast<cudaStream_t>(stream));
+  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, 0, 0, 1, split_off,
+                  splits, max_splits, num_splits, err_word, static_cast<cudaStream_t>(stream));
   return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
 }
 

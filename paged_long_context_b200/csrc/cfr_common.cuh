@@ -46,6 +46,8 @@ struct DecodeParams {
   float sigma_log2e;    // softmax scale times log2(e)
   int gmax;             // largest group size
   int sink, window;     // window > 0: only tokens j < sink or j >= n - window take part
+  int nq;               // query tokens per sequence (the last nq positions, causal)
+  int hq_real;          // query heads; the Hq = nq * hq_real query rows are qi * hq_real + h
   int16_t grp_off[kMaxQHeads + 1];  // heads of kv head g: grp_heads[grp_off[g] .. grp_off[g+1])
   int16_t grp_heads[kMaxQHeads];
 };
@@ -225,6 +227,13 @@ __device__ __forceinline__ void mask_set_range(uint32_t (&m)[4], int lo, int hi)
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int r) {
   const uint32_t w = r < 32 ? m[0] : r < 64 ? m[1] : r < 96 ? m[2] : m[3];
   return (w >> (r & 31)) & 1u;
+}
+
+// ALiBi slope index and causal offset of query row vh (= qi * hq_real + h): the
+// row is query qi of the last nq positions and sees tokens j <= n - 1 - offset.
+__device__ __forceinline__ int row_head(const DecodeParams &p, int vh) { return vh % p.hq_real; }
+__device__ __forceinline__ int row_offset(const DecodeParams &p, int vh) {
+  return p.nq - 1 - vh / p.hq_real;
 }
 
 // Token j of a sequence of n tokens takes part in the softmax: every token, or

@@ -162,6 +162,7 @@ struct CcLayout {
   float *sc;       // [2][GT][T]
   float *alpha;    // [2][GT]
   float *slope2;   // [GT] slope * log2(e)
+  int *qoff;       // [GT] causal offset of each query row
   float *red;      // [CC_WARPS][4][D]
   int *flag;       // [1] wait outcome broadcast
   uint8_t *ring;   // [stages][2][T][pitch]
@@ -174,7 +175,7 @@ __host__ __device__ inline size_t cc_fixed_bytes(int stages) {
   o = (o + 15) & ~size_t(15);
   o += stages * sizeof(CcStageMeta);
   o = (o + 15) & ~size_t(15);
-  o += GT * D * 4 + 2 * GT * CC_T * 4 + 2 * GT * 4 + GT * 4 + CC_WARPS * 4 * D * 4 + 16;
+  o += GT * D * 4 + 2 * GT * CC_T * 4 + 2 * GT * 4 + GT * 4 + GT * 4 + CC_WARPS * 4 * D * 4 + 16;
   o = (o + 127) & ~size_t(127);
   return o;
 }
@@ -197,6 +198,8 @@ __device__ inline CcLayout cc_layout(uint8_t *smem, int stages, int pitch) {
   L.alpha = reinterpret_cast<float *>(smem + o);
   o += 2 * GT * 4;
   L.slope2 = reinterpret_cast<float *>(smem + o);
+  o += GT * 4;
+  L.qoff = reinterpret_cast<int *>(smem + o);
   o += GT * 4;
   L.red = reinterpret_cast<float *>(smem + o);
   o += CC_WARPS * 4 * D * 4;
@@ -328,8 +331,11 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
       }
       L.q_s[i] = v;
     }
-    if (tid < GT)
-      L.slope2[tid] = (p.slopes && tid < cnt) ? p.slopes[p.grp_heads[h0 + tid]] * kLog2e : 0.f;
+    if (tid < GT) {
+      L.slope2[tid] =
+          (p.slopes && tid < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + tid])] * kLog2e : 0.f;
+      L.qoff[tid] = tid < cnt ? row_offset(p, p.grp_heads[h0 + tid]) : 0;
+    }
     consumers_sync();
 
     float acc[GT][DPL];
@@ -392,12 +398,15 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
           dot[h] += __shfl_xor_sync(0xffffffffu, dot[h], 4);
         }
         if (r < CC_T) {
-          const float dist = static_cast<float>(n - 1 - (m.t0 + r));
 #pragma unroll
           for (int h = 0; h < GT; ++h)
-            if ((h & 7) == j8)
-              sc[h * CC_T + r] =
-                  valid ? fmaf(dot[h] * ks, p.sigma_log2e, -L.slope2[h] * dist) : -INFINITY;
+            if ((h & 7) == j8) {
+              // query row h sits at position n - 1 - qoff[h] and sees tokens up to it
+              const int dist = n - 1 - L.qoff[h] - (m.t0 + r);
+              sc[h * CC_T + r] = (valid && dist >= 0) ? fmaf(dot[h] * ks, p.sigma_log2e,
+                                                             -L.slope2[h] * static_cast<float>(dist))
+                                                      : -INFINITY;
+            }
         }
       }
       consumers_sync();

@@ -81,9 +81,10 @@ __host__ __device__ constexpr size_t f32_smem_bytes() {
   return f32_ring_offset<D, GT>() + static_cast<size_t>(F_STAGES) * 2 * F32Cfg<D>::TILE_BYTES + 1024;
 }
 
-// one tile of the producer warp: lane 0 waits for the stage; lane f resolves page
+// one tile of the producer warp: lane f resolves page
 // piece f of the tile and issues its boxes; lane 0 publishes which rows are valid
-// and the expected byte count.
+// and the expected byte count.  Pages are resolved before the wait for the
+// stage, so that only the publication and the copies follow it.
 template <int D>
 __device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F32Maps &maps,
                                                  uint64_t *full, uint64_t *empty, F32Meta *meta,
@@ -92,9 +93,6 @@ __device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F3
                                                  uint32_t phase, bool *timed_out, int lane) {
   using C = F32Cfg<D>;
   const int P = p.P;
-  int ok = 1;
-  if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
-  if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
   const int rows = min(C::T, tok_end - t0);
   const int npiece = (rows + box_rows - 1) / box_rows;  // <= 16
   bool pvalid = false;
@@ -113,12 +111,18 @@ __device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F3
     }
   }
   const uint32_t vb = __ballot_sync(0xffffffffu, pvalid);
+  uint32_t valid[4] = {0u, 0u, 0u, 0u};
   if (lane == 0) {
-    F32Meta &m = meta[stage];
-    uint32_t valid[4] = {0u, 0u, 0u, 0u};
     for (int f = 0; f < npiece; ++f)
       if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
     mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
+  }
+  // the stage is needed only from here on
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
+  if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+  if (lane == 0) {
+    F32Meta &m = meta[stage];
     for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
     m.rows = rows;
     m.t0 = t0;
@@ -200,9 +204,11 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
 
     float q[GT][32];
     float slope2[GT];
+    int qoff[GT];  // causal offset of each query row (0 with one query per sequence)
 #pragma unroll
     for (int h = 0; h < GT; ++h) {
       slope2[h] = 0.f;
+      qoff[h] = 0;
       if (h < cnt) {
         const int head = p.grp_heads[h0 + h];
         const long long base = (static_cast<long long>(b) * p.Hq + head) * D + 32 * q_blk;
@@ -226,7 +232,8 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
             }
           }
         }
-        if (p.slopes) slope2[h] = p.slopes[head] * kLog2e;
+        if (p.slopes) slope2[h] = p.slopes[row_head(p, head)] * kLog2e;
+        qoff[h] = row_offset(p, head);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) q[h][i] = 0.f;
@@ -278,10 +285,15 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
         }
         if (q_blk == 0) {
           const bool valid = (m.valid[q_row >> 5] >> (q_row & 31)) & 1u;
-          const float dist = static_cast<float>(n - 1 - (m.t0 + q_row));
+          const int j = m.t0 + q_row;
 #pragma unroll
-          for (int h = 0; h < GT; ++h)
-            sc[h][q_row] = valid ? fmaf(dot[h], p.sigma_log2e, -slope2[h] * dist) : -INFINITY;
+          for (int h = 0; h < GT; ++h) {
+            // query row h sits at position n - 1 - qoff[h] and sees tokens up to it
+            const int dist = n - 1 - qoff[h] - j;
+            sc[h][q_row] = (valid && dist >= 0)
+                               ? fmaf(dot[h], p.sigma_log2e, -slope2[h] * static_cast<float>(dist))
+                               : -INFINITY;
+          }
         }
       }
       f_sync();

@@ -51,6 +51,8 @@ constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V 
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
 constexpr int TC_RAW_BYTES = 2 * TC_T * TC_D;  // raw int8 / FP8 K + V rows (int4 uses half)
 constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2, KIND_FP8 = 3;
+// compile-time variants: plain decode, multi-query rows, sink + window subset
+constexpr int TC_FEAT_PLAIN = 0, TC_FEAT_MULTI = 1, TC_FEAT_SUBSET = 2;
 
 struct TcMeta {
   uint32_t valid[4];
@@ -211,7 +213,7 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 
 // ---- roles ------------------------------------------------------------------
 
-template <int NCOL, bool INTP>
+template <int NCOL, bool INTP, int FEAT>
 struct TcCtx {
   const DecodeParams &p;
   const TcMaps &maps;
@@ -266,21 +268,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// one tile of the producer warp: lane 0 waits for the stage; lane f resolves
-// page piece f of the tile and issues its copies, so a tile made of many small
-// pages is issued in parallel; lane 0 publishes the tile description and the
-// expected byte count.
-template <int NCOL, bool INTP>
-__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int g, int n, int t0,
+// one tile of the producer warp.  Everything that does not need the stage --
+// page resolution (lane f resolves page piece f, so a tile made of many small
+// pages is resolved in parallel), the row mask, scales, byte count -- is done
+// first; then lane 0 waits for the stage, and the moment it is free lane 0
+// publishes the tile description and the expected byte count while every lane
+// issues its own copies.
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int b, int g, int n, int t0,
                                                 int tok_end, int stage, uint32_t phase,
                                                 bool *timed_out, int lane) {
   const DecodeParams &p = c.p;
   const PageCache &pc = c.S.pc;
   const int P = p.P;
   const int box_rows = P < TC_T ? P : TC_T;
-  int ok = 1;
-  if (lane == 0) ok = mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
-  if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
   const int rows = min(TC_T, tok_end - t0);
   const int npiece = (rows + box_rows - 1) / box_rows;  // <= 16
   // ---- resolve piece `lane` ----
@@ -310,15 +311,16 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
                     : fmt == CFR_FMT_FP8   ? KIND_FP8
                                            : KIND_BF16;
   const int kind = __shfl_sync(0xffffffffu, kind0, 0);
-  uint64_t *done = nullptr;
+  // ---- the tile description (lane 0) ----
+  uint32_t valid[4] = {0u, 0u, 0u, 0u};
+  float ks = 1.f, vs = 1.f;
+  uint32_t bytes = 0;
+  bool direct = false;
   if (lane == 0) {
-    TcMeta &m = c.S.meta[stage];
-    uint32_t valid[4] = {0u, 0u, 0u, 0u};
     for (int f = 0; f < npiece; ++f)
       if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
-    mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
-    float ks = 1.f, vs = 1.f;
-    uint32_t bytes;
+    if constexpr (FEAT == TC_FEAT_SUBSET)
+      mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
     if (kind == KIND_BF16) {
       bytes = static_cast<uint32_t>(__popc(vb)) * 4u * box_rows * 128u;
     } else {
@@ -329,7 +331,17 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
     }
     // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA; every
     // other tile passes through the staging warps
-    const bool direct = kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu;
+    direct = kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu;
+  }
+  // every lane learns where its copies complete
+  uint64_t *done = __shfl_sync(0xffffffffu, direct ? 1 : 0, 0) ? &c.S.op_full[stage]
+                                                               : &c.S.raw_full[stage];
+  // ---- wait for the stage ----
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
+  if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+  if (lane == 0) {
+    TcMeta &m = c.S.meta[stage];
     for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
     m.rows = rows;
     m.t0 = t0;
@@ -337,13 +349,9 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
     m.direct = direct ? 1 : 0;
     m.ks = ks;
     m.vs = vs;
-    done = direct ? &c.S.op_full[stage] : &c.S.raw_full[stage];
     if (direct) mbar_arrive(&c.S.raw_full[stage]);  // lets the staging warps skip this tile
     mbar_arrive_expect_tx(done, bytes);
   }
-  // every lane learns where its copies complete
-  const int dsel = __shfl_sync(0xffffffffu, (lane == 0 && done == &c.S.op_full[stage]) ? 1 : 0, 0);
-  done = dsel ? &c.S.op_full[stage] : &c.S.raw_full[stage];
   if (pvalid) {
     const int tin = (t0 + r) % P;
     uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
@@ -366,8 +374,8 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP> &c, int b, int
 
 // Producer warp: all 32 lanes keep the page-table cache filled and issue the
 // copies of each tile together.
-template <int NCOL, bool INTP>
-__device__ void tc_producer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT>
+__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
@@ -397,8 +405,8 @@ __device__ void tc_producer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
 }
 
 // staging warpgroup: thread r (0..127) owns row r of every tile that is not direct
-template <int NCOL, bool INTP>
-__device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT>
+__device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int r = threadIdx.x - 192;
@@ -435,7 +443,9 @@ __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
           }
         } else if (INTP) {
           const uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
-#pragma unroll
+          // K then V through one copy of the code (the kernel's roles share the
+          // SM's instruction cache; unrolling this loop costs more than it saves)
+#pragma unroll 1
           for (int kv = 0; kv < 2; ++kv) {
             uint8_t *dst = op + kv * 2 * TC_HALF;
             if (!valid) {
@@ -522,8 +532,8 @@ __device__ void tc_staging(TcCtx<NCOL, INTP> &c, bool *timed_out) {
 
 // QK issuer (warp 1, one thread): for every tile in order, once its operands
 // are staged and an S buffer is free, S^T = K . [q_hi | q_lo]^T into TMEM.
-template <int NCOL, bool INTP>
-__device__ void tc_qk_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT>
+__device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
@@ -572,8 +582,8 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
 // P.V issuer (warp 10, one thread): for every tile in order, once its
 // probabilities are written and an O buffer is free, O^T = V^T . [p_hi | p_lo]^T
 // into TMEM; the commit then frees the stage, the P buffer and signals the fold.
-template <int NCOL, bool INTP>
-__device__ void tc_pv_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT>
+__device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
@@ -618,8 +628,8 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP> &c, bool *timed_out) {
 }
 
 // folds the P.V product of tile i into the running accumulators (dim t of each head)
-template <int NCOL, bool INTP>
-__device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint32_t tmem, int lane,
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT> &c, long long i, uint32_t tmem, int lane,
                                         int cnt, float (&acc)[NCOL / 2],
                                         const float (&alpha_prev)[NCOL / 2], float vscale_prev,
                                         bool *timed_out) {
@@ -640,8 +650,8 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP> &c, long long i, uint3
 
 // writes the hi/lo query operand of item `it` (both bf16 and fp16 copies); the
 // warpgroup's 128 threads (index tsm) share the work, each warp then arrives on q_full
-template <int NCOL, bool INTP>
-__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP> &c, long long it, int tsm, int lane) {
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT> &c, long long it, int tsm, int lane) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   {
@@ -701,8 +711,8 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP> &c, long long it, i
 // softmax / fold warpgroup.  Every thread waits on the mbarriers itself; a
 // thread whose wait gives up keeps the same control flow (later waits return at
 // once), so the one named barrier per tile is always reached by all 128 threads.
-template <int NCOL, bool INTP>
-__device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT>
+__device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   constexpr int GM = NCOL / 2;  // most query heads per tile
   const DecodeParams &p = c.p;
@@ -730,9 +740,13 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
     // folds lag two tiles behind the scores: tiles prev2 (older) and prev1 wait,
     // each with its rescale factors and V scale
     float slope2[GM], m_run[GM], l_part[GM], acc[GM], alpha1[GM], alpha2[GM];
+    // causal offsets of the query rows, 4 bits each (at most 16 rows of offset <= 15)
+    uint32_t qoff[2] = {0u, 0u};
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
-      slope2[h] = (p.slopes && h < cnt) ? p.slopes[p.grp_heads[h0 + h]] * kLog2e : 0.f;
+      slope2[h] = (p.slopes && h < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + h])] * kLog2e : 0.f;
+      if constexpr (FEAT == TC_FEAT_MULTI)
+        if (h < cnt) qoff[h >> 3] |= static_cast<uint32_t>(row_offset(p, p.grp_heads[h0 + h])) << (4 * (h & 7));
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
       acc[h] = 0.f;
@@ -758,13 +772,22 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
       const TcMeta &m = c.S.meta[stage];
       const bool valid = (m.valid[t >> 5] >> (t & 31)) & 1u;
       const float scale = m.ks * p.sigma_log2e;
-      const float dist = static_cast<float>(n - 1 - (m.t0 + t));
       const int kind = m.kind;
       const float vsc = kind == KIND_BF16 ? 1.f : m.vs * (1.f / 32768.f);
+      // ALiBi from the last position; a query row at offset o before it differs by the
+      // row constant slope * o, added back to its maximum at the partial write
+      const int j = m.t0 + t;
+      const float dist = static_cast<float>(n - 1 - j);
       float s[GM];
 #pragma unroll
       for (int h = 0; h < GM; ++h)
         s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
+      if (FEAT == TC_FEAT_MULTI && m.t0 + TC_T - 1 > n - p.nq) {
+        // the tile reaches the query positions: row h sees tokens j <= n - 1 - offset_h
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (j > n - 1 - static_cast<int>((qoff[h >> 3] >> (4 * (h & 7))) & 15u)) s[h] = -INFINITY;
+      }
       {
         int hm;
         const float mx = warp_multi_max<GM>(s, lane, &hm);
@@ -875,6 +898,11 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
 #pragma unroll
       for (int h = 0; h < GM; ++h)
         if (h == tsm) mrun = m_run[h];
+      if constexpr (FEAT == TC_FEAT_MULTI) {
+        const int vh = p.grp_heads[h0 + tsm];
+        const float sl = p.slopes ? p.slopes[row_head(p, vh)] * kLog2e : 0.f;
+        if (mrun != -INFINITY) mrun = fmaf(sl, static_cast<float>(row_offset(p, vh)), mrun);
+      }
       p.part_m[cidx] = mrun;
       p.part_l[cidx] = (c.S.red_l[0][tsm] + c.S.red_l[1][tsm]) + (c.S.red_l[2][tsm] + c.S.red_l[3][tsm]);
     }
@@ -882,7 +910,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP> &c, bool *timed_out) {
   }
 }
 
-template <int NCOL, bool INTP>
+template <int NCOL, bool INTP, int FEAT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -924,19 +952,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_after();
   griddep_wait();  // the split schedule comes from the previous kernel
 
-  TcCtx<NCOL, INTP> c{p, maps, S, smem + L::op, smem + L::raw, smem + L::q, smem + L::pbuf,
+  TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::raw, smem + L::q, smem + L::pbuf,
                       static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
   bool timed_out = false;
   if (warp == 0) {
-    tc_producer<NCOL, INTP>(c, &timed_out);
+    tc_producer<NCOL, INTP, FEAT>(c, &timed_out);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP>(c, &timed_out);
+    if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP, FEAT>(c, &timed_out);
   } else if (warp == 10) {
-    if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP>(c, &timed_out);
+    if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP, FEAT>(c, &timed_out);
   } else if (warp < 6) {
-    tc_softmax<NCOL, INTP>(c, &timed_out);
+    tc_softmax<NCOL, INTP, FEAT>(c, &timed_out);
   } else {
-    tc_staging<NCOL, INTP>(c, &timed_out);
+    tc_staging<NCOL, INTP, FEAT>(c, &timed_out);
   }
   tc_fence_before();
   __syncthreads();
@@ -981,7 +1009,7 @@ bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
   return true;
 }
 
-template <int NCOL, bool INTP>
+template <int NCOL, bool INTP, int FEAT>
 static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t stream) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -996,20 +1024,30 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
   }
   constexpr size_t smem = TcLayout<NCOL, INTP>::launch_bytes;
   static_assert(smem <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<NCOL, INTP>,
+  cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<NCOL, INTP, FEAT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_after_previous(tc_decode_kernel<NCOL, INTP>, dim3(grid), dim3(TC_THREADS), smem, stream,
+  e = launch_after_previous(tc_decode_kernel<NCOL, INTP, FEAT>, dim3(grid), dim3(TC_THREADS), smem, stream,
                             p, maps);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream) {
+template <int FEAT>
+static cudaError_t tc_launch_f(const DecodeParams &p, int grid, cudaStream_t stream) {
   const bool ints = tc_int_pools(p, p.page_fmt != nullptr);
   if (p.gmax <= 8)
-    return ints ? tc_launch_t<16, true>(p, grid, stream) : tc_launch_t<16, false>(p, grid, stream);
-  return ints ? tc_launch_t<32, true>(p, grid, stream) : tc_launch_t<32, false>(p, grid, stream);
+    return ints ? tc_launch_t<16, true, FEAT>(p, grid, stream)
+                : tc_launch_t<16, false, FEAT>(p, grid, stream);
+  return ints ? tc_launch_t<32, true, FEAT>(p, grid, stream)
+              : tc_launch_t<32, false, FEAT>(p, grid, stream);
+}
+
+cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream) {
+  // plain decode runs neither the per-row causal masks nor the subset masks
+  if (p.nq > 1) return tc_launch_f<TC_FEAT_MULTI>(p, grid, stream);
+  if (p.window > 0) return tc_launch_f<TC_FEAT_SUBSET>(p, grid, stream);
+  return tc_launch_f<TC_FEAT_PLAIN>(p, grid, stream);
 }
 
 }  // namespace cfr

@@ -7,7 +7,9 @@
 // the sequence lengths).  With a sink + recent window subset (window > 0) only
 // the pages holding tokens of the subset are scheduled: the pages of the first
 // `sink` tokens and those of the last `window` tokens, two page ranges when a
-// gap separates them.  Writes split_off[B+1], the (b, first page, end page)
+// gap separates them.  A sequence shorter than its number of query tokens (or
+// empty, or longer than its page table) gets no split and sets
+// CFR_DEVERR_SEQ_LEN.  Writes split_off[B+1], the (b, first page, end page)
 // triple of every split, and (total splits, chunk).  Deterministic.
 #include "cfr_common.cuh"
 
@@ -63,8 +65,9 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *red, int *total)
   return r;
 }
 
-__device__ __forceinline__ int valid_pages(int n, int P, int max_pages) {
-  if (n <= 0 || n > max_pages * P) return -1;
+// pages of a sequence of n tokens; -1 when n is outside [min_len, max_pages * P]
+__device__ __forceinline__ int valid_pages(int n, int P, int max_pages, int min_len) {
+  if (n <= 0 || n < min_len || n > max_pages * P) return -1;
   return (n + P - 1) / P;
 }
 
@@ -85,7 +88,7 @@ __device__ __forceinline__ void page_ranges(int n, int np, int P, int sink, int 
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     const int32_t *__restrict__ seq_lens, int batch, int P, int max_pages, int target, int sink,
-    int window, int32_t *__restrict__ split_off, int32_t *__restrict__ splits, int max_splits,
+    int window, int nq, int32_t *__restrict__ split_off, int32_t *__restrict__ splits, int max_splits,
     int32_t *__restrict__ num_splits, uint32_t *err) {
   griddep_launch_dependents();
   __shared__ long long red_ll[33];
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
   long long local = 0;
   for (int b = threadIdx.x; b < batch; b += blockDim.x) {
     const int n = seq_lens[b];
-    const int np = valid_pages(n, P, max_pages);
+    const int np = valid_pages(n, P, max_pages, nq);
     if (np < 0) {
       set_err(err, CFR_DEVERR_SEQ_LEN);
     } else {
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
   for (int base = 0; base < batch; base += blockDim.x) {
     const int b = base + threadIdx.x;
     const int n = b < batch ? seq_lens[b] : 0;
-    int np = b < batch ? valid_pages(n, P, max_pages) : -1;
+    int np = b < batch ? valid_pages(n, P, max_pages, nq) : -1;
     if (np < 0) np = 0;
     int a_end, b_begin;
     page_ranges(n, np, P, sink, window, &a_end, &b_begin);
@@ -149,10 +152,10 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
 }
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
-                     int sink, int window, int32_t *split_off, int32_t *splits, int max_splits,
-                     int32_t *num_splits, uint32_t *err, cudaStream_t stream) {
+                     int sink, int window, int nq, int32_t *split_off, int32_t *splits,
+                     int max_splits, int32_t *num_splits, uint32_t *err, cudaStream_t stream) {
   schedule_kernel<<<1, kSchedThreads, 0, stream>>>(seq_lens, batch, P, max_pages, target, sink,
-                                                   window, split_off, splits, max_splits,
+                                                   window, nq, split_off, splits, max_splits,
                                                    num_splits, err);
 }
 

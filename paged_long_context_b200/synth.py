@@ -446,10 +446,15 @@ WORKLOADS = {
 }
 
 
-def workload(name: str, device="cpu") -> DecodeCase:
-    """One of the five page-shaped workloads, with its fixed seed."""
+def workload(name: str, device="cpu", num_queries: int = 1) -> DecodeCase:
+    """One of the five page-shaped workloads, with its fixed seed (optionally with
+    several query tokens per sequence)."""
     fn, seed = WORKLOADS[name]
-    return make_case(fn(), seed, device)
+    spec = fn()
+    if num_queries > 1:
+        spec = dataclasses.replace(spec, num_queries=num_queries,
+                                   name=f"{spec.name}_q{num_queries}")
+    return make_case(spec, seed, device)
 
 
 def merge_inputs(num_splits: Sequence[int], num_q_heads: int, head_dim: int, seed: int,
