@@ -238,7 +238,7 @@ cfr_status cfr_paged_decode_multi(const void *q, int32_t q_fmt, const cfr_kv_poo
  * Bytes of the scratch array compiled into the library for
  * cfr_paged_decode_static_workspace (one array per GPU that loads the library).
  */
-#define CFR_STATIC_WORKSPACE_BYTES (8u << 20)
+#define CFR_STATIC_WORKSPACE_BYTES (16u << 20)
 
 /*
  * cfr_paged_decode for callers that cannot allocate device memory: plugin or

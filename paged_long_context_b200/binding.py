@@ -30,7 +30,7 @@ EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_dec
            "cfr_paged_decode_static_workspace", "cfr_demote_pages", "cfr_append_kv",
            "cfr_paged_decode_sink_window", "cfr_paged_decode_multi"]
 FMT_COUNT = 5
-STATIC_WORKSPACE_BYTES = 8 << 20
+STATIC_WORKSPACE_BYTES = 16 << 20
 
 
 class CfrError(RuntimeError):

@@ -69,11 +69,16 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Target number of splits over the whole batch: about eight work items
+// Target number of splits over the whole batch: about `per_sm` work items
 // (split x kv head) per SM, so that a persistent grid of one CTA per SM gets
-// an even share.
-int target_splits(int sms, int hkv) {
-  const long long items = 8LL * sms;
+// an even share.  A cache of mixed storage formats has items of unequal cost
+// (a page of int4 codes is a quarter of the bytes of a bf16 page, but takes
+// longer to expand), so it is cut finer; a uniform cache keeps longer items,
+// each of which pays one pipeline drain at its end.
+constexpr int kItemsPerSm = 8, kItemsPerSmMixed = 16;
+
+int target_splits(int sms, int hkv, int per_sm = kItemsPerSmMixed) {
+  const long long items = static_cast<long long>(per_sm) * sms;
   long long t = (items + hkv - 1) / hkv;
   if (t < 1) t = 1;
   if (t > (1 << 20)) t = 1 << 20;
@@ -297,7 +302,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
 
   DeviceInfo di;
   if (!device_info(&di)) return CFR_ERR_CUDA;
-  const int target = target_splits(di.sms, kv->num_kv_heads);
+  const int target =
+      target_splits(di.sms, kv->num_kv_heads, page_fmt ? kItemsPerSmMixed : kItemsPerSm);
   WsLayout w;
   if (!ws_layout(batch, rows, kv->head_dim, max_pages, target, &w)) return CFR_ERR_OVERFLOW;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return CFR_ERR_WORKSPACE;

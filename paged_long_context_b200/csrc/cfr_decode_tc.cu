@@ -950,7 +950,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_wait();  // the split schedule comes from the previous kernel
+  griddep_wait();  // the split schedule comes from the previous kernel (returns at once
+                   // when the launch did not overlap it)
 
   TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::raw, smem + L::q, smem + L::pbuf,
                       static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
@@ -1028,8 +1029,10 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_after_previous(tc_decode_kernel<NCOL, INTP, FEAT>, dim3(grid), dim3(TC_THREADS), smem, stream,
-                            p, maps);
+  // a plain launch: overlapping this kernel's start with the schedule kernel
+  // (programmatic dependent launch) measured slower for this kernel
+  tc_decode_kernel<NCOL, INTP, FEAT><<<dim3(grid), dim3(TC_THREADS), smem, stream>>>(p, maps);
+  e = cudaSuccess;
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
