@@ -180,10 +180,10 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, path: int):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary,
-    only when the kernel sources are unchanged since the capture."""
-    name = os.path.join(PROFILE_TRAFFIC, f"decode_kernel_{workload}.md")
+def profiled_traffic(summary: str, key: str):
+    """DRAM bytes (read + write) from a committed ncu summary under profiles/, only
+    when the kernel sources are unchanged since the capture."""
+    name = os.path.join(PROFILE_TRAFFIC, summary)
     if not os.path.exists(name):
         return None
     vals = {}
@@ -194,7 +194,7 @@ def profiled_traffic(workload: str, path: int):
     if vals.get("kernel_source_digest") != kernel_source_digest():
         return None
     try:
-        return int(vals["dram_bytes_per_launch"])
+        return int(vals[key])
     except (KeyError, ValueError):
         return None
 
@@ -371,7 +371,9 @@ def run_ours(args, dist):
 
     peak, peak_kind = measured_peaks()
     achieved = acct["total"] / (kern_ms_max * 1e-3) / 1e9
-    traffic = profiled_traffic(args.workload, path)
+    # the committed capture is of the plain decode (no subset, one query per sequence)
+    traffic = (profiled_traffic(f"decode_kernel_{args.workload}.md", "dram_bytes_per_launch")
+               if sw is None and args.queries == 1 else None)
     world = dist.world
     value = world * kv_bytes / (step_ms_max * 1e-3) / 1e9
     res = {
@@ -556,7 +558,7 @@ def run_demote(args, dist):
 
     peak, peak_kind = measured_peaks()
     achieved = acct["total"] / (launch_ms_max * 1e-3) / 1e9
-    traffic = profiled_traffic("demote", 0)
+    traffic = profiled_traffic("demote_kernel_demote.md", "dram_bytes_per_step")
     world = dist.world
     res = {
         "metric": DEMOTE_METRIC,
