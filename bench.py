@@ -4,6 +4,7 @@ every (sequence, query head) of the workload (schedule + decode + merge).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload cfr|tiny|gqa|tiered|alibi1m|demote]
+                    [--queries Q] [--sink S --window W]
 
 Prints one JSON line (rank 0).  `value` is the effective KV-read bandwidth
 (algorithmic K/V bytes of all ranks / step time, GB/s) with every input resident
@@ -15,7 +16,10 @@ and (out, lse) read back, the KV cache staying resident.  `--impl reference`
 times the fp64 CPU oracle on the host cores instead.  With N > 1 (torchrun) each
 rank runs an independent replica of the workload (no collective on the path).
 
-`--workload demote` measures page demotion instead: one step re-encodes the
+`--queries Q` makes the last Q positions of every sequence causal query rows
+(cfr_paged_decode_multi); `--sink S --window W` restricts every softmax to the
+first S and last W tokens (cfr_paged_decode_sink_window), the byte count then
+covering only those tokens.  `--workload demote` measures page demotion instead: one step re-encodes the
 cold pages of the tiered cache shape (768 bf16 pages of 8 kv heads x 256 tokens
 x 128 dims) into int4 and int8 with cfr_demote_pages; `value` is HBM bytes
 (read + written) per second.
@@ -27,6 +31,7 @@ import glob
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -173,10 +178,19 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C++ source with its comments and blank lines removed (the kernel sources
+    hold no string literal that contains a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
 def kernel_source_digest() -> str:
+    """Digest of the kernel sources' code (comments do not change a capture's validity)."""
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "paged_long_context_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+        h.update(_code_only(open(f, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -2,7 +2,8 @@
 // (tcgen05, accumulators in TMEM) for bf16, FP8 (E4M3), int8 and int4 K/V pages,
 // head_dim 128.
 //
-// For a kv head serving G query heads, one 128-token tile is two small dense
+// For a kv head serving G query rows (its query heads, times the queries per
+// sequence in multi-query decode), one 128-token tile is two small dense
 // contractions:
 //   S^T[128 tok x N] = K_tile[128 x 128] . Q^T           (M = tokens, K = head_dim)
 //   O^T[128 dim x N] = V_tile^T[128 x 128] . P^T          (M = head_dim, K = tokens)
@@ -35,6 +36,13 @@
 //               never meet a zero probability inside the MMA.
 // Every mbarrier wait is bounded; on a timeout the error word is set, every
 // role leaves its loop, the MMA pipe is drained and TMEM is freed.
+//
+// Three compile-time variants: plain decode; multi-query rows (per-row causal
+// limits in the tiles that reach the query positions, and the row's ALiBi
+// constant added to its maximum at the partial write); sink + recent-window
+// subsets (gap rows cleared from the producer's row mask).  The roles share
+// the SM's instruction cache, so code that is not on the current variant's
+// path is kept out of it and loops off the critical path stay rolled.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 

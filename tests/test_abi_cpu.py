@@ -276,3 +276,25 @@ def test_sink_window_rejects(lib):
     assert L.cfr_paged_decode_sink_window(*args, 4, 0, binding.PHASE_ALL) == INVALID
     assert L.cfr_paged_decode_sink_window(*args, 4, 16, 0) == INVALID
     assert L.cfr_paged_decode_sink_window(*args, 4, 16, 0x10) == INVALID
+
+
+def test_multi_query_rejects(lib):
+    case = _case()
+    bufs = FakeBufs(case)
+    pool = binding.kv_pool_struct(case)
+    L = binding.lib()
+
+    def call(nq, hq=case.num_q_heads, hkv=None, phases=binding.PHASE_ALL):
+        p = binding.kv_pool_struct(case)
+        if hkv is not None:
+            p.num_kv_heads = hkv
+        return L.cfr_paged_decode_multi(
+            binding._p(case.q), case.q_fmt, ctypes.byref(p), binding._p(case.page_table),
+            case.max_pages, binding._p(case.seq_lens), case.batch, binding._p(case.page_fmt),
+            case.uniform_fmt, hq, nq, None, None, 0.0, binding._p(bufs.out), binding._p(bufs.lse),
+            binding._p(bufs.workspace), bufs.workspace.numel(), binding._p(bufs.err), None, phases)
+    assert call(0) == INVALID                     # at least one query per sequence
+    assert call(17) == UNSUP                      # at most 16
+    assert call(4, hq=8, hkv=1) == UNSUP          # 8 heads x 4 queries = 32 rows per kv head
+    assert call(2, hq=130, hkv=130) == UNSUP      # 260 query rows per sequence
+    assert call(2, phases=0) == INVALID
