@@ -186,17 +186,22 @@ def _code_only(text: str) -> str:
     return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
 
 
-def kernel_source_digest() -> str:
-    """Digest of the kernel sources' code (comments do not change a capture's validity)."""
+def kernel_source_digest(files=None) -> str:
+    """Digest of kernel sources' code (comments do not change a capture's validity):
+    the named files under csrc/, or all of them."""
+    csrc = os.path.join(ROOT, "paged_long_context_b200", "csrc")
+    paths = ([os.path.join(csrc, f) for f in files] if files else
+             sorted(glob.glob(os.path.join(csrc, "*"))))
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "paged_long_context_b200", "csrc", "*"))):
+    for f in paths:
         h.update(_code_only(open(f, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(summary: str, key: str):
     """DRAM bytes (read + write) from a committed ncu summary under profiles/, only
-    when the kernel sources are unchanged since the capture."""
+    when the profiled kernel's sources (listed in the summary) are unchanged since
+    the capture."""
     name = os.path.join(PROFILE_TRAFFIC, summary)
     if not os.path.exists(name):
         return None
@@ -205,7 +210,8 @@ def profiled_traffic(summary: str, key: str):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_digest") != kernel_source_digest():
+    files = [f.strip() for f in vals.get("kernel_sources", "").split(",") if f.strip()]
+    if not files or vals.get("kernel_source_digest") != kernel_source_digest(files):
         return None
     try:
         return int(vals[key])

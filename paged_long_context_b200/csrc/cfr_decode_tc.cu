@@ -57,7 +57,7 @@ constexpr int TC_D = 128;            // head_dim
 constexpr int TC_THREADS = 352;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
-constexpr int TC_RAW_BYTES = 2 * TC_T * TC_D;  // raw int8 / FP8 K + V rows (int4 uses half)
+constexpr int TC_RAW_K = TC_T * TC_D;  // raw code offset of V inside a stage's V region (K at 0)
 constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2, KIND_FP8 = 3;
 // compile-time variants: plain decode, multi-query rows, sink + window subset
 constexpr int TC_FEAT_PLAIN = 0, TC_FEAT_MULTI = 1, TC_FEAT_SUBSET = 2;
@@ -75,7 +75,9 @@ struct TcMaps {
 
 template <int NCOL, bool INTP>
 struct TcCfg {
-  static constexpr int STAGES = INTP ? 2 : 3;
+  // quantised codes are copied into the stage's own V region and expanded in
+  // place, so the variant with quantised pools keeps the same three stages
+  static constexpr int STAGES = 3;
   static constexpr int Q_BYTES = NCOL * 256;       // [NCOL rows][128 cols] 16-bit, 2 halves
   static constexpr int P_BYTES = NCOL * TC_T * 2;  // [128 tokens][NCOL] 16-bit
   static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
@@ -99,8 +101,7 @@ template <int NCOL, bool INTP>
 struct TcLayout {
   static constexpr size_t head = (sizeof(TcSmem<NCOL, INTP>) + 1023) / 1024 * 1024;
   static constexpr size_t op = head;
-  static constexpr size_t raw = op + TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_OP_BYTES);
-  static constexpr size_t q = raw + (INTP ? TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_RAW_BYTES) : 0);
+  static constexpr size_t q = op + TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_OP_BYTES);
   static constexpr size_t pbuf = q + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::Q_BYTES);
   static constexpr size_t total = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
   static constexpr size_t launch_bytes = total + 1024;  // slack for 1024-byte alignment
@@ -226,7 +227,7 @@ struct TcCtx {
   const DecodeParams &p;
   const TcMaps &maps;
   TcSmem<NCOL, INTP> &S;
-  uint8_t *op, *raw, *qop, *pop;
+  uint8_t *op, *qop, *pop;
   long long nitems;
   int nsplit;
 };
@@ -372,9 +373,11 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int 
     } else if (INTP) {
       const int rb = row_bytes(fmt, TC_D);
       const long long off = ((id * p.Hkv + g) * P + tin) * rb;
-      uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
+      // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in);
+      // the staging warps expand them in place
+      uint8_t *raw = op + 2 * TC_HALF;
       bulk_g2s(raw, p.k_pool[fmt] + off, rows * rb, done);
-      bulk_g2s(raw + TC_T * TC_D, p.v_pool[fmt] + off, rows * rb, done);
+      bulk_g2s(raw + TC_RAW_K, p.v_pool[fmt] + off, rows * rb, done);
     }
   }
   return true;
@@ -450,12 +453,29 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
             }
           }
         } else if (INTP) {
-          const uint8_t *raw = c.raw + static_cast<size_t>(stage) * TC_RAW_BYTES;
+          // the codes sit in this stage's V region (K codes at 0, V codes at
+          // TC_RAW_K); a thread loads its whole row before converting it, and the
+          // V rows, which are expanded over the codes, are all loaded before any
+          // is written
+          const uint8_t *raw = op + 2 * TC_HALF;
+          const bool i4 = m.kind == KIND_I4;
+          const int rb = i4 ? TC_D / 2 : TC_D;  // row bytes of the codes
           // K then V through one copy of the code (the kernel's roles share the
           // SM's instruction cache; unrolling this loop costs more than it saves)
 #pragma unroll 1
           for (int kv = 0; kv < 2; ++kv) {
             uint8_t *dst = op + kv * 2 * TC_HALF;
+            const uint8_t *src = raw + kv * TC_RAW_K + r * rb;
+            // 16-byte chunks, starting at a row-dependent chunk (no bank conflicts)
+            uint4 w[8];
+            if (valid) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int ci = i4 ? ((j + (r >> 1)) & 3) : ((j + r) & 7);
+                if (!i4 || j < 4) w[j] = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+              }
+            }
+            if (kv == 1) named_sync(3, 128);  // every V row has been read
             if (!valid) {
 #pragma unroll
               for (int ch = 0; ch < 8; ++ch) {
@@ -465,17 +485,14 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
               continue;
             }
             if (m.kind == KIND_I8) {
-              // 128 codes = 8 chunks of 16 bytes; start at a row-dependent chunk (no bank conflicts)
-              const uint8_t *src = raw + kv * TC_T * TC_D + r * TC_D;
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const int ci = (j + r) & 7;  // input chunk: codes 16ci .. 16ci+15
-                const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+                const int ci = (j + r) & 7;  // codes 16ci .. 16ci+15
                 uint32_t o[8];
-                i8x4_to_h2x2(w.x, o[0], o[1]);
-                i8x4_to_h2x2(w.y, o[2], o[3]);
-                i8x4_to_h2x2(w.z, o[4], o[5]);
-                i8x4_to_h2x2(w.w, o[6], o[7]);
+                i8x4_to_h2x2(w[j].x, o[0], o[1]);
+                i8x4_to_h2x2(w[j].y, o[2], o[3]);
+                i8x4_to_h2x2(w[j].z, o[4], o[5]);
+                i8x4_to_h2x2(w[j].w, o[6], o[7]);
                 // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
                 uint8_t *hb = dst + (ci >> 2) * TC_HALF;
                 const int oc = (2 * ci) & 7;
@@ -483,13 +500,10 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
                 *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
               }
             } else if (m.kind == KIND_FP8) {
-              // 128 E4M3 codes = 8 chunks of 16 bytes, each to two fp16 output chunks
-              const uint8_t *src = raw + kv * TC_T * TC_D + r * TC_D;
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const int ci = (j + r) & 7;
-                const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
-                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                const int ci = (j + r) & 7;  // E4M3 codes 16ci .. 16ci+15
+                const uint32_t wv[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
                 uint32_t o[8];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -502,14 +516,11 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
                 *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
               }
             } else {
-              // 128 codes = 64 bytes = 4 chunks of 16 bytes (32 codes each)
-              const uint8_t *src = raw + kv * TC_T * TC_D + r * (TC_D / 2);
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const int ci = (j + (r >> 1)) & 3;  // input chunk: codes 32ci .. 32ci+31
-                const uint4 w = *reinterpret_cast<const uint4 *>(src + 16 * ci);
-                const uint32_t wv[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u,
-                                        w.w ^ 0x88888888u};
+                const int ci = (j + (r >> 1)) & 3;  // codes 32ci .. 32ci+31
+                const uint32_t wv[4] = {w[j].x ^ 0x88888888u, w[j].y ^ 0x88888888u,
+                                        w[j].z ^ 0x88888888u, w[j].w ^ 0x88888888u};
                 uint32_t o[16];
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -961,7 +972,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   griddep_wait();  // the split schedule comes from the previous kernel (returns at once
                    // when the launch did not overlap it)
 
-  TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::raw, smem + L::q, smem + L::pbuf,
+  TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::q, smem + L::pbuf,
                       static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
   bool timed_out = false;
   if (warp == 0) {
