@@ -72,17 +72,27 @@ def parse():
 # --------------------------------------------------------------------------
 
 class Dist:
-    def __init__(self, want: int):
+    """One process per GPU, each an independent replica of the workload; the
+    process group only carries the barriers around the timed region and the
+    max over ranks of the measured times (no collective on the data path).
+    `backend` "gloo" runs the same logic on CPU processes."""
+
+    def __init__(self, want: int, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cpu"
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                self.device = f"cuda:{self.local}"
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.pg = dist
         elif torch.cuda.is_available():
             torch.cuda.set_device(0)
@@ -94,7 +104,7 @@ class Dist:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
