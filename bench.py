@@ -27,6 +27,7 @@ x 128 dims) into int4 and int8 with cfr_demote_pages; `value` is HBM bytes
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import glob
 import hashlib
 import json
@@ -361,25 +362,44 @@ def run_ours(args, dist):
     err = int(bufs.err.item())
 
     # ---- end to end through the public call, host buffers ----
-    q_h = case.q.cpu().pin_memory()
-    sl_h = case.seq_lens.cpu().pin_memory()
-    pt_h = case.page_table.cpu().pin_memory()
-    pf_h = case.page_fmt.cpu().pin_memory() if case.page_fmt is not None else None
-    out_h = torch.empty_like(bufs.out, device="cpu").pin_memory()
-    lse_h = torch.empty_like(bufs.lse, device="cpu").pin_memory()
-    h2d = q_h.numel() * q_h.element_size() + sl_h.numel() * 4 + pt_h.numel() * 4 + \
-        (pf_h.numel() if pf_h is not None else 0)
-    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+    # The step's inputs (q, seq_lens, page table, page formats) travel in one
+    # pinned buffer and its results (out, lse) come back in one: one copy each
+    # way per step.  The library is called on views into the packed device
+    # buffers, exactly as a caller that packs its per-step tensors would.
+    def layout(tensors):
+        offs, o = [], 0
+        for t in tensors:
+            offs.append(o)
+            o = (o + t.numel() * t.element_size() + 255) // 256 * 256
+        return offs, o
+
+    def views_of(buf, offs, tensors):
+        return [buf[a:a + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                for a, t in zip(offs, tensors)]
+
+    ins = [case.q, case.seq_lens, case.page_table] + \
+        ([case.page_fmt] if case.page_fmt is not None else [])
+    in_offs, in_total = layout(ins)
+    in_d = torch.empty((in_total,), dtype=torch.uint8, device=dev)
+    in_h = torch.zeros((in_total,), dtype=torch.uint8).pin_memory()
+    for v, t in zip(views_of(in_h, in_offs, ins), ins):
+        v.copy_(t.cpu())
+    in_v = views_of(in_d, in_offs, ins)
+    e2e_case = dataclasses.replace(case, q=in_v[0], seq_lens=in_v[1], page_table=in_v[2],
+                                   page_fmt=in_v[3] if case.page_fmt is not None else None)
+    outs = [bufs.out, bufs.lse]
+    out_offs, out_total = layout(outs)
+    out_d = torch.empty((out_total,), dtype=torch.uint8, device=dev)
+    e2e_bufs = binding.DecodeBuffers.__new__(binding.DecodeBuffers)
+    e2e_bufs.out, e2e_bufs.lse = views_of(out_d, out_offs, outs)
+    e2e_bufs.workspace, e2e_bufs.err = bufs.workspace, bufs.err
+    out_h = torch.empty((out_total,), dtype=torch.uint8).pin_memory()
+    h2d, d2h = in_total, out_total
 
     def e2e_step():
-        case.q.copy_(q_h, non_blocking=True)
-        case.seq_lens.copy_(sl_h, non_blocking=True)
-        case.page_table.copy_(pt_h, non_blocking=True)
-        if pf_h is not None:
-            case.page_fmt.copy_(pf_h, non_blocking=True)
-        binding.paged_decode_raw(case, bufs, stream, sink_window=sw)
-        out_h.copy_(bufs.out, non_blocking=True)
-        lse_h.copy_(bufs.lse, non_blocking=True)
+        in_d.copy_(in_h, non_blocking=True)
+        binding.paged_decode_raw(e2e_case, e2e_bufs, stream, sink_window=sw)
+        out_h.copy_(out_d, non_blocking=True)
 
     for _ in range(min(args.warmup, 10)):
         e2e_step()
@@ -397,7 +417,8 @@ def run_ours(args, dist):
     torch.cuda.synchronize()
     dist.barrier()
     e2e_ms = dist.max(sum(a.elapsed_time(b) for a, b in ee) / Ke)
-    assert torch.equal(out_h, bufs.out.cpu())
+    # the result read back through the packed buffer is the device-resident result
+    assert torch.equal(views_of(out_h, out_offs, outs)[0], bufs.out.cpu())
 
     peak, peak_kind = measured_peaks()
     achieved = acct["total"] / (kern_ms_max * 1e-3) / 1e9
