@@ -257,23 +257,27 @@ __device__ __forceinline__ void mask_clear_gap(uint32_t (&m)[4], const DecodePar
 }
 
 // Page ids and formats of a run of pages of one sequence, staged in shared
-// memory by the producer warp so that resolving a tile reads no global memory.
-constexpr int kPageCache = 128;
-struct PageCache {
-  int32_t id[kPageCache];
-  uint8_t fmt[kPageCache];
+// memory by a producer warp so that resolving a tile reads no global memory.
+template <int N>
+struct PageCacheT {
+  static constexpr int kEntries = N;
+  int32_t id[N];
+  uint8_t fmt[N];
   int seq, base, count;
 };
+constexpr int kPageCache = 128;
+using PageCache = PageCacheT<kPageCache>;
 
 // Called by all 32 lanes of one warp: makes pages [pg, pg_last] of sequence b
-// available in the cache (pg_last - pg < kPageCache, pg_last < pg_end),
-// refilling it from pg with one coalesced read of the page table (up to pg_end)
-// when they are not all cached.
-__device__ __forceinline__ void page_cache_ensure(PageCache &pc, const DecodeParams &p, int b,
+// available in the cache (pg_last - pg < N, pg_last < pg_end), refilling it from
+// pg with one coalesced read of the page table (up to pg_end) when they are not
+// all cached.
+template <int N>
+__device__ __forceinline__ void page_cache_ensure(PageCacheT<N> &pc, const DecodeParams &p, int b,
                                                   int pg, int pg_last, int pg_end, int lane) {
   __syncwarp();
   if (b == pc.seq && pg >= pc.base && pg_last < pc.base + pc.count) return;
-  const int n = min(kPageCache, pg_end - pg);
+  const int n = min(N, pg_end - pg);
   const long long row = static_cast<long long>(b) * p.max_pages + pg;
   for (int i = lane; i < n; i += 32) {
     pc.id[i] = p.page_table[row + i];
@@ -288,7 +292,8 @@ __device__ __forceinline__ void page_cache_ensure(PageCache &pc, const DecodePar
   __syncwarp();
 }
 
-__device__ __forceinline__ void page_cache_reset(PageCache &pc, int lane) {
+template <int N>
+__device__ __forceinline__ void page_cache_reset(PageCacheT<N> &pc, int lane) {
   if (lane == 0) {
     pc.seq = -1;
     pc.base = 0;

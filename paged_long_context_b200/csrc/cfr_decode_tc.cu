@@ -16,11 +16,14 @@
 // result, both in fp32 (ARGUS page, "Transient FP16 Reconstruction ... in GPU
 // SRAM": pages are expanded on chip only, attention runs at 16-bit).
 //
-// Warp roles (352 threads, one CTA per SM, persistent over work items =
+// Warp roles (384 threads, one CTA per SM, persistent over work items =
 // (split of a sequence, kv head)):
-//   warp 0      TMA producer: resolves pages, bf16 tiles by 2-D tensor-map
-//               boxes straight into the 128-byte-swizzled operand layout,
-//               int tiles by 1-D bulk copies of the raw rows.
+//   warps 0, 11 TMA producers, taking alternate tiles: resolve pages, bf16
+//               tiles by 2-D tensor-map boxes straight into the 128-byte-swizzled
+//               operand layout, int tiles by 1-D bulk copies of the raw rows.
+//               Resolving and issuing a tile of many small pages is a serial
+//               chain of dependent steps inside one warp, so two warps run two
+//               such chains at once.
 //   warp 1      TMEM allocation; lane 0 issues the QK products.
 //   warp 10     lane 0 issues the P.V products (a thread of its own, so the two
 //               kinds of MMA never wait for each other's issue).
@@ -54,7 +57,9 @@ namespace cfr {
 
 constexpr int TC_T = 128;            // tokens per tile
 constexpr int TC_D = 128;            // head_dim
-constexpr int TC_THREADS = 352;
+constexpr int TC_THREADS = 384;
+constexpr int TC_PRODUCERS = 2;      // producer warps 0 and TC_PROD2_WARP, alternate tiles
+constexpr int TC_PROD2_WARP = 11;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
 constexpr int TC_RAW_K = TC_T * TC_D;  // raw code offset of V inside a stage's V region (K at 0)
@@ -82,6 +87,11 @@ struct TcCfg {
   static constexpr int P_BYTES = NCOL * TC_T * 2;  // [128 tokens][NCOL] 16-bit
   static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
   static constexpr int TMEM_COLS = NCOL == 16 ? 128 : 256;  // S x2 + O x3 columns, power of two
+  // page-table entries each producer keeps on chip; with 32 columns the q and P
+  // buffers leave room for two caches of 88 beside the three stages (with
+  // 16-token pages, one refill then serves 11 tiles)
+  static constexpr int PAGE_CACHE = NCOL == 16 ? 128 : 88;
+  using PageCache = PageCacheT<PAGE_CACHE>;
 };
 
 template <int NCOL, bool INTP>
@@ -94,7 +104,7 @@ struct TcSmem {
   TcMeta meta[3];
   alignas(16) float red_max[2][4][16];
   alignas(16) float red_l[4][16];
-  PageCache pc;
+  typename TcCfg<NCOL, INTP>::PageCache pc[TC_PRODUCERS];
 };
 
 template <int NCOL, bool INTP>
@@ -277,42 +287,61 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// one tile of the producer warp.  Everything that does not need the stage --
+// Per-kernel constants of a producer warp: which formats have their pools (and
+// scales) and the geometry of a tile's copy boxes.
+struct TcProdGeom {
+  uint32_t fmt_ok;  // bit f: format f can be read on this path
+  int box_rows;     // rows of one copy box: min(P, 128); a power of two
+  int box_shift;    // log2(box_rows)
+};
+
+// one tile of a producer warp.  Everything that does not need the stage --
 // page resolution (lane f resolves page piece f, so a tile made of many small
-// pages is resolved in parallel), the row mask, scales, byte count -- is done
-// first; then lane 0 waits for the stage, and the moment it is free lane 0
-// publishes the tile description and the expected byte count while every lane
-// issues its own copies.
+// pages is resolved in parallel), the row mask (one ballot per 32 rows), scales,
+// byte count -- is done first; then lane 0 waits for the stage, and the moment
+// it is free lane 0 publishes the tile description and the expected byte count
+// while every lane issues its own copies.  The tile starts at row tin0 of
+// logical page pg0 (tin0 = 0 when pages are shorter than a tile).
 template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int b, int g, int n, int t0,
-                                                int tok_end, int stage, uint32_t phase,
-                                                bool *timed_out, int lane) {
+__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c,
+                                                const typename TcCfg<NCOL, INTP>::PageCache &pc,
+                                                const TcProdGeom &geo, int b, int g, int n,
+                                                int t0, int rows, int npiece, int pg0, int tin0,
+                                                int stage, uint32_t phase, bool *timed_out,
+                                                int lane) {
   const DecodeParams &p = c.p;
-  const PageCache &pc = c.S.pc;
-  const int P = p.P;
-  const int box_rows = P < TC_T ? P : TC_T;
-  const int rows = min(TC_T, tok_end - t0);
-  const int npiece = (rows + box_rows - 1) / box_rows;  // <= 16
+  const int box_rows = geo.box_rows;
   // ---- resolve piece `lane` ----
   bool pvalid = false;
   int fmt = -1;
   long long id = 0;
-  const int r = lane * box_rows;
   if (lane < npiece) {
-    const int pg = (t0 + r) / P;
-    fmt = pc.fmt[pg - pc.base];
-    id = pc.id[pg - pc.base];
-    if (fmt < 0 || fmt >= kFmtCount) {
+    fmt = pc.fmt[pg0 + lane - pc.base];
+    id = pc.id[pg0 + lane - pc.base];
+    long long lim = 0;
+#pragma unroll
+    for (int f = 0; f < kFmtCount; ++f)
+      if (f == fmt) lim = p.pool_pages[f];
+    if (fmt >= kFmtCount) {
       set_err(p.err, CFR_DEVERR_PAGE_FMT);
-    } else if (fmt == CFR_FMT_F32 || !p.k_pool[fmt] || (is_quantised(fmt) && !p.scales[fmt])) {
+    } else if (((geo.fmt_ok >> fmt) & 1u) == 0u) {
       set_err(p.err, CFR_DEVERR_POOL);
-    } else if (id < 0 || id >= p.pool_pages[fmt]) {
+    } else if (id < 0 || id >= lim) {
       set_err(p.err, CFR_DEVERR_PAGE_ID);
     } else {
       pvalid = true;
     }
   }
   const uint32_t vb = __ballot_sync(0xffffffffu, pvalid);
+  // rows of valid pieces that hold tokens, 32 rows per ballot (every lane gets the mask)
+  uint32_t valid[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int row = 32 * w + lane;
+    valid[w] = __ballot_sync(0xffffffffu, row < rows && ((vb >> (row >> geo.box_shift)) & 1u));
+  }
+  if constexpr (FEAT == TC_FEAT_SUBSET)
+    mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
   // quantised pages need page_tokens >= 128: the tile is then one piece (lane 0)
   const int kind0 = !pvalid                ? KIND_BF16
                     : fmt == CFR_FMT_I8    ? KIND_I8
@@ -320,16 +349,13 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int 
                     : fmt == CFR_FMT_FP8   ? KIND_FP8
                                            : KIND_BF16;
   const int kind = __shfl_sync(0xffffffffu, kind0, 0);
-  // ---- the tile description (lane 0) ----
-  uint32_t valid[4] = {0u, 0u, 0u, 0u};
+  // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA; every
+  // other tile passes through the staging warps
+  const bool direct = kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu;
+  // ---- the tile's byte count and scales (lane 0) ----
   float ks = 1.f, vs = 1.f;
   uint32_t bytes = 0;
-  bool direct = false;
   if (lane == 0) {
-    for (int f = 0; f < npiece; ++f)
-      if ((vb >> f) & 1u) mask_set_range(valid, f * box_rows, min(rows, (f + 1) * box_rows));
-    if constexpr (FEAT == TC_FEAT_SUBSET)
-      mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
     if (kind == KIND_BF16) {
       bytes = static_cast<uint32_t>(__popc(vb)) * 4u * box_rows * 128u;
     } else {
@@ -338,13 +364,8 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int 
       vs = sc.y;
       bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, TC_D));
     }
-    // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA; every
-    // other tile passes through the staging warps
-    direct = kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu;
   }
-  // every lane learns where its copies complete
-  uint64_t *done = __shfl_sync(0xffffffffu, direct ? 1 : 0, 0) ? &c.S.op_full[stage]
-                                                               : &c.S.raw_full[stage];
+  uint64_t *done = direct ? &c.S.op_full[stage] : &c.S.raw_full[stage];
   // ---- wait for the stage ----
   int ok = 1;
   if (lane == 0) ok = mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
@@ -361,18 +382,19 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int 
     if (direct) mbar_arrive(&c.S.raw_full[stage]);  // lets the staging warps skip this tile
     mbar_arrive_expect_tx(done, bytes);
   }
+  __syncwarp();
   if (pvalid) {
-    const int tin = (t0 + r) % P;
+    const int r = lane * box_rows;
     uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
     if (kind == KIND_BF16) {
-      const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
+      const int y = static_cast<int>((id * p.Hkv + g) * p.P + tin0);
       tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, done);
       tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
       tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, done);
       tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
     } else if (INTP) {
       const int rb = row_bytes(fmt, TC_D);
-      const long long off = ((id * p.Hkv + g) * P + tin) * rb;
+      const long long off = ((id * p.Hkv + g) * p.P + tin0) * rb;
       // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in);
       // the staging warps expand them in place
       uint8_t *raw = op + 2 * TC_HALF;
@@ -383,30 +405,57 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c, int 
   return true;
 }
 
-// Producer warp: all 32 lanes keep the page-table cache filled and issue the
-// copies of each tile together.
+// Producer warp `k` (0 or 1): walks every tile of the CTA's items in order and
+// produces tiles k, k + 2, k + 4, ...  Two producers never hold one stage at a
+// time: tile i waits for the consumers of tile i - 3 (the same stage), and the
+// warp's previous tile i - 2 waited for tile i - 5, so the stage's barrier can
+// never be two phases behind when tile i starts waiting on it.
 template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
+__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int k) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
   const int lane = threadIdx.x & 31;
+  typename Cfg::PageCache &pc = c.S.pc[k];
+  TcProdGeom geo;
+  geo.fmt_ok = 0u;
+#pragma unroll
+  for (int f = 0; f < kFmtCount; ++f)
+    if (f != CFR_FMT_F32 && p.k_pool[f] && (!is_quantised(f) || p.scales[f])) geo.fmt_ok |= 1u << f;
+  // the path takes P a power of two dividing 128, or a multiple of 128
+  geo.box_rows = P < TC_T ? P : TC_T;
+  geo.box_shift = 31 - __clz(geo.box_rows);
+  const int pages_per_tile = P < TC_T ? TC_T / P : 0;
   int stage = 0;
   uint32_t phase = 0;
   if (lane == 0 && p.k_pool[CFR_FMT_BF16]) {
     prefetch_map(&c.maps.k);
     prefetch_map(&c.maps.v);
   }
-  page_cache_reset(c.S.pc, lane);
+  page_cache_reset(pc, lane);
+  long long tile = 0;
   for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
-      page_cache_ensure(c.S.pc, p, b, t0 / P, (min(t0 + TC_T, tok_end) - 1) / P, pe, lane);
-      if (!tc_produce_tile(c, b, g, n, t0, tok_end, stage, phase, timed_out, lane)) return;
+    int pg0 = pb, tin0 = 0;
+    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T, ++tile) {
+      if ((tile & (TC_PRODUCERS - 1)) == k) {
+        const int rows = min(TC_T, tok_end - t0);
+        const int npiece = (rows + geo.box_rows - 1) >> geo.box_shift;  // <= 16
+        page_cache_ensure(pc, p, b, pg0, pages_per_tile ? pg0 + npiece - 1 : pg0, pe, lane);
+        if (!tc_produce_tile(c, pc, geo, b, g, n, t0, rows, npiece, pg0, tin0, stage, phase,
+                             timed_out, lane))
+          return;
+      }
+      if (pages_per_tile) {
+        pg0 += pages_per_tile;
+      } else if ((tin0 += TC_T) == P) {
+        tin0 = 0;
+        ++pg0;
+      }
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -541,6 +590,9 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
         named_sync(3, 128);
         if (r == 0) mbar_arrive(&c.S.op_full[stage]);
       }
+      // the stage (and its description) may be refilled only once this
+      // warpgroup is done with it, as well as the P.V product
+      if (r == 0) mbar_arrive(&c.S.op_empty[stage]);
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -941,7 +993,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 3; ++s) {
       mbar_init(&S.op_full[s], 1);
-      mbar_init(&S.op_empty[s], 1);
+      mbar_init(&S.op_empty[s], 2);  // P.V commit + staging warpgroup
       mbar_init(&S.raw_full[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -975,8 +1027,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::q, smem + L::pbuf,
                       static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
   bool timed_out = false;
-  if (warp == 0) {
-    tc_producer<NCOL, INTP, FEAT>(c, &timed_out);
+  if (warp == 0 || warp == TC_PROD2_WARP) {
+    tc_producer<NCOL, INTP, FEAT>(c, &timed_out, warp == 0 ? 0 : 1);
   } else if (warp == 1) {
     if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP, FEAT>(c, &timed_out);
   } else if (warp == 10) {
