@@ -9,7 +9,8 @@ namespace cfr {
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
                      int sink, int window, int nq, int32_t *split_off, int32_t *splits,
-                     int max_splits, int32_t *num_splits, uint32_t *err, cudaStream_t stream);
+                     int max_splits, int32_t *num_splits, uint32_t *item_ctr, uint32_t *err,
+                     cudaStream_t stream);
 void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
                   const int32_t *split_off, int batch, int Hq, int D, float *out, float *lse,
                   cudaStream_t stream);
@@ -84,6 +85,10 @@ int target_splits(int sms, int hkv, int per_sm = kItemsPerSmMixed) {
   if (t > (1 << 20)) t = 1 << 20;
   return static_cast<int>(t);
 }
+
+// workspace header: [0] split count, [1] split length in pages; at byte
+// kItemCtrOffset the decode kernel's work-item claim counter and finished-CTA count
+constexpr size_t kItemCtrOffset = 64;
 
 struct WsLayout {
   size_t header, split_off, splits, part_m, part_l, part_acc, total;
@@ -310,6 +315,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   int32_t *num_splits = reinterpret_cast<int32_t *>(ws + w.header);
+  uint32_t *item_ctr = reinterpret_cast<uint32_t *>(ws + w.header + kItemCtrOffset);
   int32_t *split_off = reinterpret_cast<int32_t *>(ws + w.split_off);
   int32_t *splits = reinterpret_cast<int32_t *>(ws + w.splits);
   p.q = q;
@@ -324,6 +330,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.part_l = reinterpret_cast<float *>(ws + w.part_l);
   p.splits = splits;
   p.num_splits = num_splits;
+  p.item_ctr = item_ctr;
   p.err = err_word;
   p.batch = batch;
   p.max_pages = max_pages;
@@ -343,7 +350,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   }
   if (phases & CFR_PHASE_SCHEDULE) {
     launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, nq,
-                    split_off, splits, w.max_splits, num_splits, err_word, s);
+                    split_off, splits, w.max_splits, num_splits, item_ctr, err_word, s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_DECODE) {
@@ -431,7 +438,8 @@ cfr_status cfr_schedule_splits(const int32_t *seq_lens, int32_t batch, int32_t p
     return CFR_ERR_INVALID_ARG;
   if (static_cast<long long>(max_pages) * page_tokens > INT_MAX) return CFR_ERR_OVERFLOW;
   launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, 0, 0, 1, split_off,
-                  splits, max_splits, num_splits, err_word, static_cast<cudaStream_t>(stream));
+                  splits, max_splits, num_splits, nullptr, err_word,
+                  static_cast<cudaStream_t>(stream));
   return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
 }
 

@@ -38,6 +38,7 @@ struct DecodeParams {
   float *part_l;        // [S][Hq]
   const int32_t *splits;     // [S][3]: b, page begin, page end
   const int32_t *num_splits; // [0] = S
+  uint32_t *item_ctr;   // [0] work items claimed past the first per CTA, [1] CTAs finished; or null
   uint32_t *err;
   int q_fmt, uniform_fmt;
   int batch, max_pages, Hq, Hkv, D, P;

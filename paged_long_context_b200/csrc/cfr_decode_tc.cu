@@ -60,6 +60,11 @@ constexpr int TC_D = 128;            // head_dim
 constexpr int TC_THREADS = 384;
 constexpr int TC_PRODUCERS = 2;      // producer warps 0 and TC_PROD2_WARP, alternate tiles
 constexpr int TC_PROD2_WARP = 11;
+// work items reach the CTA's warps through a ring of this many slots; every
+// slot is read by producer warp 11, the two MMA issuers and one thread of each of
+// the softmax and staging warpgroups
+constexpr int TC_ITEM_RING = 4;
+constexpr int TC_ITEM_READERS = 5;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
 constexpr int TC_RAW_K = TC_T * TC_D;  // raw code offset of V inside a stage's V region (K at 0)
@@ -88,9 +93,9 @@ struct TcCfg {
   static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
   static constexpr int TMEM_COLS = NCOL == 16 ? 128 : 256;  // S x2 + O x3 columns, power of two
   // page-table entries each producer keeps on chip; with 32 columns the q and P
-  // buffers leave room for two caches of 88 beside the three stages (with
-  // 16-token pages, one refill then serves 11 tiles)
-  static constexpr int PAGE_CACHE = NCOL == 16 ? 128 : 88;
+  // buffers leave room for two caches of 80 beside the three stages (with
+  // 16-token pages, one refill then serves 10 tiles)
+  static constexpr int PAGE_CACHE = NCOL == 16 ? 128 : 80;
   using PageCache = PageCacheT<PAGE_CACHE>;
 };
 
@@ -99,6 +104,9 @@ struct TcSmem {
   uint64_t op_full[3], op_empty[3], raw_full[3];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[3], o_empty[3];
   uint64_t q_full, drain;
+  uint64_t item_full[TC_ITEM_RING], item_empty[TC_ITEM_RING];
+  int item_q[TC_ITEM_RING];  // work item of each ring slot, -1 past the last
+  int item_bc[2][2];         // [softmax, staging][k & 1]: the item broadcast in a warpgroup
   uint32_t tmem_base;
   int flag_st[3];
   TcMeta meta[3];
@@ -287,6 +295,84 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// ---- work items --------------------------------------------------------------
+// Two ways of sharing the items among the CTAs, chosen per variant by measurement:
+//  - fixed: CTA x takes items x, x + grid, x + 2 grid, ...
+//  - claimed (bf16-only plain and multi-query decode): CTA x starts with item x
+//    and claims every further item from a global counter when producer warp 0
+//    reaches it, so SMs that the memory system serves faster take more items and
+//    all CTAs finish together.  Warp 0 publishes item k of the CTA in ring slot
+//    k % TC_ITEM_RING; the other warps read the slots in order and free them.  A
+//    slot holds -1 past the CTA's last item, which ends every loop.  On quantised
+//    tiles (whose expansion sets the pace) and on subset decode the ring's
+//    per-item hand-off cost more than the balance gained, so those keep the
+//    fixed share.
+template <bool INTP, int FEAT>
+__host__ __device__ constexpr bool tc_claimed_items() {
+  return !INTP && FEAT != TC_FEAT_SUBSET;
+}
+
+// item k of the fixed share, or -1
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ int tc_fixed_item(const TcCtx<NCOL, INTP, FEAT> &c, int k) {
+  const long long it = static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
+  return it < c.nitems ? static_cast<int>(it) : -1;
+}
+
+// producer warp 0 (all lanes): claims and publishes item k; returns it, or -1.
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ int tc_claim_item(TcCtx<NCOL, INTP, FEAT> &c, int k, bool *timed_out,
+                                             int lane) {
+  const int s = k & (TC_ITEM_RING - 1);
+  int item = -1;
+  if (lane == 0) {
+    if (mbar_wait(&c.S.item_empty[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1) ^ 1u, c.p.err,
+                  timed_out)) {
+      const long long it =
+          k == 0 ? static_cast<long long>(blockIdx.x)
+          : c.p.item_ctr ? static_cast<long long>(gridDim.x) + atomicAdd(c.p.item_ctr, 1u)
+                         : static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
+      item = it < c.nitems ? static_cast<int>(it) : -1;
+      c.S.item_q[s] = item;
+      mbar_arrive(&c.S.item_full[s]);
+    }
+  }
+  return __shfl_sync(0xffffffffu, item, 0);
+}
+
+// item k read by one thread (an MMA issuer) or by every lane of a warp
+// (producer warp 11; lane 0 waits and frees the slot); -1 past the last item
+// or when the wait gave up.
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ int tc_read_item(TcCtx<NCOL, INTP, FEAT> &c, int k, bool *timed_out,
+                                            bool warp_wide) {
+  if constexpr (!tc_claimed_items<INTP, FEAT>()) return tc_fixed_item(c, k);
+  const int s = k & (TC_ITEM_RING - 1);
+  int item = -1;
+  if (!warp_wide || (threadIdx.x & 31) == 0) {
+    if (mbar_wait(&c.S.item_full[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1), c.p.err,
+                  timed_out)) {
+      item = c.S.item_q[s];
+      mbar_arrive(&c.S.item_empty[s]);
+    }
+  }
+  return warp_wide ? __shfl_sync(0xffffffffu, item, 0) : item;
+}
+
+// item k read by a 128-thread warpgroup that synchronises on named barrier
+// `bar` (2: softmax, 3: staging): thread t = 0 waits, reads and frees the slot,
+// and the barrier hands the value to all 128 threads, so they leave their loop
+// together even when the wait gave up (named barriers have no time limit).
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ int tc_read_item_wg(TcCtx<NCOL, INTP, FEAT> &c, int k, int bar, int t,
+                                               bool *timed_out) {
+  if constexpr (!tc_claimed_items<INTP, FEAT>()) return tc_fixed_item(c, k);
+  int *bc = &c.S.item_bc[bar - 2][k & 1];
+  if (t == 0) *bc = tc_read_item(c, k, timed_out, false);
+  named_sync(bar, 128);
+  return *reinterpret_cast<volatile int *>(bc);
+}
+
 // Per-kernel constants of a producer warp: which formats have their pools (and
 // scales) and the geometry of a tile's copy boxes.
 struct TcProdGeom {
@@ -405,18 +491,18 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c,
   return true;
 }
 
-// Producer warp `k` (0 or 1): walks every tile of the CTA's items in order and
-// produces tiles k, k + 2, k + 4, ...  Two producers never hold one stage at a
+// Producer warp `pk` (0 or 1): walks every tile of the CTA's items in order and
+// produces tiles pk, pk + 2, pk + 4, ...; warp 0 also claims the items.  Two producers never hold one stage at a
 // time: tile i waits for the consumers of tile i - 3 (the same stage), and the
 // warp's previous tile i - 2 waited for tile i - 5, so the stage's barrier can
 // never be two phases behind when tile i starts waiting on it.
 template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int k) {
+__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int pk) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
   const int lane = threadIdx.x & 31;
-  typename Cfg::PageCache &pc = c.S.pc[k];
+  typename Cfg::PageCache &pc = c.S.pc[pk];
   TcProdGeom geo;
   geo.fmt_ok = 0u;
 #pragma unroll
@@ -434,7 +520,11 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int k) 
   }
   page_cache_reset(pc, lane);
   long long tile = 0;
-  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
+  for (int k = 0;; ++k) {
+    const int item = !tc_claimed_items<INTP, FEAT>() ? tc_fixed_item(c, k)
+                     : pk == 0 ? tc_claim_item(c, k, timed_out, lane)
+                               : tc_read_item(c, k, timed_out, true);
+    if (item < 0) break;
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
@@ -442,7 +532,7 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int k) 
     const int tok_end = min(n, pe * P);
     int pg0 = pb, tin0 = 0;
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T, ++tile) {
-      if ((tile & (TC_PRODUCERS - 1)) == k) {
+      if ((tile & (TC_PRODUCERS - 1)) == pk) {
         const int rows = min(TC_T, tok_end - t0);
         const int npiece = (rows + geo.box_rows - 1) >> geo.box_shift;  // <= 16
         page_cache_ensure(pc, p, b, pg0, pages_per_tile ? pg0 + npiece - 1 : pg0, pe, lane);
@@ -473,7 +563,9 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   const int P = p.P;
   int stage = 0;
   uint32_t phase = 0;
-  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
+  for (int k = 0;; ++k) {
+    const int item = tc_read_item_wg(c, k, 3, r, timed_out);
+    if (item < 0) break;
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     (void)g;
@@ -613,8 +705,9 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   int stage = 0;
   uint32_t phase = 0;
   long long tc = 0;
-  int item_k = 0;
-  for (long long item = blockIdx.x; item < c.nitems && !*timed_out; item += gridDim.x, ++item_k) {
+  for (int item_k = 0; !*timed_out; ++item_k) {
+    const int item = tc_read_item(c, item_k, timed_out, false);
+    if (item < 0) break;
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     (void)g;
@@ -662,7 +755,9 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   const uint32_t op0 = smem_u32(c.op), p0 = smem_u32(c.pop);
   int stage = 0;
   long long tc = 0;
-  for (long long item = blockIdx.x; item < c.nitems && !*timed_out; item += gridDim.x) {
+  for (int k = 0; !*timed_out; ++k) {
+    const int item = tc_read_item(c, k, timed_out, false);
+    if (item < 0) break;
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     (void)g;
@@ -797,8 +892,12 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   uint32_t phase = 0;
   long long tc = 0;
   bool q_ready = false;
+  // the next item is read at the last tile of the current one (to write its
+  // query operand early); nxt_read says whether that read has happened
+  int k = 0, nxt = -1;
+  bool nxt_read = false;
 
-  for (long long item = blockIdx.x; item < c.nitems; item += gridDim.x) {
+  for (int item = tc_read_item_wg(c, 0, 2, tsm, timed_out); item >= 0; ++k) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
@@ -807,6 +906,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
     if (!q_ready) tc_write_q(c, item, tsm, lane);
     q_ready = false;
+    nxt_read = false;
 
     // folds lag two tiles behind the scores: tiles prev2 (older) and prev1 wait,
     // each with its rescale factors and V scale
@@ -924,9 +1024,10 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
       if (t0 + TC_T >= tok_end) {
         // the next item's query operand can be written as soon as this item's
         // last QK product has been read
-        const long long nx = item + gridDim.x;
-        if (nx < c.nitems) {
-          tc_write_q(c, nx, tsm, lane);
+        nxt = tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
+        nxt_read = true;
+        if (nxt >= 0) {
+          tc_write_q(c, nxt, tsm, lane);
           q_ready = true;
         }
       }
@@ -978,6 +1079,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
       p.part_l[cidx] = (c.S.red_l[0][tsm] + c.S.red_l[1][tsm]) + (c.S.red_l[2][tsm] + c.S.red_l[3][tsm]);
     }
     named_sync(2, 128);
+    item = nxt_read ? nxt : tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
   }
 }
 
@@ -1005,6 +1107,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int i = 0; i < 3; ++i) {
       mbar_init(&S.o_full[i], 1);
       mbar_init(&S.o_empty[i], 4);
+    }
+    for (int i = 0; i < TC_ITEM_RING; ++i) {
+      mbar_init(&S.item_full[i], 1);
+      mbar_init(&S.item_empty[i], TC_ITEM_READERS);
     }
     mbar_init(&S.q_full, 4);
     mbar_init(&S.drain, 2);  // one commit from each MMA issuer
@@ -1040,6 +1146,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (tc_claimed_items<INTP, FEAT>() && threadIdx.x == 0 && p.item_ctr) {
+    // every CTA has stopped claiming once all have counted themselves finished;
+    // the last one leaves both counters at 0 for the next launch
+    __threadfence();
+    if (atomicAdd(&p.item_ctr[1], 1u) == gridDim.x - 1) {
+      atomicExch(&p.item_ctr[0], 0u);
+      atomicExch(&p.item_ctr[1], 0u);
+    }
+  }
   if (warp == 1) {
     if ((threadIdx.x & 31) == 0) {
       bool t2 = false;

@@ -89,8 +89,13 @@ __device__ __forceinline__ void page_ranges(int n, int np, int P, int sink, int 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     const int32_t *__restrict__ seq_lens, int batch, int P, int max_pages, int target, int sink,
     int window, int nq, int32_t *__restrict__ split_off, int32_t *__restrict__ splits, int max_splits,
-    int32_t *__restrict__ num_splits, uint32_t *err) {
+    int32_t *__restrict__ num_splits, uint32_t *__restrict__ item_ctr, uint32_t *err) {
   griddep_launch_dependents();
+  // the decode kernel's work-item claim counter and finished-CTA count start at 0
+  if (threadIdx.x == 0 && item_ctr) {
+    item_ctr[0] = 0u;
+    item_ctr[1] = 0u;
+  }
   __shared__ long long red_ll[33];
   __shared__ int red_i[33];
   long long local = 0;
@@ -153,10 +158,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
                      int sink, int window, int nq, int32_t *split_off, int32_t *splits,
-                     int max_splits, int32_t *num_splits, uint32_t *err, cudaStream_t stream) {
+                     int max_splits, int32_t *num_splits, uint32_t *item_ctr, uint32_t *err,
+                     cudaStream_t stream) {
   schedule_kernel<<<1, kSchedThreads, 0, stream>>>(seq_lens, batch, P, max_pages, target, sink,
                                                    window, nq, split_off, splits, max_splits,
-                                                   num_splits, err);
+                                                   num_splits, item_ctr, err);
 }
 
 }  // namespace cfr
