@@ -72,11 +72,23 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Target number of splits over the whole batch: about `per_sm` work items
 // (split x kv head) per SM, so that a persistent grid of one CTA per SM gets
-// an even share.  A cache of mixed storage formats has items of unequal cost
-// (a page of int4 codes is a quarter of the bytes of a bf16 page, but takes
-// longer to expand), so it is cut finer; a uniform cache keeps longer items,
-// each of which pays one pipeline drain at its end.
-constexpr int kItemsPerSm = 8, kItemsPerSmMixed = 16;
+// an even share.  Every item pays one pipeline drain at its end and one more
+// partial for the merge.
+//  - The tcgen05 path over bf16-only pools balances at run time (its CTAs
+//    claim items from a counter, or the items are few per sequence), so it
+//    takes the fewest, longest items: 4 per SM measured faster than 8 or 16.
+//  - Other uniform caches are shared out in a fixed pattern: 8 per SM.
+//  - A cache of mixed storage formats has items of unequal cost (a page of
+//    int4 codes is a quarter of the bytes of a bf16 page, but takes longer to
+//    expand), so its fixed share is cut finer: 16 per SM.
+constexpr int kItemsPerSmClaimed = 4, kItemsPerSm = 8, kItemsPerSmMixed = 16;
+
+// true when a decode over these pools expands quantised codes on chip
+bool quantised_pools(const DecodeParams &p, bool page_fmt_given) {
+  if (page_fmt_given)
+    return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4] || p.k_pool[CFR_FMT_FP8];
+  return is_quantised(p.uniform_fmt);
+}
 
 int target_splits(int sms, int hkv, int per_sm = kItemsPerSmMixed) {
   const long long items = static_cast<long long>(per_sm) * sms;
@@ -307,8 +319,16 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
 
   DeviceInfo di;
   if (!device_info(&di)) return CFR_ERR_CUDA;
-  const int target =
-      target_splits(di.sms, kv->num_kv_heads, page_fmt ? kItemsPerSmMixed : kItemsPerSm);
+  p.q = q;
+  p.q_fmt = q_fmt;
+  p.page_fmt = page_fmt;
+  p.uniform_fmt = uniform_fmt;
+  const bool use_tc = tc_supported(p, page_fmt != nullptr);
+  const bool use_f32 = !use_tc && f32_supported(p, page_fmt != nullptr);
+  const int per_sm = use_tc && !quantised_pools(p, page_fmt != nullptr) ? kItemsPerSmClaimed
+                     : page_fmt                                          ? kItemsPerSmMixed
+                                                                         : kItemsPerSm;
+  const int target = target_splits(di.sms, kv->num_kv_heads, per_sm);
   WsLayout w;
   if (!ws_layout(batch, rows, kv->head_dim, max_pages, target, &w)) return CFR_ERR_OVERFLOW;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return CFR_ERR_WORKSPACE;
@@ -318,11 +338,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   uint32_t *item_ctr = reinterpret_cast<uint32_t *>(ws + w.header + kItemCtrOffset);
   int32_t *split_off = reinterpret_cast<int32_t *>(ws + w.split_off);
   int32_t *splits = reinterpret_cast<int32_t *>(ws + w.splits);
-  p.q = q;
-  p.q_fmt = q_fmt;
   p.page_table = page_table;
-  p.page_fmt = page_fmt;
-  p.uniform_fmt = uniform_fmt;
   p.seq_lens = seq_lens;
   p.slopes = alibi_slopes;
   p.part_acc = reinterpret_cast<float *>(ws + w.part_acc);
@@ -341,8 +357,6 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.window = window;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool use_tc = tc_supported(p, page_fmt != nullptr);
-  const bool use_f32 = !use_tc && f32_supported(p, page_fmt != nullptr);
   if (!use_tc && !use_f32) {
     p.pitch = widest_row(kv, page_fmt, uniform_fmt);
     p.stages = cc_stages(p.D, cc_group_tile(p.gmax), p.pitch, di.smem_optin);
