@@ -159,9 +159,12 @@ cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
  * cfr_paged_decode split into its three stream-ordered launches, for timing
  * one launch at a time (CUDA events between calls).  Same arguments and checks
  * as cfr_paged_decode; `phases` selects which launches are enqueued.  A call
- * without CFR_PHASE_SCHEDULE relies on the workspace still holding the schedule
- * of an earlier call with the same seq_lens, batch and sizes; a call without
- * CFR_PHASE_DECODE merges the partials already in the workspace.
+ * without CFR_PHASE_SCHEDULE relies on the workspace still holding what an
+ * earlier call with the same arguments (all but q, out and lse) left there: the
+ * split schedule, and the work-item counter that the schedule launch zeroes and
+ * every completed decode launch leaves at zero.  The split count depends on the
+ * pools and formats, not only on the sizes.  A call without CFR_PHASE_DECODE
+ * merges the partials already in the workspace.
  * cfr_paged_decode(...) == cfr_paged_decode_phases(..., CFR_PHASE_ALL).
  */
 cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
@@ -189,8 +192,9 @@ cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_po
  * window_tokens >= 1 (CFR_ERR_INVALID_ARG otherwise).  With
  * sink_tokens + window_tokens >= n_b the sequence is attended in full.
  * `phases` selects launches as for cfr_paged_decode_phases (CFR_PHASE_ALL for
- * one whole step); a call without CFR_PHASE_SCHEDULE needs the schedule of an
- * earlier call with the same seq_lens, sizes, sink_tokens and window_tokens.
+ * one whole step); a call without CFR_PHASE_SCHEDULE needs the workspace of an
+ * earlier call with the same arguments (all but q, out and lse), including
+ * sink_tokens and window_tokens.
  */
 cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
                                         const int32_t *page_table, int32_t max_pages,
