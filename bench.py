@@ -3,8 +3,12 @@
 every (sequence, query head) of the workload (schedule + decode + merge).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload cfr|tiny|gqa|tiered|alibi1m|demote]
+                    [--workload alibi1m|cfr|tiny|gqa|tiered|demote] [--context N]
                     [--queries Q] [--sink S --window W]
+    python bench.py --record-traffic NCU_CSV --workload W [--context N]
+
+The default workload is the largest single-GPU one: 1,048,576 tokens of a
+64-query / 8-kv-head bf16 cache with ALiBi (4 GiB of K/V).
 
 Prints one JSON line (rank 0).  `value` is the effective KV-read bandwidth
 (algorithmic K/V bytes of all ranks / step time, GB/s) with every input resident
@@ -46,7 +50,11 @@ sys.path.insert(0, ROOT)
 from paged_long_context_b200 import accounting, binding, demote_workload, synth  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "traffic.json")
+# the kernel sources whose code a traffic record is valid for
+DECODE_SOURCES = ["cfr_decode_tc.cu", "cfr_decode_f32.cu", "cfr_decode_cc.cu", "cfr_common.cuh",
+                  "cfr_tmap.cuh", "cfr_tmap.cu"]
+DEMOTE_SOURCES = ["cfr_demote.cu", "cfr_common.cuh"]
 
 
 def parse():
@@ -55,7 +63,13 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="cfr", choices=sorted(synth.WORKLOADS) + ["demote"])
+    ap.add_argument("--workload", default="alibi1m", choices=sorted(synth.WORKLOADS) + ["demote"])
+    ap.add_argument("--context", type=int, default=None,
+                    help="cut every sequence to CONTEXT tokens (the same shape, smaller)")
+    ap.add_argument("--record-traffic", default=None, metavar="NCU_CSV",
+                    help="store the DRAM traffic of the decode kernel from an ncu --csv "
+                         "capture of this workload (at --context, scaled to the full size) "
+                         "in profiles/traffic.json, then exit")
     ap.add_argument("--sink", type=int, default=0,
                     help="with --window: attend to the first SINK tokens of each sequence too")
     ap.add_argument("--window", type=int, default=0,
@@ -209,25 +223,82 @@ def kernel_source_digest(files=None) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(summary: str, key: str):
-    """DRAM bytes (read + write) from a committed ncu summary under profiles/, only
-    when the profiled kernel's sources (listed in the summary) are unchanged since
-    the capture."""
-    name = os.path.join(PROFILE_TRAFFIC, summary)
-    if not os.path.exists(name):
+def traffic_record(key: str):
+    """The ncu DRAM figures of one kernel on one workload from profiles/traffic.json,
+    only when the kernel's sources are unchanged since the capture (else None)."""
+    if not os.path.exists(TRAFFIC_JSON):
         return None
-    vals = {}
-    for line in open(name):
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip()
-    files = [f.strip() for f in vals.get("kernel_sources", "").split(",") if f.strip()]
-    if not files or vals.get("kernel_source_digest") != kernel_source_digest(files):
+    rec = json.load(open(TRAFFIC_JSON)).get(key)
+    if not rec or rec.get("kernel_source_digest") != kernel_source_digest(rec["kernel_sources"]):
         return None
-    try:
-        return int(vals[key])
-    except (KeyError, ValueError):
-        return None
+    return rec
+
+
+_UNITS = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+          "nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6, "%": 1.0, "": 1.0}
+
+
+def ncu_csv_metrics(path: str, kernel_regex: str):
+    """Per-launch metric values (bytes, microseconds, percent) of the launches whose
+    kernel name matches, from `ncu --metrics ... --csv --log-file path`."""
+    import csv
+    launches = {}
+    lines = [l for l in open(path) if l.startswith('"')]
+    for row in csv.DictReader(lines):
+        if not re.search(kernel_regex, row.get("Kernel Name", "")):
+            continue
+        unit = row.get("Metric Unit", "").strip().lower()
+        val = float(row["Metric Value"].replace(",", "")) * _UNITS.get(unit, 1.0)
+        launches.setdefault(row["ID"], {"kernel": row["Kernel Name"]})[row["Metric Name"]] = val
+    return list(launches.values())
+
+
+def record_traffic(args):
+    """Writes the decode (or demotion) kernel's DRAM figures from an ncu CSV into
+    profiles/traffic.json under this workload's key, scaled from the captured size
+    to the full workload by the K/V bytes (DRAM traffic of these kernels grows in
+    proportion to the tokens read)."""
+    demote = args.workload == "demote"
+    regex = r"demote_kernel" if demote else r"decode_kernel"
+    rows = ncu_csv_metrics(args.record_traffic, regex)
+    if not rows:
+        raise SystemExit(f"no {regex} launch in {args.record_traffic}")
+    r = rows[-1]
+    rd, wr = r["dram__bytes_read.sum"], r["dram__bytes_write.sum"]
+    scale = 1.0
+    if demote:
+        # a demotion step is two launches (int4 and int8 destinations): the
+        # capture holds whole steps, and the record is per step
+        steps = max(1, len(rows) // 2)
+        rd = sum(x["dram__bytes_read.sum"] for x in rows) / steps
+        wr = sum(x["dram__bytes_write.sum"] for x in rows) / steps
+    elif args.context is not None:
+        # K/V traffic grows with the tokens read; the workload's lengths come from
+        # its shape alone (no cache is generated for this)
+        spec = synth.WORKLOADS[args.workload][0]()
+        if not spec.seq_lens:
+            raise SystemExit("--context scaling needs a workload of fixed lengths")
+        scale = sum(spec.seq_lens) / (args.context * spec.batch)
+    rec = {
+        "kernel": r["kernel"].split("(")[0],
+        "workload": args.workload,
+        "captured_context": args.context,
+        "scale_to_workload": round(scale, 6),
+        "dram_bytes_read_per_launch": int(round(rd * scale)),
+        "dram_bytes_write_per_launch": int(round(wr * scale)),
+        "dram_bytes_per_launch": int(round((rd + wr) * scale)),
+        "dram_throughput_pct_of_peak_sustained_elapsed":
+            r.get("dram__throughput.avg.pct_of_peak_sustained_elapsed"),
+        "captured_gpu_time_us": r.get("gpu__time_duration.sum"),
+        "kernel_sources": DEMOTE_SOURCES if demote else DECODE_SOURCES,
+    }
+    rec["kernel_source_digest"] = kernel_source_digest(rec["kernel_sources"])
+    db = json.load(open(TRAFFIC_JSON)) if os.path.exists(TRAFFIC_JSON) else {}
+    db[args.workload] = rec
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(db, f, indent=1, sort_keys=True)
+        f.write("\n")
+    print(json.dumps(rec))
 
 
 def dtype_name(case) -> str:
@@ -294,7 +365,8 @@ def cpu_baseline(case, budget_s: float, host=None, sink: int = 0, window: int = 
 
 def run_ours(args, dist):
     dev = torch.device("cuda", dist.local)
-    case = synth.workload(args.workload, device=dev, num_queries=args.queries)
+    case = synth.workload(args.workload, device=dev, num_queries=args.queries,
+                          context=args.context)
     sw = (args.sink, args.window) if args.window > 0 else None
     acct = accounting.step_bytes(case, args.sink, args.window)
     kv_bytes = acct["kv"] + acct["scales"]
@@ -434,9 +506,11 @@ def run_ours(args, dist):
 
     peak, peak_kind = measured_peaks()
     achieved = acct["total"] / (kern_ms_max * 1e-3) / 1e9
-    # the committed capture is of the plain decode (no subset, one query per sequence)
-    traffic = (profiled_traffic(f"decode_kernel_{args.workload}.md", "dram_bytes_per_launch")
-               if sw is None and args.queries == 1 else None)
+    # the committed capture is of the plain decode (no subset, one query per
+    # sequence) at the workload's full size
+    rec = (traffic_record(args.workload)
+           if sw is None and args.queries == 1 and args.context is None else None)
+    traffic = rec["dram_bytes_per_launch"] if rec else None
     world = dist.world
     value = world * kv_bytes / (step_ms_max * 1e-3) / 1e9
     res = {
@@ -458,6 +532,10 @@ def run_ours(args, dist):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_kind": peak_kind,
+                     "ncu_dram_throughput_pct": (
+                         rec["dram_throughput_pct_of_peak_sustained_elapsed"] if rec else None),
+                     "traffic_source": ("profiles/traffic.json (ncu, kernel sources unchanged)"
+                                        if rec else None),
                      "kernel_us": round(kern_ms_max * 1e3, 2),
                      "kernel_us_median": round(statistics.median(kern_times) * 1e3, 2),
                      "kernel_us_min": round(min(kern_times) * 1e3, 2),
@@ -477,7 +555,8 @@ def run_reference(args, dist):
     """The fp64 CPU oracle, as it stands, timed on the host cores (rank 0 only)."""
     import oracle
     oracle.build()
-    case = synth.workload(args.workload, device="cpu", num_queries=args.queries)
+    case = synth.workload(args.workload, device="cpu", num_queries=args.queries,
+                          context=args.context)
     pairs = [(b, h) for b in range(case.batch) for h in range(case.num_q_heads * case.num_queries)]
     sub = dict(sink_tokens=args.sink, window_tokens=args.window)
     threads = oracle.default_threads()
@@ -626,7 +705,8 @@ def run_demote(args, dist):
 
     peak, peak_kind = measured_peaks()
     achieved = acct["total"] / (launch_ms_max * 1e-3) / 1e9
-    traffic = profiled_traffic("demote_kernel_demote.md", "dram_bytes_per_step")
+    rec = traffic_record("demote")
+    traffic = rec["dram_bytes_per_launch"] if rec else None   # per step (both launches)
     world = dist.world
     res = {
         "metric": DEMOTE_METRIC,
@@ -673,6 +753,9 @@ def run_reference_demote(args):
 
 def main():
     args = parse()
+    if args.record_traffic:
+        record_traffic(args)
+        return 0
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:

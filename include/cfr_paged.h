@@ -76,6 +76,11 @@ typedef enum {
 #define CFR_DEVERR_SEQ_LEN 0x4u   /* seq_lens[b] < 1 or > max_pages * page_tokens */
 #define CFR_DEVERR_POOL 0x8u      /* page refers to a format whose pool (or scales) is NULL */
 #define CFR_DEVERR_TIMEOUT 0x10u  /* a bounded on-device wait gave up; outputs undefined */
+#define CFR_DEVERR_SCHEDULE 0x20u /* a call without CFR_PHASE_SCHEDULE found a split schedule in
+                                     the workspace that does not fit its own arguments (more
+                                     splits than its arrays hold, or a split outside its batch or
+                                     page table); the extra or bad splits were skipped and the
+                                     outputs are not the attention result */
 
 /*
  * The paged K/V pools of one layer.  One pool per storage format; a page's
@@ -164,7 +169,11 @@ cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
  * split schedule, and the work-item counter that the schedule launch zeroes and
  * every completed decode launch leaves at zero.  The split count depends on the
  * pools and formats, not only on the sizes.  A call without CFR_PHASE_DECODE
- * merges the partials already in the workspace.
+ * merges the partials already in the workspace.  A call that breaks this rule
+ * gets wrong outputs but no write outside its own workspace: the decode and
+ * merge launches cap the split count and the split offsets at the capacity that
+ * this call's workspace size provides, skip splits that name a sequence or page
+ * outside this call's batch and page table, and set CFR_DEVERR_SCHEDULE.
  * cfr_paged_decode(...) == cfr_paged_decode_phases(..., CFR_PHASE_ALL).
  */
 cfr_status cfr_paged_decode_phases(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
@@ -407,6 +416,27 @@ cfr_status cfr_append_kv(const cfr_kv_pool *kv, const int32_t *page_table, int32
 int32_t cfr_paged_decode_path(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_pages,
                               const uint8_t *page_fmt, int32_t uniform_fmt,
                               int32_t num_q_heads, const int32_t *head_map);
+
+/*
+ * Diagnostic of the device-side failure handling (the pages have no
+ * counterpart; it exists so that the bounded waits can be tested).  Every
+ * wait of the decode kernels on an on-chip barrier gives up after a cycle limit
+ * (about 4e9 SM cycles, two seconds at the top clock), ORs CFR_DEVERR_TIMEOUT
+ * into *err_word and lets the kernel return, so a stalled pipeline ends as an
+ * error bit the host reads rather than a hung GPU.  This call launches one
+ * thread that runs that same wait on a shared-memory barrier, with a limit of
+ * limit_cycles SM cycles, after arriving on the barrier itself when `arrive` is
+ * non-zero and not arriving at all otherwise.
+ *
+ *  limit_cycles  1 .. 4e9 (CFR_ERR_INVALID_ARG otherwise).
+ *  err_word      device uint32 or NULL; gets CFR_DEVERR_TIMEOUT when the wait gives up.
+ *  result        device uint32 or NULL; written 1 when the barrier phase completed,
+ *                0 when the wait gave up.
+ * The kernel holds no copy or tensor-core operation in flight, so a wait that
+ * gives up leaves the context usable.
+ */
+cfr_status cfr_wait_probe(int64_t limit_cycles, int32_t arrive, uint32_t *err_word,
+                          uint32_t *result, void *stream);
 
 /* Static description of a status code. */
 const char *cfr_status_str(cfr_status status);

@@ -21,6 +21,8 @@ CFR_OK = 0
 STATUS = {0: "CFR_OK", 1: "CFR_ERR_INVALID_ARG", 2: "CFR_ERR_UNSUPPORTED", 3: "CFR_ERR_OVERFLOW",
           4: "CFR_ERR_PAGE_INDEX", 5: "CFR_ERR_CUDA", 6: "CFR_ERR_TIMEOUT", 7: "CFR_ERR_WORKSPACE"}
 DEVERR_PAGE_ID, DEVERR_PAGE_FMT, DEVERR_SEQ_LEN, DEVERR_POOL, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+DEVERR_SCHEDULE = 0x20
+STATUS_CODES = {v: k for k, v in STATUS.items()}
 PATH_CUDA_CORE, PATH_TENSOR_CORE, PATH_F32_TMA = 1, 2, 3
 
 # every exported symbol the header declares
@@ -28,9 +30,22 @@ EXPORTS = ["cfr_paged_decode_workspace_size", "cfr_paged_decode", "cfr_paged_dec
            "cfr_merge_partials",
            "cfr_schedule_splits", "cfr_gather_pages", "cfr_paged_decode_path", "cfr_status_str",
            "cfr_paged_decode_static_workspace", "cfr_demote_pages", "cfr_append_kv",
-           "cfr_paged_decode_sink_window", "cfr_paged_decode_multi"]
+           "cfr_paged_decode_sink_window", "cfr_paged_decode_multi", "cfr_wait_probe"]
 FMT_COUNT = 5
-STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def _header_static_workspace_bytes() -> int:
+    """CFR_STATIC_WORKSPACE_BYTES as the header defines it (one source of truth)."""
+    import re
+    hdr = os.path.join(os.path.dirname(_PKG), "include", "cfr_paged.h")
+    m = re.search(r"#define\s+CFR_STATIC_WORKSPACE_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)",
+                  open(hdr).read())
+    if not m:
+        raise RuntimeError("CFR_STATIC_WORKSPACE_BYTES not found in include/cfr_paged.h")
+    return int(m.group(1)) << int(m.group(2))
+
+
+STATIC_WORKSPACE_BYTES = _header_static_workspace_bytes()
 
 
 class CfrError(RuntimeError):
@@ -94,6 +109,8 @@ def lib():
         L.cfr_append_kv.restype = ctypes.c_int
         L.cfr_append_kv.argtypes = [ctypes.POINTER(KvPool), _VP, _I32, _VP, _I32, _VP, _I32,
                                     _VP, _VP, _I32, _VP, _VP]
+        L.cfr_wait_probe.restype = ctypes.c_int
+        L.cfr_wait_probe.argtypes = [_I64, _I32, _VP, _VP, _VP]
         L.cfr_status_str.restype = ctypes.c_char_p
         L.cfr_status_str.argtypes = [ctypes.c_int]
         _lib = L
@@ -253,6 +270,13 @@ def paged_decode_static_workspace(case, out, lse=None, err=None, stream=None) ->
         _p(case.seq_lens), case.batch, _p(case.page_fmt), case.uniform_fmt, case.num_q_heads, hmp,
         _p(case.alibi_slopes), float(case.softmax_scale), _p(out), _p(lse), _p(err),
         _stream(stream)))
+
+
+def wait_probe(limit_cycles: int, arrive: bool, err=None, result=None, stream=None) -> int:
+    """cfr_wait_probe: the decode kernels' bounded on-chip wait, run once with a
+    short cycle limit on a barrier that is (arrive) or is not arrived on."""
+    return int(lib().cfr_wait_probe(int(limit_cycles), 1 if arrive else 0, _p(err), _p(result),
+                                    _stream(stream)))
 
 
 def demote_pages(pool: KvPool, src_fmt: int, dst_fmt: int, dst_k, dst_v, dst_scales,

@@ -12,8 +12,8 @@ void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, i
                      int max_splits, int32_t *num_splits, uint32_t *item_ctr, uint32_t *err,
                      cudaStream_t stream);
 void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
-                  const int32_t *split_off, int batch, int Hq, int D, float *out, float *lse,
-                  cudaStream_t stream);
+                  const int32_t *split_off, int batch, int Hq, int D, int max_splits, float *out,
+                  float *lse, uint32_t *err, cudaStream_t stream);
 void launch_gather(const DecodeParams &p, int b, int g, int n_tokens, void *k_out, void *v_out,
                    long long pitch, cudaStream_t stream);
 cudaError_t launch_decode_cc(const DecodeParams &p, int grid, cudaStream_t stream);
@@ -346,6 +346,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.part_l = reinterpret_cast<float *>(ws + w.part_l);
   p.splits = splits;
   p.num_splits = num_splits;
+  p.max_splits = w.max_splits;
   p.item_ctr = item_ctr;
   p.err = err_word;
   p.batch = batch;
@@ -374,8 +375,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
     if (e != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_MERGE) {
-    launch_merge(p.part_acc, p.part_m, p.part_l, split_off, batch, rows, kv->head_dim, out, lse,
-                 s);
+    launch_merge(p.part_acc, p.part_m, p.part_l, split_off, batch, rows, kv->head_dim,
+                 w.max_splits, out, lse, err_word, s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   return CFR_OK;
@@ -438,8 +439,8 @@ cfr_status cfr_merge_partials(const float *part_acc, const float *part_m, const 
   if (head_dim != 64 && head_dim != 128) return CFR_ERR_UNSUPPORTED;
   if (!aligned(part_acc, 16) || !aligned(out, 16)) return CFR_ERR_INVALID_ARG;
   if (static_cast<long long>(batch) * num_q_heads > INT_MAX) return CFR_ERR_OVERFLOW;
-  launch_merge(part_acc, part_m, part_l, split_off, batch, num_q_heads, head_dim, out, lse,
-               static_cast<cudaStream_t>(stream));
+  launch_merge(part_acc, part_m, part_l, split_off, batch, num_q_heads, head_dim, INT_MAX, out,
+               lse, nullptr, static_cast<cudaStream_t>(stream));
   return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
 }
 

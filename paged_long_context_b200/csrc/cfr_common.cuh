@@ -38,6 +38,7 @@ struct DecodeParams {
   float *part_l;        // [S][Hq]
   const int32_t *splits;     // [S][3]: b, page begin, page end
   const int32_t *num_splits; // [0] = S
+  int max_splits;            // capacity of this call's split arrays (part_*, splits)
   uint32_t *item_ctr;   // [0] work items claimed past the first per CTA, [1] CTAs finished; or null
   uint32_t *err;
   int q_fmt, uniform_fmt;
@@ -111,16 +112,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
 // Waits for the phase of `parity` to complete.  Returns false (and flags the
-// error word) when the wait exceeded kWaitLimitCycles; `*timed_out` then stays
-// set so that callers stop waiting on anything else.
+// error word) when the wait exceeded `limit` cycles (kWaitLimitCycles unless a
+// caller asks for less); `*timed_out` then stays set so that callers stop
+// waiting on anything else.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *err,
-                                          bool *timed_out) {
+                                          bool *timed_out,
+                                          long long limit = kWaitLimitCycles) {
   if (*timed_out) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t spins = 1;; ++spins) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((spins & 63u) == 0 && clock64() - t0 > kWaitLimitCycles) {
+    if ((spins & 63u) == 0 && clock64() - t0 > limit) {
       set_err(err, CFR_DEVERR_TIMEOUT);
       *timed_out = true;
       return false;
@@ -301,6 +304,37 @@ __device__ __forceinline__ void page_cache_reset(PageCacheT<N> &pc, int lane) {
     pc.count = 0;
   }
   __syncwarp();
+}
+
+// Number of splits of the schedule in the workspace, capped at the capacity of
+// this call's split arrays.  The schedule launch of the same call never writes
+// more; a larger (or negative) count can only come from a decode-only call on a
+// workspace scheduled with other arguments, and sets CFR_DEVERR_SCHEDULE (when
+// `report`) instead of letting the partial writes run past their arrays.
+__device__ __forceinline__ int schedule_split_count(const DecodeParams &p, bool report) {
+  const int s = p.num_splits[0];
+  if (s >= 0 && s <= p.max_splits) return s;
+  if (report) set_err(p.err, CFR_DEVERR_SCHEDULE);
+  return s < 0 ? 0 : p.max_splits;
+}
+
+// Split `slot` of the schedule: sequence b and its page range [pb, pe).  An
+// entry that is not a page range of this call's batch (again only possible on a
+// workspace scheduled with other arguments) becomes an empty range of sequence 0
+// and sets CFR_DEVERR_SCHEDULE, so no page-table row or sequence length outside
+// the call's arrays is read.
+struct SplitRange {
+  int b, pb, pe;
+};
+__device__ __forceinline__ SplitRange split_at(const DecodeParams &p, int slot) {
+  SplitRange r{p.splits[3 * slot], p.splits[3 * slot + 1], p.splits[3 * slot + 2]};
+  if (r.b < 0 || r.b >= p.batch || r.pb < 0 || r.pe < r.pb || r.pe > p.max_pages) {
+    set_err(p.err, CFR_DEVERR_SCHEDULE);
+    r.b = 0;
+    r.pb = 0;
+    r.pe = 0;
+  }
+  return r;
 }
 
 // Work item -> (split slot, kv head).  Items are numbered split-fastest, so the

@@ -220,8 +220,9 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
   const int P = p.P;
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, p.num_splits[0], slot, g);
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += CC_T) {
@@ -313,8 +314,9 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, p.num_splits[0], slot, g);
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
@@ -517,7 +519,8 @@ __global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_c
   griddep_launch_dependents();
   __syncthreads();
   griddep_wait();  // the split schedule comes from the previous kernel
-  const long long nitems = static_cast<long long>(p.num_splits[0]) * p.Hkv;
+  const long long nitems =
+      static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.Hkv;
   bool timed_out = false;
   if (threadIdx.x >= CC_WARPS * 32) {
     if (threadIdx.x == CC_WARPS * 32) cc_producer<D>(p, L, nitems, &timed_out);

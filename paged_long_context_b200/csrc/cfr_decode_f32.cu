@@ -161,8 +161,9 @@ __device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_
   page_cache_reset(pc, lane);
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, p.num_splits[0], slot, g);
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += C::T) {
@@ -196,8 +197,9 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, p.num_splits[0], slot, g);
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
@@ -426,7 +428,8 @@ __global__ void __launch_bounds__(F_THREADS, 1)
   griddep_launch_dependents();
   __syncthreads();
   griddep_wait();  // the split schedule comes from the previous kernel
-  const long long nitems = static_cast<long long>(p.num_splits[0]) * p.Hkv;
+  const long long nitems =
+      static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.Hkv;
   bool timed_out = false;
   if (threadIdx.x >= F_WARPS * 32) {
     f32_producer<D>(p, maps, S.full, S.empty, S.meta, ring, S.pc, nitems, &timed_out);

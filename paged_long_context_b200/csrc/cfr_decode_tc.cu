@@ -373,6 +373,18 @@ __device__ __forceinline__ int tc_read_item_wg(TcCtx<NCOL, INTP, FEAT> &c, int k
   return *reinterpret_cast<volatile int *>(bc);
 }
 
+// true when item `it` has at least one tile.  Every split of a schedule this
+// call wrote does; an item that split_at emptied (a foreign schedule) has none,
+// and then neither writes nor waits for a query operand, so the q_full phases
+// of the softmax warpgroup and the QK issuer stay paired.
+template <int NCOL, bool INTP, int FEAT>
+__device__ __forceinline__ bool tc_item_has_tiles(const TcCtx<NCOL, INTP, FEAT> &c, long long it) {
+  int slot, g;
+  item_coords(it, c.nsplit, slot, g);
+  const SplitRange sr = split_at(c.p, slot);
+  return sr.pb * c.p.P < min(c.p.seq_lens[sr.b], sr.pe * c.p.P);
+}
+
 // Per-kernel constants of a producer warp: which formats have their pools (and
 // scales) and the geometry of a tile's copy boxes.
 struct TcProdGeom {
@@ -527,7 +539,8 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int pk)
     if (item < 0) break;
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     int pg0 = pb, tin0 = 0;
@@ -569,7 +582,8 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     (void)g;
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int tok_end = min(p.seq_lens[b], pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       // elected bounded wait; the outcome slot is per stage, so a slow reader can
@@ -705,15 +719,18 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   int stage = 0;
   uint32_t phase = 0;
   long long tc = 0;
+  int q_items = 0;  // items with tiles so far: one q_full phase each
   for (int item_k = 0; !*timed_out; ++item_k) {
     const int item = tc_read_item(c, item_k, timed_out, false);
     if (item < 0) break;
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     (void)g;
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int tok_end = min(p.seq_lens[b], pe * P);
-    if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(item_k & 1), p.err, timed_out)) break;
+    if (pb * P >= tok_end) continue;
+    if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(q_items++ & 1), p.err, timed_out)) break;
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       if (!mbar_wait(&c.S.op_full[stage], phase, p.err, timed_out)) break;
       if (!mbar_wait(&c.S.s_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err,
@@ -761,7 +778,8 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
     (void)g;
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int tok_end = min(p.seq_lens[b], pe * P);
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       const int ob = static_cast<int>(tc % Cfg::O_BUFS);
@@ -823,7 +841,7 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT> &c, long long
   {
     int slot, g;
     item_coords(it, c.nsplit, slot, g);
-    const int b = p.splits[3 * slot];
+    const int b = split_at(p, slot).b;
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
     for (int idx = tsm; idx < NCOL * 16; idx += 128) {
       const int n = idx >> 4, ch = idx & 15;  // row n, 8-element chunk ch of 16
@@ -900,11 +918,12 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   for (int item = tc_read_item_wg(c, 0, 2, tsm, timed_out); item >= 0; ++k) {
     int slot, g;
     item_coords(item, c.nsplit, slot, g);
-    const int b = p.splits[3 * slot], pb = p.splits[3 * slot + 1], pe = p.splits[3 * slot + 2];
+    const SplitRange sr = split_at(p, slot);
+    const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
-    if (!q_ready) tc_write_q(c, item, tsm, lane);
+    if (!q_ready && pb * P < tok_end) tc_write_q(c, item, tsm, lane);
     q_ready = false;
     nxt_read = false;
 
@@ -1026,7 +1045,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
         // last QK product has been read
         nxt = tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
         nxt_read = true;
-        if (nxt >= 0) {
+        if (nxt >= 0 && tc_item_has_tiles(c, nxt)) {
           tc_write_q(c, nxt, tsm, lane);
           q_ready = true;
         }
@@ -1130,8 +1149,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   griddep_wait();  // the split schedule comes from the previous kernel (returns at once
                    // when the launch did not overlap it)
 
+  const int nsplit = schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0);
   TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::q, smem + L::pbuf,
-                      static_cast<long long>(p.num_splits[0]) * p.Hkv, p.num_splits[0]};
+                            static_cast<long long>(nsplit) * p.Hkv, nsplit};
   bool timed_out = false;
   if (warp == 0 || warp == TC_PROD2_WARP) {
     tc_producer<NCOL, INTP, FEAT>(c, &timed_out, warp == 0 ? 0 : 1);

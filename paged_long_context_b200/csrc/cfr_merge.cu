@@ -25,7 +25,7 @@ template <int D>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const float *__restrict__ part_acc, const float *__restrict__ part_m,
     const float *__restrict__ part_l, const int32_t *__restrict__ split_off, int batch, int Hq,
-    float *__restrict__ out, float *__restrict__ lse) {
+    int max_splits, float *__restrict__ out, float *__restrict__ lse, uint32_t *err) {
   __shared__ float w_s[kMergeChunk];
   __shared__ float red[kMergeThreads / 32];
   __shared__ float gsum[kMergeGroups][D];
@@ -34,8 +34,15 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   const long long pair = blockIdx.x;
   if (pair >= static_cast<long long>(batch) * Hq) return;
   const int b = static_cast<int>(pair / Hq), h = static_cast<int>(pair % Hq);
-  const int s0 = split_off[b], s1 = split_off[b + 1];
+  int s0 = split_off[b], s1 = split_off[b + 1];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (s0 < 0 || s1 < s0 || s1 > max_splits) {
+    // offsets that do not index this call's partial arrays (a merge-only call on
+    // a workspace scheduled with other arguments): merge only what is in range
+    if (tid == 0) set_err(err, CFR_DEVERR_SCHEDULE);
+    s0 = min(max(s0, 0), max_splits);
+    s1 = min(max(s1, s0), max_splits);
+  }
 
   // M = max over non-empty splits
   float M = -INFINITY;
@@ -112,17 +119,17 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
 }
 
 void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
-                  const int32_t *split_off, int batch, int Hq, int D, float *out, float *lse,
-                  cudaStream_t stream) {
+                  const int32_t *split_off, int batch, int Hq, int D, int max_splits, float *out,
+                  float *lse, uint32_t *err, cudaStream_t stream) {
   const long long pairs = static_cast<long long>(batch) * Hq;
   if (pairs <= 0) return;
   const unsigned blocks = static_cast<unsigned>(pairs);
   if (D == 64)
     (void)launch_after_previous(merge_kernel<64>, dim3(blocks), dim3(kMergeThreads), 0, stream,
-                                part_acc, part_m, part_l, split_off, batch, Hq, out, lse);
+                                part_acc, part_m, part_l, split_off, batch, Hq, max_splits, out, lse, err);
   else
     (void)launch_after_previous(merge_kernel<128>, dim3(blocks), dim3(kMergeThreads), 0, stream,
-                                part_acc, part_m, part_l, split_off, batch, Hq, out, lse);
+                                part_acc, part_m, part_l, split_off, batch, Hq, max_splits, out, lse, err);
 }
 
 }  // namespace cfr

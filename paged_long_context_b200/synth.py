@@ -446,14 +446,19 @@ WORKLOADS = {
 }
 
 
-def workload(name: str, device="cpu", num_queries: int = 1) -> DecodeCase:
+def workload(name: str, device="cpu", num_queries: int = 1,
+             context: Optional[int] = None) -> DecodeCase:
     """One of the five page-shaped workloads, with its fixed seed (optionally with
-    several query tokens per sequence)."""
+    several query tokens per sequence, or with every sequence cut to `context`
+    tokens: the same shape at a smaller size, e.g. for a profiler capture)."""
     fn, seed = WORKLOADS[name]
     spec = fn()
     if num_queries > 1:
         spec = dataclasses.replace(spec, num_queries=num_queries,
                                    name=f"{spec.name}_q{num_queries}")
+    if context is not None:
+        spec = dataclasses.replace(spec, seq_lens=[int(context)] * spec.batch, len_range=None,
+                                   name=f"{spec.name}_n{int(context)}")
     return make_case(spec, seed, device)
 
 

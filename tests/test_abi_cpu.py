@@ -298,3 +298,10 @@ def test_multi_query_rejects(lib):
     assert call(4, hq=8, hkv=1) == UNSUP          # 8 heads x 4 queries = 32 rows per kv head
     assert call(2, hq=130, hkv=130) == UNSUP      # 260 query rows per sequence
     assert call(2, phases=0) == INVALID
+
+
+def test_wait_probe_rejects_limits_out_of_range(lib):
+    # rejected on the host, before any launch
+    assert binding.wait_probe(0, False) == 1
+    assert binding.wait_probe(-5, True) == 1
+    assert binding.wait_probe(4_000_000_001, False) == 1

@@ -54,3 +54,54 @@ def test_phases_and_repeated_decode(name):
         assert int(bufs.err.item()) == 0
         assert torch.equal(bufs.out, out0)
         assert torch.equal(bufs.lse, lse0)
+
+
+FOREIGN = {
+    # tcgen05 path, bf16 pages, claimed items
+    "bf16": dict(d=128, fmt="bf16", q_fmt="bf16"),
+    # tcgen05 path, quantised tiers, fixed share
+    "tiered": dict(d=128, fmt="tiered", tiers=[(0.5, "i8"), (0.5, "bf16")], q_fmt="bf16", P=128),
+    # fp32 TMA kernel
+    "f32": dict(d=64, fmt="f32", q_fmt="f32", Hq=4, Hkv=4),
+    # general CUDA-core kernel (bf16 pages of head_dim 64)
+    "cc": dict(d=64, fmt="bf16", q_fmt="bf16"),
+}
+
+
+@pytest.mark.parametrize("name", list(FOREIGN))
+def test_decode_only_call_on_a_foreign_schedule_stays_in_its_workspace(name):
+    """A decode-only call (no schedule launch) on a workspace that a call with
+    other arguments scheduled breaks the documented rule of split-phase calls.
+    The kernels must then cap the split count and skip foreign splits, report
+    CFR_DEVERR_SCHEDULE, and write nothing past the bytes this call was given."""
+    kw = dict(Hq=16, Hkv=4, P=16)
+    kw.update(FOREIGN[name])
+    P = kw.pop("P")
+    big = small_case(seed=21, B=8, P=P, lens=(8192,) * 8, **kw)
+    small = small_case(seed=22, B=1, P=P, lens=(4 * P,), **kw)
+    assert small.max_pages == 4
+    bb, sb = binding.DecodeBuffers(big), binding.DecodeBuffers(small)
+    ws_big, ws_small = bb.workspace.numel(), sb.workspace.numel()
+    assert ws_small < ws_big
+    arena = torch.zeros(ws_big + (1 << 20), dtype=torch.uint8, device="cuda")
+    bb.workspace = arena[:ws_big]
+    sb.workspace = arena[:ws_small]
+    assert binding.decode_path(small) == binding.decode_path(big)
+
+    assert binding.paged_decode_raw(big, bb) == binding.CFR_OK
+    torch.cuda.synchronize()
+    assert int(bb.err.item()) == 0
+    guard = arena[ws_small:].clone()
+
+    assert binding.paged_decode_raw(
+        small, sb, phases=binding.PHASE_DECODE | binding.PHASE_MERGE) == binding.CFR_OK
+    torch.cuda.synchronize()
+    assert int(sb.err.item()) & binding.DEVERR_SCHEDULE
+    assert torch.equal(arena[ws_small:], guard)
+
+    # the same call with its own schedule is clean and correct again
+    sb.err.zero_()
+    assert binding.paged_decode_raw(small, sb) == binding.CFR_OK
+    torch.cuda.synchronize()
+    assert int(sb.err.item()) == 0
+    check(small, sb.out.cpu(), sb.lse.cpu())
