@@ -235,7 +235,8 @@ def traffic_record(key: str):
 
 
 _UNITS = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
-          "nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6, "%": 1.0, "": 1.0}
+          "nsecond": 1e-3, "usecond": 1.0, "msecond": 1e3, "second": 1e6,
+          "ns": 1e-3, "us": 1.0, "ms": 1e3, "s": 1e6, "%": 1.0, "": 1.0}
 
 
 def ncu_csv_metrics(path: str, kernel_regex: str):

@@ -10,11 +10,22 @@
 // N = 16 (G <= 8) or 32 (G <= 16) columns: N/2 "hi" and N/2 "lo" columns, so that q
 // (fp32 or bf16) and the probabilities p enter the 16-bit MMA as hi + lo pairs
 // (about 16 significant bits for bf16, 22 for fp16), accumulated in fp32.
-// bf16 pages run bf16 MMAs; FP8 / int8 / int4 pages are expanded to fp16 codes
-// in shared memory (their codes are exact in fp16) and run fp16 MMAs; their per-page
-// K scale multiplies the scores, their V scale multiplies the tile's P.V
-// result, both in fp32 (ARGUS page, "Transient FP16 Reconstruction ... in GPU
-// SRAM": pages are expanded on chip only, attention runs at 16-bit).
+// bf16 pages run bf16 MMAs; FP8 pages are expanded to fp16 codes in shared
+// memory (every E4M3 value is exact in fp16) and run fp16 MMAs.  int8 / int4
+// pages take one of two routes:
+//  - IMMA variants (at most 4 query rows per kv head): int8 MMAs (kind::i8,
+//    int32 accumulators) on the codes themselves.  int8 tiles are loaded by TMA
+//    straight into the operand layout; int4 codes are widened to one byte per
+//    code (16 * code, exact).  The query enters as 4 signed digit columns per
+//    head, q * 127 / max|q| = d0 + d1/128 + d2/128^2 + d3/128^3, and the
+//    probabilities as 4 unsigned digit columns, p * 255 = e0 + e1/256 + e2/256^2
+//    + e3/256^3; every int32 column sum stays below 2^23, so the fp32
+//    recombination of the digit products loses only the usual fp32 rounding.
+//  - otherwise the codes are expanded to fp16 in shared memory (exact) and run
+//    fp16 MMAs like FP8 pages.
+// Per-page K scales multiply the scores and V scales the tile's P.V result, in
+// fp32 (ARGUS page, "Transient FP16 Reconstruction ... in GPU SRAM": pages are
+// expanded on chip only).
 //
 // Warp roles (384 threads, one CTA per SM, persistent over work items =
 // (split of a sequence, kv head)):
@@ -34,9 +45,11 @@
 //               and the exact fold acc = acc*2^(m_old-m_new) + O_tile of the
 //               previous tile (CFR-Atlas page, "exact folded online-softmax
 //               attention pass").
-//   warps 6-9   staging: FP8/int8/int4 rows -> fp16 operand rows; zeroes V rows of
+//   warps 6-9   staging: FP8/int8/int4 rows -> fp16 operand rows (int4 rows ->
+//               int8 rows in IMMA variants); zeroes V rows of 16-bit tiles for
 //               tokens that are not part of the input so stale or NaN bytes
-//               never meet a zero probability inside the MMA.
+//               never meet a zero probability inside the MMA (8-bit codes are
+//               always finite, and meet an exact zero digit).
 // Every mbarrier wait is bounded; on a timeout the error word is set, every
 // role leaves its loop, the MMA pipe is drained and TMEM is freed.
 //
@@ -79,8 +92,10 @@ struct TcMeta {
 };
 
 struct TcMaps {
-  CUtensorMap k;
+  CUtensorMap k;   // bf16 pool
   CUtensorMap v;
+  CUtensorMap k8;  // int8 pool (tiles loaded straight into the 8-bit operand layout)
+  CUtensorMap v8;
 };
 
 template <int NCOL, bool INTP>
@@ -89,6 +104,8 @@ struct TcCfg {
   // place, so the variant with quantised pools keeps the same three stages
   static constexpr int STAGES = 3;
   static constexpr int Q_BYTES = NCOL * 256;       // [NCOL rows][128 cols] 16-bit, 2 halves
+  // [NCOL rows][128 cols] int8 query digits (int8 MMAs, 16 columns only)
+  static constexpr int Q8_BYTES = (INTP && NCOL == 16) ? NCOL * 128 : 0;
   static constexpr int P_BYTES = NCOL * TC_T * 2;  // [128 tokens][NCOL] 16-bit
   static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
   static constexpr int TMEM_COLS = NCOL == 16 ? 128 : 256;  // S x2 + O x3 columns, power of two
@@ -111,7 +128,7 @@ struct TcSmem {
   int flag_st[3];
   TcMeta meta[3];
   alignas(16) float red_max[2][4][16];
-  alignas(16) float red_l[4][16];
+  alignas(16) float red_l[4][16];  // also the per-warp max|q_h| of the int8 query digits
   typename TcCfg<NCOL, INTP>::PageCache pc[TC_PRODUCERS];
 };
 
@@ -120,7 +137,8 @@ struct TcLayout {
   static constexpr size_t head = (sizeof(TcSmem<NCOL, INTP>) + 1023) / 1024 * 1024;
   static constexpr size_t op = head;
   static constexpr size_t q = op + TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_OP_BYTES);
-  static constexpr size_t pbuf = q + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::Q_BYTES);
+  static constexpr size_t q8 = q + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::Q_BYTES);
+  static constexpr size_t pbuf = q8 + static_cast<size_t>(TcCfg<NCOL, INTP>::Q8_BYTES);
   static constexpr size_t total = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
   static constexpr size_t launch_bytes = total + 1024;  // slack for 1024-byte alignment
 };
@@ -130,6 +148,14 @@ struct TcLayout {
 // instruction descriptor, kind::f16, fp32 accumulator, M = 128
 __host__ __device__ constexpr uint32_t tc_idesc(int ab_bf16, int a_mn, int b_mn, int n) {
   return (1u << 4) | (static_cast<uint32_t>(ab_bf16) << 7) | (static_cast<uint32_t>(ab_bf16) << 10) |
+         (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+         (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// instruction descriptor, kind::i8, s32 accumulator, M = 128: A signed 8-bit
+// codes, B signed (query digits) or unsigned (probability digits) 8-bit
+__host__ __device__ constexpr uint32_t tc_idesc_i8(int b_signed, int a_mn, int b_mn, int n) {
+  return (2u << 4) | (1u << 7) | (static_cast<uint32_t>(b_signed) << 10) |
          (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
          (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
 }
@@ -148,6 +174,15 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, 
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -240,7 +275,7 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 
 // ---- roles ------------------------------------------------------------------
 
-template <int NCOL, bool INTP, int FEAT>
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
 struct TcCtx {
   const DecodeParams &p;
   const TcMaps &maps;
@@ -248,7 +283,16 @@ struct TcCtx {
   uint8_t *op, *qop, *pop;
   long long nitems;
   int nsplit;
+  uint8_t *q8op;  // int8 query digits (IMMA variants)
 };
+
+// With IMMA, int8 and int4 tiles run kind::i8 MMAs on 8-bit operands: int8 codes
+// as stored, int4 codes widened to bytes (times 16, so that the sign needs no
+// extension), query and probability as base-128 / base-256 digit columns.
+template <bool IMMA>
+__device__ __forceinline__ bool tc_int_tile(int kind) {
+  return IMMA && (kind == KIND_I8 || kind == KIND_I4);
+}
 
 
 // Maximum over the 32 lanes of each of NV values per lane (NV a power of two,
@@ -307,21 +351,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 //    tiles (whose expansion sets the pace) and on subset decode the ring's
 //    per-item hand-off cost more than the balance gained, so those keep the
 //    fixed share.
-template <bool INTP, int FEAT>
+template <bool INTP, int FEAT, bool IMMA>
 __host__ __device__ constexpr bool tc_claimed_items() {
   return !INTP && FEAT != TC_FEAT_SUBSET;
 }
 
 // item k of the fixed share, or -1
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ int tc_fixed_item(const TcCtx<NCOL, INTP, FEAT> &c, int k) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ int tc_fixed_item(const TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k) {
   const long long it = static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
   return it < c.nitems ? static_cast<int>(it) : -1;
 }
 
 // producer warp 0 (all lanes): claims and publishes item k; returns it, or -1.
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ int tc_claim_item(TcCtx<NCOL, INTP, FEAT> &c, int k, bool *timed_out,
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ int tc_claim_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, bool *timed_out,
                                              int lane) {
   const int s = k & (TC_ITEM_RING - 1);
   int item = -1;
@@ -343,10 +387,10 @@ __device__ __forceinline__ int tc_claim_item(TcCtx<NCOL, INTP, FEAT> &c, int k, 
 // item k read by one thread (an MMA issuer) or by every lane of a warp
 // (producer warp 11; lane 0 waits and frees the slot); -1 past the last item
 // or when the wait gave up.
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ int tc_read_item(TcCtx<NCOL, INTP, FEAT> &c, int k, bool *timed_out,
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ int tc_read_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, bool *timed_out,
                                             bool warp_wide) {
-  if constexpr (!tc_claimed_items<INTP, FEAT>()) return tc_fixed_item(c, k);
+  if constexpr (!tc_claimed_items<INTP, FEAT, IMMA>()) return tc_fixed_item(c, k);
   const int s = k & (TC_ITEM_RING - 1);
   int item = -1;
   if (!warp_wide || (threadIdx.x & 31) == 0) {
@@ -363,10 +407,10 @@ __device__ __forceinline__ int tc_read_item(TcCtx<NCOL, INTP, FEAT> &c, int k, b
 // `bar` (2: softmax, 3: staging): thread t = 0 waits, reads and frees the slot,
 // and the barrier hands the value to all 128 threads, so they leave their loop
 // together even when the wait gave up (named barriers have no time limit).
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ int tc_read_item_wg(TcCtx<NCOL, INTP, FEAT> &c, int k, int bar, int t,
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ int tc_read_item_wg(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, int bar, int t,
                                                bool *timed_out) {
-  if constexpr (!tc_claimed_items<INTP, FEAT>()) return tc_fixed_item(c, k);
+  if constexpr (!tc_claimed_items<INTP, FEAT, IMMA>()) return tc_fixed_item(c, k);
   int *bc = &c.S.item_bc[bar - 2][k & 1];
   if (t == 0) *bc = tc_read_item(c, k, timed_out, false);
   named_sync(bar, 128);
@@ -377,8 +421,8 @@ __device__ __forceinline__ int tc_read_item_wg(TcCtx<NCOL, INTP, FEAT> &c, int k
 // call wrote does; an item that split_at emptied (a foreign schedule) has none,
 // and then neither writes nor waits for a query operand, so the q_full phases
 // of the softmax warpgroup and the QK issuer stay paired.
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ bool tc_item_has_tiles(const TcCtx<NCOL, INTP, FEAT> &c, long long it) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ bool tc_item_has_tiles(const TcCtx<NCOL, INTP, FEAT, IMMA> &c, long long it) {
   int slot, g;
   item_coords(it, c.nsplit, slot, g);
   const SplitRange sr = split_at(c.p, slot);
@@ -400,8 +444,8 @@ struct TcProdGeom {
 // it is free lane 0 publishes the tile description and the expected byte count
 // while every lane issues its own copies.  The tile starts at row tin0 of
 // logical page pg0 (tin0 = 0 when pages are shorter than a tile).
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c,
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c,
                                                 const typename TcCfg<NCOL, INTP>::PageCache &pc,
                                                 const TcProdGeom &geo, int b, int g, int n,
                                                 int t0, int rows, int npiece, int pg0, int tin0,
@@ -447,15 +491,23 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c,
                     : fmt == CFR_FMT_FP8   ? KIND_FP8
                                            : KIND_BF16;
   const int kind = __shfl_sync(0xffffffffu, kind0, 0);
-  // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA; every
+  // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA, and so
+  // does every int8 tile of an IMMA variant (its codes are the operand; rows
+  // that hold no token carry finite codes that meet a zero probability); every
   // other tile passes through the staging warps
-  const bool direct = kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu;
+  const bool direct = (kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu) ||
+                      (IMMA && kind == KIND_I8);
   // ---- the tile's byte count and scales (lane 0) ----
   float ks = 1.f, vs = 1.f;
   uint32_t bytes = 0;
   if (lane == 0) {
     if (kind == KIND_BF16) {
       bytes = static_cast<uint32_t>(__popc(vb)) * 4u * box_rows * 128u;
+    } else if (IMMA && kind == KIND_I8) {
+      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+      ks = sc.x;
+      vs = sc.y;
+      bytes = 2u * TC_T * 128u;  // one full 128-row box of K and of V
     } else {
       const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
       ks = sc.x;
@@ -490,6 +542,18 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c,
       tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
       tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, done);
       tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
+    } else if (IMMA && kind == KIND_I8) {
+      // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows
+      const int y = static_cast<int>((id * p.Hkv + g) * p.P + tin0);
+      tma_load_2d(op, &c.maps.k8, 0, y, done);
+      tma_load_2d(op + 2 * TC_HALF, &c.maps.v8, 0, y, done);
+    } else if (IMMA && kind == KIND_I4) {
+      // raw codes above the int8 operands the staging warps write (K at TC_HALF,
+      // V at 3 * TC_HALF)
+      const int rb = row_bytes(fmt, TC_D);
+      const long long off = ((id * p.Hkv + g) * p.P + tin0) * rb;
+      bulk_g2s(op + TC_HALF, p.k_pool[fmt] + off, rows * rb, done);
+      bulk_g2s(op + 3 * TC_HALF, p.v_pool[fmt] + off, rows * rb, done);
     } else if (INTP) {
       const int rb = row_bytes(fmt, TC_D);
       const long long off = ((id * p.Hkv + g) * p.P + tin0) * rb;
@@ -508,8 +572,8 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT> &c,
 // time: tile i waits for the consumers of tile i - 3 (the same stage), and the
 // warp's previous tile i - 2 waited for tile i - 5, so the stage's barrier can
 // never be two phases behind when tile i starts waiting on it.
-template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int pk) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ void tc_producer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out, int pk) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
@@ -530,10 +594,14 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int pk)
     prefetch_map(&c.maps.k);
     prefetch_map(&c.maps.v);
   }
+  if (IMMA && lane == 0 && p.k_pool[CFR_FMT_I8]) {
+    prefetch_map(&c.maps.k8);
+    prefetch_map(&c.maps.v8);
+  }
   page_cache_reset(pc, lane);
   long long tile = 0;
   for (int k = 0;; ++k) {
-    const int item = !tc_claimed_items<INTP, FEAT>() ? tc_fixed_item(c, k)
+    const int item = !tc_claimed_items<INTP, FEAT, IMMA>() ? tc_fixed_item(c, k)
                      : pk == 0 ? tc_claim_item(c, k, timed_out, lane)
                                : tc_read_item(c, k, timed_out, true);
     if (item < 0) break;
@@ -568,8 +636,8 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out, int pk)
 }
 
 // staging warpgroup: thread r (0..127) owns row r of every tile that is not direct
-template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int r = threadIdx.x - 192;
@@ -605,6 +673,36 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
             for (int ch = 0; ch < 8; ++ch) {
               *reinterpret_cast<uint4 *>(op + 2 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
               *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+            }
+          }
+        } else if (IMMA && m.kind == KIND_I4) {
+          // int4 codes (raw rows of 64 bytes at TC_HALF for K, 3 * TC_HALF for V)
+          // -> one byte per code, 16 * code, in the 128-byte-swizzled int8 operand
+          // rows at 0 (K) and 2 * TC_HALF (V).  Raw and widened rows do not
+          // overlap; rows past the tile's tokens hold finite codes that meet a
+          // zero probability.
+#pragma unroll 1
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint8_t *src = op + (2 * kv + 1) * TC_HALF + r * (TC_D / 2);
+            uint8_t *dst = op + kv * 2 * TC_HALF;
+            uint4 w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              w[j] = *reinterpret_cast<const uint4 *>(src + 16 * ((j + (r >> 1)) & 3));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int ci = (j + (r >> 1)) & 3;  // codes 32ci .. 32ci+31: output chunks 2ci, 2ci+1
+              const uint32_t wv[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+              uint32_t o[8];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint32_t lo = (wv[q] << 4) & 0xF0F0F0F0u;  // 16 * even elements
+                const uint32_t hi = wv[q] & 0xF0F0F0F0u;         // 16 * odd elements
+                o[2 * q] = prmt(lo, hi, 0x5140u);
+                o[2 * q + 1] = prmt(lo, hi, 0x7362u);
+              }
+              *reinterpret_cast<uint4 *>(dst + sw128(r, 2 * ci)) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4 *>(dst + sw128(r, 2 * ci + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
             }
           }
         } else if (INTP) {
@@ -709,8 +807,8 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
 
 // QK issuer (warp 1, one thread): for every tile in order, once its operands
 // are staged and an S buffer is free, S^T = K . [q_hi | q_lo]^T into TMEM.
-template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
@@ -738,15 +836,27 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
         break;
       tc_fence_after();
       const int kind = c.S.meta[stage].kind;
-      const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
       const uint32_t kbase = op0 + stage * TC_OP_BYTES;
-      const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
       const uint32_t d = tmem + static_cast<uint32_t>(tc & 1) * NCOL;
+      if (tc_int_tile<IMMA>(kind)) {
+        // int8 codes [128 tok][128 dims] x query digits [NCOL][128 dims], K = 32 per MMA
+        const uint32_t idesc = tc_idesc_i8(1, 0, 0, NCOL);
+        const uint32_t q8 = smem_u32(c.q8op);
 #pragma unroll
-      for (int k = 0; k < TC_D / 16; ++k) {
-        const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
-        const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
-        tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        for (int k = 0; k < TC_D / 32; ++k) {
+          const uint64_t a = tc_sdesc(kbase + k * 32, 16, 1024, 2);
+          const uint64_t bd = tc_sdesc(q8 + k * 32, 16, 1024, 2);
+          tc_mma_i8(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
+      } else {
+        const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
+        const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
+#pragma unroll
+        for (int k = 0; k < TC_D / 16; ++k) {
+          const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
+          const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
+          tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
       }
       tc_commit(&c.S.s_full[tc & 1]);
       ++tc;
@@ -763,8 +873,8 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
 // P.V issuer (warp 10, one thread): for every tile in order, once its
 // probabilities are written and an O buffer is free, O^T = V^T . [p_hi | p_lo]^T
 // into TMEM; the commit then frees the stage, the P buffer and signals the fold.
-template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   const int P = p.P;
@@ -791,15 +901,27 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
       tc_fence_after();
       // the tile description stays valid until this P.V has freed the stage
       const int kind = c.S.meta[stage].kind;
-      const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
       const uint32_t vbase = op0 + stage * TC_OP_BYTES + 2 * TC_HALF;
       const uint32_t pbase = p0 + static_cast<uint32_t>(tc & 1) * Cfg::P_BYTES;
       const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(ob) * NCOL;
+      if (tc_int_tile<IMMA>(kind)) {
+        // V^T: int8 codes [128 tok][128 dims] read dim-major; P^T: unsigned digits
+        // [128 tok][16 columns]; K = 32 tokens per MMA
+        const uint32_t idesc = tc_idesc_i8(0, 1, 1, NCOL);
 #pragma unroll
-      for (int k = 0; k < TC_T / 16; ++k) {
-        const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
-        const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
-        tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        for (int k = 0; k < TC_T / 32; ++k) {
+          const uint64_t a = tc_sdesc(vbase + k * 4096, TC_HALF, 1024, 2);
+          const uint64_t bd = tc_sdesc(pbase + k * 512, 128, 2048, 0);
+          tc_mma_i8(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
+      } else {
+        const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 1, 1, NCOL);
+#pragma unroll
+        for (int k = 0; k < TC_T / 16; ++k) {
+          const uint64_t a = tc_sdesc(vbase + k * 2048, TC_HALF, 1024, 2);
+          const uint64_t bd = tc_sdesc(pbase + k * 256, 128, 2048, 0);
+          tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
+        }
       }
       tc_commit(&c.S.o_full[ob]);
       tc_commit(&c.S.p_empty[tc & 1]);
@@ -811,12 +933,14 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   tc_commit(&c.S.drain);
 }
 
-// folds the P.V product of tile i into the running accumulators (dim t of each head)
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT> &c, long long i, uint32_t tmem, int lane,
+// folds the P.V product of tile i into the running accumulators (dim t of each
+// head); `oint`: the product is in int32 digit columns (an int tile of an IMMA
+// variant), column 4 * l + h holding digit l of head h
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long long i, uint32_t tmem, int lane,
                                         int cnt, float (&acc)[NCOL / 2],
                                         const float (&alpha_prev)[NCOL / 2], float vscale_prev,
-                                        bool *timed_out) {
+                                        bool oint, bool *timed_out) {
   const int ob = static_cast<int>(i % TcCfg<NCOL, INTP>::O_BUFS);
   (void)mbar_wait(&c.S.o_full[ob], static_cast<uint32_t>((i / TcCfg<NCOL, INTP>::O_BUFS) & 1),
                   c.p.err, timed_out);
@@ -827,15 +951,42 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT> &c, long long i,
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(&c.S.o_empty[ob]);
+  if (IMMA && oint) {
+    // sum_l digit_l 256^-l in fp32 (every int32 product sum is below 2^23, exact)
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      if (h < cnt) {
+        float t = fmaf(static_cast<float>(__float_as_int(o[12 + h])), 1.f / 256.f,
+                       static_cast<float>(__float_as_int(o[8 + h])));
+        t = fmaf(t, 1.f / 256.f, static_cast<float>(__float_as_int(o[4 + h])));
+        t = fmaf(t, 1.f / 256.f, static_cast<float>(__float_as_int(o[h])));
+        acc[h] = fmaf(acc[h], alpha_prev[h], t * vscale_prev);
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int h = 0; h < NCOL / 2; ++h)
     if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
 }
 
-// writes the hi/lo query operand of item `it` (both bf16 and fp16 copies); the
-// warpgroup's 128 threads (index tsm) share the work, each warp then arrives on q_full
-template <int NCOL, bool INTP, int FEAT>
-__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT> &c, long long it, int tsm, int lane) {
+// element `dim` of query row vh of sequence b, as fp32
+__device__ __forceinline__ float q_elem(const DecodeParams &p, int b, int vh, int dim) {
+  const long long i = (static_cast<long long>(b) * p.Hq + vh) * TC_D + dim;
+  return p.q_fmt == CFR_FMT_F32
+             ? static_cast<const float *>(p.q)[i]
+             : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
+}
+
+// writes the hi/lo query operand of item `it` (both bf16 and fp16 copies) and,
+// in IMMA variants, its int8 digit operand: row 4 * l + h holds digit l of head
+// h (h < 4) of q_h * 127 / max|q_h| = d0 + d1 / 128 + d2 / 128^2 + d3 / 128^3,
+// d0 in [-127, 127], d1..d3 in [-64, 64]; qsc[h] receives max|q_h| / 127.  The
+// warpgroup's 128 threads (index tsm) share the work, each warp then arrives on
+// q_full.
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long long it, int tsm, int lane,
+                                           float (&qsc)[4]) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
   {
@@ -886,6 +1037,51 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT> &c, long long
       *reinterpret_cast<uint4 *>(c.qop + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
       *reinterpret_cast<uint4 *>(c.qop + Cfg::Q_BYTES + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
     }
+    if constexpr (IMMA) {
+      static_assert(NCOL == 16, "int8 digit operand: 4 digits x 4 heads");
+      // max|q_h| over the 128 dims: thread tsm holds dim tsm of every head
+      const int warp4 = tsm >> 5;
+      float mx[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float v = 0.f;
+        if (h < cnt) v = fabsf(q_elem(p, b, p.grp_heads[h0 + h], tsm));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        mx[h] = v;
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) c.S.red_l[warp4][h] = mx[h];
+      }
+      named_sync(2, 128);
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        qsc[h] = fmaxf(fmaxf(c.S.red_l[0][h], c.S.red_l[1][h]), fmaxf(c.S.red_l[2][h], c.S.red_l[3][h])) *
+                 (1.f / 127.f);
+      named_sync(2, 128);  // red_l is free again (the partial write reuses it)
+      // row n = 4 * l + h, 16-dim chunk ch of it
+      const int n = tsm >> 3, ch = tsm & 7, l = n >> 2, h = n & 3;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (h < cnt && qsc[h] > 0.f) {
+        const float inv = 1.f / qsc[h];
+        const int head = p.grp_heads[h0 + h];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float r = q_elem(p, b, head, 16 * ch + e) * inv;
+          float d = rintf(r);
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            if (k < l) {
+              r = (r - d) * 128.f;
+              d = rintf(r);
+            }
+          }
+          w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(d)) & 0xFFu) << (8 * (e & 3));
+        }
+      }
+      *reinterpret_cast<uint4 *>(c.q8op + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&c.S.q_full);
@@ -895,8 +1091,8 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT> &c, long long
 // softmax / fold warpgroup.  Every thread waits on the mbarriers itself; a
 // thread whose wait gives up keeps the same control flow (later waits return at
 // once), so the one named barrier per tile is always reached by all 128 threads.
-template <int NCOL, bool INTP, int FEAT>
-__device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   constexpr int GM = NCOL / 2;  // most query heads per tile
   const DecodeParams &p = c.p;
@@ -914,6 +1110,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   // query operand early); nxt_read says whether that read has happened
   int k = 0, nxt = -1;
   bool nxt_read = false;
+  float qs_nxt[4] = {0.f, 0.f, 0.f, 0.f};  // int8 digit scales of the last query operand written
 
   for (int item = tc_read_item_wg(c, 0, 2, tsm, timed_out); item >= 0; ++k) {
     int slot, g;
@@ -923,9 +1120,12 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * P);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
-    if (!q_ready && pb * P < tok_end) tc_write_q(c, item, tsm, lane);
+    if (!q_ready && pb * P < tok_end) tc_write_q(c, item, tsm, lane, qs_nxt);
     q_ready = false;
     nxt_read = false;
+    float qs[4];  // this item's int8 digit scales (max|q_h| / 127)
+#pragma unroll
+    for (int h = 0; h < 4; ++h) qs[h] = qs_nxt[h];
 
     // folds lag two tiles behind the scores: tiles prev2 (older) and prev1 wait,
     // each with its rescale factors and V scale
@@ -944,6 +1144,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
       alpha2[h] = 1.f;
     }
     float vs1 = 1.f, vs2 = 1.f;
+    bool oi1 = false, oi2 = false;  // the pending P.V products are int32 digit columns
     long long prev1 = -1, prev2 = -1;
 
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
@@ -961,17 +1162,37 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
       (void)mbar_try_wait(&c.S.op_full[stage], phase);
       const TcMeta &m = c.S.meta[stage];
       const bool valid = (m.valid[t >> 5] >> (t & 31)) & 1u;
-      const float scale = m.ks * p.sigma_log2e;
       const int kind = m.kind;
-      const float vsc = kind == KIND_BF16 ? 1.f : m.vs * (1.f / 32768.f);
+      const bool itile = tc_int_tile<IMMA>(kind);
+      // int4 codes enter the int8 MMAs times 16; probability digits are of p * 255
+      const float i4f = itile && kind == KIND_I4 ? 1.f / 16.f : 1.f;
+      const float scale = m.ks * p.sigma_log2e * i4f;
+      const float vsc = kind == KIND_BF16 ? 1.f
+                        : itile           ? m.vs * i4f * (1.f / 255.f)
+                                          : m.vs * (1.f / 32768.f);
       // ALiBi from the last position; a query row at offset o before it differs by the
       // row constant slope * o, added back to its maximum at the partial write
       const int j = m.t0 + t;
       const float dist = static_cast<float>(n - 1 - j);
       float s[GM];
+      if (IMMA && itile) {
+        // column 4 * l + h: digit l of head h; sum_l S_l 128^-l, exact terms below 2^22
 #pragma unroll
-      for (int h = 0; h < GM; ++h)
-        s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
+        for (int h = 0; h < GM; ++h) {
+          s[h] = -INFINITY;
+          if (h < 4 && valid && h < cnt) {
+            float u = fmaf(static_cast<float>(__float_as_int(sv[12 + h])), 1.f / 128.f,
+                           static_cast<float>(__float_as_int(sv[8 + h])));
+            u = fmaf(u, 1.f / 128.f, static_cast<float>(__float_as_int(sv[4 + h])));
+            u = fmaf(u, 1.f / 128.f, static_cast<float>(__float_as_int(sv[h])));
+            s[h] = fmaf(u, scale * qs[h], -slope2[h] * dist);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
+      }
       if (FEAT == TC_FEAT_MULTI && m.t0 + TC_T - 1 > n - p.nq) {
         // the tile reaches the query positions: row h sees tokens j <= n - 1 - offset_h
 #pragma unroll
@@ -1011,8 +1232,24 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
         l_part[h] = fmaf(l_part[h], alpha[h], pr[h]);
         m_run[h] = m_new;
       }
-      // P^T row t: columns [hi(0..GM) | lo(0..GM)]
-      {
+      if (IMMA && itile) {
+        // P^T row t: 16 unsigned digit columns, column 4 * l + h = digit l of
+        // p_h * 255 = e0 + e1 / 256 + e2 / 256^2 + e3 / 256^3 (floor digits, the
+        // last rounded; every e in [0, 255])
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float x = pr[h] * 255.f;
+#pragma unroll
+          for (int l = 0; l < 4; ++l) {
+            const float d = l < 3 ? floorf(x) : fminf(rintf(x), 255.f);
+            w[l] |= static_cast<uint32_t>(d) << (8 * h);
+            x = (x - d) * 256.f;
+          }
+        }
+        *reinterpret_cast<uint4 *>(c.pop + (tc & 1) * Cfg::P_BYTES + t * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        // P^T row t: columns [hi(0..GM) | lo(0..GM)]
         float colv[NCOL];
 #pragma unroll
         for (int k = 0; k < NCOL; ++k) colv[k] = 0.f;
@@ -1046,14 +1283,15 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
         nxt = tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
         nxt_read = true;
         if (nxt >= 0 && tc_item_has_tiles(c, nxt)) {
-          tc_write_q(c, nxt, tsm, lane);
+          tc_write_q(c, nxt, tsm, lane, qs_nxt);
           q_ready = true;
         }
       }
       // fold the tile two behind (its P.V has long been issued)
-      if (prev2 >= 0) tc_fold(c, prev2, tmem, lane, cnt, acc, alpha2, vs2, timed_out);
+      if (prev2 >= 0) tc_fold(c, prev2, tmem, lane, cnt, acc, alpha2, vs2, oi2, timed_out);
       prev2 = prev1;
       vs2 = vs1;
+      oi2 = oi1;
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         alpha2[h] = alpha1[h];
@@ -1061,14 +1299,15 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
       }
       prev1 = tc;
       vs1 = vsc;
+      oi1 = itile;
       ++tc;
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
       }
     }
-    if (prev2 >= 0) tc_fold(c, prev2, tmem, lane, cnt, acc, alpha2, vs2, timed_out);
-    if (prev1 >= 0) tc_fold(c, prev1, tmem, lane, cnt, acc, alpha1, vs1, timed_out);
+    if (prev2 >= 0) tc_fold(c, prev2, tmem, lane, cnt, acc, alpha2, vs2, oi2, timed_out);
+    if (prev1 >= 0) tc_fold(c, prev1, tmem, lane, cnt, acc, alpha1, vs1, oi1, timed_out);
 
     // split partial: acc (dim t), m, and l summed over the 128 token slots
 #pragma unroll
@@ -1102,7 +1341,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT> &c, bool *timed_out) {
   }
 }
 
-template <int NCOL, bool INTP, int FEAT>
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1150,23 +1389,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    // when the launch did not overlap it)
 
   const int nsplit = schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0);
-  TcCtx<NCOL, INTP, FEAT> c{p, maps, S, smem + L::op, smem + L::q, smem + L::pbuf,
-                            static_cast<long long>(nsplit) * p.Hkv, nsplit};
+  TcCtx<NCOL, INTP, FEAT, IMMA> c{p,
+                                  maps,
+                                  S,
+                                  smem + L::op,
+                                  smem + L::q,
+                                  smem + L::pbuf,
+                                  static_cast<long long>(nsplit) * p.Hkv,
+                                  nsplit,
+                                  smem + L::q8};
   bool timed_out = false;
   if (warp == 0 || warp == TC_PROD2_WARP) {
-    tc_producer<NCOL, INTP, FEAT>(c, &timed_out, warp == 0 ? 0 : 1);
+    tc_producer<NCOL, INTP, FEAT, IMMA>(c, &timed_out, warp == 0 ? 0 : 1);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP, FEAT>(c, &timed_out);
+    if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   } else if (warp == 10) {
-    if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP, FEAT>(c, &timed_out);
+    if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   } else if (warp < 6) {
-    tc_softmax<NCOL, INTP, FEAT>(c, &timed_out);
+    tc_softmax<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   } else {
-    tc_staging<NCOL, INTP, FEAT>(c, &timed_out);
+    tc_staging<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   }
   tc_fence_before();
   __syncthreads();
-  if (tc_claimed_items<INTP, FEAT>() && threadIdx.x == 0 && p.item_ctr) {
+  if (tc_claimed_items<INTP, FEAT, IMMA>() && threadIdx.x == 0 && p.item_ctr) {
     // every CTA has stopped claiming once all have counted themselves finished;
     // the last one leaves both counters at 0 for the next launch
     __threadfence();
@@ -1213,10 +1459,13 @@ bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
   }
   const long long rows = p.pool_pages[CFR_FMT_BF16] * p.Hkv * static_cast<long long>(p.P);
   if (rows > 0x7fffffffLL) return false;
+  // int8 pools are read through a tensor map when their tiles run int8 MMAs
+  const long long rows8 = p.pool_pages[CFR_FMT_I8] * p.Hkv * static_cast<long long>(p.P);
+  if (p.k_pool[CFR_FMT_I8] && p.gmax <= 4 && rows8 > 0x7fffffffLL) return false;
   return true;
 }
 
-template <int NCOL, bool INTP, int FEAT>
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
 static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t stream) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -1229,27 +1478,45 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                          TC_D, box_rows))
       return cudaErrorInvalidValue;
   }
+  if (IMMA && p.k_pool[CFR_FMT_I8] && p.pool_pages[CFR_FMT_I8] > 0) {
+    // int pages have page_tokens a multiple of 128: one 128-row box per tile
+    const long long rows = p.pool_pages[CFR_FMT_I8] * p.Hkv * static_cast<long long>(p.P);
+    if (!encode_pool_map(&maps.k8, p.k_pool[CFR_FMT_I8], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows,
+                         TC_D, TC_T) ||
+        !encode_pool_map(&maps.v8, p.v_pool[CFR_FMT_I8], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows,
+                         TC_D, TC_T))
+      return cudaErrorInvalidValue;
+  }
   constexpr size_t smem = TcLayout<NCOL, INTP>::launch_bytes;
   static_assert(smem <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<NCOL, INTP, FEAT>,
+  cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel<NCOL, INTP, FEAT, IMMA>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   // a plain launch: overlapping this kernel's start with the schedule kernel
   // (programmatic dependent launch) measured slower for this kernel
-  tc_decode_kernel<NCOL, INTP, FEAT><<<dim3(grid), dim3(TC_THREADS), smem, stream>>>(p, maps);
+  tc_decode_kernel<NCOL, INTP, FEAT, IMMA><<<dim3(grid), dim3(TC_THREADS), smem, stream>>>(p, maps);
   e = cudaSuccess;
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// int8 or int4 pools whose tiles can run the int8 MMAs: up to 4 query rows per
+// kv head (4 digit columns each fill the 16-column operand)
+static bool tc_imma(const DecodeParams &p, bool page_fmt_given) {
+  if (p.gmax > 4) return false;
+  if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4];
+  return p.uniform_fmt == CFR_FMT_I8 || p.uniform_fmt == CFR_FMT_I4;
 }
 
 template <int FEAT>
 static cudaError_t tc_launch_f(const DecodeParams &p, int grid, cudaStream_t stream) {
   const bool ints = tc_int_pools(p, p.page_fmt != nullptr);
+  if (ints && tc_imma(p, p.page_fmt != nullptr)) return tc_launch_t<16, true, FEAT, true>(p, grid, stream);
   if (p.gmax <= 8)
-    return ints ? tc_launch_t<16, true, FEAT>(p, grid, stream)
-                : tc_launch_t<16, false, FEAT>(p, grid, stream);
-  return ints ? tc_launch_t<32, true, FEAT>(p, grid, stream)
-              : tc_launch_t<32, false, FEAT>(p, grid, stream);
+    return ints ? tc_launch_t<16, true, FEAT, false>(p, grid, stream)
+                : tc_launch_t<16, false, FEAT, false>(p, grid, stream);
+  return ints ? tc_launch_t<32, true, FEAT, false>(p, grid, stream)
+              : tc_launch_t<32, false, FEAT, false>(p, grid, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream) {
