@@ -81,9 +81,18 @@ constexpr int TC_ITEM_READERS = 5;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
 constexpr int TC_RAW_K = TC_T * TC_D;  // raw code offset of V inside a stage's V region (K at 0)
+constexpr int TC_QRAW_BUF = 8 * 512;   // query rows of one item (16-column variants: <= 8 rows of <= 512 B)
 constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2, KIND_FP8 = 3;
 // compile-time variants: plain decode, multi-query rows, sink + window subset
 constexpr int TC_FEAT_PLAIN = 0, TC_FEAT_MULTI = 1, TC_FEAT_SUBSET = 2;
+
+// one work item as producer warp 0 publishes it (see tc_publish_item)
+struct TcItem {
+  int item;        // -1: past the CTA's last item, or a wait gave up
+  int slot, g, b;  // split slot, kv head, sequence
+  int pb, pe;      // the split's logical pages [pb, pe)
+  int n, t_end;    // sequence length; the split's tokens are [pb * P, t_end)
+};
 
 struct TcMeta {
   uint32_t valid[4];
@@ -110,9 +119,12 @@ struct TcCfg {
   static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
   static constexpr int TMEM_COLS = NCOL == 16 ? 128 : 256;  // S x2 + O x3 columns, power of two
   // page-table entries each producer keeps on chip; with 32 columns the q and P
-  // buffers leave room for two caches of 80 beside the three stages (with
-  // 16-token pages, one refill then serves 10 tiles)
-  static constexpr int PAGE_CACHE = NCOL == 16 ? 128 : 80;
+  // buffers leave room for two caches of 48 beside the three stages (with
+  // 16-token pages, one refill then serves 6 tiles)
+  static constexpr int PAGE_CACHE = NCOL == 16 ? 128 : 48;
+  // the 16-column variants keep each item's ALiBi slopes in shared memory (the
+  // 32-column ones, which fill shared memory, read them at the item's start)
+  static constexpr int RING_SLOPES = NCOL == 16 ? NCOL / 2 : 1;
   using PageCache = PageCacheT<PAGE_CACHE>;
 };
 
@@ -122,8 +134,12 @@ struct TcSmem {
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[3], o_empty[3];
   uint64_t q_full, drain;
   uint64_t item_full[TC_ITEM_RING], item_empty[TC_ITEM_RING];
-  int item_q[TC_ITEM_RING];  // work item of each ring slot, -1 past the last
-  int item_bc[2][2];         // [softmax, staging][k & 1]: the item broadcast in a warpgroup
+  uint64_t qraw_full[2], qraw_empty[2];
+  TcItem ring[TC_ITEM_RING];  // work item k in slot k % TC_ITEM_RING
+  // ALiBi slope * log2(e) of its query rows (16-column variants)
+  float ring_slope[TC_ITEM_RING][TcCfg<NCOL, INTP>::RING_SLOPES];
+  TcItem item_bc[2][2];       // [softmax, staging][k & 1]: the item in a warpgroup
+  float slope_bc[2][TcCfg<NCOL, INTP>::RING_SLOPES];  // [k & 1]: its slopes, for the softmax
   uint32_t tmem_base;
   int flag_st[3];
   TcMeta meta[3];
@@ -139,7 +155,8 @@ struct TcLayout {
   static constexpr size_t q = op + TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_OP_BYTES);
   static constexpr size_t q8 = q + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::Q_BYTES);
   static constexpr size_t pbuf = q8 + static_cast<size_t>(TcCfg<NCOL, INTP>::Q8_BYTES);
-  static constexpr size_t total = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
+  static constexpr size_t qraw = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
+  static constexpr size_t total = qraw + (NCOL == 16 ? 2 * static_cast<size_t>(TC_QRAW_BUF) : 0);
   static constexpr size_t launch_bytes = total + 1024;  // slack for 1024-byte alignment
 };
 
@@ -284,6 +301,7 @@ struct TcCtx {
   long long nitems;
   int nsplit;
   uint8_t *q8op;  // int8 query digits (IMMA variants)
+  uint8_t *qraw;  // [2][TC_QRAW_BUF]: query rows of the next items (16-column variants)
 };
 
 // With IMMA, int8 and int4 tiles run kind::i8 MMAs on 8-bit operands: int8 codes
@@ -340,93 +358,151 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 }
 
 // ---- work items --------------------------------------------------------------
-// Two ways of sharing the items among the CTAs, chosen per variant by measurement:
+// An item is one split of one kv head.  Producer warp 0 takes the CTA's items in
+// order and publishes item k in ring slot k % TC_ITEM_RING together with what
+// every other role needs to know about it (split, sequence length, token range,
+// the ALiBi slopes of its query rows), so that no other role reads global
+// memory at an item boundary; a slot whose item is -1 ends every loop.  In the
+// 16-column variants warp 0 also bulk-copies the item's query rows into shared
+// memory (qraw), so that the softmax warpgroup builds the query operand without
+// a global round trip.  Two ways of choosing the items, by measurement:
 //  - fixed: CTA x takes items x, x + grid, x + 2 grid, ...
 //  - claimed (bf16-only plain and multi-query decode): CTA x starts with item x
 //    and claims every further item from a global counter when producer warp 0
 //    reaches it, so SMs that the memory system serves faster take more items and
-//    all CTAs finish together.  Warp 0 publishes item k of the CTA in ring slot
-//    k % TC_ITEM_RING; the other warps read the slots in order and free them.  A
-//    slot holds -1 past the CTA's last item, which ends every loop.  On quantised
-//    tiles (whose expansion sets the pace) and on subset decode the ring's
-//    per-item hand-off cost more than the balance gained, so those keep the
-//    fixed share.
+//    all CTAs finish together.
 template <bool INTP, int FEAT, bool IMMA>
 __host__ __device__ constexpr bool tc_claimed_items() {
   return !INTP && FEAT != TC_FEAT_SUBSET;
 }
 
-// item k of the fixed share, or -1
-template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ int tc_fixed_item(const TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k) {
-  const long long it = static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
-  return it < c.nitems ? static_cast<int>(it) : -1;
+// query rows of one item staged in shared memory (16-column variants)
+template <int NCOL>
+__host__ __device__ constexpr bool tc_qraw() {
+  return NCOL == 16;
 }
 
-// producer warp 0 (all lanes): claims and publishes item k; returns it, or -1.
+// producer warp 0 (all lanes): takes item k, publishes it and (16-column
+// variants) starts the copy of its query rows into qraw buffer kq & 1, kq
+// counting the items with tiles.  Returns the item (item = -1 past the last, or
+// when a wait gave up).
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ int tc_claim_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, bool *timed_out,
-                                             int lane) {
+__device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, int &kq,
+                                                  bool *timed_out, int lane) {
+  const DecodeParams &p = c.p;
   const int s = k & (TC_ITEM_RING - 1);
-  int item = -1;
-  if (lane == 0) {
-    if (mbar_wait(&c.S.item_empty[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1) ^ 1u, c.p.err,
-                  timed_out)) {
-      const long long it =
-          k == 0 ? static_cast<long long>(blockIdx.x)
-          : c.p.item_ctr ? static_cast<long long>(gridDim.x) + atomicAdd(c.p.item_ctr, 1u)
-                         : static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
-      item = it < c.nitems ? static_cast<int>(it) : -1;
-      c.S.item_q[s] = item;
-      mbar_arrive(&c.S.item_full[s]);
+  TcItem d;
+  d.item = -1;
+  d.slot = d.g = d.b = d.pb = d.pe = d.n = d.t_end = 0;
+  int ok = 1;
+  if (lane == 0)
+    ok = mbar_wait(&c.S.item_empty[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1) ^ 1u, p.err,
+                   timed_out) ? 1 : 0;
+  if (!__shfl_sync(0xffffffffu, ok, 0)) return d;
+  long long it = 0;
+  if (lane == 0)
+    it = k == 0 ? static_cast<long long>(blockIdx.x)
+         : (tc_claimed_items<INTP, FEAT, IMMA>() && p.item_ctr)
+             ? static_cast<long long>(gridDim.x) + atomicAdd(p.item_ctr, 1u)
+             : static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
+  it = __shfl_sync(0xffffffffu, it, 0);
+  if (it < c.nitems) {
+    d.item = static_cast<int>(it);
+    item_coords(it, c.nsplit, d.slot, d.g);
+    const SplitRange sr = split_at(p, d.slot);
+    d.b = sr.b;
+    d.pb = sr.pb;
+    d.pe = sr.pe;
+    d.n = p.seq_lens[d.b];
+    d.t_end = min(d.n, d.pe * p.P);
+    const int h0 = p.grp_off[d.g], cnt = p.grp_off[d.g + 1] - h0;
+    if (tc_qraw<NCOL>() && lane < NCOL / 2)
+      c.S.ring_slope[s][lane] =
+          (p.slopes && lane < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + lane])] * kLog2e : 0.f;
+    if (tc_qraw<NCOL>() && d.pb * p.P < d.t_end) {
+      // the query rows of the group, one bulk copy per row
+      const int buf = kq & 1;
+      const uint32_t rb = static_cast<uint32_t>(TC_D) * (p.q_fmt == CFR_FMT_F32 ? 4u : 2u);
+      int qok = 1;
+      if (lane == 0) {
+        qok = mbar_wait(&c.S.qraw_empty[buf], static_cast<uint32_t>((kq >> 1) & 1) ^ 1u, p.err,
+                        timed_out) ? 1 : 0;
+        if (qok) mbar_arrive_expect_tx(&c.S.qraw_full[buf], static_cast<uint32_t>(cnt) * rb);
+      }
+      if (!__shfl_sync(0xffffffffu, qok, 0)) {
+        d.item = -1;
+      } else if (lane < cnt) {
+        const uint8_t *src = static_cast<const uint8_t *>(p.q) +
+                             (static_cast<long long>(d.b) * p.Hq + p.grp_heads[h0 + lane]) * rb;
+        bulk_g2s(c.qraw + buf * TC_QRAW_BUF + lane * 512, src, rb, &c.S.qraw_full[buf]);
+      }
+      ++kq;
     }
   }
-  return __shfl_sync(0xffffffffu, item, 0);
+  if (lane == 0) c.S.ring[s] = d;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&c.S.item_full[s]);
+  return d;
 }
 
 // item k read by one thread (an MMA issuer) or by every lane of a warp
-// (producer warp 11; lane 0 waits and frees the slot); -1 past the last item
-// or when the wait gave up.
+// (producer warp 11: lane 0 waits, reads and frees the slot, the lanes get the
+// fields by shuffles).  item = -1 past the last item or when the wait gave up.
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ int tc_read_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, bool *timed_out,
-                                            bool warp_wide) {
-  if constexpr (!tc_claimed_items<INTP, FEAT, IMMA>()) return tc_fixed_item(c, k);
+__device__ __forceinline__ TcItem tc_read_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, bool *timed_out,
+                                               bool warp_wide) {
   const int s = k & (TC_ITEM_RING - 1);
-  int item = -1;
+  TcItem d;
+  d.item = -1;
+  d.slot = d.g = d.b = d.pb = d.pe = d.n = d.t_end = 0;
   if (!warp_wide || (threadIdx.x & 31) == 0) {
     if (mbar_wait(&c.S.item_full[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1), c.p.err,
                   timed_out)) {
-      item = c.S.item_q[s];
+      d = c.S.ring[s];
       mbar_arrive(&c.S.item_empty[s]);
     }
   }
-  return warp_wide ? __shfl_sync(0xffffffffu, item, 0) : item;
+  if (warp_wide) {
+    d.item = __shfl_sync(0xffffffffu, d.item, 0);
+    d.slot = __shfl_sync(0xffffffffu, d.slot, 0);
+    d.g = __shfl_sync(0xffffffffu, d.g, 0);
+    d.b = __shfl_sync(0xffffffffu, d.b, 0);
+    d.pb = __shfl_sync(0xffffffffu, d.pb, 0);
+    d.pe = __shfl_sync(0xffffffffu, d.pe, 0);
+    d.n = __shfl_sync(0xffffffffu, d.n, 0);
+    d.t_end = __shfl_sync(0xffffffffu, d.t_end, 0);
+  }
+  return d;
 }
 
 // item k read by a 128-thread warpgroup that synchronises on named barrier
-// `bar` (2: softmax, 3: staging): thread t = 0 waits, reads and frees the slot,
-// and the barrier hands the value to all 128 threads, so they leave their loop
-// together even when the wait gave up (named barriers have no time limit).
+// `bar` (2: softmax, 3: staging): thread t = 0 waits, copies the slot (and the
+// ALiBi slopes) to the warpgroup's broadcast area and frees it; the barrier
+// hands the copy to all 128 threads, so they leave their loop together even when
+// the wait gave up (named barriers have no time limit).
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ int tc_read_item_wg(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, int bar, int t,
-                                               bool *timed_out) {
-  if constexpr (!tc_claimed_items<INTP, FEAT, IMMA>()) return tc_fixed_item(c, k);
-  int *bc = &c.S.item_bc[bar - 2][k & 1];
-  if (t == 0) *bc = tc_read_item(c, k, timed_out, false);
+__device__ __forceinline__ TcItem tc_read_item_wg(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, int bar, int t,
+                                                  bool *timed_out) {
+  TcItem *bc = &c.S.item_bc[bar - 2][k & 1];
+  if (t == 0) {
+    const int s = k & (TC_ITEM_RING - 1);
+    TcItem d;
+    d.item = -1;
+    d.slot = d.g = d.b = d.pb = d.pe = d.n = d.t_end = 0;
+    if (mbar_wait(&c.S.item_full[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1), c.p.err,
+                  timed_out)) {
+      d = c.S.ring[s];
+      if (tc_qraw<NCOL>() && bar == 2) {
+#pragma unroll
+        for (int h = 0; h < TcCfg<NCOL, INTP>::RING_SLOPES; ++h)
+          c.S.slope_bc[k & 1][h] = c.S.ring_slope[s][h];
+      }
+      mbar_arrive(&c.S.item_empty[s]);
+    }
+    *bc = d;
+  }
   named_sync(bar, 128);
-  return *reinterpret_cast<volatile int *>(bc);
-}
-
-// true when item `it` has at least one tile.  Every split of a schedule this
-// call wrote does; an item that split_at emptied (a foreign schedule) has none,
-// and then neither writes nor waits for a query operand, so the q_full phases
-// of the softmax warpgroup and the QK issuer stay paired.
-template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ bool tc_item_has_tiles(const TcCtx<NCOL, INTP, FEAT, IMMA> &c, long long it) {
-  int slot, g;
-  item_coords(it, c.nsplit, slot, g);
-  const SplitRange sr = split_at(c.p, slot);
-  return sr.pb * c.p.P < min(c.p.seq_lens[sr.b], sr.pe * c.p.P);
+  return *const_cast<const TcItem *>(bc);
 }
 
 // Per-kernel constants of a producer warp: which formats have their pools (and
@@ -600,17 +676,12 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out, i
   }
   page_cache_reset(pc, lane);
   long long tile = 0;
+  int kq = 0;  // items with tiles so far (query-row buffers)
   for (int k = 0;; ++k) {
-    const int item = !tc_claimed_items<INTP, FEAT, IMMA>() ? tc_fixed_item(c, k)
-                     : pk == 0 ? tc_claim_item(c, k, timed_out, lane)
-                               : tc_read_item(c, k, timed_out, true);
-    if (item < 0) break;
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    const SplitRange sr = split_at(p, slot);
-    const int b = sr.b, pb = sr.pb, pe = sr.pe;
-    const int n = p.seq_lens[b];
-    const int tok_end = min(n, pe * P);
+    const TcItem it = pk == 0 ? tc_publish_item(c, k, kq, timed_out, lane)
+                              : tc_read_item(c, k, timed_out, true);
+    if (it.item < 0) break;
+    const int b = it.b, g = it.g, pb = it.pb, pe = it.pe, n = it.n, tok_end = it.t_end;
     int pg0 = pb, tin0 = 0;
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T, ++tile) {
       if ((tile & (TC_PRODUCERS - 1)) == pk) {
@@ -645,14 +716,9 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   int stage = 0;
   uint32_t phase = 0;
   for (int k = 0;; ++k) {
-    const int item = tc_read_item_wg(c, k, 3, r, timed_out);
-    if (item < 0) break;
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    (void)g;
-    const SplitRange sr = split_at(p, slot);
-    const int b = sr.b, pb = sr.pb, pe = sr.pe;
-    const int tok_end = min(p.seq_lens[b], pe * P);
+    const TcItem it = tc_read_item_wg(c, k, 3, r, timed_out);
+    if (it.item < 0) break;
+    const int pb = it.pb, tok_end = it.t_end;
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       // elected bounded wait; the outcome slot is per stage, so a slow reader can
       // never see the next use of the slot (that needs every thread's barrier)
@@ -819,14 +885,9 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
   long long tc = 0;
   int q_items = 0;  // items with tiles so far: one q_full phase each
   for (int item_k = 0; !*timed_out; ++item_k) {
-    const int item = tc_read_item(c, item_k, timed_out, false);
-    if (item < 0) break;
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    (void)g;
-    const SplitRange sr = split_at(p, slot);
-    const int b = sr.b, pb = sr.pb, pe = sr.pe;
-    const int tok_end = min(p.seq_lens[b], pe * P);
+    const TcItem it = tc_read_item(c, item_k, timed_out, false);
+    if (it.item < 0) break;
+    const int pb = it.pb, tok_end = it.t_end;
     if (pb * P >= tok_end) continue;
     if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(q_items++ & 1), p.err, timed_out)) break;
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
@@ -883,14 +944,9 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
   int stage = 0;
   long long tc = 0;
   for (int k = 0; !*timed_out; ++k) {
-    const int item = tc_read_item(c, k, timed_out, false);
-    if (item < 0) break;
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    (void)g;
-    const SplitRange sr = split_at(p, slot);
-    const int b = sr.b, pb = sr.pb, pe = sr.pe;
-    const int tok_end = min(p.seq_lens[b], pe * P);
+    const TcItem it = tc_read_item(c, k, timed_out, false);
+    if (it.item < 0) break;
+    const int pb = it.pb, tok_end = it.t_end;
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       const int ob = static_cast<int>(tc % Cfg::O_BUFS);
       if (!mbar_wait(&c.S.p_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), p.err, timed_out))
@@ -970,121 +1026,145 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long l
     if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
 }
 
-// element `dim` of query row vh of sequence b, as fp32
-__device__ __forceinline__ float q_elem(const DecodeParams &p, int b, int vh, int dim) {
-  const long long i = (static_cast<long long>(b) * p.Hq + vh) * TC_D + dim;
-  return p.q_fmt == CFR_FMT_F32
-             ? static_cast<const float *>(p.q)[i]
-             : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
-}
+// Query rows of one item: in the 16-column variants from the qraw buffer that
+// producer warp 0 filled (row h at h * 512 bytes), otherwise from global memory.
+template <int NCOL>
+struct TcQRows {
+  const DecodeParams &p;
+  const uint8_t *raw;  // qraw buffer, or null
+  int b, h0;
+  __device__ __forceinline__ float elem(int h, int dim) const {
+    if (tc_qraw<NCOL>()) {
+      return p.q_fmt == CFR_FMT_F32
+                 ? reinterpret_cast<const float *>(raw + h * 512)[dim]
+                 : __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t *>(raw + h * 512)[dim]) << 16);
+    }
+    const long long i = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + h]) * TC_D + dim;
+    return p.q_fmt == CFR_FMT_F32
+               ? static_cast<const float *>(p.q)[i]
+               : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
+  }
+  // elements 8 * ch .. 8 * ch + 7 of row h
+  __device__ __forceinline__ void chunk8(int h, int ch, float (&x)[8]) const {
+    if (p.q_fmt == CFR_FMT_F32) {
+      const float *src = tc_qraw<NCOL>()
+                             ? reinterpret_cast<const float *>(raw + h * 512) + 8 * ch
+                             : static_cast<const float *>(p.q) +
+                                   (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + h]) * TC_D + 8 * ch;
+      const float4 a = reinterpret_cast<const float4 *>(src)[0];
+      const float4 bb = reinterpret_cast<const float4 *>(src)[1];
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = bb.x; x[5] = bb.y; x[6] = bb.z; x[7] = bb.w;
+    } else {
+      const uint16_t *src = tc_qraw<NCOL>()
+                                ? reinterpret_cast<const uint16_t *>(raw + h * 512) + 8 * ch
+                                : static_cast<const uint16_t *>(p.q) +
+                                      (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + h]) * TC_D + 8 * ch;
+      const uint4 w = *reinterpret_cast<const uint4 *>(src);
+      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[2 * k] = bf16_lo(a[k]);
+        x[2 * k + 1] = bf16_hi(a[k]);
+      }
+    }
+  }
+};
 
 // writes the hi/lo query operand of item `it` (both bf16 and fp16 copies) and,
 // in IMMA variants, its int8 digit operand: row 4 * l + h holds digit l of head
 // h (h < 4) of q_h * 127 / max|q_h| = d0 + d1 / 128 + d2 / 128^2 + d3 / 128^3,
-// d0 in [-127, 127], d1..d3 in [-64, 64]; qsc[h] receives max|q_h| / 127.  The
+// d0 in [-127, 127], d1..d3 in [-64, 64]; qsc[h] receives max|q_h| / 127.  In
+// the 16-column variants the rows come from qraw buffer kq & 1 (kq counts the
+// items with tiles), which is handed back to producer warp 0 afterwards.  The
 // warpgroup's 128 threads (index tsm) share the work, each warp then arrives on
 // q_full.
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long long it, int tsm, int lane,
-                                           float (&qsc)[4]) {
+__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, const TcItem &it, int kq,
+                                           int tsm, int lane, float (&qsc)[4], bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
-  {
-    int slot, g;
-    item_coords(it, c.nsplit, slot, g);
-    const int b = split_at(p, slot).b;
-    const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
-    for (int idx = tsm; idx < NCOL * 16; idx += 128) {
-      const int n = idx >> 4, ch = idx & 15;  // row n, 8-element chunk ch of 16
-      constexpr int GM = NCOL / 2;            // rows [0, GM): hi parts, [GM, NCOL): lo parts
-      const bool lo_part = n >= GM;
-      const int head = lo_part ? n - GM : n;
-      float x[8];
+  const int h0 = p.grp_off[it.g], cnt = p.grp_off[it.g + 1] - h0;
+  const int buf = kq & 1;
+  if (tc_qraw<NCOL>())
+    (void)mbar_wait(&c.S.qraw_full[buf], static_cast<uint32_t>((kq >> 1) & 1), p.err, timed_out);
+  const TcQRows<NCOL> q{p, c.qraw + buf * TC_QRAW_BUF, it.b, h0};
+  for (int idx = tsm; idx < NCOL * 16; idx += 128) {
+    const int n = idx >> 4, ch = idx & 15;  // row n, 8-element chunk ch of 16
+    constexpr int GM = NCOL / 2;            // rows [0, GM): hi parts, [GM, NCOL): lo parts
+    const bool lo_part = n >= GM;
+    const int head = lo_part ? n - GM : n;
+    float x[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = 0.f;
-      if (head < cnt) {
-        const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * TC_D + 8 * ch;
-        if (p.q_fmt == CFR_FMT_F32) {
-          const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi);
-          const float4 bb = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi + 4);
-          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = bb.x; x[5] = bb.y; x[6] = bb.z; x[7] = bb.w;
-        } else {
-          const uint4 w = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + qi);
-          const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+    for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    if (head < cnt) q.chunk8(head, ch, x);
+    uint32_t wb[4], wh[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            x[2 * k] = bf16_lo(a[k]);
-            x[2 * k + 1] = bf16_hi(a[k]);
+    for (int k = 0; k < 4; ++k) {
+      float bl[2], fl[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float v = x[2 * k + e];
+        const float bh = __bfloat162float(__float2bfloat16_rn(v));
+        const float fh = __half2float(__float2half_rn(v));
+        bl[e] = lo_part ? v - bh : bh;
+        fl[e] = lo_part ? v - fh : fh;
+      }
+      wb[k] = pack_bf16(bl[0], bl[1]);
+      wh[k] = pack_f16(fl[0], fl[1]);
+    }
+    const int off = (ch >> 3) * (NCOL * 128) + sw128(n, ch & 7);
+    *reinterpret_cast<uint4 *>(c.qop + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    *reinterpret_cast<uint4 *>(c.qop + Cfg::Q_BYTES + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+  }
+  if constexpr (IMMA) {
+    static_assert(NCOL == 16, "int8 digit operand: 4 digits x 4 heads");
+    // max|q_h| over the 128 dims: thread tsm holds dim tsm of every head
+    const int warp4 = tsm >> 5;
+    float mx[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float v = 0.f;
+      if (h < cnt) v = fabsf(q.elem(h, tsm));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+      mx[h] = v;
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) c.S.red_l[warp4][h] = mx[h];
+    }
+    named_sync(2, 128);
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      qsc[h] = fmaxf(fmaxf(c.S.red_l[0][h], c.S.red_l[1][h]), fmaxf(c.S.red_l[2][h], c.S.red_l[3][h])) *
+               (1.f / 127.f);
+    named_sync(2, 128);  // red_l is free again (the partial write reuses it)
+    // row n = 4 * l + h, 16-dim chunk ch of it
+    const int n = tsm >> 3, ch = tsm & 7, l = n >> 2, h = n & 3;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (h < cnt && qsc[h] > 0.f) {
+      const float inv = 1.f / qsc[h];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float r = q.elem(h, 16 * ch + e) * inv;
+        float d = rintf(r);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          if (k < l) {
+            r = (r - d) * 128.f;
+            d = rintf(r);
           }
         }
+        w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(d)) & 0xFFu) << (8 * (e & 3));
       }
-      uint32_t wb[4], wh[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float bl[2], fl[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float v = x[2 * k + e];
-          const float bh = __bfloat162float(__float2bfloat16_rn(v));
-          const float fh = __half2float(__float2half_rn(v));
-          bl[e] = lo_part ? v - bh : bh;
-          fl[e] = lo_part ? v - fh : fh;
-        }
-        wb[k] = pack_bf16(bl[0], bl[1]);
-        wh[k] = pack_f16(fl[0], fl[1]);
-      }
-      const int off = (ch >> 3) * (NCOL * 128) + sw128(n, ch & 7);
-      *reinterpret_cast<uint4 *>(c.qop + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-      *reinterpret_cast<uint4 *>(c.qop + Cfg::Q_BYTES + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
     }
-    if constexpr (IMMA) {
-      static_assert(NCOL == 16, "int8 digit operand: 4 digits x 4 heads");
-      // max|q_h| over the 128 dims: thread tsm holds dim tsm of every head
-      const int warp4 = tsm >> 5;
-      float mx[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        float v = 0.f;
-        if (h < cnt) v = fabsf(q_elem(p, b, p.grp_heads[h0 + h], tsm));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        mx[h] = v;
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) c.S.red_l[warp4][h] = mx[h];
-      }
-      named_sync(2, 128);
-#pragma unroll
-      for (int h = 0; h < 4; ++h)
-        qsc[h] = fmaxf(fmaxf(c.S.red_l[0][h], c.S.red_l[1][h]), fmaxf(c.S.red_l[2][h], c.S.red_l[3][h])) *
-                 (1.f / 127.f);
-      named_sync(2, 128);  // red_l is free again (the partial write reuses it)
-      // row n = 4 * l + h, 16-dim chunk ch of it
-      const int n = tsm >> 3, ch = tsm & 7, l = n >> 2, h = n & 3;
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      if (h < cnt && qsc[h] > 0.f) {
-        const float inv = 1.f / qsc[h];
-        const int head = p.grp_heads[h0 + h];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float r = q_elem(p, b, head, 16 * ch + e) * inv;
-          float d = rintf(r);
-#pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            if (k < l) {
-              r = (r - d) * 128.f;
-              d = rintf(r);
-            }
-          }
-          w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(d)) & 0xFFu) << (8 * (e & 3));
-        }
-      }
-      *reinterpret_cast<uint4 *>(c.q8op + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    fence_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&c.S.q_full);
+    *reinterpret_cast<uint4 *>(c.q8op + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    mbar_arrive(&c.S.q_full);
+    if (tc_qraw<NCOL>()) mbar_arrive(&c.S.qraw_empty[buf]);  // this warp has read its rows
   }
 }
 
@@ -1108,19 +1188,17 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   bool q_ready = false;
   // the next item is read at the last tile of the current one (to write its
   // query operand early); nxt_read says whether that read has happened
-  int k = 0, nxt = -1;
+  int k = 0;
+  int kq = 0;  // items with tiles whose query operand has been written
+  TcItem nxt;
+  nxt.item = -1;
   bool nxt_read = false;
   float qs_nxt[4] = {0.f, 0.f, 0.f, 0.f};  // int8 digit scales of the last query operand written
 
-  for (int item = tc_read_item_wg(c, 0, 2, tsm, timed_out); item >= 0; ++k) {
-    int slot, g;
-    item_coords(item, c.nsplit, slot, g);
-    const SplitRange sr = split_at(p, slot);
-    const int b = sr.b, pb = sr.pb, pe = sr.pe;
-    const int n = p.seq_lens[b];
-    const int tok_end = min(n, pe * P);
+  for (TcItem it = tc_read_item_wg(c, 0, 2, tsm, timed_out); it.item >= 0; ++k) {
+    const int slot = it.slot, g = it.g, pb = it.pb, n = it.n, tok_end = it.t_end;
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
-    if (!q_ready && pb * P < tok_end) tc_write_q(c, item, tsm, lane, qs_nxt);
+    if (!q_ready && pb * P < tok_end) tc_write_q(c, it, kq++, tsm, lane, qs_nxt, timed_out);
     q_ready = false;
     nxt_read = false;
     float qs[4];  // this item's int8 digit scales (max|q_h| / 127)
@@ -1134,7 +1212,11 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
     uint32_t qoff[2] = {0u, 0u};
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
-      slope2[h] = (p.slopes && h < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + h])] * kLog2e : 0.f;
+      // 0 past the group's rows and without ALiBi
+      if constexpr (tc_qraw<NCOL>())
+        slope2[h] = c.S.slope_bc[k & 1][h];
+      else
+        slope2[h] = (p.slopes && h < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + h])] * kLog2e : 0.f;
       if constexpr (FEAT == TC_FEAT_MULTI)
         if (h < cnt) qoff[h >> 3] |= static_cast<uint32_t>(row_offset(p, p.grp_heads[h0 + h])) << (4 * (h & 7));
       m_run[h] = -INFINITY;
@@ -1282,8 +1364,8 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         // last QK product has been read
         nxt = tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
         nxt_read = true;
-        if (nxt >= 0 && tc_item_has_tiles(c, nxt)) {
-          tc_write_q(c, nxt, tsm, lane, qs_nxt);
+        if (nxt.item >= 0 && nxt.pb * P < nxt.t_end) {
+          tc_write_q(c, nxt, kq++, tsm, lane, qs_nxt, timed_out);
           q_ready = true;
         }
       }
@@ -1330,14 +1412,17 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         if (h == tsm) mrun = m_run[h];
       if constexpr (FEAT == TC_FEAT_MULTI) {
         const int vh = p.grp_heads[h0 + tsm];
-        const float sl = p.slopes ? p.slopes[row_head(p, vh)] * kLog2e : 0.f;
+        float sl = 0.f;
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h == tsm) sl = slope2[h];
         if (mrun != -INFINITY) mrun = fmaf(sl, static_cast<float>(row_offset(p, vh)), mrun);
       }
       p.part_m[cidx] = mrun;
       p.part_l[cidx] = (c.S.red_l[0][tsm] + c.S.red_l[1][tsm]) + (c.S.red_l[2][tsm] + c.S.red_l[3][tsm]);
     }
     named_sync(2, 128);
-    item = nxt_read ? nxt : tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
+    it = nxt_read ? nxt : tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
   }
 }
 
@@ -1371,6 +1456,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&S.item_empty[i], TC_ITEM_READERS);
     }
     mbar_init(&S.q_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.qraw_full[i], 1);
+      mbar_init(&S.qraw_empty[i], 4);  // the softmax warps, once they read the rows
+    }
     mbar_init(&S.drain, 2);  // one commit from each MMA issuer
     fence_mbar_init();
   }
@@ -1397,7 +1486,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                   smem + L::pbuf,
                                   static_cast<long long>(nsplit) * p.Hkv,
                                   nsplit,
-                                  smem + L::q8};
+                                  smem + L::q8,
+                                  smem + L::qraw};
   bool timed_out = false;
   if (warp == 0 || warp == TC_PROD2_WARP) {
     tc_producer<NCOL, INTP, FEAT, IMMA>(c, &timed_out, warp == 0 ? 0 : 1);
