@@ -304,6 +304,19 @@ struct TcCtx {
   uint8_t *qraw;  // [2][TC_QRAW_BUF]: query rows of the next items (16-column variants)
 };
 
+// query rows one tile holds: 4 in IMMA variants (their int8 digit columns are 4
+// digits x 4 rows), else NCOL / 2 (hi + lo columns per row)
+template <int NCOL, bool IMMA>
+__host__ __device__ constexpr int tc_rows() {
+  return IMMA ? 4 : NCOL / 2;
+}
+
+// an int32 value |x| < 2^22 as fp32, exactly, with two full-rate operations:
+// 1.5 * 2^23 + x has x in its low mantissa bits
+__device__ __forceinline__ float small_i2f(float bits) {
+  return __int_as_float(__float_as_int(bits) + 0x4B400000) - 12582912.f;
+}
+
 // With IMMA, int8 and int4 tiles run kind::i8 MMAs on 8-bit operands: int8 codes
 // as stored, int4 codes widened to bytes (times 16, so that the sign needs no
 // extension), query and probability as base-128 / base-256 digit columns.
@@ -994,9 +1007,9 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
 // variant), column 4 * l + h holding digit l of head h
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long long i, uint32_t tmem, int lane,
-                                        int cnt, float (&acc)[NCOL / 2],
-                                        const float (&alpha_prev)[NCOL / 2], float vscale_prev,
-                                        bool oint, bool *timed_out) {
+                                        int cnt, float (&acc)[tc_rows<NCOL, IMMA>()],
+                                        const float (&alpha_prev)[tc_rows<NCOL, IMMA>()],
+                                        float vscale_prev, bool oint, bool *timed_out) {
   const int ob = static_cast<int>(i % TcCfg<NCOL, INTP>::O_BUFS);
   (void)mbar_wait(&c.S.o_full[ob], static_cast<uint32_t>((i / TcCfg<NCOL, INTP>::O_BUFS) & 1),
                   c.p.err, timed_out);
@@ -1008,21 +1021,20 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long l
   __syncwarp();
   if (lane == 0) mbar_arrive(&c.S.o_empty[ob]);
   if (IMMA && oint) {
-    // sum_l digit_l 256^-l in fp32 (every int32 product sum is below 2^23, exact)
+    // sum_l digit_l 256^-l in fp32 (every int32 product sum is below 2^22, exact)
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       if (h < cnt) {
-        float t = fmaf(static_cast<float>(__float_as_int(o[12 + h])), 1.f / 256.f,
-                       static_cast<float>(__float_as_int(o[8 + h])));
-        t = fmaf(t, 1.f / 256.f, static_cast<float>(__float_as_int(o[4 + h])));
-        t = fmaf(t, 1.f / 256.f, static_cast<float>(__float_as_int(o[h])));
+        float t = fmaf(small_i2f(o[12 + h]), 1.f / 256.f, small_i2f(o[8 + h]));
+        t = fmaf(t, 1.f / 256.f, small_i2f(o[4 + h]));
+        t = fmaf(t, 1.f / 256.f, small_i2f(o[h]));
         acc[h] = fmaf(acc[h], alpha_prev[h], t * vscale_prev);
       }
     }
     return;
   }
 #pragma unroll
-  for (int h = 0; h < NCOL / 2; ++h)
+  for (int h = 0; h < tc_rows<NCOL, IMMA>(); ++h)
     if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
 }
 
@@ -1174,7 +1186,8 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, con
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
-  constexpr int GM = NCOL / 2;  // most query heads per tile
+  constexpr int GM = NCOL / 2;  // offset of the lo columns of the 16-bit operands
+  constexpr int GH = tc_rows<NCOL, IMMA>();  // query rows a tile holds
   const DecodeParams &p = c.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
@@ -1207,11 +1220,11 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
 
     // folds lag two tiles behind the scores: tiles prev2 (older) and prev1 wait,
     // each with its rescale factors and V scale
-    float slope2[GM], m_run[GM], l_part[GM], acc[GM], alpha1[GM], alpha2[GM];
+    float slope2[GH], m_run[GH], l_part[GH], acc[GH], alpha1[GH], alpha2[GH];
     // causal offsets of the query rows, 4 bits each (at most 16 rows of offset <= 15)
     uint32_t qoff[2] = {0u, 0u};
 #pragma unroll
-    for (int h = 0; h < GM; ++h) {
+    for (int h = 0; h < GH; ++h) {
       // 0 past the group's rows and without ALiBi
       if constexpr (tc_qraw<NCOL>())
         slope2[h] = c.S.slope_bc[k & 1][h];
@@ -1256,43 +1269,42 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       // row constant slope * o, added back to its maximum at the partial write
       const int j = m.t0 + t;
       const float dist = static_cast<float>(n - 1 - j);
-      float s[GM];
+      float s[GH];
       if (IMMA && itile) {
         // column 4 * l + h: digit l of head h; sum_l S_l 128^-l, exact terms below 2^22
 #pragma unroll
-        for (int h = 0; h < GM; ++h) {
+        for (int h = 0; h < GH; ++h) {
           s[h] = -INFINITY;
           if (h < 4 && valid && h < cnt) {
-            float u = fmaf(static_cast<float>(__float_as_int(sv[12 + h])), 1.f / 128.f,
-                           static_cast<float>(__float_as_int(sv[8 + h])));
-            u = fmaf(u, 1.f / 128.f, static_cast<float>(__float_as_int(sv[4 + h])));
-            u = fmaf(u, 1.f / 128.f, static_cast<float>(__float_as_int(sv[h])));
+            float u = fmaf(small_i2f(sv[12 + h]), 1.f / 128.f, small_i2f(sv[8 + h]));
+            u = fmaf(u, 1.f / 128.f, small_i2f(sv[4 + h]));
+            u = fmaf(u, 1.f / 128.f, small_i2f(sv[h]));
             s[h] = fmaf(u, scale * qs[h], -slope2[h] * dist);
           }
         }
       } else {
 #pragma unroll
-        for (int h = 0; h < GM; ++h)
+        for (int h = 0; h < GH; ++h)
           s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
       }
       if (FEAT == TC_FEAT_MULTI && m.t0 + TC_T - 1 > n - p.nq) {
         // the tile reaches the query positions: row h sees tokens j <= n - 1 - offset_h
 #pragma unroll
-        for (int h = 0; h < GM; ++h)
+        for (int h = 0; h < GH; ++h)
           if (j > n - 1 - static_cast<int>((qoff[h >> 3] >> (4 * (h & 7))) & 15u)) s[h] = -INFINITY;
       }
       {
         int hm;
-        const float mx = warp_multi_max<GM>(s, lane, &hm);
+        const float mx = warp_multi_max<GH>(s, lane, &hm);
         // lanes whose bits below the last halving offset are zero hold head hm's max
-        if ((lane & ((32 / GM) - 1)) == 0) c.S.red_max[tc & 1][quarter][hm] = mx;
+        if ((lane & ((32 / GH) - 1)) == 0) c.S.red_max[tc & 1][quarter][hm] = mx;
       }
       // the P buffer of this tile must be free (P.V of tile tc-2 done)
       (void)mbar_wait(&c.S.p_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err, timed_out);
       named_sync(2, 128);
-      float pr[GM], alpha[GM], mt[GM];
+      float pr[GH], alpha[GH], mt[GH];
 #pragma unroll
-      for (int h4 = 0; h4 < GM; h4 += 4) {
+      for (int h4 = 0; h4 < GH; h4 += 4) {
         float4 a[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) a[q] = *reinterpret_cast<const float4 *>(&c.S.red_max[tc & 1][q][h4]);
@@ -1302,7 +1314,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         mt[h4 + 3] = fmaxf(fmaxf(a[0].w, a[1].w), fmaxf(a[2].w, a[3].w));
       }
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
+      for (int h = 0; h < GH; ++h) {
         const float m_new = fmaxf(m_run[h], mt[h]);
         if (m_new == -INFINITY) {
           alpha[h] = 1.f;
@@ -1316,20 +1328,17 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       }
       if (IMMA && itile) {
         // P^T row t: 16 unsigned digit columns, column 4 * l + h = digit l of
-        // p_h * 255 = e0 + e1 / 256 + e2 / 256^2 + e3 / 256^3 (floor digits, the
-        // last rounded; every e in [0, 255])
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        // p_h * 255 = e0 + e1 / 256 + e2 / 256^2 + e3 / 256^3: the bytes, most
+        // significant first, of X_h = round(p_h * 255 * 2^24) (< 2^32 for p <= 1)
+        uint32_t x[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          float x = pr[h] * 255.f;
-#pragma unroll
-          for (int l = 0; l < 4; ++l) {
-            const float d = l < 3 ? floorf(x) : fminf(rintf(x), 255.f);
-            w[l] |= static_cast<uint32_t>(d) << (8 * h);
-            x = (x - d) * 256.f;
-          }
-        }
-        *reinterpret_cast<uint4 *>(c.pop + (tc & 1) * Cfg::P_BYTES + t * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int h = 0; h < 4; ++h) x[h] = __float2uint_rn(pr[h] * 4278190080.f);
+        // transpose the 4 x 4 bytes: word l = byte 3 - l of x[0..3]
+        const uint32_t lo01 = prmt(x[0], x[1], 0x5140u), hi01 = prmt(x[0], x[1], 0x7362u);
+        const uint32_t lo23 = prmt(x[2], x[3], 0x5140u), hi23 = prmt(x[2], x[3], 0x7362u);
+        *reinterpret_cast<uint4 *>(c.pop + (tc & 1) * Cfg::P_BYTES + t * 16) =
+            make_uint4(prmt(hi01, hi23, 0x7632u), prmt(hi01, hi23, 0x5410u), prmt(lo01, lo23, 0x7632u),
+                       prmt(lo01, lo23, 0x5410u));
       } else {
         // P^T row t: columns [hi(0..GM) | lo(0..GM)]
         float colv[NCOL];
@@ -1337,7 +1346,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         for (int k = 0; k < NCOL; ++k) colv[k] = 0.f;
         const float pre = kind == KIND_BF16 ? 1.f : 32768.f;
 #pragma unroll
-        for (int h = 0; h < GM; ++h) {
+        for (int h = 0; h < GH; ++h) {
           const float x = pr[h] * pre;  // 0 for the padding heads h >= cnt
           const float xh = kind == KIND_BF16 ? __bfloat162float(__float2bfloat16_rn(x))
                                              : __half2float(__float2half_rn(x));
@@ -1375,7 +1384,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       vs2 = vs1;
       oi2 = oi1;
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
+      for (int h = 0; h < GH; ++h) {
         alpha2[h] = alpha1[h];
         alpha1[h] = alpha[h];
       }
@@ -1393,7 +1402,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
 
     // split partial: acc (dim t), m, and l summed over the 128 token slots
 #pragma unroll
-    for (int h = 0; h < GM; ++h) {
+    for (int h = 0; h < GH; ++h) {
       if (h < cnt) {
         const int head = p.grp_heads[h0 + h];
         p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * TC_D + t] = acc[h];
@@ -1408,13 +1417,13 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       const long long cidx = static_cast<long long>(slot) * p.Hq + p.grp_heads[h0 + tsm];
       float mrun = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < GM; ++h)
+      for (int h = 0; h < GH; ++h)
         if (h == tsm) mrun = m_run[h];
       if constexpr (FEAT == TC_FEAT_MULTI) {
         const int vh = p.grp_heads[h0 + tsm];
         float sl = 0.f;
 #pragma unroll
-        for (int h = 0; h < GM; ++h)
+        for (int h = 0; h < GH; ++h)
           if (h == tsm) sl = slope2[h];
         if (mrun != -INFINITY) mrun = fmaf(sl, static_cast<float>(row_offset(p, vh)), mrun);
       }
