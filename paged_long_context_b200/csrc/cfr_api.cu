@@ -103,11 +103,11 @@ int target_splits(int sms, int hkv, int per_sm = kItemsPerSmMixed) {
 constexpr size_t kItemCtrOffset = 64;
 
 struct WsLayout {
-  size_t header, split_off, splits, part_m, part_l, part_acc, total;
+  size_t header, split_off, splits, part_m, part_l, part_acc, qimg, qscale, total;
   int max_splits;
 };
 
-bool ws_layout(int batch, int hq, int d, int max_pages, int target, WsLayout *w) {
+bool ws_layout(int batch, int hq, int hkv, int d, int max_pages, int target, WsLayout *w) {
   // ceil(len / chunk) summed over at most two page ranges per sequence
   long long ms = static_cast<long long>(target) + 2LL * batch;
   const long long cap = static_cast<long long>(batch) * max_pages;
@@ -134,6 +134,15 @@ bool ws_layout(int batch, int hq, int d, int max_pages, int target, WsLayout *w)
   o = align_up(o, 256);
   w->part_acc = o;
   if (!mul_ok(mh, static_cast<size_t>(d) * 4, &t) || !add_ok(o, t, &o)) return false;
+  // query operand images of the tensor-core decode, one per (sequence, kv head)
+  size_t groups = 0;
+  if (!mul_ok(static_cast<size_t>(batch), static_cast<size_t>(hkv), &groups)) return false;
+  o = align_up(o, 1024);
+  w->qimg = o;
+  if (!mul_ok(groups, static_cast<size_t>(kQImgBytes), &t) || !add_ok(o, t, &o)) return false;
+  o = align_up(o, 256);
+  w->qscale = o;
+  if (!mul_ok(groups, 16, &t) || !add_ok(o, t, &o)) return false;
   w->total = align_up(o, 256);
   return true;
 }
@@ -253,7 +262,8 @@ size_t cfr_paged_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
   DeviceInfo di;
   if (!device_info(&di)) return 0;
   WsLayout w;
-  if (!ws_layout(batch, num_q_heads, head_dim, max_pages, target_splits(di.sms, num_kv_heads), &w))
+  if (!ws_layout(batch, num_q_heads, num_kv_heads, head_dim, max_pages,
+                 target_splits(di.sms, num_kv_heads), &w))
     return 0;
   return w.total;
 }
@@ -330,7 +340,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
                                                                          : kItemsPerSm;
   const int target = target_splits(di.sms, kv->num_kv_heads, per_sm);
   WsLayout w;
-  if (!ws_layout(batch, rows, kv->head_dim, max_pages, target, &w)) return CFR_ERR_OVERFLOW;
+  if (!ws_layout(batch, rows, kv->num_kv_heads, kv->head_dim, max_pages, target, &w))
+    return CFR_ERR_OVERFLOW;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return CFR_ERR_WORKSPACE;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -348,6 +359,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.num_splits = num_splits;
   p.max_splits = w.max_splits;
   p.item_ctr = item_ctr;
+  p.qimg = ws + w.qimg;
+  p.qscale = reinterpret_cast<float *>(ws + w.qscale);
   p.err = err_word;
   p.batch = batch;
   p.max_pages = max_pages;

@@ -21,6 +21,9 @@ namespace cfr {
 constexpr int kFmtCount = CFR_FMT_COUNT;
 constexpr int kMaxQHeads = 256;
 constexpr int kMaxGroup = 16;              // query heads per kv head
+// bytes of one query operand image of the tensor-core decode (16-column
+// variants): bf16 hi/lo rows, fp16 hi/lo rows, int8 digit rows
+constexpr int kQImgBytes = 16 * 256 * 2 + 16 * 128;
 
 // Parameters of one decode call, shared by both decode kernels.
 struct DecodeParams {
@@ -40,6 +43,8 @@ struct DecodeParams {
   const int32_t *num_splits; // [0] = S
   int max_splits;            // capacity of this call's split arrays (part_*, splits)
   uint32_t *item_ctr;   // [0] work items claimed past the first per CTA, [1] CTAs finished; or null
+  uint8_t *qimg;        // [B * Hkv][kQImgBytes]: query operand image of each (sequence, kv head)
+  float *qscale;        // [B * Hkv][4]: its int8 digit scales
   uint32_t *err;
   int q_fmt, uniform_fmt;
   int batch, max_pages, Hq, Hkv, D, P;

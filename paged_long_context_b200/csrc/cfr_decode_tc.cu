@@ -81,7 +81,7 @@ constexpr int TC_ITEM_READERS = 5;
 constexpr int TC_HALF = TC_T * 128;  // bytes of one 64-column half of a K or V tile
 constexpr int TC_OP_BYTES = 4 * TC_HALF;  // K (2 halves) + V (2 halves) = 64 KiB
 constexpr int TC_RAW_K = TC_T * TC_D;  // raw code offset of V inside a stage's V region (K at 0)
-constexpr int TC_QRAW_BUF = 8 * 512;   // query rows of one item (16-column variants: <= 8 rows of <= 512 B)
+
 constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2, KIND_FP8 = 3;
 // compile-time variants: plain decode, multi-query rows, sink + window subset
 constexpr int TC_FEAT_PLAIN = 0, TC_FEAT_MULTI = 1, TC_FEAT_SUBSET = 2;
@@ -115,6 +115,9 @@ struct TcCfg {
   static constexpr int Q_BYTES = NCOL * 256;       // [NCOL rows][128 cols] 16-bit, 2 halves
   // [NCOL rows][128 cols] int8 query digits (int8 MMAs, 16 columns only)
   static constexpr int Q8_BYTES = (INTP && NCOL == 16) ? NCOL * 128 : 0;
+  // one query operand buffer: bf16 hi/lo rows, then (quantised pools) fp16 hi/lo
+  // rows and int8 digit rows
+  static constexpr int QSTRIDE = INTP ? 2 * Q_BYTES + Q8_BYTES : Q_BYTES;
   static constexpr int P_BYTES = NCOL * TC_T * 2;  // [128 tokens][NCOL] 16-bit
   static constexpr int O_BUFS = 3;                 // O accumulators in flight (fold lags two tiles)
   static constexpr int TMEM_COLS = NCOL == 16 ? 128 : 256;  // S x2 + O x3 columns, power of two
@@ -134,17 +137,20 @@ struct TcSmem {
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[3], o_empty[3];
   uint64_t q_full, drain;
   uint64_t item_full[TC_ITEM_RING], item_empty[TC_ITEM_RING];
-  uint64_t qraw_full[2], qraw_empty[2];
+  uint64_t qbuf_full[2], qbuf_empty[2];  // query operand buffers (16-column variants)
   TcItem ring[TC_ITEM_RING];  // work item k in slot k % TC_ITEM_RING
   // ALiBi slope * log2(e) of its query rows (16-column variants)
   float ring_slope[TC_ITEM_RING][TcCfg<NCOL, INTP>::RING_SLOPES];
   TcItem item_bc[2][2];       // [softmax, staging][k & 1]: the item in a warpgroup
   float slope_bc[2][TcCfg<NCOL, INTP>::RING_SLOPES];  // [k & 1]: its slopes, for the softmax
+  // int8 digit scales of its query rows (16-column variants), and their copy for the softmax
+  float ring_qs[TC_ITEM_RING][TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 4 : 1];
+  float qs_bc[2][TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 4 : 1];
   uint32_t tmem_base;
   int flag_st[3];
   TcMeta meta[3];
   alignas(16) float red_max[2][4][16];
-  alignas(16) float red_l[4][16];  // also the per-warp max|q_h| of the int8 query digits
+  alignas(16) float red_l[4][16];
   typename TcCfg<NCOL, INTP>::PageCache pc[TC_PRODUCERS];
 };
 
@@ -153,10 +159,11 @@ struct TcLayout {
   static constexpr size_t head = (sizeof(TcSmem<NCOL, INTP>) + 1023) / 1024 * 1024;
   static constexpr size_t op = head;
   static constexpr size_t q = op + TcCfg<NCOL, INTP>::STAGES * static_cast<size_t>(TC_OP_BYTES);
+  // query operand buffers: one (32 columns, written by the softmax warpgroup) or
+  // two (16 columns, images copied by producer warp 0), QSTRIDE bytes apart
   static constexpr size_t q8 = q + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::Q_BYTES);
-  static constexpr size_t pbuf = q8 + static_cast<size_t>(TcCfg<NCOL, INTP>::Q8_BYTES);
-  static constexpr size_t qraw = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
-  static constexpr size_t total = qraw + (NCOL == 16 ? 2 * static_cast<size_t>(TC_QRAW_BUF) : 0);
+  static constexpr size_t pbuf = q + (NCOL == 16 ? 2 : 1) * static_cast<size_t>(TcCfg<NCOL, INTP>::QSTRIDE);
+  static constexpr size_t total = pbuf + 2 * static_cast<size_t>(TcCfg<NCOL, INTP>::P_BYTES);
   static constexpr size_t launch_bytes = total + 1024;  // slack for 1024-byte alignment
 };
 
@@ -300,8 +307,6 @@ struct TcCtx {
   uint8_t *op, *qop, *pop;
   long long nitems;
   int nsplit;
-  uint8_t *q8op;  // int8 query digits (IMMA variants)
-  uint8_t *qraw;  // [2][TC_QRAW_BUF]: query rows of the next items (16-column variants)
 };
 
 // query rows one tile holds: 4 in IMMA variants (their int8 digit columns are 4
@@ -376,9 +381,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 // every other role needs to know about it (split, sequence length, token range,
 // the ALiBi slopes of its query rows), so that no other role reads global
 // memory at an item boundary; a slot whose item is -1 ends every loop.  In the
-// 16-column variants warp 0 also bulk-copies the item's query rows into shared
-// memory (qraw), so that the softmax warpgroup builds the query operand without
-// a global round trip.  Two ways of choosing the items, by measurement:
+// 16-column variants warp 0 also bulk-copies the query operand image of the
+// item's (sequence, kv head) -- built once per decode by tc_qimage_kernel --
+// into query buffer kq & 1 (kq counting the items with tiles), so that no role
+// builds query operands inside the pipeline.  Two ways of choosing the items,
+// by measurement:
 //  - fixed: CTA x takes items x, x + grid, x + 2 grid, ...
 //  - claimed (bf16-only plain and multi-query decode): CTA x starts with item x
 //    and claims every further item from a global counter when producer warp 0
@@ -389,16 +396,16 @@ __host__ __device__ constexpr bool tc_claimed_items() {
   return !INTP && FEAT != TC_FEAT_SUBSET;
 }
 
-// query rows of one item staged in shared memory (16-column variants)
+// query operands as prebuilt images, double-buffered (16-column variants)
 template <int NCOL>
-__host__ __device__ constexpr bool tc_qraw() {
+__host__ __device__ constexpr bool tc_qimg() {
   return NCOL == 16;
 }
 
 // producer warp 0 (all lanes): takes item k, publishes it and (16-column
-// variants) starts the copy of its query rows into qraw buffer kq & 1, kq
-// counting the items with tiles.  Returns the item (item = -1 past the last, or
-// when a wait gave up).
+// variants) starts the copy of its query operand image into query buffer kq & 1,
+// kq counting the items with tiles.  Returns the item (item = -1 past the last,
+// or when a wait gave up).
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, int &kq,
                                                   bool *timed_out, int lane) {
@@ -429,26 +436,25 @@ __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> 
     d.n = p.seq_lens[d.b];
     d.t_end = min(d.n, d.pe * p.P);
     const int h0 = p.grp_off[d.g], cnt = p.grp_off[d.g + 1] - h0;
-    if (tc_qraw<NCOL>() && lane < NCOL / 2)
+    if (tc_qimg<NCOL>() && lane < NCOL / 2)
       c.S.ring_slope[s][lane] =
           (p.slopes && lane < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + lane])] * kLog2e : 0.f;
-    if (tc_qraw<NCOL>() && d.pb * p.P < d.t_end) {
-      // the query rows of the group, one bulk copy per row
+    if (tc_qimg<NCOL>() && d.pb * p.P < d.t_end) {
       const int buf = kq & 1;
-      const uint32_t rb = static_cast<uint32_t>(TC_D) * (p.q_fmt == CFR_FMT_F32 ? 4u : 2u);
+      const long long grp = static_cast<long long>(d.b) * p.Hkv + d.g;
+      constexpr uint32_t bytes = static_cast<uint32_t>(TcCfg<NCOL, INTP>::QSTRIDE);
       int qok = 1;
       if (lane == 0) {
-        qok = mbar_wait(&c.S.qraw_empty[buf], static_cast<uint32_t>((kq >> 1) & 1) ^ 1u, p.err,
+        qok = mbar_wait(&c.S.qbuf_empty[buf], static_cast<uint32_t>((kq >> 1) & 1) ^ 1u, p.err,
                         timed_out) ? 1 : 0;
-        if (qok) mbar_arrive_expect_tx(&c.S.qraw_full[buf], static_cast<uint32_t>(cnt) * rb);
+        if (qok) {
+          mbar_arrive_expect_tx(&c.S.qbuf_full[buf], bytes);
+          bulk_g2s(c.qop + buf * TcCfg<NCOL, INTP>::QSTRIDE, p.qimg + grp * kQImgBytes, bytes,
+                   &c.S.qbuf_full[buf]);
+        }
       }
-      if (!__shfl_sync(0xffffffffu, qok, 0)) {
-        d.item = -1;
-      } else if (lane < cnt) {
-        const uint8_t *src = static_cast<const uint8_t *>(p.q) +
-                             (static_cast<long long>(d.b) * p.Hq + p.grp_heads[h0 + lane]) * rb;
-        bulk_g2s(c.qraw + buf * TC_QRAW_BUF + lane * 512, src, rb, &c.S.qraw_full[buf]);
-      }
+      if (lane < 4) c.S.ring_qs[s][lane & (TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 3 : 0)] = p.qscale[grp * 4 + lane];
+      if (!__shfl_sync(0xffffffffu, qok, 0)) d.item = -1;
       ++kq;
     }
   }
@@ -505,10 +511,13 @@ __device__ __forceinline__ TcItem tc_read_item_wg(TcCtx<NCOL, INTP, FEAT, IMMA> 
     if (mbar_wait(&c.S.item_full[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1), c.p.err,
                   timed_out)) {
       d = c.S.ring[s];
-      if (tc_qraw<NCOL>() && bar == 2) {
+      if (tc_qimg<NCOL>() && bar == 2) {
 #pragma unroll
         for (int h = 0; h < TcCfg<NCOL, INTP>::RING_SLOPES; ++h)
           c.S.slope_bc[k & 1][h] = c.S.ring_slope[s][h];
+#pragma unroll
+        for (int h = 0; h < (TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 4 : 1); ++h)
+          c.S.qs_bc[k & 1][h] = c.S.ring_qs[s][h];
       }
       mbar_arrive(&c.S.item_empty[s]);
     }
@@ -896,13 +905,23 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
   int stage = 0;
   uint32_t phase = 0;
   long long tc = 0;
-  int q_items = 0;  // items with tiles so far: one q_full phase each
+  int q_items = 0;  // items with tiles so far: one query operand (phase or buffer) each
   for (int item_k = 0; !*timed_out; ++item_k) {
     const TcItem it = tc_read_item(c, item_k, timed_out, false);
     if (it.item < 0) break;
     const int pb = it.pb, tok_end = it.t_end;
     if (pb * P >= tok_end) continue;
-    if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(q_items++ & 1), p.err, timed_out)) break;
+    // the item's query operand: buffer q_items & 1 filled by producer warp 0
+    // (16 columns), or the one buffer the softmax warpgroup wrote (32 columns)
+    const int qb = tc_qimg<NCOL>() ? (q_items & 1) : 0;
+    if (tc_qimg<NCOL>()) {
+      if (!mbar_wait(&c.S.qbuf_full[qb], static_cast<uint32_t>((q_items >> 1) & 1), p.err, timed_out))
+        break;
+    } else if (!mbar_wait(&c.S.q_full, static_cast<uint32_t>(q_items & 1), p.err, timed_out)) {
+      break;
+    }
+    ++q_items;
+    const uint32_t qop = q0 + static_cast<uint32_t>(qb * Cfg::QSTRIDE);
     for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
       if (!mbar_wait(&c.S.op_full[stage], phase, p.err, timed_out)) break;
       if (!mbar_wait(&c.S.s_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err,
@@ -915,7 +934,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
       if (tc_int_tile<IMMA>(kind)) {
         // int8 codes [128 tok][128 dims] x query digits [NCOL][128 dims], K = 32 per MMA
         const uint32_t idesc = tc_idesc_i8(1, 0, 0, NCOL);
-        const uint32_t q8 = smem_u32(c.q8op);
+        const uint32_t q8 = qop + 2 * static_cast<uint32_t>(Cfg::Q_BYTES);
 #pragma unroll
         for (int k = 0; k < TC_D / 32; ++k) {
           const uint64_t a = tc_sdesc(kbase + k * 32, 16, 1024, 2);
@@ -924,7 +943,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
         }
       } else {
         const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
-        const uint32_t qbase = q0 + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
+        const uint32_t qbase = qop + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
 #pragma unroll
         for (int k = 0; k < TC_D / 16; ++k) {
           const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
@@ -939,6 +958,8 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
         phase ^= 1u;
       }
     }
+    // the buffer can be refilled once the item's products have read it
+    if (tc_qimg<NCOL>()) tc_commit(&c.S.qbuf_empty[qb]);
   }
   // drain: every MMA this thread issued has completed before TMEM is released
   tc_commit(&c.S.drain);
@@ -1038,68 +1059,32 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long l
     if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
 }
 
-// Query rows of one item: in the 16-column variants from the qraw buffer that
-// producer warp 0 filled (row h at h * 512 bytes), otherwise from global memory.
-template <int NCOL>
-struct TcQRows {
-  const DecodeParams &p;
-  const uint8_t *raw;  // qraw buffer, or null
-  int b, h0;
-  __device__ __forceinline__ float elem(int h, int dim) const {
-    if (tc_qraw<NCOL>()) {
-      return p.q_fmt == CFR_FMT_F32
-                 ? reinterpret_cast<const float *>(raw + h * 512)[dim]
-                 : __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t *>(raw + h * 512)[dim]) << 16);
-    }
-    const long long i = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + h]) * TC_D + dim;
-    return p.q_fmt == CFR_FMT_F32
-               ? static_cast<const float *>(p.q)[i]
-               : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
-  }
-  // elements 8 * ch .. 8 * ch + 7 of row h
-  __device__ __forceinline__ void chunk8(int h, int ch, float (&x)[8]) const {
-    if (p.q_fmt == CFR_FMT_F32) {
-      const float *src = tc_qraw<NCOL>()
-                             ? reinterpret_cast<const float *>(raw + h * 512) + 8 * ch
-                             : static_cast<const float *>(p.q) +
-                                   (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + h]) * TC_D + 8 * ch;
-      const float4 a = reinterpret_cast<const float4 *>(src)[0];
-      const float4 bb = reinterpret_cast<const float4 *>(src)[1];
-      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = bb.x; x[5] = bb.y; x[6] = bb.z; x[7] = bb.w;
-    } else {
-      const uint16_t *src = tc_qraw<NCOL>()
-                                ? reinterpret_cast<const uint16_t *>(raw + h * 512) + 8 * ch
-                                : static_cast<const uint16_t *>(p.q) +
-                                      (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + h]) * TC_D + 8 * ch;
-      const uint4 w = *reinterpret_cast<const uint4 *>(src);
-      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        x[2 * k] = bf16_lo(a[k]);
-        x[2 * k + 1] = bf16_hi(a[k]);
-      }
-    }
-  }
-};
+// element `dim` of query row vh of sequence b, as fp32
+__device__ __forceinline__ float q_elem(const DecodeParams &p, int b, int vh, int dim) {
+  const long long i = (static_cast<long long>(b) * p.Hq + vh) * TC_D + dim;
+  return p.q_fmt == CFR_FMT_F32
+             ? static_cast<const float *>(p.q)[i]
+             : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
+}
 
-// writes the hi/lo query operand of item `it` (both bf16 and fp16 copies) and,
-// in IMMA variants, its int8 digit operand: row 4 * l + h holds digit l of head
-// h (h < 4) of q_h * 127 / max|q_h| = d0 + d1 / 128 + d2 / 128^2 + d3 / 128^3,
-// d0 in [-127, 127], d1..d3 in [-64, 64]; qsc[h] receives max|q_h| / 127.  In
-// the 16-column variants the rows come from qraw buffer kq & 1 (kq counts the
-// items with tiles), which is handed back to producer warp 0 afterwards.  The
-// warpgroup's 128 threads (index tsm) share the work, each warp then arrives on
-// q_full.
-template <int NCOL, bool INTP, int FEAT, bool IMMA>
-__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, const TcItem &it, int kq,
-                                           int tsm, int lane, float (&qsc)[4], bool *timed_out) {
+// Builds the query operand of (sequence b, kv head g) at dst, in the shared-memory
+// layout the QK products read (dst is shared memory, or a global image that is
+// later copied byte for byte to a 1024-byte-aligned shared buffer):
+//  - dst: bf16 operand, NCOL rows x 128 dims (2 halves of 64), 128-byte swizzled:
+//    rows [0, NCOL/2) the hi parts of the group's query rows, rows [NCOL/2, NCOL)
+//    the lo parts (q - bf16(q));
+//  - dst + Q_BYTES (quantised pools): the same with fp16 hi/lo;
+//  - dst + 2 Q_BYTES (IMMA): int8 digit operand, row 4 * l + h = digit l of head
+//    h (h < 4) of q_h * 127 / max|q_h| = d0 + d1 / 128 + d2 / 128^2 + d3 / 128^3,
+//    d0 in [-127, 127], d1..d3 in [-64, 64]; qsc[h] receives max|q_h| / 127.
+// The 128 threads of a warpgroup or block (index tsm) share the work; the IMMA
+// part synchronises them once (sync()) through red[4][4] floats.
+template <int NCOL, bool INTP, bool IMMA, class Sync>
+__device__ __forceinline__ void tc_build_q(const DecodeParams &p, int b, int g, int tsm, int lane,
+                                           uint8_t *dst, float (*red)[4], Sync sync,
+                                           float (&qsc)[4]) {
   using Cfg = TcCfg<NCOL, INTP>;
-  const DecodeParams &p = c.p;
-  const int h0 = p.grp_off[it.g], cnt = p.grp_off[it.g + 1] - h0;
-  const int buf = kq & 1;
-  if (tc_qraw<NCOL>())
-    (void)mbar_wait(&c.S.qraw_full[buf], static_cast<uint32_t>((kq >> 1) & 1), p.err, timed_out);
-  const TcQRows<NCOL> q{p, c.qraw + buf * TC_QRAW_BUF, it.b, h0};
+  const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
   for (int idx = tsm; idx < NCOL * 16; idx += 128) {
     const int n = idx >> 4, ch = idx & 15;  // row n, 8-element chunk ch of 16
     constexpr int GM = NCOL / 2;            // rows [0, GM): hi parts, [GM, NCOL): lo parts
@@ -1108,7 +1093,22 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, con
     float x[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) x[e] = 0.f;
-    if (head < cnt) q.chunk8(head, ch, x);
+    if (head < cnt) {
+      const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * TC_D + 8 * ch;
+      if (p.q_fmt == CFR_FMT_F32) {
+        const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi);
+        const float4 bb = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = bb.x; x[5] = bb.y; x[6] = bb.z; x[7] = bb.w;
+      } else {
+        const uint4 w = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + qi);
+        const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[2 * k] = bf16_lo(a[k]);
+          x[2 * k + 1] = bf16_hi(a[k]);
+        }
+      }
+    }
     uint32_t wb[4], wh[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -1125,40 +1125,42 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, con
       wh[k] = pack_f16(fl[0], fl[1]);
     }
     const int off = (ch >> 3) * (NCOL * 128) + sw128(n, ch & 7);
-    *reinterpret_cast<uint4 *>(c.qop + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-    *reinterpret_cast<uint4 *>(c.qop + Cfg::Q_BYTES + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4 *>(dst + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    if (INTP) *reinterpret_cast<uint4 *>(dst + Cfg::Q_BYTES + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
   }
   if constexpr (IMMA) {
     static_assert(NCOL == 16, "int8 digit operand: 4 digits x 4 heads");
     // max|q_h| over the 128 dims: thread tsm holds dim tsm of every head
-    const int warp4 = tsm >> 5;
     float mx[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       float v = 0.f;
-      if (h < cnt) v = fabsf(q.elem(h, tsm));
+      if (h < cnt) v = fabsf(q_elem(p, b, p.grp_heads[h0 + h], tsm));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
       mx[h] = v;
     }
     if (lane == 0) {
 #pragma unroll
-      for (int h = 0; h < 4; ++h) c.S.red_l[warp4][h] = mx[h];
+      for (int h = 0; h < 4; ++h) red[tsm >> 5][h] = mx[h];
     }
-    named_sync(2, 128);
+    sync();
 #pragma unroll
     for (int h = 0; h < 4; ++h)
-      qsc[h] = fmaxf(fmaxf(c.S.red_l[0][h], c.S.red_l[1][h]), fmaxf(c.S.red_l[2][h], c.S.red_l[3][h])) *
-               (1.f / 127.f);
-    named_sync(2, 128);  // red_l is free again (the partial write reuses it)
+      qsc[h] = fmaxf(fmaxf(red[0][h], red[1][h]), fmaxf(red[2][h], red[3][h])) * (1.f / 127.f);
     // row n = 4 * l + h, 16-dim chunk ch of it
     const int n = tsm >> 3, ch = tsm & 7, l = n >> 2, h = n & 3;
+    float sc = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k == h) sc = qsc[k];
     uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (h < cnt && qsc[h] > 0.f) {
-      const float inv = 1.f / qsc[h];
+    if (h < cnt && sc > 0.f) {
+      const float inv = 1.f / sc;
+      const int head = p.grp_heads[h0 + h];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        float r = q.elem(h, 16 * ch + e) * inv;
+        float r = q_elem(p, b, head, 16 * ch + e) * inv;
         float d = rintf(r);
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
@@ -1170,14 +1172,38 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, con
         w[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(d)) & 0xFFu) << (8 * (e & 3));
       }
     }
-    *reinterpret_cast<uint4 *>(c.q8op + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4 *>(dst + 2 * Cfg::Q_BYTES + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
+}
+
+// 32-column variants: the softmax warpgroup writes the query operand of item
+// `it` into the one query buffer, then each warp arrives on q_full.
+template <int NCOL, bool INTP, int FEAT, bool IMMA>
+__device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, const TcItem &it, int tsm,
+                                           int lane) {
+  float unused[4];  // (int8 digit operands exist only in 16-column variants)
+  tc_build_q<NCOL, INTP, false>(c.p, it.b, it.g, tsm, lane, c.qop,
+                                reinterpret_cast<float (*)[4]>(c.S.red_l), [] {}, unused);
   fence_async_smem();
   __syncwarp();
-  if (lane == 0) {
-    mbar_arrive(&c.S.q_full);
-    if (tc_qraw<NCOL>()) mbar_arrive(&c.S.qraw_empty[buf]);  // this warp has read its rows
-  }
+  if (lane == 0) mbar_arrive(&c.S.q_full);
+}
+
+// The query operand image of every (sequence, kv head), one 128-thread block
+// each, for the 16-column variants: built once per decode call, copied into
+// shared memory for every work item of the group.  Sequences outside
+// [1, max_pages * page_tokens] are skipped (the decode skips them too).
+template <int NCOL, bool INTP, bool IMMA>
+__global__ void __launch_bounds__(128) tc_qimage_kernel(const __grid_constant__ DecodeParams p) {
+  __shared__ float red[4][4];
+  const long long grp = blockIdx.x;
+  const int b = static_cast<int>(grp / p.Hkv), g = static_cast<int>(grp % p.Hkv);
+  const int n = p.seq_lens[b];
+  if (n < p.nq || n > p.max_pages * p.P) return;
+  float qsc[4] = {0.f, 0.f, 0.f, 0.f};
+  tc_build_q<NCOL, INTP, IMMA>(p, b, g, threadIdx.x, threadIdx.x & 31, p.qimg + grp * kQImgBytes, red,
+                               [] { __syncthreads(); }, qsc);
+  if (threadIdx.x < 4) p.qscale[grp * 4 + threadIdx.x] = qsc[threadIdx.x];
 }
 
 // softmax / fold warpgroup.  Every thread waits on the mbarriers itself; a
@@ -1199,24 +1225,26 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   uint32_t phase = 0;
   long long tc = 0;
   bool q_ready = false;
-  // the next item is read at the last tile of the current one (to write its
-  // query operand early); nxt_read says whether that read has happened
+  // 32-column variants write the query operand themselves: the next item's is
+  // written at the last tile of the current one, right after its last QK product
+  // has been read; nxt_read says whether that read has happened
   int k = 0;
-  int kq = 0;  // items with tiles whose query operand has been written
   TcItem nxt;
   nxt.item = -1;
   bool nxt_read = false;
-  float qs_nxt[4] = {0.f, 0.f, 0.f, 0.f};  // int8 digit scales of the last query operand written
 
   for (TcItem it = tc_read_item_wg(c, 0, 2, tsm, timed_out); it.item >= 0; ++k) {
     const int slot = it.slot, g = it.g, pb = it.pb, n = it.n, tok_end = it.t_end;
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
-    if (!q_ready && pb * P < tok_end) tc_write_q(c, it, kq++, tsm, lane, qs_nxt, timed_out);
+    if constexpr (!tc_qimg<NCOL>())
+      if (!q_ready && pb * P < tok_end) tc_write_q(c, it, tsm, lane);
     q_ready = false;
     nxt_read = false;
-    float qs[4];  // this item's int8 digit scales (max|q_h| / 127)
+    float qs[4] = {0.f, 0.f, 0.f, 0.f};  // this item's int8 digit scales (max|q_h| / 127)
+    if constexpr (IMMA) {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) qs[h] = qs_nxt[h];
+      for (int h = 0; h < 4; ++h) qs[h] = c.S.qs_bc[k & 1][h];
+    }
 
     // folds lag two tiles behind the scores: tiles prev2 (older) and prev1 wait,
     // each with its rescale factors and V scale
@@ -1226,7 +1254,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
 #pragma unroll
     for (int h = 0; h < GH; ++h) {
       // 0 past the group's rows and without ALiBi
-      if constexpr (tc_qraw<NCOL>())
+      if constexpr (tc_qimg<NCOL>())
         slope2[h] = c.S.slope_bc[k & 1][h];
       else
         slope2[h] = (p.slopes && h < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + h])] * kLog2e : 0.f;
@@ -1368,13 +1396,13 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.S.p_full[tc & 1]);
 
-      if (t0 + TC_T >= tok_end) {
+      if (!tc_qimg<NCOL>() && t0 + TC_T >= tok_end) {
         // the next item's query operand can be written as soon as this item's
         // last QK product has been read
         nxt = tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
         nxt_read = true;
         if (nxt.item >= 0 && nxt.pb * P < nxt.t_end) {
-          tc_write_q(c, nxt, kq++, tsm, lane, qs_nxt, timed_out);
+          tc_write_q(c, nxt, tsm, lane);
           q_ready = true;
         }
       }
@@ -1466,8 +1494,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     mbar_init(&S.q_full, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.qraw_full[i], 1);
-      mbar_init(&S.qraw_empty[i], 4);  // the softmax warps, once they read the rows
+      mbar_init(&S.qbuf_full[i], 1);
+      mbar_init(&S.qbuf_empty[i], 1);  // the QK issuer's commit after the item's last product
     }
     mbar_init(&S.drain, 2);  // one commit from each MMA issuer
     fence_mbar_init();
@@ -1494,9 +1522,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                   smem + L::q,
                                   smem + L::pbuf,
                                   static_cast<long long>(nsplit) * p.Hkv,
-                                  nsplit,
-                                  smem + L::q8,
-                                  smem + L::qraw};
+                                  nsplit};
   bool timed_out = false;
   if (warp == 0 || warp == TC_PROD2_WARP) {
     tc_producer<NCOL, INTP, FEAT, IMMA>(c, &timed_out, warp == 0 ? 0 : 1);
@@ -1592,7 +1618,12 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  // a plain launch: overlapping this kernel's start with the schedule kernel
+  if constexpr (tc_qimg<NCOL>()) {
+    // the query operand image of every (sequence, kv head)
+    const long long groups = static_cast<long long>(p.batch) * p.Hkv;
+    tc_qimage_kernel<NCOL, INTP, IMMA><<<dim3(static_cast<unsigned>(groups)), dim3(128), 0, stream>>>(p);
+  }
+  // a plain launch: overlapping this kernel's start with the previous kernel
   // (programmatic dependent launch) measured slower for this kernel
   tc_decode_kernel<NCOL, INTP, FEAT, IMMA><<<dim3(grid), dim3(TC_THREADS), smem, stream>>>(p, maps);
   e = cudaSuccess;
