@@ -129,8 +129,10 @@ size_t cfr_paged_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
  *              every page has format uniform_fmt.
  *  head_map    host, int32 [num_q_heads]: kv head of each query head, or NULL:
  *              h -> h / (num_q_heads / num_kv_heads) (MHA, MQA, GQA; CFR-Atlas
- *              page, "MHA/MQA/GQA head mapping").  At most 16 query heads may
- *              share one kv head.
+ *              page, "MHA/MQA/GQA head mapping").  The query heads of a kv head
+ *              are decoded together, reading its pages once, in groups of at
+ *              most 16: a kv head serving more (MQA, wide GQA) has its pages
+ *              read once per group of 16.
  *  alibi_slopes device, float [num_q_heads] or NULL: bias -slope_h * (n_b - 1 - j) is
  *              added to the score of token j (CFR-Atlas page, "RoPE/ALiBi
  *              positional policy").
@@ -231,10 +233,12 @@ cfr_status cfr_paged_decode_sink_window(const void *q, int32_t q_fmt, const cfr_
  *  out  device float [batch][num_queries][num_q_heads][head_dim];
  *  lse  device float [batch][num_queries][num_q_heads] or NULL.
  *  workspace  >= cfr_paged_decode_workspace_size(batch, num_q_heads * num_queries, ...).
- * Every K/V page is read once for all Q queries of the kv head's group: the
- * query rows (qi, h) of one kv head form its group, at most 16 rows
- * (num_queries * query heads per kv head <= 16, CFR_ERR_UNSUPPORTED otherwise;
- * num_queries in [1, 16], CFR_ERR_INVALID_ARG below 1).  A sequence with
+ * Every K/V page is read once for all Q queries of a kv head's group: the
+ * query rows (qi, h) of one kv head are decoded together in groups of at most
+ * 16 rows (num_queries * query heads per kv head above 16 makes several
+ * groups, each reading the kv head's pages).  num_queries in [1, 16]
+ * (CFR_ERR_INVALID_ARG below 1, CFR_ERR_UNSUPPORTED above 16); at most 256
+ * query rows (num_queries * num_q_heads) per sequence.  A sequence with
  * n_b < num_queries gets out = 0 and lse = -inf for every row and sets
  * CFR_DEVERR_SEQ_LEN.  `phases` as for cfr_paged_decode_phases.
  */

@@ -134,9 +134,11 @@ bool ws_layout(int batch, int hq, int hkv, int d, int max_pages, int target, WsL
   o = align_up(o, 256);
   w->part_acc = o;
   if (!mul_ok(mh, static_cast<size_t>(d) * 4, &t) || !add_ok(o, t, &o)) return false;
-  // query operand images of the tensor-core decode, one per (sequence, kv head)
+  // query operand images of the tensor-core decode, one per (sequence, row
+  // group); a kv head's rows make at most count / kMaxGroup + 1 groups
   size_t groups = 0;
-  if (!mul_ok(static_cast<size_t>(batch), static_cast<size_t>(hkv), &groups)) return false;
+  const size_t ngmax = static_cast<size_t>(hkv) + (static_cast<size_t>(hq) + kMaxGroup - 1) / kMaxGroup;
+  if (!mul_ok(static_cast<size_t>(batch), ngmax, &groups)) return false;
   o = align_up(o, 1024);
   w->qimg = o;
   if (!mul_ok(groups, static_cast<size_t>(kQImgBytes), &t) || !add_ok(o, t, &o)) return false;
@@ -192,16 +194,31 @@ cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *
     if (g < 0 || g >= hkv) return CFR_ERR_INVALID_ARG;
     count[g] += nq;
   }
-  int gmax = 0, off = 0;
+  // the rows of each kv head in order; a kv head with more than kMaxGroup rows
+  // (MQA, wide GQA, many query tokens) is cut into ceil(count / kMaxGroup)
+  // groups of near-equal size
+  int start[kMaxQHeads + 1];
+  int off = 0;
   for (int g = 0; g < hkv; ++g) {
-    p->grp_off[g] = static_cast<int16_t>(off);
+    start[g] = off;
     off += count[g];
-    if (count[g] > gmax) gmax = count[g];
   }
-  p->grp_off[hkv] = static_cast<int16_t>(off);
-  if (gmax > kMaxGroup) return CFR_ERR_UNSUPPORTED;
+  int gmax = 0, ng = 0;
+  for (int g = 0; g < hkv; ++g) {
+    const int nblk = count[g] <= kMaxGroup ? 1 : (count[g] + kMaxGroup - 1) / kMaxGroup;
+    for (int j = 0; j < nblk; ++j) {
+      const int lo = start[g] + count[g] * j / nblk, hi = start[g] + count[g] * (j + 1) / nblk;
+      if (ng >= kMaxGroups) return CFR_ERR_UNSUPPORTED;
+      p->grp_off[ng] = static_cast<int16_t>(lo);
+      p->grp_kv[ng] = static_cast<int16_t>(g);
+      if (hi - lo > gmax) gmax = hi - lo;
+      ++ng;
+    }
+  }
+  p->grp_off[ng] = static_cast<int16_t>(off);
+  p->ngroups = ng;
   int fill[kMaxQHeads];
-  for (int g = 0; g < hkv; ++g) fill[g] = p->grp_off[g];
+  for (int g = 0; g < hkv; ++g) fill[g] = start[g];
   for (int vh = 0; vh < rows; ++vh) {
     const int h = vh % hq;
     const int g = head_map ? head_map[h] : h / (hq / hkv);
@@ -338,7 +355,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   const int per_sm = use_tc && !quantised_pools(p, page_fmt != nullptr) ? kItemsPerSmClaimed
                      : page_fmt                                          ? kItemsPerSmMixed
                                                                          : kItemsPerSm;
-  const int target = target_splits(di.sms, kv->num_kv_heads, per_sm);
+  const int target = target_splits(di.sms, p.ngroups, per_sm);
   WsLayout w;
   if (!ws_layout(batch, rows, kv->num_kv_heads, kv->head_dim, max_pages, target, &w))
     return CFR_ERR_OVERFLOW;

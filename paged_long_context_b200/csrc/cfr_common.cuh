@@ -20,7 +20,10 @@ namespace cfr {
 
 constexpr int kFmtCount = CFR_FMT_COUNT;
 constexpr int kMaxQHeads = 256;
-constexpr int kMaxGroup = 16;              // query heads per kv head
+constexpr int kMaxGroup = 16;              // query rows of one work-item group
+// groups: a kv head with more than kMaxGroup query rows is split into several
+// groups of at most kMaxGroup rows (each reads the kv head's pages itself)
+constexpr int kMaxGroups = kMaxQHeads + kMaxQHeads / kMaxGroup;
 // bytes of one query operand image of the tensor-core decode (16-column
 // variants): bf16 hi/lo rows, fp16 hi/lo rows, int8 digit rows
 constexpr int kQImgBytes = 16 * 256 * 2 + 16 * 128;
@@ -43,8 +46,8 @@ struct DecodeParams {
   const int32_t *num_splits; // [0] = S
   int max_splits;            // capacity of this call's split arrays (part_*, splits)
   uint32_t *item_ctr;   // [0] work items claimed past the first per CTA, [1] CTAs finished; or null
-  uint8_t *qimg;        // [B * Hkv][kQImgBytes]: query operand image of each (sequence, kv head)
-  float *qscale;        // [B * Hkv][4]: its int8 digit scales
+  uint8_t *qimg;        // [B * ngroups][kQImgBytes]: query operand image of each (sequence, group)
+  float *qscale;        // [B * ngroups][4]: its int8 digit scales
   uint32_t *err;
   int q_fmt, uniform_fmt;
   int batch, max_pages, Hq, Hkv, D, P;
@@ -55,7 +58,9 @@ struct DecodeParams {
   int sink, window;     // window > 0: only tokens j < sink or j >= n - window take part
   int nq;               // query tokens per sequence (the last nq positions, causal)
   int hq_real;          // query heads; the Hq = nq * hq_real query rows are qi * hq_real + h
-  int16_t grp_off[kMaxQHeads + 1];  // heads of kv head g: grp_heads[grp_off[g] .. grp_off[g+1])
+  int ngroups;          // row groups (Hkv, or more when a kv head has over kMaxGroup rows)
+  int16_t grp_off[kMaxGroups + 1];  // rows of group g: grp_heads[grp_off[g] .. grp_off[g+1])
+  int16_t grp_kv[kMaxGroups];       // the kv head whose pages group g reads
   int16_t grp_heads[kMaxQHeads];
 };
 

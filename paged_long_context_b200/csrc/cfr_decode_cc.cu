@@ -220,7 +220,7 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
   const int P = p.P;
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
@@ -255,7 +255,7 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
         } else {
           f.ok = 1;
           if (is_quantised(fmt)) {
-            const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+            const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
             f.ks = s.x;
             f.vs = s.y;
           }
@@ -277,7 +277,7 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
           const long long cell = static_cast<long long>(b) * p.max_pages + pg;
           const long long id = p.page_table[cell];
           const int rb = row_bytes(f.fmt, D);
-          const long long off = ((id * p.Hkv + g) * P + tin) * rb;
+          const long long off = ((id * p.Hkv + p.grp_kv[g]) * P + tin) * rb;
           const uint8_t *ks = p.k_pool[f.fmt] + off;
           const uint8_t *vs = p.v_pool[f.fmt] + off;
           if (rb == p.pitch) {
@@ -314,7 +314,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_c
   __syncthreads();
   griddep_wait();  // the split schedule comes from the previous kernel
   const long long nitems =
-      static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.Hkv;
+      static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.ngroups;
   bool timed_out = false;
   if (threadIdx.x >= CC_WARPS * 32) {
     if (threadIdx.x == CC_WARPS * 32) cc_producer<D>(p, L, nitems, &timed_out);

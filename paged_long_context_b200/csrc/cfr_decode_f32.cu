@@ -132,7 +132,7 @@ __device__ __forceinline__ bool f32_produce_tile(const DecodeParams &p, const F3
     uint8_t *kst = ring + static_cast<size_t>(stage) * 2 * C::TILE_BYTES;
     uint8_t *vst = kst + C::TILE_BYTES;
     const int tin = (t0 + r) % P;
-    const int y = static_cast<int>((id * p.Hkv + g) * P + tin);
+    const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * P + tin);
 #pragma unroll
     for (int blk = 0; blk < C::NB; ++blk) {
       tma_load_2d(kst + blk * C::BLOCK_BYTES + r * 128, &maps.k, 32 * blk, y, &full[stage]);
@@ -161,7 +161,7 @@ __device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_
   page_cache_reset(pc, lane);
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
@@ -197,7 +197,7 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.Hkv), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
   __syncthreads();
   griddep_wait();  // the split schedule comes from the previous kernel
   const long long nitems =
-      static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.Hkv;
+      static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.ngroups;
   bool timed_out = false;
   if (threadIdx.x >= F_WARPS * 32) {
     f32_producer<D>(p, maps, S.full, S.empty, S.meta, ring, S.pc, nitems, &timed_out);

@@ -441,7 +441,7 @@ __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> 
           (p.slopes && lane < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + lane])] * kLog2e : 0.f;
     if (tc_qimg<NCOL>() && d.pb * p.P < d.t_end) {
       const int buf = kq & 1;
-      const long long grp = static_cast<long long>(d.b) * p.Hkv + d.g;
+      const long long grp = static_cast<long long>(d.b) * p.ngroups + d.g;
       constexpr uint32_t bytes = static_cast<uint32_t>(TcCfg<NCOL, INTP>::QSTRIDE);
       int qok = 1;
       if (lane == 0) {
@@ -602,12 +602,12 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     if (kind == KIND_BF16) {
       bytes = static_cast<uint32_t>(__popc(vb)) * 4u * box_rows * 128u;
     } else if (IMMA && kind == KIND_I8) {
-      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
       ks = sc.x;
       vs = sc.y;
       bytes = 2u * TC_T * 128u;  // one full 128-row box of K and of V
     } else {
-      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + g) * 2);
+      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
       ks = sc.x;
       vs = sc.y;
       bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, TC_D));
@@ -635,26 +635,26 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     const int r = lane * box_rows;
     uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
     if (kind == KIND_BF16) {
-      const int y = static_cast<int>((id * p.Hkv + g) * p.P + tin0);
+      const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
       tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, done);
       tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
       tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, done);
       tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
     } else if (IMMA && kind == KIND_I8) {
       // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows
-      const int y = static_cast<int>((id * p.Hkv + g) * p.P + tin0);
+      const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
       tma_load_2d(op, &c.maps.k8, 0, y, done);
       tma_load_2d(op + 2 * TC_HALF, &c.maps.v8, 0, y, done);
     } else if (IMMA && kind == KIND_I4) {
       // raw codes above the int8 operands the staging warps write (K at TC_HALF,
       // V at 3 * TC_HALF)
       const int rb = row_bytes(fmt, TC_D);
-      const long long off = ((id * p.Hkv + g) * p.P + tin0) * rb;
+      const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
       bulk_g2s(op + TC_HALF, p.k_pool[fmt] + off, rows * rb, done);
       bulk_g2s(op + 3 * TC_HALF, p.v_pool[fmt] + off, rows * rb, done);
     } else if (INTP) {
       const int rb = row_bytes(fmt, TC_D);
-      const long long off = ((id * p.Hkv + g) * p.P + tin0) * rb;
+      const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
       // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in);
       // the staging warps expand them in place
       uint8_t *raw = op + 2 * TC_HALF;
@@ -1197,7 +1197,7 @@ template <int NCOL, bool INTP, bool IMMA>
 __global__ void __launch_bounds__(128) tc_qimage_kernel(const __grid_constant__ DecodeParams p) {
   __shared__ float red[4][4];
   const long long grp = blockIdx.x;
-  const int b = static_cast<int>(grp / p.Hkv), g = static_cast<int>(grp % p.Hkv);
+  const int b = static_cast<int>(grp / p.ngroups), g = static_cast<int>(grp % p.ngroups);
   const int n = p.seq_lens[b];
   if (n < p.nq || n > p.max_pages * p.P) return;
   float qsc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1521,7 +1521,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                   smem + L::op,
                                   smem + L::q,
                                   smem + L::pbuf,
-                                  static_cast<long long>(nsplit) * p.Hkv,
+                                  static_cast<long long>(nsplit) * p.ngroups,
                                   nsplit};
   bool timed_out = false;
   if (warp == 0 || warp == TC_PROD2_WARP) {
@@ -1620,7 +1620,7 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
   if (e != cudaSuccess) return e;
   if constexpr (tc_qimg<NCOL>()) {
     // the query operand image of every (sequence, kv head)
-    const long long groups = static_cast<long long>(p.batch) * p.Hkv;
+    const long long groups = static_cast<long long>(p.batch) * p.ngroups;
     tc_qimage_kernel<NCOL, INTP, IMMA><<<dim3(static_cast<unsigned>(groups)), dim3(128), 0, stream>>>(p);
   }
   // a plain launch: overlapping this kernel's start with the previous kernel

@@ -437,12 +437,19 @@ def spec_alibi_1m() -> CaseSpec:
                     fmt="bf16", q_fmt="bf16", permute=True, alibi=True)
 
 
+def spec_mqa() -> CaseSpec:
+    """8 x 32,768 tokens, 32 q heads on 1 kv head (MQA), d 128, bf16, 256-token pages."""
+    return CaseSpec("mqa_b8_32k_32q1kv_p256_bf16", 8, 32, 1, 128, 256, seq_lens=[32768] * 8,
+                    fmt="bf16", q_fmt="bf16", permute=True)
+
+
 WORKLOADS = {
     "tiny": (spec_tiny_exact_fold, 1),
     "cfr": (spec_cfr_shaped, 2),
     "gqa": (spec_gqa_ragged, 3),
     "tiered": (spec_tiered, 4),
     "alibi1m": (spec_alibi_1m, 5),
+    "mqa": (spec_mqa, 6),
 }
 
 

@@ -106,10 +106,14 @@ def test_sequence_shorter_than_queries():
     check_mq(case, out, lse, sel=[(b, r) for b in (0, 2) for r in range(rows)])
 
 
-def test_group_too_large_is_rejected():
-    case = mq_case(4, Hq=16, Hkv=2)          # 8 heads x 4 queries = 32 rows per kv head
-    bufs = binding.DecodeBuffers(case)
-    assert binding.paged_decode_raw(case, bufs) == 2
+@pytest.mark.parametrize("fmt", ["bf16", "i8", "f32"])
+def test_more_than_16_rows_per_kv_head(fmt):
+    # 8 heads x 4 queries = 32 rows per kv head: decoded as two groups of 16
+    case = mq_case(4, Hq=16, Hkv=2, fmt=fmt, q_fmt="f32" if fmt == "f32" else "bf16",
+                   P=128 if fmt == "i8" else 64)
+    out, lse, err = run_mq(case)
+    assert err == 0
+    check_mq(case, out, lse)
 
 
 @pytest.mark.parametrize("name,Q", [("gqa", 4), ("alibi1m", 2)])
