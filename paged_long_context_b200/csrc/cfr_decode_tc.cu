@@ -29,23 +29,23 @@
 //
 // Warp roles (384 threads, one CTA per SM, persistent over work items =
 // (split of a sequence, kv head)):
-//   warps 0, 11 TMA producers, taking alternate tiles: resolve pages, bf16
+//   warps 0, 3  TMA producers, taking alternate tiles: resolve pages, bf16
 //               tiles by 2-D tensor-map boxes straight into the 128-byte-swizzled
 //               operand layout, int tiles by 1-D bulk copies of the raw rows.
 //               Resolving and issuing a tile of many small pages is a serial
 //               chain of dependent steps inside one warp, so two warps run two
 //               such chains at once.
 //   warp 1      TMEM allocation; lane 0 issues the QK products.
-//   warp 10     lane 0 issues the P.V products (a thread of its own, so the two
+//   warp 2      lane 0 issues the P.V products (a thread of its own, so the two
 //               kinds of MMA never wait for each other's issue).
-//   warps 2-5   softmax / fold: thread t owns TMEM lane t = token t of S and
+//   warps 4-7   softmax / fold: thread t owns TMEM lane t = token t of S and
 //               dim t of O.  Per tile: scores (scale, ALiBi from the integer
 //               distance), tile max across the 128 tokens, p = 2^(s - m),
 //               running normaliser, hi/lo split of p into the MMA's B operand,
 //               and the exact fold acc = acc*2^(m_old-m_new) + O_tile of the
 //               previous tile (CFR-Atlas page, "exact folded online-softmax
 //               attention pass").
-//   warps 6-9   staging: FP8/int8/int4 rows -> fp16 operand rows (int4 rows ->
+//   warps 8-11  staging: FP8/int8/int4 rows -> fp16 operand rows (int4 rows ->
 //               int8 rows in IMMA variants); zeroes V rows of 16-bit tiles for
 //               tokens that are not part of the input so stale or NaN bytes
 //               never meet a zero probability inside the MMA (8-bit codes are
@@ -71,10 +71,19 @@ namespace cfr {
 constexpr int TC_T = 128;            // tokens per tile
 constexpr int TC_D = 128;            // head_dim
 constexpr int TC_THREADS = 384;
+// warp roles, one warpgroup each for the register split (setmaxnreg):
+// warpgroup 0 = producers and MMA issuers, 1 = softmax, 2 = staging
 constexpr int TC_PRODUCERS = 2;      // producer warps 0 and TC_PROD2_WARP, alternate tiles
-constexpr int TC_PROD2_WARP = 11;
+constexpr int TC_PROD2_WARP = 3;
+constexpr int TC_QK_WARP = 1;
+constexpr int TC_PV_WARP = 2;
+constexpr int TC_SOFTMAX_T0 = 128;   // first thread of the softmax warpgroup (warps 4-7)
+constexpr int TC_STAGING_T0 = 256;   // first thread of the staging warpgroup (warps 8-11)
+// registers per thread of each warpgroup after the split; the launch gives
+// 384 x 168 = 64,512 and the split takes 128 x (104 + 224 + 136) = 59,392
+constexpr int TC_REGS_IO = 104, TC_REGS_SOFTMAX = 224, TC_REGS_STAGING = 136;
 // work items reach the CTA's warps through a ring of this many slots; every
-// slot is read by producer warp 11, the two MMA issuers and one thread of each of
+// slot is read by producer warp 3, the two MMA issuers and one thread of each of
 // the softmax and staging warpgroups
 constexpr int TC_ITEM_RING = 4;
 constexpr int TC_ITEM_READERS = 5;
@@ -465,7 +474,7 @@ __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> 
 }
 
 // item k read by one thread (an MMA issuer) or by every lane of a warp
-// (producer warp 11: lane 0 waits, reads and frees the slot, the lanes get the
+// (producer warp 3: lane 0 waits, reads and frees the slot, the lanes get the
 // fields by shuffles).  item = -1 past the last item or when the wait gave up.
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __device__ __forceinline__ TcItem tc_read_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c, int k, bool *timed_out,
@@ -733,7 +742,7 @@ template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   using Cfg = TcCfg<NCOL, INTP>;
   const DecodeParams &p = c.p;
-  const int r = threadIdx.x - 192;
+  const int r = threadIdx.x - TC_STAGING_T0;
   const int P = p.P;
   int stage = 0;
   uint32_t phase = 0;
@@ -965,7 +974,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
   tc_commit(&c.S.drain);
 }
 
-// P.V issuer (warp 10, one thread): for every tile in order, once its
+// P.V issuer (warp 2, one thread): for every tile in order, once its
 // probabilities are written and an O buffer is free, O^T = V^T . [p_hi | p_lo]^T
 // into TMEM; the commit then frees the stage, the P buffer and signals the fold.
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
@@ -1218,7 +1227,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;
   const int t = 32 * quarter + lane;  // TMEM lane: token t of S, dim t of O
-  const int tsm = threadIdx.x - 64;   // 0..127 within the warpgroup
+  const int tsm = threadIdx.x - TC_SOFTMAX_T0;  // 0..127 within the warpgroup
   const uint32_t tmem = c.S.tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
   const int P = p.P;
   int stage = 0;
@@ -1524,15 +1533,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                   static_cast<long long>(nsplit) * p.ngroups,
                                   nsplit};
   bool timed_out = false;
-  if (warp == 0 || warp == TC_PROD2_WARP) {
-    tc_producer<NCOL, INTP, FEAT, IMMA>(c, &timed_out, warp == 0 ? 0 : 1);
-  } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
-  } else if (warp == 10) {
-    if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
-  } else if (warp < 6) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(TC_REGS_IO));
+    if (warp == 0 || warp == TC_PROD2_WARP) {
+      tc_producer<NCOL, INTP, FEAT, IMMA>(c, &timed_out, warp == 0 ? 0 : 1);
+    } else if (warp == TC_QK_WARP) {
+      if ((threadIdx.x & 31) == 0) tc_qk_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
+    } else {
+      if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
+    }
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(TC_REGS_SOFTMAX));
     tc_softmax<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(TC_REGS_STAGING));
     tc_staging<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   }
   tc_fence_before();
