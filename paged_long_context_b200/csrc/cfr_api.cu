@@ -74,9 +74,10 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // (split x kv head) per SM, so that a persistent grid of one CTA per SM gets
 // an even share.  Every item pays one pipeline drain at its end and one more
 // partial for the merge.
-//  - The tcgen05 path over bf16-only pools balances at run time (its CTAs
-//    claim items from a counter, or the items are few per sequence), so it
-//    takes the fewest, longest items: 4 per SM measured faster than 8 or 16.
+//  - The tcgen05 path over bf16-only pools, and over uniform int8 / int4 pools
+//    in its int8-MMA variant, balances at run time (its CTAs claim items from a
+//    counter), so it takes the fewest, longest items: 4 per SM measured faster
+//    than 8 or 16.
 //  - Other uniform caches are shared out in a fixed pattern: 8 per SM.
 //  - A cache of mixed storage formats has items of unequal cost (a page of
 //    int4 codes is a quarter of the bytes of a bf16 page, but takes longer to
@@ -352,9 +353,13 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.uniform_fmt = uniform_fmt;
   const bool use_tc = tc_supported(p, page_fmt != nullptr);
   const bool use_f32 = !use_tc && f32_supported(p, page_fmt != nullptr);
-  const int per_sm = use_tc && !quantised_pools(p, page_fmt != nullptr) ? kItemsPerSmClaimed
-                     : page_fmt                                          ? kItemsPerSmMixed
-                                                                         : kItemsPerSm;
+  // the tcgen05 path claims its items at run time over bf16 pools and over
+  // uniform int8 / int4 pools of up to 4 rows per group (the int8-MMA variant)
+  const bool claimed =
+      use_tc && (!quantised_pools(p, page_fmt != nullptr) ||
+                 (!page_fmt && p.gmax <= 4 &&
+                  (uniform_fmt == CFR_FMT_I8 || uniform_fmt == CFR_FMT_I4)));
+  const int per_sm = claimed ? kItemsPerSmClaimed : page_fmt ? kItemsPerSmMixed : kItemsPerSm;
   const int target = target_splits(di.sms, p.ngroups, per_sm);
   WsLayout w;
   if (!ws_layout(batch, rows, kv->num_kv_heads, kv->head_dim, max_pages, target, &w))
@@ -375,7 +380,9 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.splits = splits;
   p.num_splits = num_splits;
   p.max_splits = w.max_splits;
-  p.item_ctr = item_ctr;
+  // mixed-format caches with quantised pages share their items out in a fixed
+  // pattern (no claim counter); see tc_claimed_items
+  p.item_ctr = (page_fmt && quantised_pools(p, true)) ? nullptr : item_ctr;
   p.qimg = ws + w.qimg;
   p.qscale = reinterpret_cast<float *>(ws + w.qscale);
   p.err = err_word;

@@ -396,13 +396,16 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 // builds query operands inside the pipeline.  Two ways of choosing the items,
 // by measurement:
 //  - fixed: CTA x takes items x, x + grid, x + 2 grid, ...
-//  - claimed (bf16-only plain and multi-query decode): CTA x starts with item x
-//    and claims every further item from a global counter when producer warp 0
+//  - claimed (plain and multi-query decode over bf16 pools, or over int8 / int4
+//    pools of one format in the IMMA variants): CTA x starts with item x and
+//    claims every further item from a global counter when producer warp 0
 //    reaches it, so SMs that the memory system serves faster take more items and
-//    all CTAs finish together.
+//    all CTAs finish together.  Over pools of mixed formats the items differ in
+//    cost several-fold and the fixed share measured faster; the host then passes
+//    no counter (item_ctr = null), which selects the fixed share.
 template <bool INTP, int FEAT, bool IMMA>
 __host__ __device__ constexpr bool tc_claimed_items() {
-  return !INTP && FEAT != TC_FEAT_SUBSET;
+  return (!INTP || IMMA) && FEAT != TC_FEAT_SUBSET;
 }
 
 // query operands as prebuilt images, double-buffered (16-column variants)
