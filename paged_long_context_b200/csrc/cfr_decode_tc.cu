@@ -82,6 +82,23 @@ constexpr int TC_STAGING_T0 = 256;   // first thread of the staging warpgroup (w
 // registers per thread of each warpgroup after the split; the launch gives
 // 384 x 168 = 64,512 and the split takes 128 x (104 + 224 + 136) = 59,392
 constexpr int TC_REGS_IO = 104, TC_REGS_SOFTMAX = 224, TC_REGS_STAGING = 136;
+// registers per thread at launch: the register file (65,536) over the block's
+// threads, rounded down to the allocation unit of 8 (what __launch_bounds__ with
+// one block per SM gives ptxas); the launch checks the kernel really has it
+constexpr int TC_REGS_LAUNCH = 65536 / TC_THREADS / 8 * 8;
+static_assert(128 * (TC_REGS_IO + TC_REGS_SOFTMAX + TC_REGS_STAGING) <= TC_REGS_LAUNCH * TC_THREADS,
+              "the split must fit the registers the block was launched with");
+
+// move this warpgroup's register count to N: setmaxnreg.dec below the launch
+// count, .inc above it (a decrease must not name a larger count)
+template <int N>
+__device__ __forceinline__ void tc_setmaxnreg() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+  if constexpr (N < TC_REGS_LAUNCH)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+  else if constexpr (N > TC_REGS_LAUNCH)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 // work items reach the CTA's warps through a ring of this many slots; every
 // slot is read by producer warp 3, the two MMA issuers and one thread of each of
 // the softmax and staging warpgroups
@@ -143,7 +160,8 @@ struct TcCfg {
 template <int NCOL, bool INTP>
 struct TcSmem {
   uint64_t op_full[3], op_empty[3], raw_full[3];
-  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[3], o_empty[3];
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t o_full[TcCfg<NCOL, INTP>::O_BUFS], o_empty[TcCfg<NCOL, INTP>::O_BUFS];
   uint64_t q_full, drain;
   uint64_t item_full[TC_ITEM_RING], item_empty[TC_ITEM_RING];
   uint64_t qbuf_full[2], qbuf_empty[2];  // query operand buffers (16-column variants)
@@ -1496,7 +1514,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&S.p_full[i], 4);
       mbar_init(&S.p_empty[i], 1);
     }
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < TcCfg<NCOL, INTP>::O_BUFS; ++i) {
       mbar_init(&S.o_full[i], 1);
       mbar_init(&S.o_empty[i], 4);
     }
@@ -1537,7 +1555,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                   nsplit};
   bool timed_out = false;
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(TC_REGS_IO));
+    tc_setmaxnreg<TC_REGS_IO>();
     if (warp == 0 || warp == TC_PROD2_WARP) {
       tc_producer<NCOL, INTP, FEAT, IMMA>(c, &timed_out, warp == 0 ? 0 : 1);
     } else if (warp == TC_QK_WARP) {
@@ -1546,10 +1564,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if ((threadIdx.x & 31) == 0) tc_pv_issuer<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
     }
   } else if (warp < 8) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(TC_REGS_SOFTMAX));
+    tc_setmaxnreg<TC_REGS_SOFTMAX>();
     tc_softmax<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(TC_REGS_STAGING));
+    tc_setmaxnreg<TC_REGS_STAGING>();
     tc_staging<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   }
   tc_fence_before();
@@ -1635,6 +1653,14 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  // the warpgroups' register split assumes the launch count it was written for
+  static const int launch_regs = [] {
+    cudaFuncAttributes fa;
+    return cudaFuncGetAttributes(&fa, tc_decode_kernel<NCOL, INTP, FEAT, IMMA>) == cudaSuccess
+               ? fa.numRegs
+               : -1;
+  }();
+  if (launch_regs != TC_REGS_LAUNCH) return cudaErrorInvalidConfiguration;
   if constexpr (tc_qimg<NCOL>()) {
     // the query operand image of every (sequence, kv head)
     const long long groups = static_cast<long long>(p.batch) * p.ngroups;
