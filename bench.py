@@ -403,6 +403,12 @@ def run_ours(args, dist):
             flush.fill_(1.0)
         full_step()
     torch.cuda.synchronize()
+    # this library's kernels per step, counted from the device's own launch
+    # record (outside the timed regions): the public call, and the phase-split
+    # step of timed region 2
+    n_full, names_full = count_launches(full_step)
+    n_phased, names_phased = count_launches(
+        lambda: phased_step([torch.cuda.Event(enable_timing=True) for _ in range(2)]))
 
     # timed region 1: K steps through the public call (schedule, decode, merge
     # launched back to back as a caller sees them)
@@ -544,12 +550,37 @@ def run_ours(args, dist):
         "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": round(e2e_ms * 1e3, 2)},
-        "gpu_launches": 3 * K,
-        "gpu_launches_note": "3 per step (schedule, decode, merge); region 2 repeats them for the kernel time",
+        "gpu_launches": (n_full + n_phased) * K if n_full is not None else None,
+        "gpu_launches_note": (
+            f"{n_full} per step through the public call ({', '.join(names_full)}); the "
+            f"kernel-time region repeats each step as separate schedule, decode and merge "
+            f"calls ({n_phased}: {', '.join(names_phased)})" if n_full is not None else
+            "the launch record could not be read"),
         "clocks": clk.summary(),
         "device_err_word": err,
     }
     return case, res
+
+
+OUR_KERNELS = re.compile(r"(schedule|qimage|decode|merge|demote)_kernel")
+
+
+def count_launches(step):
+    """Kernels of this library that one call of `step` launches, read from the
+    CUDA activity record (torch.profiler / CUPTI): (count, sorted kernel names),
+    or (None, []) when the record is unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events()
+                 if e.device_type == torch.autograd.DeviceType.CUDA and OUR_KERNELS.search(e.name)]
+    except Exception:  # noqa: BLE001 - the count is a report, not part of the measurement
+        return None, []
+    short = sorted({OUR_KERNELS.search(n).group(0) for n in names})
+    return len(names), short
 
 
 def run_reference(args, dist):

@@ -32,6 +32,13 @@ CASES = {
                          tiers=[(0.3, "i4"), (0.4, "i8"), (0.3, "bf16")], q_fmt="bf16"),
     # fp32, d 64: the fp32 kernel
     "f32": dict(B=2, Hq=4, Hkv=4, d=64, P=64, lens=(1000, 4000), fmt="f32", q_fmt="f32"),
+    # bf16, d 64: the CUDA-core kernel
+    "cc": dict(B=3, Hq=8, Hkv=2, d=64, P=32, lens=(2500, 31, 900), fmt="bf16", q_fmt="bf16"),
+    # uniform int8, 4 rows per kv head: tcgen05 int8-MMA variant, items claimed
+    "i8_claimed": dict(B=3, Hq=8, Hkv=2, d=128, P=128, lens=(3000, 129, 5000), fmt="i8",
+                       q_fmt="bf16", alibi=True),
+    # 32 query heads on one kv head: two row groups per sequence, merged separately
+    "mqa": dict(B=2, Hq=32, Hkv=1, d=128, P=64, lens=(4000, 700), fmt="bf16", q_fmt="bf16"),
 }
 
 
