@@ -69,7 +69,7 @@
 namespace cfr {
 
 constexpr int TC_T = 128;            // tokens per tile
-constexpr int TC_D = 128;            // head_dim
+constexpr int TC_D = 128;            // head_dim of the operand layout (64 is read as its first half)
 constexpr int TC_THREADS = 384;
 // warp roles, one warpgroup each for the register split (setmaxnreg):
 // warpgroup 0 = producers and MMA issuers, 1 = softmax, 2 = staging
@@ -80,8 +80,8 @@ constexpr int TC_PV_WARP = 2;
 constexpr int TC_SOFTMAX_T0 = 128;   // first thread of the softmax warpgroup (warps 4-7)
 constexpr int TC_STAGING_T0 = 256;   // first thread of the staging warpgroup (warps 8-11)
 // registers per thread of each warpgroup after the split; the launch gives
-// 384 x 168 = 64,512 and the split takes 128 x (104 + 224 + 136) = 59,392
-constexpr int TC_REGS_IO = 104, TC_REGS_SOFTMAX = 224, TC_REGS_STAGING = 136;
+// 384 x 168 = 64,512 and the split takes 128 x (104 + 224 + 152) = 61,440
+constexpr int TC_REGS_IO = 104, TC_REGS_SOFTMAX = 224, TC_REGS_STAGING = 152;
 // registers per thread at launch: the register file (65,536) over the block's
 // threads, rounded down to the allocation unit of 8 (what __launch_bounds__ with
 // one block per SM gives ptxas); the launch checks the kernel really has it
@@ -630,7 +630,8 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   uint32_t bytes = 0;
   if (lane == 0) {
     if (kind == KIND_BF16) {
-      bytes = static_cast<uint32_t>(__popc(vb)) * 4u * box_rows * 128u;
+      // a K and a V box per 64 dims (2 with head_dim 64, 4 with 128) per valid piece
+      bytes = static_cast<uint32_t>(__popc(vb)) * static_cast<uint32_t>(p.D / 32) * box_rows * 128u;
     } else if (IMMA && kind == KIND_I8) {
       const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
       ks = sc.x;
@@ -640,7 +641,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
       const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
       ks = sc.x;
       vs = sc.y;
-      bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, TC_D));
+      bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, p.D));
     }
   }
   uint64_t *done = direct ? &c.S.op_full[stage] : &c.S.raw_full[stage];
@@ -666,10 +667,12 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
     if (kind == KIND_BF16) {
       const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
+      // head_dim 64 fills only the first half of K and of V: the QK products
+      // stop at dim 64 and the P.V rows of dims 64..127 are never read
       tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, done);
-      tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
+      if (p.D == TC_D) tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
       tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, done);
-      tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
+      if (p.D == TC_D) tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
     } else if (IMMA && kind == KIND_I8) {
       // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows
       const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
@@ -683,7 +686,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
       bulk_g2s(op + TC_HALF, p.k_pool[fmt] + off, rows * rb, done);
       bulk_g2s(op + 3 * TC_HALF, p.v_pool[fmt] + off, rows * rb, done);
     } else if (INTP) {
-      const int rb = row_bytes(fmt, TC_D);
+      const int rb = row_bytes(fmt, p.D);
       const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
       // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in);
       // the staging warps expand them in place
@@ -758,6 +761,99 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out, i
   }
 }
 
+// Staging of row r of a quantised tile for the fp16 MMAs: the int8 / int4 /
+// E4M3 codes of K and V, copied raw into the stage's V region (K codes at 0, V
+// codes TC_RAW_K bytes in), become fp16 operand rows (K halves at 0, V halves at
+// 2 * TC_HALF), 128-byte swizzled.  HD = head_dim: 128 fills both 64-dim halves,
+// 64 the first (the QK products stop at dim 64; the P.V rows of dims 64..127 are
+// never read).  A thread loads its whole row before converting it, starting at
+// a row-dependent 16-byte chunk (no bank conflicts), and the V rows, which are
+// expanded over the codes, are all loaded (named barrier 3) before any is
+// written.  Rows that hold no token become zeros.
+template <int HD>
+__device__ __forceinline__ void tc_expand_codes(uint8_t *op, int r, bool valid, int kind) {
+  constexpr int NCH = HD / 16;   // 16-byte chunks of an int8 / E4M3 code row
+  constexpr int NCH4 = HD / 32;  // 16-byte chunks of an int4 code row
+  const uint8_t *raw = op + 2 * TC_HALF;
+  const bool i4 = kind == KIND_I4;
+  const int rb = i4 ? HD / 2 : HD;  // row bytes of the codes
+  // K then V through one copy of the code (the kernel's roles share the SM's
+  // instruction cache; unrolling this loop costs more than it saves)
+#pragma unroll 1
+  for (int kv = 0; kv < 2; ++kv) {
+    uint8_t *dst = op + kv * 2 * TC_HALF;
+    const uint8_t *src = raw + kv * TC_RAW_K + r * rb;
+    uint4 w[NCH];
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        const int ci = i4 ? ((j + (r >> 1)) & (NCH4 - 1)) : ((j + r) & (NCH - 1));
+        if (!i4 || j < NCH4) w[j] = *reinterpret_cast<const uint4 *>(src + 16 * ci);
+      }
+    }
+    if (kv == 1) named_sync(3, 128);  // every V row has been read
+    if (!valid) {
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        *reinterpret_cast<uint4 *>(dst + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+        if (HD == TC_D) *reinterpret_cast<uint4 *>(dst + TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+      }
+      continue;
+    }
+    if (kind == KIND_I8) {
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        const int ci = (j + r) & (NCH - 1);  // codes 16ci .. 16ci+15
+        uint32_t o[8];
+        i8x4_to_h2x2(w[j].x, o[0], o[1]);
+        i8x4_to_h2x2(w[j].y, o[2], o[3]);
+        i8x4_to_h2x2(w[j].z, o[4], o[5]);
+        i8x4_to_h2x2(w[j].w, o[6], o[7]);
+        // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
+        uint8_t *hb = dst + (ci >> 2) * TC_HALF;
+        const int oc = (2 * ci) & 7;
+        *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    } else if (kind == KIND_FP8) {
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        const int ci = (j + r) & (NCH - 1);  // E4M3 codes 16ci .. 16ci+15
+        const uint32_t wv[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+        uint32_t o[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          o[2 * q] = e4m3x2_to_h2(wv[q], 0);
+          o[2 * q + 1] = e4m3x2_to_h2(wv[q], 1);
+        }
+        uint8_t *hb = dst + (ci >> 2) * TC_HALF;
+        const int oc = (2 * ci) & 7;
+        *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < NCH4; ++j) {
+        const int ci = (j + (r >> 1)) & (NCH4 - 1);  // codes 32ci .. 32ci+31
+        const uint32_t wv[4] = {w[j].x ^ 0x88888888u, w[j].y ^ 0x88888888u, w[j].z ^ 0x88888888u,
+                                w[j].w ^ 0x88888888u};
+        uint32_t o[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) o[4 * q + k] = i4x2_to_h2(wv[q], k);
+        // output chunks 4ci .. 4ci+3 in half ci/2
+        uint8_t *hb = dst + (ci >> 1) * TC_HALF;
+        const int oc = (4 * ci) & 7;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4 *>(hb + sw128(r, oc + q)) =
+              make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+    }
+  }
+}
+
 // staging warpgroup: thread r (0..127) owns row r of every tile that is not direct
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
 __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
@@ -824,89 +920,10 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
             }
           }
         } else if (INTP) {
-          // the codes sit in this stage's V region (K codes at 0, V codes at
-          // TC_RAW_K); a thread loads its whole row before converting it, and the
-          // V rows, which are expanded over the codes, are all loaded before any
-          // is written
-          const uint8_t *raw = op + 2 * TC_HALF;
-          const bool i4 = m.kind == KIND_I4;
-          const int rb = i4 ? TC_D / 2 : TC_D;  // row bytes of the codes
-          // K then V through one copy of the code (the kernel's roles share the
-          // SM's instruction cache; unrolling this loop costs more than it saves)
-#pragma unroll 1
-          for (int kv = 0; kv < 2; ++kv) {
-            uint8_t *dst = op + kv * 2 * TC_HALF;
-            const uint8_t *src = raw + kv * TC_RAW_K + r * rb;
-            // 16-byte chunks, starting at a row-dependent chunk (no bank conflicts)
-            uint4 w[8];
-            if (valid) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int ci = i4 ? ((j + (r >> 1)) & 3) : ((j + r) & 7);
-                if (!i4 || j < 4) w[j] = *reinterpret_cast<const uint4 *>(src + 16 * ci);
-              }
-            }
-            if (kv == 1) named_sync(3, 128);  // every V row has been read
-            if (!valid) {
-#pragma unroll
-              for (int ch = 0; ch < 8; ++ch) {
-                *reinterpret_cast<uint4 *>(dst + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(dst + TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-              }
-              continue;
-            }
-            if (m.kind == KIND_I8) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int ci = (j + r) & 7;  // codes 16ci .. 16ci+15
-                uint32_t o[8];
-                i8x4_to_h2x2(w[j].x, o[0], o[1]);
-                i8x4_to_h2x2(w[j].y, o[2], o[3]);
-                i8x4_to_h2x2(w[j].z, o[4], o[5]);
-                i8x4_to_h2x2(w[j].w, o[6], o[7]);
-                // output chunks 2ci, 2ci+1 (8 fp16 each) in half ci/4
-                uint8_t *hb = dst + (ci >> 2) * TC_HALF;
-                const int oc = (2 * ci) & 7;
-                *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-              }
-            } else if (m.kind == KIND_FP8) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int ci = (j + r) & 7;  // E4M3 codes 16ci .. 16ci+15
-                const uint32_t wv[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
-                uint32_t o[8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  o[2 * q] = e4m3x2_to_h2(wv[q], 0);
-                  o[2 * q + 1] = e4m3x2_to_h2(wv[q], 1);
-                }
-                uint8_t *hb = dst + (ci >> 2) * TC_HALF;
-                const int oc = (2 * ci) & 7;
-                *reinterpret_cast<uint4 *>(hb + sw128(r, oc)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(hb + sw128(r, oc + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int ci = (j + (r >> 1)) & 3;  // codes 32ci .. 32ci+31
-                const uint32_t wv[4] = {w[j].x ^ 0x88888888u, w[j].y ^ 0x88888888u,
-                                        w[j].z ^ 0x88888888u, w[j].w ^ 0x88888888u};
-                uint32_t o[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                  for (int k = 0; k < 4; ++k) o[4 * q + k] = i4x2_to_h2(wv[q], k);
-                // output chunks 4ci .. 4ci+3 in half ci/2
-                uint8_t *hb = dst + (ci >> 1) * TC_HALF;
-                const int oc = (4 * ci) & 7;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  *reinterpret_cast<uint4 *>(hb + sw128(r, oc + q)) =
-                      make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-              }
-            }
-          }
+          if (IMMA || p.D == TC_D)  // int8-MMA variants only run head_dim 128
+            tc_expand_codes<TC_D>(op, r, valid, m.kind);
+          else
+            tc_expand_codes<TC_D / 2>(op, r, valid, m.kind);
         }
         fence_async_smem();
         named_sync(3, 128);
@@ -974,8 +991,9 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
       } else {
         const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
         const uint32_t qbase = qop + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
-#pragma unroll
-        for (int k = 0; k < TC_D / 16; ++k) {
+        const int ksteps = p.D / 16;  // 8, or 4 for head_dim 64 (the first half)
+#pragma unroll 8
+        for (int k = 0; k < ksteps; ++k) {
           const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
           const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
           tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
@@ -1091,7 +1109,7 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long l
 
 // element `dim` of query row vh of sequence b, as fp32
 __device__ __forceinline__ float q_elem(const DecodeParams &p, int b, int vh, int dim) {
-  const long long i = (static_cast<long long>(b) * p.Hq + vh) * TC_D + dim;
+  const long long i = (static_cast<long long>(b) * p.Hq + vh) * p.D + dim;
   return p.q_fmt == CFR_FMT_F32
              ? static_cast<const float *>(p.q)[i]
              : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
@@ -1123,8 +1141,8 @@ __device__ __forceinline__ void tc_build_q(const DecodeParams &p, int b, int g, 
     float x[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) x[e] = 0.f;
-    if (head < cnt) {
-      const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * TC_D + 8 * ch;
+    if (head < cnt && 8 * ch < p.D) {  // dims past head_dim 64 stay 0
+      const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * p.D + 8 * ch;
       if (p.q_fmt == CFR_FMT_F32) {
         const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi);
         const float4 bb = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi + 4);
@@ -1463,7 +1481,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
     for (int h = 0; h < GH; ++h) {
       if (h < cnt) {
         const int head = p.grp_heads[h0 + h];
-        p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * TC_D + t] = acc[h];
+        if (t < p.D) p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * p.D + t] = acc[h];
         float l = l_part[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -1601,7 +1619,7 @@ static bool tc_int_pools(const DecodeParams &p, bool page_fmt_given) {
 }
 
 bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
-  if (p.D != TC_D || p.gmax > 16) return false;
+  if ((p.D != TC_D && p.D != TC_D / 2) || p.gmax > 16) return false;
   if ((reinterpret_cast<uintptr_t>(p.q) & 15) != 0) return false;
   if (page_fmt_given) {
     if (p.k_pool[CFR_FMT_F32]) return false;
@@ -1633,9 +1651,9 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
     const long long rows = p.pool_pages[CFR_FMT_BF16] * p.Hkv * static_cast<long long>(p.P);
     const int box_rows = p.P < TC_T ? p.P : TC_T;
     if (!encode_pool_map(&maps.k, p.k_pool[CFR_FMT_BF16], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows,
-                         TC_D, box_rows) ||
+                         p.D, box_rows) ||
         !encode_pool_map(&maps.v, p.v_pool[CFR_FMT_BF16], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows,
-                         TC_D, box_rows))
+                         p.D, box_rows))
       return cudaErrorInvalidValue;
   }
   if (IMMA && p.k_pool[CFR_FMT_I8] && p.pool_pages[CFR_FMT_I8] > 0) {
@@ -1676,7 +1694,7 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
 // int8 or int4 pools whose tiles can run the int8 MMAs: up to 4 query rows per
 // kv head (4 digit columns each fill the 16-column operand)
 static bool tc_imma(const DecodeParams &p, bool page_fmt_given) {
-  if (p.gmax > 4) return false;
+  if (p.gmax > 4 || p.D != TC_D) return false;
   if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4];
   return p.uniform_fmt == CFR_FMT_I8 || p.uniform_fmt == CFR_FMT_I4;
 }

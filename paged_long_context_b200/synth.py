@@ -443,6 +443,20 @@ def spec_mqa() -> CaseSpec:
                     fmt="bf16", q_fmt="bf16", permute=True)
 
 
+def spec_gqa_d64() -> CaseSpec:
+    """The ragged GQA batch at head_dim 64: 16 sequences of 1K-32K tokens, 32 q / 8 kv
+    heads, bf16, 16-token pages (the tensor-core kernel, first half of its operands)."""
+    return CaseSpec("gqa_ragged_b16_1k32k_p16_bf16_d64", 16, 32, 8, 64, 16,
+                    len_range=(1024, 32768), fmt="bf16", q_fmt="bf16", permute=True)
+
+
+def spec_gqa_d64_i8_p16() -> CaseSpec:
+    """The same batch as int8 pages of 16 tokens, head_dim 64: a shape only the
+    general CUDA-core kernel takes (quantised pages under 128 tokens)."""
+    return CaseSpec("gqa_ragged_b16_1k32k_p16_i8_d64", 16, 32, 8, 64, 16,
+                    len_range=(1024, 32768), fmt="i8", q_fmt="bf16", permute=True)
+
+
 WORKLOADS = {
     "tiny": (spec_tiny_exact_fold, 1),
     "cfr": (spec_cfr_shaped, 2),
@@ -450,12 +464,14 @@ WORKLOADS = {
     "tiered": (spec_tiered, 4),
     "alibi1m": (spec_alibi_1m, 5),
     "mqa": (spec_mqa, 6),
+    "gqa_d64": (spec_gqa_d64, 7),
+    "gqa_d64_i8p16": (spec_gqa_d64_i8_p16, 7),
 }
 
 
 def workload(name: str, device="cpu", num_queries: int = 1,
              context: Optional[int] = None) -> DecodeCase:
-    """One of the five page-shaped workloads, with its fixed seed (optionally with
+    """One of the page-shaped workloads, with its fixed seed (optionally with
     several query tokens per sequence, or with every sequence cut to `context`
     tokens: the same shape at a smaller size, e.g. for a profiler capture)."""
     fn, seed = WORKLOADS[name]

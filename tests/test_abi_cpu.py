@@ -186,6 +186,11 @@ def test_path_selection_is_host_only(lib):
     assert binding.decode_path(_case(fmt="f32", page_tokens=24)) == binding.PATH_CUDA_CORE
     assert binding.decode_path(_case(fmt="tiered", tiers=[(0.5, "i8"), (0.5, "f32")])) == \
         binding.PATH_CUDA_CORE
+    # bf16 caches of head_dim 64 take the tensor-core kernel (the first half of
+    # its 128-dim operands); int8 pages under 128 tokens take the general kernel
+    assert binding.decode_path(_case()) == binding.PATH_TENSOR_CORE
+    assert binding.decode_path(_case(fmt="i8")) == binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="i8", page_tokens=128)) == binding.PATH_TENSOR_CORE
     # rejected configurations report 0
     assert binding.decode_path(_case(num_q_heads=3, num_kv_heads=2)) == 0
 

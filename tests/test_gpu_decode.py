@@ -176,7 +176,7 @@ def test_full_page_table():
 def test_bad_sequence_length(bad_len, path):
     # a sequence that gets no split: its rows are written as a merge of nothing
     # (0, lse -inf) by the decode that merges, on each kernel
-    kw = {"cc": dict(d=64, fmt="bf16"), "tc": dict(d=128, fmt="bf16", q_fmt="bf16"),
+    kw = {"cc": dict(d=64, fmt="i8"), "tc": dict(d=128, fmt="bf16", q_fmt="bf16"),
           "f32": dict(d=64, fmt="f32", q_fmt="f32")}[path]
     case = small_case(B=3, Hq=4, Hkv=2, P=16, lens=(50, 33, 70), **kw)
     assert binding.decode_path(case) == {"cc": binding.PATH_CUDA_CORE, "tc": binding.PATH_TENSOR_CORE,

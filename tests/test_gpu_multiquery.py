@@ -68,6 +68,9 @@ CONFIGS = {
                             tiers=[(0.3, "i4"), (0.3, "i8"), (0.2, "fp8"), (0.2, "bf16")]),
     "cuda-core-d64": dict(Q=4, Hq=8, Hkv=2, d=64, P=16, fmt="tiered",
                           tiers=[(0.3, "i4"), (0.3, "i8"), (0.2, "fp8"), (0.2, "bf16")]),
+    "tcgen05-d64": dict(Q=2, Hq=8, Hkv=2, d=64, P=32),
+    "tcgen05-d64-int": dict(Q=3, Hq=8, Hkv=2, d=64, P=128, fmt="tiered",
+                            tiers=[(0.3, "i4"), (0.3, "i8"), (0.2, "fp8"), (0.2, "bf16")]),
     "f32-tma": dict(Q=2, Hq=4, Hkv=4, d=64, fmt="f32", q_fmt="f32"),
     "cuda-core-f32": dict(Q=4, Hq=8, Hkv=4, d=64, fmt="f32", q_fmt="f32"),
 }

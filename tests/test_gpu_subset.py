@@ -51,9 +51,11 @@ PATHS = {
                         tiers=[(0.3, "i4"), (0.3, "i8"), (0.2, "fp8"), (0.2, "bf16")]),
     "cuda-core": dict(d=64, P=16, fmt="tiered", q_fmt="bf16", Hq=8, Hkv=2,
                       tiers=[(0.3, "i4"), (0.3, "i8"), (0.2, "fp8"), (0.2, "bf16")]),
+    "tcgen05-d64": dict(d=64, P=32, fmt="bf16", q_fmt="bf16", Hq=8, Hkv=2),
 }
 WANT = {"f32-tma": binding.PATH_F32_TMA, "tcgen05-bf16": binding.PATH_TENSOR_CORE,
-        "tcgen05-int": binding.PATH_TENSOR_CORE, "cuda-core": binding.PATH_CUDA_CORE}
+        "tcgen05-int": binding.PATH_TENSOR_CORE, "cuda-core": binding.PATH_CUDA_CORE,
+        "tcgen05-d64": binding.PATH_TENSOR_CORE}
 
 
 @pytest.mark.parametrize("path", list(PATHS))

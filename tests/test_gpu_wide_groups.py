@@ -2,8 +2,8 @@
 
 The query rows of a kv head are decoded in groups of at most 16 (each group
 reads the kv head's pages); every path -- the tensor-core kernel for bf16,
-FP8, int8 and int4 pages, the CUDA-core kernels for fp32 pages and head_dim 64
--- must match the oracle at the stated tolerance, with contiguous and
+FP8, int8 and int4 pages (head_dim 128, and 64 for bf16), the CUDA-core kernels
+for fp32 pages and small int8 pages -- must match the oracle at the stated tolerance, with contiguous and
 arbitrary head maps, ALiBi, and several query tokens per sequence."""
 import numpy as np
 import pytest
@@ -41,8 +41,11 @@ def test_wide_groups_tensor_core_shapes(fmt, heads):
 
 @pytest.mark.parametrize("fmt", ["bf16", "i8"])
 def test_wide_groups_head_dim_64(fmt):
-    # head_dim 64: the CUDA-core kernel
+    # head_dim 64: the tensor-core kernel (bf16) or the CUDA-core kernel (int8
+    # pages of 16 tokens)
     case = small_case(B=2, Hq=32, Hkv=1, d=64, P=16, lens=(700, 33), fmt=fmt, seed=3)
+    assert binding.decode_path(case) == (binding.PATH_TENSOR_CORE if fmt == "bf16"
+                                         else binding.PATH_CUDA_CORE)
     out, lse, err = run(case)
     assert err == 0
     check(case, out, lse)
