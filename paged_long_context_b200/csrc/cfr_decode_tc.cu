@@ -120,10 +120,17 @@ struct TcItem {
   int n, t_end;    // sequence length; the split's tokens are [pb * P, t_end)
 };
 
-struct TcMeta {
+template <int NP>
+struct TcMetaT {
   uint32_t valid[4];
   int rows, t0, kind, direct;
-  float ks, vs;
+  // quantised tiles: the K and V scale of each page piece (one piece when pages
+  // hold 128 tokens or more; up to NP = 16 pieces of a uniform-format cache with
+  // smaller pages in the 16-column variants), and vs, the largest V scale, which
+  // the fold applies to the tile's product (each row's probability carries its
+  // piece's vsp / vs)
+  float vs;
+  float ksp[NP], vsp[NP];
 };
 
 struct TcMaps {
@@ -175,7 +182,9 @@ struct TcSmem {
   float qs_bc[2][TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 4 : 1];
   uint32_t tmem_base;
   int flag_st[3];
-  TcMeta meta[3];
+  // tile descriptions; the 32-column variants, which fill shared memory, take
+  // quantised pages of 128 tokens or more only (one piece)
+  TcMetaT<NCOL == 16 ? 16 : 1> meta[3];
   alignas(16) float red_max[2][4][16];
   alignas(16) float red_l[4][16];
   typename TcCfg<NCOL, INTP>::PageCache pc[TC_PRODUCERS];
@@ -612,36 +621,43 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   }
   if constexpr (FEAT == TC_FEAT_SUBSET)
     mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
-  // quantised pages need page_tokens >= 128: the tile is then one piece (lane 0)
+  // the tile's kind is the format of its first valid piece: a cache whose page
+  // formats differ has quantised pages of 128 tokens or more (one piece per
+  // tile), and a uniform-format cache gives every piece the same format
   const int kind0 = !pvalid                ? KIND_BF16
                     : fmt == CFR_FMT_I8    ? KIND_I8
                     : fmt == CFR_FMT_I4    ? KIND_I4
                     : fmt == CFR_FMT_FP8   ? KIND_FP8
                                            : KIND_BF16;
-  const int kind = __shfl_sync(0xffffffffu, kind0, 0);
+  const int kind = __shfl_sync(0xffffffffu, kind0, vb ? __ffs(vb) - 1 : 0);
   // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA, and so
   // does every int8 tile of an IMMA variant (its codes are the operand; rows
   // that hold no token carry finite codes that meet a zero probability); every
   // other tile passes through the staging warps
   const bool direct = (kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu) ||
                       (IMMA && kind == KIND_I8);
-  // ---- the tile's byte count and scales (lane 0) ----
+  // ---- the tile's byte count (lane 0) and its pieces' scales (lane f: piece f) ----
   float ks = 1.f, vs = 1.f;
+  if (kind != KIND_BF16 && pvalid) {
+    const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
+    ks = sc.x;
+    vs = sc.y;
+  }
+  float vs_max = pvalid ? vs : 0.f;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) vs_max = fmaxf(vs_max, __shfl_xor_sync(0xffffffffu, vs_max, o));
   uint32_t bytes = 0;
   if (lane == 0) {
     if (kind == KIND_BF16) {
       // a K and a V box per 64 dims (2 with head_dim 64, 4 with 128) per valid piece
       bytes = static_cast<uint32_t>(__popc(vb)) * static_cast<uint32_t>(p.D / 32) * box_rows * 128u;
     } else if (IMMA && kind == KIND_I8) {
-      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
-      ks = sc.x;
-      vs = sc.y;
       bytes = 2u * TC_T * 128u;  // one full 128-row box of K and of V
+    } else if (p.P >= TC_T) {
+      bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, p.D));  // the tile's rows of one page
     } else {
-      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
-      ks = sc.x;
-      vs = sc.y;
-      bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, p.D));
+      // whole pieces of box_rows rows (a uniform format: every piece's row bytes)
+      bytes = static_cast<uint32_t>(__popc(vb)) * 2u * box_rows * static_cast<uint32_t>(row_bytes(fmt, p.D));
     }
   }
   uint64_t *done = direct ? &c.S.op_full[stage] : &c.S.raw_full[stage];
@@ -650,14 +666,21 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   if (lane == 0) ok = mbar_wait(&c.S.op_empty[stage], phase ^ 1u, p.err, timed_out) ? 1 : 0;
   if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
   if (lane == 0) {
-    TcMeta &m = c.S.meta[stage];
+    auto &m = c.S.meta[stage];
     for (int w = 0; w < 4; ++w) m.valid[w] = valid[w];
     m.rows = rows;
     m.t0 = t0;
     m.kind = kind;
     m.direct = direct ? 1 : 0;
-    m.ks = ks;
-    m.vs = vs;
+    m.vs = vs_max;
+  }
+  constexpr int NP = NCOL == 16 ? 16 : 1;
+  if (lane < NP) {
+    c.S.meta[stage].ksp[lane] = ks;
+    c.S.meta[stage].vsp[lane] = vs;
+  }
+  __syncwarp();  // the whole description is written before lane 0 publishes it
+  if (lane == 0) {
     if (direct) mbar_arrive(&c.S.raw_full[stage]);  // lets the staging warps skip this tile
     mbar_arrive_expect_tx(done, bytes);
   }
@@ -688,11 +711,12 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     } else if (INTP) {
       const int rb = row_bytes(fmt, p.D);
       const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
-      // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in);
-      // the staging warps expand them in place
-      uint8_t *raw = op + 2 * TC_HALF;
-      bulk_g2s(raw, p.k_pool[fmt] + off, rows * rb, done);
-      bulk_g2s(raw + TC_RAW_K, p.v_pool[fmt] + off, rows * rb, done);
+      // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in),
+      // piece `lane` at row r; the staging warps expand them in place
+      const int nrows = p.P >= TC_T ? rows : box_rows;
+      uint8_t *raw = op + 2 * TC_HALF + r * rb;
+      bulk_g2s(raw, p.k_pool[fmt] + off, nrows * rb, done);
+      bulk_g2s(raw + TC_RAW_K, p.v_pool[fmt] + off, nrows * rb, done);
     }
   }
   return true;
@@ -877,7 +901,7 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         return;
       }
       (void)mbar_try_wait(&c.S.raw_full[stage], phase);
-      const TcMeta &m = c.S.meta[stage];
+      const auto &m = c.S.meta[stage];
       if (!m.direct) {
         const bool valid = (m.valid[r >> 5] >> (r & 31)) & 1u;
         uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
@@ -1269,6 +1293,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   const int tsm = threadIdx.x - TC_SOFTMAX_T0;  // 0..127 within the warpgroup
   const uint32_t tmem = c.S.tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
   const int P = p.P;
+  const int pshift = 31 - __clz(P < TC_T ? P : TC_T);  // log2 of a page piece's rows
   int stage = 0;
   uint32_t phase = 0;
   long long tc = 0;
@@ -1331,16 +1356,20 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       // acquire the tile description published through the stage's op_full phase
       // (that phase cannot move on before this tile's P.V has run)
       (void)mbar_try_wait(&c.S.op_full[stage], phase);
-      const TcMeta &m = c.S.meta[stage];
+      const auto &m = c.S.meta[stage];
       const bool valid = (m.valid[t >> 5] >> (t & 31)) & 1u;
       const int kind = m.kind;
       const bool itile = tc_int_tile<IMMA>(kind);
       // int4 codes enter the int8 MMAs times 16; probability digits are of p * 255
       const float i4f = itile && kind == KIND_I4 ? 1.f / 16.f : 1.f;
-      const float scale = m.ks * p.sigma_log2e * i4f;
+      // token t's page piece: its K scale, and its V scale relative to the tile's
+      // (1 with one piece per tile: pages of 128 tokens or more)
+      const int piece = NCOL == 16 ? t >> pshift : 0;
+      const float scale = m.ksp[piece] * p.sigma_log2e * i4f;
       const float vsc = kind == KIND_BF16 ? 1.f
                         : itile           ? m.vs * i4f * (1.f / 255.f)
                                           : m.vs * (1.f / 32768.f);
+      const float vratio = kind == KIND_BF16 || m.vs <= 0.f ? 1.f : m.vsp[piece] / m.vs;
       // ALiBi from the last position; a query row at offset o before it differs by the
       // row constant slope * o, added back to its maximum at the partial write
       const int j = m.t0 + t;
@@ -1420,7 +1449,9 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         float colv[NCOL];
 #pragma unroll
         for (int k = 0; k < NCOL; ++k) colv[k] = 0.f;
-        const float pre = kind == KIND_BF16 ? 1.f : 32768.f;
+        // fp16 probabilities of quantised tiles are scaled up by 2^15 (and by the
+        // row's V-scale ratio) to use the fp16 range
+        const float pre = kind == KIND_BF16 ? 1.f : 32768.f * vratio;
 #pragma unroll
         for (int h = 0; h < GH; ++h) {
           const float x = pr[h] * pre;  // 0 for the padding heads h >= cnt
@@ -1630,11 +1661,11 @@ bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
     return false;
   }
   const bool ints = tc_int_pools(p, page_fmt_given);
-  if (ints) {
-    if (p.P % TC_T != 0) return false;
-  } else if (!((p.P <= TC_T && TC_T % p.P == 0) || p.P % TC_T == 0)) {
-    return false;
-  }
+  const bool p_ok = (p.P <= TC_T && TC_T % p.P == 0) || p.P % TC_T == 0;
+  // quantised pages shorter than a tile only in a uniform-format cache (a tile
+  // then holds pieces of one format, each with its own scales) and with at most
+  // 8 rows per group (the 16-column variants keep the pieces' scales)
+  if (!p_ok || (ints && p.P % TC_T != 0 && (page_fmt_given || p.gmax > 8))) return false;
   const long long rows = p.pool_pages[CFR_FMT_BF16] * p.Hkv * static_cast<long long>(p.P);
   if (rows > 0x7fffffffLL) return false;
   // int8 pools are read through a tensor map when their tiles run int8 MMAs
@@ -1694,7 +1725,7 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
 // int8 or int4 pools whose tiles can run the int8 MMAs: up to 4 query rows per
 // kv head (4 digit columns each fill the 16-column operand)
 static bool tc_imma(const DecodeParams &p, bool page_fmt_given) {
-  if (p.gmax > 4 || p.D != TC_D) return false;
+  if (p.gmax > 4 || p.D != TC_D || p.P % TC_T != 0) return false;
   if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4];
   return p.uniform_fmt == CFR_FMT_I8 || p.uniform_fmt == CFR_FMT_I4;
 }

@@ -451,10 +451,19 @@ def spec_gqa_d64() -> CaseSpec:
 
 
 def spec_gqa_d64_i8_p16() -> CaseSpec:
-    """The same batch as int8 pages of 16 tokens, head_dim 64: a shape only the
-    general CUDA-core kernel takes (quantised pages under 128 tokens)."""
+    """The same batch as int8 pages of 16 tokens, head_dim 64 (the tensor-core
+    kernel: a tile holds 8 pages, each with its own scales)."""
     return CaseSpec("gqa_ragged_b16_1k32k_p16_i8_d64", 16, 32, 8, 64, 16,
                     len_range=(1024, 32768), fmt="i8", q_fmt="bf16", permute=True)
+
+
+def spec_gqa_d64_mixed_p16() -> CaseSpec:
+    """The same batch with int8 and bf16 pages of 16 tokens mixed, head_dim 64: a
+    shape only the general CUDA-core kernel takes (quantised pages under 128
+    tokens among other formats)."""
+    return CaseSpec("gqa_ragged_b16_1k32k_p16_i8bf16_d64", 16, 32, 8, 64, 16,
+                    len_range=(1024, 32768), fmt="tiered", tiers=[(0.5, "i8"), (0.5, "bf16")],
+                    q_fmt="bf16", permute=True)
 
 
 WORKLOADS = {
@@ -466,6 +475,7 @@ WORKLOADS = {
     "mqa": (spec_mqa, 6),
     "gqa_d64": (spec_gqa_d64, 7),
     "gqa_d64_i8p16": (spec_gqa_d64_i8_p16, 7),
+    "gqa_d64_mixed_p16": (spec_gqa_d64_mixed_p16, 7),
 }
 
 

@@ -187,10 +187,16 @@ def test_path_selection_is_host_only(lib):
     assert binding.decode_path(_case(fmt="tiered", tiers=[(0.5, "i8"), (0.5, "f32")])) == \
         binding.PATH_CUDA_CORE
     # bf16 caches of head_dim 64 take the tensor-core kernel (the first half of
-    # its 128-dim operands); int8 pages under 128 tokens take the general kernel
+    # its 128-dim operands), and so do uniform int8 caches of any page size up to
+    # 8 rows per group; quantised pages under 128 tokens in a cache of mixed
+    # formats, or with wider groups, take the general kernel
     assert binding.decode_path(_case()) == binding.PATH_TENSOR_CORE
-    assert binding.decode_path(_case(fmt="i8")) == binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="i8")) == binding.PATH_TENSOR_CORE
     assert binding.decode_path(_case(fmt="i8", page_tokens=128)) == binding.PATH_TENSOR_CORE
+    assert binding.decode_path(_case(fmt="i8", num_q_heads=32, num_kv_heads=2)) == \
+        binding.PATH_CUDA_CORE
+    assert binding.decode_path(_case(fmt="tiered", tiers=[(0.5, "i8"), (0.5, "bf16")])) == \
+        binding.PATH_CUDA_CORE
     # rejected configurations report 0
     assert binding.decode_path(_case(num_q_heads=3, num_kv_heads=2)) == 0
 
@@ -199,9 +205,12 @@ def test_path_selection_fp8(lib):
     # FP8 pages: head_dim 128 with 128-token pages take the tensor-core kernel
     assert binding.decode_path(_case(fmt="fp8", head_dim=128, page_tokens=128)) == \
         binding.PATH_TENSOR_CORE
-    # other shapes take the general kernel
-    assert binding.decode_path(_case(fmt="fp8")) == binding.PATH_CUDA_CORE
+    # and so do uniform FP8 caches with smaller pages; FP8 pages under 128
+    # tokens among other formats take the general kernel
+    assert binding.decode_path(_case(fmt="fp8")) == binding.PATH_TENSOR_CORE
     assert binding.decode_path(_case(fmt="fp8", head_dim=128, page_tokens=64)) == \
+        binding.PATH_TENSOR_CORE
+    assert binding.decode_path(_case(fmt="tiered", tiers=[(0.5, "fp8"), (0.5, "bf16")])) == \
         binding.PATH_CUDA_CORE
 
 

@@ -176,7 +176,8 @@ def test_full_page_table():
 def test_bad_sequence_length(bad_len, path):
     # a sequence that gets no split: its rows are written as a merge of nothing
     # (0, lse -inf) by the decode that merges, on each kernel
-    kw = {"cc": dict(d=64, fmt="i8"), "tc": dict(d=128, fmt="bf16", q_fmt="bf16"),
+    kw = {"cc": dict(d=64, fmt="tiered", tiers=[(0.5, "i8"), (0.5, "bf16")]),
+          "tc": dict(d=128, fmt="bf16", q_fmt="bf16"),
           "f32": dict(d=64, fmt="f32", q_fmt="f32")}[path]
     case = small_case(B=3, Hq=4, Hkv=2, P=16, lens=(50, 33, 70), **kw)
     assert binding.decode_path(case) == {"cc": binding.PATH_CUDA_CORE, "tc": binding.PATH_TENSOR_CORE,
@@ -345,3 +346,18 @@ def test_merge_matches_oracle():
     assert np.array_equal(np.isfinite(lse.cpu().numpy()), fin)
     np.testing.assert_allclose(lse.cpu().double().numpy()[fin], rl[fin], rtol=1e-5, atol=1e-5)
     assert torch.all(out[2] == 0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("P", [8, 16, 32, 64])
+@pytest.mark.parametrize("fmt", ["i8", "i4", "fp8"])
+def test_small_quantised_pages_on_the_tensor_core_kernel(fmt, P, d):
+    # uniform int8 / int4 / FP8 caches with pages shorter than a 128-token tile:
+    # a tile holds 128 / P pages, each with its own K and V scale
+    lens = (1, P + 3, 3 * 128 + 5, 1000)
+    case = small_case(B=len(lens), Hq=8, Hkv=2, d=d, P=P, lens=lens, fmt=fmt, q_fmt="bf16",
+                      alibi=True, seed=P + d)
+    assert binding.decode_path(case) == binding.PATH_TENSOR_CORE
+    out, lse, err = run(case)
+    assert err == 0
+    check(case, out, lse)

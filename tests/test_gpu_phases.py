@@ -32,8 +32,12 @@ CASES = {
                          tiers=[(0.3, "i4"), (0.4, "i8"), (0.3, "bf16")], q_fmt="bf16"),
     # fp32, d 64: the fp32 kernel
     "f32": dict(B=2, Hq=4, Hkv=4, d=64, P=64, lens=(1000, 4000), fmt="f32", q_fmt="f32"),
-    # int8 pages of 32 tokens, d 64: the CUDA-core kernel
-    "cc": dict(B=3, Hq=8, Hkv=2, d=64, P=32, lens=(2500, 31, 900), fmt="i8", q_fmt="bf16"),
+    # int8 and bf16 pages of 32 tokens, d 64: the CUDA-core kernel
+    "cc": dict(B=3, Hq=8, Hkv=2, d=64, P=32, lens=(2500, 31, 900), fmt="tiered",
+               tiers=[(0.5, "i8"), (0.5, "bf16")], q_fmt="bf16"),
+    # uniform int4 pages of 32 tokens: the tcgen05 path, per-page scales in a tile
+    "i4_small_pages": dict(B=3, Hq=8, Hkv=2, d=128, P=32, lens=(2500, 31, 900), fmt="i4",
+                           q_fmt="bf16", alibi=True),
     # bf16, d 64: the tcgen05 path reading the first half of its operands
     "bf16_d64": dict(B=3, Hq=8, Hkv=2, d=64, P=32, lens=(2500, 31, 900), fmt="bf16", q_fmt="bf16"),
     # uniform int8, 4 rows per kv head: tcgen05 int8-MMA variant, items claimed
@@ -72,8 +76,8 @@ FOREIGN = {
     "tiered": dict(d=128, fmt="tiered", tiers=[(0.5, "i8"), (0.5, "bf16")], q_fmt="bf16", P=128),
     # fp32 TMA kernel
     "f32": dict(d=64, fmt="f32", q_fmt="f32", Hq=4, Hkv=4),
-    # general CUDA-core kernel (int8 pages of 16 tokens, head_dim 64)
-    "cc": dict(d=64, fmt="i8", q_fmt="bf16"),
+    # general CUDA-core kernel (int8 and bf16 pages of 16 tokens, head_dim 64)
+    "cc": dict(d=64, fmt="tiered", tiers=[(0.5, "i8"), (0.5, "bf16")], q_fmt="bf16"),
 }
 
 
