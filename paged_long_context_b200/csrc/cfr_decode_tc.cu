@@ -82,6 +82,7 @@ constexpr int TC_STAGING_T0 = 256;   // first thread of the staging warpgroup (w
 // registers per thread of each warpgroup after the split; the launch gives
 // 384 x 168 = 64,512 and the split takes 128 x (104 + 224 + 152) = 61,440
 constexpr int TC_REGS_IO = 104, TC_REGS_SOFTMAX = 224, TC_REGS_STAGING = 152;
+constexpr int TC_REGS_STAGING_IMMA = 136;
 // registers per thread at launch: the register file (65,536) over the block's
 // threads, rounded down to the allocation unit of 8 (what __launch_bounds__ with
 // one block per SM gives ptxas); the launch checks the kernel really has it
@@ -124,11 +125,11 @@ template <int NP>
 struct TcMetaT {
   uint32_t valid[4];
   int rows, t0, kind, direct;
-  // quantised tiles: the K and V scale of each page piece (one piece when pages
-  // hold 128 tokens or more; up to NP = 16 pieces of a uniform-format cache with
-  // smaller pages in the 16-column variants), and vs, the largest V scale, which
-  // the fold applies to the tile's product (each row's probability carries its
-  // piece's vsp / vs)
+  // quantised tiles: the K scale of each page piece (one piece when pages hold
+  // 128 tokens or more; up to NP = 16 pieces of a uniform-format cache with
+  // smaller pages in the 16-column variants), vs, the largest V scale, which the
+  // fold applies to the tile's product, and vsp, each piece's V scale over vs,
+  // which its rows' probabilities carry
   float vs;
   float ksp[NP], vsp[NP];
 };
@@ -143,8 +144,11 @@ struct TcMaps {
 template <int NCOL, bool INTP>
 struct TcCfg {
   // quantised codes are copied into the stage's own V region and expanded in
-  // place, so the variant with quantised pools keeps the same three stages
+  // place, so the variant with quantised pools keeps the same three stages of
+  // 64 KiB; with head_dim 64 the 16-column variants cut the same bytes into six
+  // stages of 32 KiB (K half, V half), twice the tiles in flight
   static constexpr int STAGES = 3;
+  static constexpr int MAX_STAGES = NCOL == 16 ? 6 : 3;
   static constexpr int Q_BYTES = NCOL * 256;       // [NCOL rows][128 cols] 16-bit, 2 halves
   // [NCOL rows][128 cols] int8 query digits (int8 MMAs, 16 columns only)
   static constexpr int Q8_BYTES = (INTP && NCOL == 16) ? NCOL * 128 : 0;
@@ -166,7 +170,8 @@ struct TcCfg {
 
 template <int NCOL, bool INTP>
 struct TcSmem {
-  uint64_t op_full[3], op_empty[3], raw_full[3];
+  uint64_t op_full[TcCfg<NCOL, INTP>::MAX_STAGES], op_empty[TcCfg<NCOL, INTP>::MAX_STAGES],
+      raw_full[TcCfg<NCOL, INTP>::MAX_STAGES];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   uint64_t o_full[TcCfg<NCOL, INTP>::O_BUFS], o_empty[TcCfg<NCOL, INTP>::O_BUFS];
   uint64_t q_full, drain;
@@ -181,10 +186,10 @@ struct TcSmem {
   float ring_qs[TC_ITEM_RING][TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 4 : 1];
   float qs_bc[2][TcCfg<NCOL, INTP>::RING_SLOPES >= 4 ? 4 : 1];
   uint32_t tmem_base;
-  int flag_st[3];
+  int flag_st[TcCfg<NCOL, INTP>::MAX_STAGES];
   // tile descriptions; the 32-column variants, which fill shared memory, take
   // quantised pages of 128 tokens or more only (one piece)
-  TcMetaT<NCOL == 16 ? 16 : 1> meta[3];
+  TcMetaT<NCOL == 16 ? 16 : 1> meta[TcCfg<NCOL, INTP>::MAX_STAGES];
   alignas(16) float red_max[2][4][16];
   alignas(16) float red_l[4][16];
   typename TcCfg<NCOL, INTP>::PageCache pc[TC_PRODUCERS];
@@ -343,6 +348,21 @@ struct TcCtx {
   uint8_t *op, *qop, *pop;
   long long nitems;
   int nsplit;
+  // head_dim 64 in a 16-column variant other than int8-MMA: six stages of 32 KiB
+  // (K half, V half) instead of three of 64 KiB
+  bool compact;
+  // stage geometry: nst() stages of sbytes() bytes; the V operand (and the raw
+  // codes of quantised tiles) at voff() in a stage, the raw V codes rawv() bytes
+  // after the raw K codes.  Compile-time constants where compact cannot hold.
+  static constexpr bool kMayCompact = NCOL == 16 && !IMMA;
+  __device__ __forceinline__ int nst() const {
+    return kMayCompact && compact ? 2 * TcCfg<NCOL, INTP>::STAGES : TcCfg<NCOL, INTP>::STAGES;
+  }
+  __device__ __forceinline__ int sbytes() const {
+    return kMayCompact && compact ? TC_OP_BYTES / 2 : TC_OP_BYTES;
+  }
+  __device__ __forceinline__ int voff() const { return kMayCompact && compact ? TC_HALF : 2 * TC_HALF; }
+  __device__ __forceinline__ int rawv() const { return kMayCompact && compact ? TC_RAW_K / 2 : TC_RAW_K; }
 };
 
 // query rows one tile holds: 4 in IMMA variants (their int8 digit columns are 4
@@ -433,6 +453,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 template <bool INTP, int FEAT, bool IMMA>
 __host__ __device__ constexpr bool tc_claimed_items() {
   return (!INTP || IMMA) && FEAT != TC_FEAT_SUBSET;
+}
+
+// quantised pages shorter than a tile (several pages, each with its scales, in
+// one tile) reach the 16-column fp16-staging variants only
+template <int NCOL, bool INTP, bool IMMA>
+__host__ __device__ constexpr bool tc_pieces() {
+  return NCOL == 16 && INTP && !IMMA;
 }
 
 // query operands as prebuilt images, double-buffered (16-column variants)
@@ -636,16 +663,27 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   // other tile passes through the staging warps
   const bool direct = (kind == KIND_BF16 && (valid[0] & valid[1] & valid[2] & valid[3]) == 0xFFFFFFFFu) ||
                       (IMMA && kind == KIND_I8);
-  // ---- the tile's byte count (lane 0) and its pieces' scales (lane f: piece f) ----
-  float ks = 1.f, vs = 1.f;
-  if (kind != KIND_BF16 && pvalid) {
-    const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
-    ks = sc.x;
-    vs = sc.y;
-  }
-  float vs_max = pvalid ? vs : 0.f;
+  // ---- the tile's byte count (lane 0) and, for quantised tiles, its pieces'
+  // scales (lane f: piece f) and their largest V scale ----
+  float ks = 1.f, vs = 1.f, vs_max = 1.f;
+  if (!tc_pieces<NCOL, INTP, IMMA>()) {
+    // one piece per quantised tile (pages of 128 tokens or more): lane 0's scales
+    if (lane == 0 && kind != KIND_BF16) {
+      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
+      ks = sc.x;
+      vs = vs_max = sc.y;
+    }
+  } else if (kind != KIND_BF16) {  // the same in every lane
+    if (pvalid) {
+      const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
+      ks = sc.x;
+      vs = sc.y;
+    }
+    vs_max = pvalid ? vs : 0.f;
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) vs_max = fmaxf(vs_max, __shfl_xor_sync(0xffffffffu, vs_max, o));
+    for (int o = 8; o > 0; o >>= 1) vs_max = fmaxf(vs_max, __shfl_xor_sync(0xffffffffu, vs_max, o));
+    vs_max = __shfl_sync(0xffffffffu, vs_max, 0);
+  }
   uint32_t bytes = 0;
   if (lane == 0) {
     if (kind == KIND_BF16) {
@@ -674,12 +712,15 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     m.direct = direct ? 1 : 0;
     m.vs = vs_max;
   }
-  constexpr int NP = NCOL == 16 ? 16 : 1;
-  if (lane < NP) {
-    c.S.meta[stage].ksp[lane] = ks;
-    c.S.meta[stage].vsp[lane] = vs;
+  if constexpr (tc_pieces<NCOL, INTP, IMMA>()) {
+    if (kind != KIND_BF16 && lane < 16) {
+      c.S.meta[stage].ksp[lane] = ks;
+      c.S.meta[stage].vsp[lane] = vs_max > 0.f ? vs / vs_max : 1.f;  // 1 with one piece
+    }
+    __syncwarp();  // the whole description is written before lane 0 publishes it
+  } else if (lane == 0) {
+    c.S.meta[stage].ksp[0] = ks;  // the softmax reads no V-scale ratio here
   }
-  __syncwarp();  // the whole description is written before lane 0 publishes it
   if (lane == 0) {
     if (direct) mbar_arrive(&c.S.raw_full[stage]);  // lets the staging warps skip this tile
     mbar_arrive_expect_tx(done, bytes);
@@ -687,14 +728,14 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   __syncwarp();
   if (pvalid) {
     const int r = lane * box_rows;
-    uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
+    uint8_t *op = c.op + static_cast<size_t>(stage) * c.sbytes();
     if (kind == KIND_BF16) {
       const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
       // head_dim 64 fills only the first half of K and of V: the QK products
       // stop at dim 64 and the P.V rows of dims 64..127 are never read
       tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, done);
       if (p.D == TC_D) tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
-      tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v, 0, y, done);
+      tma_load_2d(op + c.voff() + r * 128, &c.maps.v, 0, y, done);
       if (p.D == TC_D) tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
     } else if (IMMA && kind == KIND_I8) {
       // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows
@@ -711,12 +752,12 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     } else if (INTP) {
       const int rb = row_bytes(fmt, p.D);
       const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
-      // codes go to the stage's V region (K codes first, V codes TC_RAW_K bytes in),
+      // codes go to the stage's V region (K codes first, V codes rawv bytes in),
       // piece `lane` at row r; the staging warps expand them in place
       const int nrows = p.P >= TC_T ? rows : box_rows;
-      uint8_t *raw = op + 2 * TC_HALF + r * rb;
+      uint8_t *raw = op + c.voff() + r * rb;
       bulk_g2s(raw, p.k_pool[fmt] + off, nrows * rb, done);
-      bulk_g2s(raw + TC_RAW_K, p.v_pool[fmt] + off, nrows * rb, done);
+      bulk_g2s(raw + c.rawv(), p.v_pool[fmt] + off, nrows * rb, done);
     }
   }
   return true;
@@ -777,7 +818,7 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out, i
         tin0 = 0;
         ++pg0;
       }
-      if (++stage == Cfg::STAGES) {
+      if (++stage == c.nst()) {
         stage = 0;
         phase ^= 1u;
       }
@@ -786,27 +827,28 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out, i
 }
 
 // Staging of row r of a quantised tile for the fp16 MMAs: the int8 / int4 /
-// E4M3 codes of K and V, copied raw into the stage's V region (K codes at 0, V
-// codes TC_RAW_K bytes in), become fp16 operand rows (K halves at 0, V halves at
-// 2 * TC_HALF), 128-byte swizzled.  HD = head_dim: 128 fills both 64-dim halves,
+// E4M3 codes of K and V, copied raw into the stage's V region at voff (K codes
+// first, V codes rawv bytes in), become fp16 operand rows (K halves at 0, V
+// halves at voff), 128-byte swizzled.  HD = head_dim: 128 fills both 64-dim halves,
 // 64 the first (the QK products stop at dim 64; the P.V rows of dims 64..127 are
 // never read).  A thread loads its whole row before converting it, starting at
 // a row-dependent 16-byte chunk (no bank conflicts), and the V rows, which are
 // expanded over the codes, are all loaded (named barrier 3) before any is
 // written.  Rows that hold no token become zeros.
 template <int HD>
-__device__ __forceinline__ void tc_expand_codes(uint8_t *op, int r, bool valid, int kind) {
+__device__ __forceinline__ void tc_expand_codes(uint8_t *op, int voff, int rawv, int r, bool valid,
+                                                int kind) {
   constexpr int NCH = HD / 16;   // 16-byte chunks of an int8 / E4M3 code row
   constexpr int NCH4 = HD / 32;  // 16-byte chunks of an int4 code row
-  const uint8_t *raw = op + 2 * TC_HALF;
+  const uint8_t *raw = op + voff;
   const bool i4 = kind == KIND_I4;
   const int rb = i4 ? HD / 2 : HD;  // row bytes of the codes
   // K then V through one copy of the code (the kernel's roles share the SM's
   // instruction cache; unrolling this loop costs more than it saves)
 #pragma unroll 1
   for (int kv = 0; kv < 2; ++kv) {
-    uint8_t *dst = op + kv * 2 * TC_HALF;
-    const uint8_t *src = raw + kv * TC_RAW_K + r * rb;
+    uint8_t *dst = op + kv * voff;
+    const uint8_t *src = raw + kv * rawv + r * rb;
     uint4 w[NCH];
     if (valid) {
 #pragma unroll
@@ -904,13 +946,15 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       const auto &m = c.S.meta[stage];
       if (!m.direct) {
         const bool valid = (m.valid[r >> 5] >> (r & 31)) & 1u;
-        uint8_t *op = c.op + static_cast<size_t>(stage) * TC_OP_BYTES;
+        uint8_t *op = c.op + static_cast<size_t>(stage) * c.sbytes();
         if (m.kind == KIND_BF16) {
           if (!valid) {
+            // V rows that hold no token become zeros (their probability is 0)
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-              *reinterpret_cast<uint4 *>(op + 2 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4 *>(op + c.voff() + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
+              if (p.D == TC_D)
+                *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
             }
           }
         } else if (IMMA && m.kind == KIND_I4) {
@@ -945,9 +989,9 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
           }
         } else if (INTP) {
           if (IMMA || p.D == TC_D)  // int8-MMA variants only run head_dim 128
-            tc_expand_codes<TC_D>(op, r, valid, m.kind);
+            tc_expand_codes<TC_D>(op, c.voff(), c.rawv(), r, valid, m.kind);
           else
-            tc_expand_codes<TC_D / 2>(op, r, valid, m.kind);
+            tc_expand_codes<TC_D / 2>(op, c.voff(), c.rawv(), r, valid, m.kind);
         }
         fence_async_smem();
         named_sync(3, 128);
@@ -956,7 +1000,7 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       // the stage (and its description) may be refilled only once this
       // warpgroup is done with it, as well as the P.V product
       if (r == 0) mbar_arrive(&c.S.op_empty[stage]);
-      if (++stage == Cfg::STAGES) {
+      if (++stage == c.nst()) {
         stage = 0;
         phase ^= 1u;
       }
@@ -1000,7 +1044,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
         break;
       tc_fence_after();
       const int kind = c.S.meta[stage].kind;
-      const uint32_t kbase = op0 + stage * TC_OP_BYTES;
+      const uint32_t kbase = op0 + stage * c.sbytes();
       const uint32_t d = tmem + static_cast<uint32_t>(tc & 1) * NCOL;
       if (tc_int_tile<IMMA>(kind)) {
         // int8 codes [128 tok][128 dims] x query digits [NCOL][128 dims], K = 32 per MMA
@@ -1015,9 +1059,10 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
       } else {
         const uint32_t idesc = tc_idesc(kind == KIND_BF16 ? 1 : 0, 0, 0, NCOL);
         const uint32_t qbase = qop + (kind == KIND_BF16 ? 0u : static_cast<uint32_t>(Cfg::Q_BYTES));
-        const int ksteps = p.D / 16;  // 8, or 4 for head_dim 64 (the first half)
-#pragma unroll 8
-        for (int k = 0; k < ksteps; ++k) {
+        // 8 K-steps of 16 dims, or 4 for head_dim 64 (the first half)
+#pragma unroll
+        for (int k = 0; k < TC_D / 16; ++k) {
+          if (k >= 4 && p.D != TC_D) break;
           const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
           const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
           tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
@@ -1025,7 +1070,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
       }
       tc_commit(&c.S.s_full[tc & 1]);
       ++tc;
-      if (++stage == Cfg::STAGES) {
+      if (++stage == c.nst()) {
         stage = 0;
         phase ^= 1u;
       }
@@ -1063,7 +1108,10 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
       tc_fence_after();
       // the tile description stays valid until this P.V has freed the stage
       const int kind = c.S.meta[stage].kind;
-      const uint32_t vbase = op0 + stage * TC_OP_BYTES + 2 * TC_HALF;
+      // with the 32 KiB stages of head_dim 64 the MMA's rows of dims 64..127
+      // read the next 16 KiB of shared memory (another stage, or the query
+      // buffers): their products are never read
+      const uint32_t vbase = op0 + stage * c.sbytes() + c.voff();
       const uint32_t pbase = p0 + static_cast<uint32_t>(tc & 1) * Cfg::P_BYTES;
       const uint32_t d = tmem + 2 * NCOL + static_cast<uint32_t>(ob) * NCOL;
       if (tc_int_tile<IMMA>(kind)) {
@@ -1089,7 +1137,7 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
       tc_commit(&c.S.p_empty[tc & 1]);
       tc_commit(&c.S.op_empty[stage]);
       ++tc;
-      if (++stage == Cfg::STAGES) stage = 0;
+      if (++stage == c.nst()) stage = 0;
     }
   }
   tc_commit(&c.S.drain);
@@ -1131,9 +1179,10 @@ __device__ __forceinline__ void tc_fold(TcCtx<NCOL, INTP, FEAT, IMMA> &c, long l
     if (h < cnt) acc[h] = fmaf(acc[h], alpha_prev[h], (o[h] + o[NCOL / 2 + h]) * vscale_prev);
 }
 
-// element `dim` of query row vh of sequence b, as fp32
+// element `dim` of query row vh of sequence b, as fp32 (head_dim 128: the int8
+// digit operands of the int8-MMA variants)
 __device__ __forceinline__ float q_elem(const DecodeParams &p, int b, int vh, int dim) {
-  const long long i = (static_cast<long long>(b) * p.Hq + vh) * p.D + dim;
+  const long long i = (static_cast<long long>(b) * p.Hq + vh) * TC_D + dim;
   return p.q_fmt == CFR_FMT_F32
              ? static_cast<const float *>(p.q)[i]
              : __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t *>(p.q)[i]) << 16);
@@ -1151,8 +1200,8 @@ __device__ __forceinline__ float q_elem(const DecodeParams &p, int b, int vh, in
 //    d0 in [-127, 127], d1..d3 in [-64, 64]; qsc[h] receives max|q_h| / 127.
 // The 128 threads of a warpgroup or block (index tsm) share the work; the IMMA
 // part synchronises them once (sync()) through red[4][4] floats.
-template <int NCOL, bool INTP, bool IMMA, class Sync>
-__device__ __forceinline__ void tc_build_q(const DecodeParams &p, int b, int g, int tsm, int lane,
+template <int HD, int NCOL, bool INTP, bool IMMA, class Sync>
+__device__ __forceinline__ void tc_build_q_d(const DecodeParams &p, int b, int g, int tsm, int lane,
                                            uint8_t *dst, float (*red)[4], Sync sync,
                                            float (&qsc)[4]) {
   using Cfg = TcCfg<NCOL, INTP>;
@@ -1165,8 +1214,8 @@ __device__ __forceinline__ void tc_build_q(const DecodeParams &p, int b, int g, 
     float x[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) x[e] = 0.f;
-    if (head < cnt && 8 * ch < p.D) {  // dims past head_dim 64 stay 0
-      const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * p.D + 8 * ch;
+    if (head < cnt && 8 * ch < HD) {  // dims past head_dim 64 stay 0
+      const long long qi = (static_cast<long long>(b) * p.Hq + p.grp_heads[h0 + head]) * HD + 8 * ch;
       if (p.q_fmt == CFR_FMT_F32) {
         const float4 a = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi);
         const float4 bb = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qi + 4);
@@ -1246,6 +1295,18 @@ __device__ __forceinline__ void tc_build_q(const DecodeParams &p, int b, int g, 
     }
     *reinterpret_cast<uint4 *>(dst + 2 * Cfg::Q_BYTES + sw128(n, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
+}
+
+// head_dim 128 or 64 (the operand's second half left at 0), with the row
+// stride as a compile-time constant
+template <int NCOL, bool INTP, bool IMMA, class Sync>
+__device__ __forceinline__ void tc_build_q(const DecodeParams &p, int b, int g, int tsm, int lane,
+                                           uint8_t *dst, float (*red)[4], Sync sync,
+                                           float (&qsc)[4]) {
+  if (IMMA || p.D == TC_D)  // int8-MMA variants only run head_dim 128
+    tc_build_q_d<TC_D, NCOL, INTP, IMMA>(p, b, g, tsm, lane, dst, red, sync, qsc);
+  else if constexpr (!IMMA)
+    tc_build_q_d<TC_D / 2, NCOL, INTP, IMMA>(p, b, g, tsm, lane, dst, red, sync, qsc);
 }
 
 // 32-column variants: the softmax warpgroup writes the query operand of item
@@ -1362,14 +1423,18 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       const bool itile = tc_int_tile<IMMA>(kind);
       // int4 codes enter the int8 MMAs times 16; probability digits are of p * 255
       const float i4f = itile && kind == KIND_I4 ? 1.f / 16.f : 1.f;
-      // token t's page piece: its K scale, and its V scale relative to the tile's
-      // (1 with one piece per tile: pages of 128 tokens or more)
-      const int piece = NCOL == 16 ? t >> pshift : 0;
-      const float scale = m.ksp[piece] * p.sigma_log2e * i4f;
+      // quantised tiles: token t's page piece gives its K scale and its V scale
+      // relative to the tile's (1 with one piece per tile: pages of 128 tokens
+      // or more)
+      float scale = p.sigma_log2e, vratio = 1.f;
+      if (kind != KIND_BF16) {
+        const int piece = tc_pieces<NCOL, INTP, IMMA>() ? t >> pshift : 0;
+        scale = m.ksp[piece] * p.sigma_log2e * i4f;
+        if (tc_pieces<NCOL, INTP, IMMA>()) vratio = m.vsp[piece];
+      }
       const float vsc = kind == KIND_BF16 ? 1.f
                         : itile           ? m.vs * i4f * (1.f / 255.f)
                                           : m.vs * (1.f / 32768.f);
-      const float vratio = kind == KIND_BF16 || m.vs <= 0.f ? 1.f : m.vsp[piece] / m.vs;
       // ALiBi from the last position; a query row at offset o before it differs by the
       // row constant slope * o, added back to its maximum at the partial write
       const int j = m.t0 + t;
@@ -1499,7 +1564,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       vs1 = vsc;
       oi1 = itile;
       ++tc;
-      if (++stage == Cfg::STAGES) {
+      if (++stage == c.nst()) {
         stage = 0;
         phase ^= 1u;
       }
@@ -1512,7 +1577,10 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
     for (int h = 0; h < GH; ++h) {
       if (h < cnt) {
         const int head = p.grp_heads[h0 + h];
-        if (t < p.D) p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * p.D + t] = acc[h];
+        if (p.D == TC_D)  // (head_dim 64: dims 64..127 of O hold nothing)
+          p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * TC_D + t] = acc[h];
+        else if (t < TC_D / 2)
+          p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * (TC_D / 2) + t] = acc[h];
         float l = l_part[h];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -1552,7 +1620,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   TcSmem<NCOL, INTP> &S = *reinterpret_cast<TcSmem<NCOL, INTP> *>(smem);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < TcCfg<NCOL, INTP>::MAX_STAGES; ++s) {
       mbar_init(&S.op_full[s], 1);
       mbar_init(&S.op_empty[s], 2);  // P.V commit + staging warpgroup
       mbar_init(&S.raw_full[s], 1);
@@ -1601,7 +1669,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                   smem + L::q,
                                   smem + L::pbuf,
                                   static_cast<long long>(nsplit) * p.ngroups,
-                                  nsplit};
+                                  nsplit,
+                                  NCOL == 16 && !IMMA && p.D == TC_D / 2};
   bool timed_out = false;
   if (warp < 4) {
     tc_setmaxnreg<TC_REGS_IO>();
@@ -1616,7 +1685,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_setmaxnreg<TC_REGS_SOFTMAX>();
     tc_softmax<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   } else {
-    tc_setmaxnreg<TC_REGS_STAGING>();
+    // the int8-MMA variants' staging (int4 widening only) runs in fewer registers,
+    // which measured faster there
+    tc_setmaxnreg<IMMA ? TC_REGS_STAGING_IMMA : TC_REGS_STAGING>();
     tc_staging<NCOL, INTP, FEAT, IMMA>(c, &timed_out);
   }
   tc_fence_before();
