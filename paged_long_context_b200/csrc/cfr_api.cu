@@ -204,9 +204,12 @@ cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *
     start[g] = off;
     off += count[g];
   }
-  int gmax = 0, ng = 0;
+  int gmax = 0, ng = 0, nblk0 = -1;
+  bool uniform = true;  // every kv head cut into the same number of groups
   for (int g = 0; g < hkv; ++g) {
     const int nblk = count[g] <= kMaxGroup ? 1 : (count[g] + kMaxGroup - 1) / kMaxGroup;
+    if (nblk0 < 0) nblk0 = nblk;
+    uniform = uniform && nblk == nblk0;
     for (int j = 0; j < nblk; ++j) {
       const int lo = start[g] + count[g] * j / nblk, hi = start[g] + count[g] * (j + 1) / nblk;
       if (ng >= kMaxGroups) return CFR_ERR_UNSUPPORTED;
@@ -218,6 +221,7 @@ cfr_status build_groups(int hq, int hkv, const int32_t *head_map, DecodeParams *
   }
   p->grp_off[ng] = static_cast<int16_t>(off);
   p->ngroups = ng;
+  p->gsub = uniform && nblk0 > 1 ? nblk0 : 1;
   int fill[kMaxQHeads];
   for (int g = 0; g < hkv; ++g) fill[g] = start[g];
   for (int vh = 0; vh < rows; ++vh) {

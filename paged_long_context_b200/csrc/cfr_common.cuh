@@ -59,6 +59,7 @@ struct DecodeParams {
   int nq;               // query tokens per sequence (the last nq positions, causal)
   int hq_real;          // query heads; the Hq = nq * hq_real query rows are qi * hq_real + h
   int ngroups;          // row groups (Hkv, or more when a kv head has over kMaxGroup rows)
+  int gsub;             // groups per kv head when every kv head has the same number (else 1)
   int16_t grp_off[kMaxGroups + 1];  // rows of group g: grp_heads[grp_off[g] .. grp_off[g+1])
   int16_t grp_kv[kMaxGroups];       // the kv head whose pages group g reads
   int16_t grp_heads[kMaxQHeads];
@@ -347,12 +348,23 @@ __device__ __forceinline__ SplitRange split_at(const DecodeParams &p, int slot) 
   return r;
 }
 
-// Work item -> (split slot, kv head).  Items are numbered split-fastest, so the
-// CTAs that start together read different page slots of the pool rather than
-// the kv heads of one slot (those sit a fixed sub-page stride apart).
-__device__ __forceinline__ void item_coords(long long item, int nsplit, int &slot, int &g) {
-  slot = static_cast<int>(item % nsplit);
-  g = static_cast<int>(item / nsplit);
+// Work item -> (split slot, row group).  Items are numbered split-fastest, so
+// the CTAs that start together read different page slots of the pool rather
+// than the kv heads of one slot (those sit a fixed sub-page stride apart).  When
+// every kv head's rows form gsub > 1 groups (MQA, wide GQA), the gsub groups of
+// one kv head and split are numbered next to each other, so the CTAs that take
+// them read the same pages at about the same time and all but the first find
+// them in L2.
+__device__ __forceinline__ void item_coords(long long item, int nsplit, int gsub, int &slot, int &g) {
+  if (gsub > 1) {
+    const long long per = static_cast<long long>(nsplit) * gsub;  // items of one kv head
+    const long long r = item % per;
+    slot = static_cast<int>(r / gsub);
+    g = static_cast<int>(item / per) * gsub + static_cast<int>(r % gsub);
+  } else {
+    slot = static_cast<int>(item % nsplit);
+    g = static_cast<int>(item / nsplit);
+  }
 }
 
 }  // namespace cfr

@@ -220,7 +220,7 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
   const int P = p.P;
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), p.gsub, slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
@@ -314,7 +314,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), p.gsub, slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];

@@ -161,7 +161,7 @@ __device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_
   page_cache_reset(pc, lane);
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), p.gsub, slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
@@ -197,7 +197,7 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
 
   for (long long item = blockIdx.x; item < nitems; item += gridDim.x) {
     int slot, g;
-    item_coords(item, static_cast<int>(nitems / p.ngroups), slot, g);
+    item_coords(item, static_cast<int>(nitems / p.ngroups), p.gsub, slot, g);
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];

@@ -494,7 +494,7 @@ __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> 
   it = __shfl_sync(0xffffffffu, it, 0);
   if (it < c.nitems) {
     d.item = static_cast<int>(it);
-    item_coords(it, c.nsplit, d.slot, d.g);
+    item_coords(it, c.nsplit, p.gsub, d.slot, d.g);
     const SplitRange sr = split_at(p, d.slot);
     d.b = sr.b;
     d.pb = sr.pb;
