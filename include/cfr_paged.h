@@ -416,6 +416,13 @@ cfr_status cfr_append_kv(const cfr_kv_pool *kv, const int32_t *page_table, int32
  * benchmarks): 1 = general CUDA-core kernel (any format mix), 2 = tensor-core
  * (tcgen05) kernel, 3 = fp32 CUDA-core kernel with TMA tensor-map tiles, 0 if
  * the arguments would be rejected.  Host only; launches nothing.
+ *
+ * The tensor-core kernel takes bf16, FP8, int8 and int4 pages (no fp32) of
+ * head_dim 64 or 128 with a 16-byte-aligned q, page_tokens dividing 128 or a
+ * multiple of 128; quantised pages shorter than 128 tokens only when the cache
+ * has one format (page_fmt NULL) and at most 8 query rows per kv head.  The
+ * fp32 kernel takes fp32 caches with at most 2 query rows per kv head and the
+ * same page sizes.  Everything else runs on the general kernel.
  */
 int32_t cfr_paged_decode_path(int32_t q_fmt, const cfr_kv_pool *kv, int32_t max_pages,
                               const uint8_t *page_fmt, int32_t uniform_fmt,
