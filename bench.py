@@ -3,7 +3,8 @@
 every (sequence, query head) of the workload (schedule + decode + merge).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload alibi1m|cfr|tiny|gqa|tiered|mqa|gqa_d64|gqa_d64_i8p16|gqa_d64_mixed_p16|demote]
+                    [--workload alibi1m|cfr|tiny|gqa|tiered|mqa|gqa_d64|gqa_d64_i8p16|gqa_d64_mixed_p16|
+                                gqa_i8p16|demote]
                     [--context N]
                     [--queries Q] [--sink S --window W]
     python bench.py --record-traffic NCU_CSV --workload W [--context N]

@@ -361,7 +361,7 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   // uniform int8 / int4 pools of up to 4 rows per group (the int8-MMA variant)
   const bool claimed =
       use_tc && (!quantised_pools(p, page_fmt != nullptr) ||
-                 (!page_fmt && p.gmax <= 4 && kv->head_dim == 128 && kv->page_tokens % 128 == 0 &&
+                 (!page_fmt && p.gmax <= 4 && kv->head_dim == 128 &&
                   (uniform_fmt == CFR_FMT_I8 || uniform_fmt == CFR_FMT_I4)));
   const int per_sm = claimed ? kItemsPerSmClaimed : page_fmt ? kItemsPerSmMixed : kItemsPerSm;
   const int target = target_splits(di.sms, p.ngroups, per_sm);

@@ -112,6 +112,11 @@ constexpr int TC_RAW_K = TC_T * TC_D;  // raw code offset of V inside a stage's 
 constexpr int KIND_BF16 = 0, KIND_I8 = 1, KIND_I4 = 2, KIND_FP8 = 3;
 // compile-time variants: plain decode, multi-query rows, sink + window subset
 constexpr int TC_FEAT_PLAIN = 0, TC_FEAT_MULTI = 1, TC_FEAT_SUBSET = 2;
+// OR'ed into the feature: quantised pages shorter than a tile in a uniform-format
+// cache (a tile holds several pages, each with its own scales); its own
+// instantiations, so that the variants for larger pages carry none of it
+constexpr int TC_FEAT_SMALL_PAGES = 4;
+__host__ __device__ constexpr int tc_feat(int feat) { return feat & 3; }
 
 // one work item as producer warp 0 publishes it (see tc_publish_item)
 struct TcItem {
@@ -452,14 +457,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 //    no counter (item_ctr = null), which selects the fixed share.
 template <bool INTP, int FEAT, bool IMMA>
 __host__ __device__ constexpr bool tc_claimed_items() {
-  return (!INTP || IMMA) && FEAT != TC_FEAT_SUBSET;
+  return (!INTP || IMMA) && tc_feat(FEAT) != TC_FEAT_SUBSET;
 }
 
 // quantised pages shorter than a tile (several pages, each with its scales, in
-// one tile) reach the 16-column fp16-staging variants only
-template <int NCOL, bool INTP, bool IMMA>
+// one tile): the small-page instantiations of the 16-column variants with
+// quantised pools
+template <int NCOL, bool INTP, int FEAT>
 __host__ __device__ constexpr bool tc_pieces() {
-  return NCOL == 16 && INTP && !IMMA;
+  return NCOL == 16 && INTP && (FEAT & TC_FEAT_SMALL_PAGES) != 0;
 }
 
 // query operands as prebuilt images, double-buffered (16-column variants)
@@ -646,7 +652,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     const int row = 32 * w + lane;
     valid[w] = __ballot_sync(0xffffffffu, row < rows && ((vb >> (row >> geo.box_shift)) & 1u));
   }
-  if constexpr (FEAT == TC_FEAT_SUBSET)
+  if constexpr (tc_feat(FEAT) == TC_FEAT_SUBSET)
     mask_clear_gap(valid, p, n, t0, rows);  // tokens between the sinks and the recent window
   // the tile's kind is the format of its first valid piece: a cache whose page
   // formats differ has quantised pages of 128 tokens or more (one piece per
@@ -666,7 +672,8 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   // ---- the tile's byte count (lane 0) and, for quantised tiles, its pieces'
   // scales (lane f: piece f) and their largest V scale ----
   float ks = 1.f, vs = 1.f, vs_max = 1.f;
-  if (!tc_pieces<NCOL, INTP, IMMA>()) {
+  constexpr bool pieces = tc_pieces<NCOL, INTP, FEAT>();
+  if (!pieces) {
     // one piece per quantised tile (pages of 128 tokens or more): lane 0's scales
     if (lane == 0 && kind != KIND_BF16) {
       const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
@@ -690,7 +697,9 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
       // a K and a V box per 64 dims (2 with head_dim 64, 4 with 128) per valid piece
       bytes = static_cast<uint32_t>(__popc(vb)) * static_cast<uint32_t>(p.D / 32) * box_rows * 128u;
     } else if (IMMA && kind == KIND_I8) {
-      bytes = 2u * TC_T * 128u;  // one full 128-row box of K and of V
+      // a full box of K and of V per valid piece (one 128-row box with pages of
+      // 128 tokens or more)
+      bytes = static_cast<uint32_t>(p.P >= TC_T ? 1 : __popc(vb)) * 2u * box_rows * 128u;
     } else if (p.P >= TC_T) {
       bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, p.D));  // the tile's rows of one page
     } else {
@@ -712,14 +721,14 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     m.direct = direct ? 1 : 0;
     m.vs = vs_max;
   }
-  if constexpr (tc_pieces<NCOL, INTP, IMMA>()) {
+  if constexpr (pieces) {
     if (kind != KIND_BF16 && lane < 16) {
       c.S.meta[stage].ksp[lane] = ks;
-      c.S.meta[stage].vsp[lane] = vs_max > 0.f ? vs / vs_max : 1.f;  // 1 with one piece
+      c.S.meta[stage].vsp[lane] = vs_max > 0.f ? vs / vs_max : 1.f;
     }
     __syncwarp();  // the whole description is written before lane 0 publishes it
   } else if (lane == 0) {
-    c.S.meta[stage].ksp[0] = ks;  // the softmax reads no V-scale ratio here
+    c.S.meta[stage].ksp[0] = ks;
   }
   if (lane == 0) {
     if (direct) mbar_arrive(&c.S.raw_full[stage]);  // lets the staging warps skip this tile
@@ -738,17 +747,19 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
       tma_load_2d(op + c.voff() + r * 128, &c.maps.v, 0, y, done);
       if (p.D == TC_D) tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
     } else if (IMMA && kind == KIND_I8) {
-      // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows
+      // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows; piece
+      // `lane` at row r (boxes of min(P, 128) rows)
       const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
-      tma_load_2d(op, &c.maps.k8, 0, y, done);
-      tma_load_2d(op + 2 * TC_HALF, &c.maps.v8, 0, y, done);
+      tma_load_2d(op + r * 128, &c.maps.k8, 0, y, done);
+      tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v8, 0, y, done);
     } else if (IMMA && kind == KIND_I4) {
       // raw codes above the int8 operands the staging warps write (K at TC_HALF,
-      // V at 3 * TC_HALF)
+      // V at 3 * TC_HALF), piece `lane` at row r
       const int rb = row_bytes(fmt, TC_D);
       const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
-      bulk_g2s(op + TC_HALF, p.k_pool[fmt] + off, rows * rb, done);
-      bulk_g2s(op + 3 * TC_HALF, p.v_pool[fmt] + off, rows * rb, done);
+      const int nrows = p.P >= TC_T ? rows : box_rows;
+      bulk_g2s(op + TC_HALF + r * rb, p.k_pool[fmt] + off, nrows * rb, done);
+      bulk_g2s(op + 3 * TC_HALF + r * rb, p.v_pool[fmt] + off, nrows * rb, done);
     } else if (INTP) {
       const int rb = row_bytes(fmt, p.D);
       const long long off = ((id * p.Hkv + p.grp_kv[g]) * p.P + tin0) * rb;
@@ -1392,7 +1403,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         slope2[h] = c.S.slope_bc[k & 1][h];
       else
         slope2[h] = (p.slopes && h < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + h])] * kLog2e : 0.f;
-      if constexpr (FEAT == TC_FEAT_MULTI)
+      if constexpr (tc_feat(FEAT) == TC_FEAT_MULTI)
         if (h < cnt) qoff[h >> 3] |= static_cast<uint32_t>(row_offset(p, p.grp_heads[h0 + h])) << (4 * (h & 7));
       m_run[h] = -INFINITY;
       l_part[h] = 0.f;
@@ -1428,9 +1439,10 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
       // or more)
       float scale = p.sigma_log2e, vratio = 1.f;
       if (kind != KIND_BF16) {
-        const int piece = tc_pieces<NCOL, INTP, IMMA>() ? t >> pshift : 0;
+        constexpr bool pieces = tc_pieces<NCOL, INTP, FEAT>();
+        const int piece = pieces ? t >> pshift : 0;
         scale = m.ksp[piece] * p.sigma_log2e * i4f;
-        if (tc_pieces<NCOL, INTP, IMMA>()) vratio = m.vsp[piece];
+        if (pieces) vratio = m.vsp[piece];
       }
       const float vsc = kind == KIND_BF16 ? 1.f
                         : itile           ? m.vs * i4f * (1.f / 255.f)
@@ -1457,7 +1469,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         for (int h = 0; h < GH; ++h)
           s[h] = (valid && h < cnt) ? fmaf(sv[h] + sv[GM + h], scale, -slope2[h] * dist) : -INFINITY;
       }
-      if (FEAT == TC_FEAT_MULTI && m.t0 + TC_T - 1 > n - p.nq) {
+      if (tc_feat(FEAT) == TC_FEAT_MULTI && m.t0 + TC_T - 1 > n - p.nq) {
         // the tile reaches the query positions: row h sees tokens j <= n - 1 - offset_h
 #pragma unroll
         for (int h = 0; h < GH; ++h)
@@ -1502,7 +1514,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         // significant first, of X_h = round(p_h * 255 * 2^24) (< 2^32 for p <= 1)
         uint32_t x[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) x[h] = __float2uint_rn(pr[h] * 4278190080.f);
+        for (int h = 0; h < 4; ++h) x[h] = __float2uint_rn(pr[h] * vratio * 4278190080.f);
         // transpose the 4 x 4 bytes: word l = byte 3 - l of x[0..3]
         const uint32_t lo01 = prmt(x[0], x[1], 0x5140u), hi01 = prmt(x[0], x[1], 0x7362u);
         const uint32_t lo23 = prmt(x[2], x[3], 0x5140u), hi23 = prmt(x[2], x[3], 0x7362u);
@@ -1594,7 +1606,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
 #pragma unroll
       for (int h = 0; h < GH; ++h)
         if (h == tsm) mrun = m_run[h];
-      if constexpr (FEAT == TC_FEAT_MULTI) {
+      if constexpr (tc_feat(FEAT) == TC_FEAT_MULTI) {
         const int vh = p.grp_heads[h0 + tsm];
         float sl = 0.f;
 #pragma unroll
@@ -1759,12 +1771,13 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
       return cudaErrorInvalidValue;
   }
   if (IMMA && p.k_pool[CFR_FMT_I8] && p.pool_pages[CFR_FMT_I8] > 0) {
-    // int pages have page_tokens a multiple of 128: one 128-row box per tile
+    // one box per page piece: 128 rows, or a whole page when pages are shorter
     const long long rows = p.pool_pages[CFR_FMT_I8] * p.Hkv * static_cast<long long>(p.P);
+    const int box_rows = p.P < TC_T ? p.P : TC_T;
     if (!encode_pool_map(&maps.k8, p.k_pool[CFR_FMT_I8], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows,
-                         TC_D, TC_T) ||
+                         TC_D, box_rows) ||
         !encode_pool_map(&maps.v8, p.v_pool[CFR_FMT_I8], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows,
-                         TC_D, TC_T))
+                         TC_D, box_rows))
       return cudaErrorInvalidValue;
   }
   constexpr size_t smem = TcLayout<NCOL, INTP>::launch_bytes;
@@ -1796,7 +1809,8 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
 // int8 or int4 pools whose tiles can run the int8 MMAs: up to 4 query rows per
 // kv head (4 digit columns each fill the 16-column operand)
 static bool tc_imma(const DecodeParams &p, bool page_fmt_given) {
-  if (p.gmax > 4 || p.D != TC_D || p.P % TC_T != 0) return false;
+  // (quantised pages under 128 tokens: uniform-format caches only)
+  if (p.gmax > 4 || p.D != TC_D || (p.P % TC_T != 0 && page_fmt_given)) return false;
   if (page_fmt_given) return p.k_pool[CFR_FMT_I8] || p.k_pool[CFR_FMT_I4];
   return p.uniform_fmt == CFR_FMT_I8 || p.uniform_fmt == CFR_FMT_I4;
 }
@@ -1804,7 +1818,12 @@ static bool tc_imma(const DecodeParams &p, bool page_fmt_given) {
 template <int FEAT>
 static cudaError_t tc_launch_f(const DecodeParams &p, int grid, cudaStream_t stream) {
   const bool ints = tc_int_pools(p, p.page_fmt != nullptr);
-  if (ints && tc_imma(p, p.page_fmt != nullptr)) return tc_launch_t<16, true, FEAT, true>(p, grid, stream);
+  // quantised pages under 128 tokens (uniform format, at most 8 rows per group)
+  const bool small = ints && p.P < TC_T;
+  if (ints && tc_imma(p, p.page_fmt != nullptr))
+    return small ? tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, true>(p, grid, stream)
+                 : tc_launch_t<16, true, FEAT, true>(p, grid, stream);
+  if (small) return tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, false>(p, grid, stream);
   if (p.gmax <= 8)
     return ints ? tc_launch_t<16, true, FEAT, false>(p, grid, stream)
                 : tc_launch_t<16, false, FEAT, false>(p, grid, stream);

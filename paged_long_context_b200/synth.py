@@ -457,6 +457,13 @@ def spec_gqa_d64_i8_p16() -> CaseSpec:
                     len_range=(1024, 32768), fmt="i8", q_fmt="bf16", permute=True)
 
 
+def spec_gqa_i8_p16() -> CaseSpec:
+    """The ragged GQA batch as int8 pages of 16 tokens, head_dim 128 (the
+    tensor-core kernel's int8 MMAs: a tile holds 8 pages, each with its scales)."""
+    return CaseSpec("gqa_ragged_b16_1k32k_p16_i8", 16, 32, 8, 128, 16, len_range=(1024, 32768),
+                    fmt="i8", q_fmt="bf16", permute=True)
+
+
 def spec_gqa_d64_mixed_p16() -> CaseSpec:
     """The same batch with int8 and bf16 pages of 16 tokens mixed, head_dim 64: a
     shape only the general CUDA-core kernel takes (quantised pages under 128
@@ -476,6 +483,7 @@ WORKLOADS = {
     "gqa_d64": (spec_gqa_d64, 7),
     "gqa_d64_i8p16": (spec_gqa_d64_i8_p16, 7),
     "gqa_d64_mixed_p16": (spec_gqa_d64_mixed_p16, 7),
+    "gqa_i8p16": (spec_gqa_i8_p16, 3),
 }
 
 
