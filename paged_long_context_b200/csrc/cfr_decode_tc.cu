@@ -695,7 +695,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   if (lane == 0) {
     if (kind == KIND_BF16) {
       // a K and a V box per 64 dims (2 with head_dim 64, 4 with 128) per valid piece
-      bytes = static_cast<uint32_t>(__popc(vb)) * static_cast<uint32_t>(p.D / 32) * box_rows * 128u;
+      bytes = static_cast<uint32_t>(__popc(vb)) * ((IMMA || p.D == TC_D) ? 4u : 2u) * box_rows * 128u;
     } else if (IMMA && kind == KIND_I8) {
       // a full box of K and of V per valid piece (one 128-row box with pages of
       // 128 tokens or more)
@@ -743,9 +743,9 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
       // head_dim 64 fills only the first half of K and of V: the QK products
       // stop at dim 64 and the P.V rows of dims 64..127 are never read
       tma_load_2d(op + 0 * TC_HALF + r * 128, &c.maps.k, 0, y, done);
-      if (p.D == TC_D) tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
+      if (IMMA || p.D == TC_D) tma_load_2d(op + 1 * TC_HALF + r * 128, &c.maps.k, 64, y, done);
       tma_load_2d(op + c.voff() + r * 128, &c.maps.v, 0, y, done);
-      if (p.D == TC_D) tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
+      if (IMMA || p.D == TC_D) tma_load_2d(op + 3 * TC_HALF + r * 128, &c.maps.v, 64, y, done);
     } else if (IMMA && kind == KIND_I8) {
       // K codes at 0, V codes at 2 * TC_HALF, 128-byte swizzled rows; piece
       // `lane` at row r (boxes of min(P, 128) rows)
@@ -964,7 +964,7 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
               *reinterpret_cast<uint4 *>(op + c.voff() + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-              if (p.D == TC_D)
+              if (IMMA || p.D == TC_D)
                 *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
             }
           }
@@ -1073,7 +1073,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
         // 8 K-steps of 16 dims, or 4 for head_dim 64 (the first half)
 #pragma unroll
         for (int k = 0; k < TC_D / 16; ++k) {
-          if (k >= 4 && p.D != TC_D) break;
+          if (!IMMA && k >= 4 && p.D != TC_D) break;  // (int8-MMA variants: head_dim 128)
           const uint64_t a = tc_sdesc(kbase + (k >> 2) * TC_HALF + (k & 3) * 32, 16, 1024, 2);
           const uint64_t bd = tc_sdesc(qbase + (k >> 2) * (NCOL * 128) + (k & 3) * 32, 16, 1024, 2);
           tc_mma(d, a, bd, idesc, k > 0 ? 1u : 0u);
@@ -1589,7 +1589,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
     for (int h = 0; h < GH; ++h) {
       if (h < cnt) {
         const int head = p.grp_heads[h0 + h];
-        if (p.D == TC_D)  // (head_dim 64: dims 64..127 of O hold nothing)
+        if (IMMA || p.D == TC_D)  // (head_dim 64: dims 64..127 of O hold nothing)
           p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * TC_D + t] = acc[h];
         else if (t < TC_D / 2)
           p.part_acc[(static_cast<long long>(slot) * p.Hq + head) * (TC_D / 2) + t] = acc[h];
