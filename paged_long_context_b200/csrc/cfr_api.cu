@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "cfr_common.cuh"
+#include "cfr_sched.cuh"
 
 namespace cfr {
 
@@ -19,7 +20,8 @@ void launch_gather(const DecodeParams &p, int b, int g, int n_tokens, void *k_ou
 cudaError_t launch_decode_cc(const DecodeParams &p, int grid, cudaStream_t stream);
 int cc_stages(int D, int gt, int pitch, size_t smem_limit);
 int cc_group_tile(int gmax);
-cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream,
+                             const SchedArgs *sched);
 bool tc_supported(const DecodeParams &p, bool page_fmt_given);
 cudaError_t launch_decode_f32(const DecodeParams &p, int grid, cudaStream_t stream);
 bool f32_supported(const DecodeParams &p, bool page_fmt_given);
@@ -404,13 +406,17 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
     p.stages = cc_stages(p.D, cc_group_tile(p.gmax), p.pitch, di.smem_optin);
     if (p.stages < 2) return CFR_ERR_UNSUPPORTED;
   }
-  if (phases & CFR_PHASE_SCHEDULE) {
+  const SchedArgs sched{seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, nq,
+                        split_off, splits, w.max_splits, num_splits, item_ctr, err_word};
+  // the tensor-core path runs a call's schedule inside its own first launch
+  const bool sched_in_decode = use_tc && (phases & CFR_PHASE_SCHEDULE) && (phases & CFR_PHASE_DECODE);
+  if ((phases & CFR_PHASE_SCHEDULE) && !sched_in_decode) {
     launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, nq,
                     split_off, splits, w.max_splits, num_splits, item_ctr, err_word, s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_DECODE) {
-    const cudaError_t e = use_tc    ? launch_decode_tc(p, di.sms, s)
+    const cudaError_t e = use_tc    ? launch_decode_tc(p, di.sms, s, sched_in_decode ? &sched : nullptr)
                           : use_f32 ? launch_decode_f32(p, di.sms, s)
                                     : launch_decode_cc(p, di.sms, s);
     if (e != cudaSuccess) return CFR_ERR_CUDA;

@@ -64,6 +64,7 @@
 
 #include <cstring>
 
+#include "cfr_sched.cuh"
 #include "cfr_tmap.cuh"
 
 namespace cfr {
@@ -1338,9 +1339,16 @@ __device__ __forceinline__ void tc_write_q(TcCtx<NCOL, INTP, FEAT, IMMA> &c, con
 // shared memory for every work item of the group.  Sequences outside
 // [1, max_pages * page_tokens] are skipped (the decode skips them too).
 template <int NCOL, bool INTP, bool IMMA>
-__global__ void __launch_bounds__(128) tc_qimage_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(128) tc_qimage_kernel(const __grid_constant__ DecodeParams p,
+                                                        const __grid_constant__ SchedArgs sched,
+                                                        int with_schedule) {
   __shared__ float red[4][4];
-  const long long grp = blockIdx.x;
+  if (with_schedule && blockIdx.x == 0) {
+    // block 0 computes the split schedule (one launch for both)
+    schedule_block(sched);
+    return;
+  }
+  const long long grp = static_cast<long long>(blockIdx.x) - with_schedule;
   const int b = static_cast<int>(grp / p.ngroups), g = static_cast<int>(grp % p.ngroups);
   const int n = p.seq_lens[b];
   if (n < p.nq || n > p.max_pages * p.P) return;
@@ -1757,8 +1765,17 @@ bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
   return true;
 }
 
+void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
+                     int sink, int window, int nq, int32_t *split_off, int32_t *splits,
+                     int max_splits, int32_t *num_splits, uint32_t *item_ctr, uint32_t *err,
+                     cudaStream_t stream);
+
+// `sched`, when set, is this call's split schedule, which runs before the decode:
+// in one extra block of the query-image kernel where the variant has one, else
+// as the schedule kernel
 template <int NCOL, bool INTP, int FEAT, bool IMMA>
-static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t stream) {
+static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t stream,
+                               const SchedArgs *sched) {
   TcMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (p.k_pool[CFR_FMT_BF16] && p.pool_pages[CFR_FMT_BF16] > 0) {
@@ -1795,9 +1812,17 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
   }();
   if (launch_regs != TC_REGS_LAUNCH) return cudaErrorInvalidConfiguration;
   if constexpr (tc_qimg<NCOL>()) {
-    // the query operand image of every (sequence, kv head)
+    // the query operand image of every (sequence, row group), after the schedule
+    // in block 0 when this call schedules
     const long long groups = static_cast<long long>(p.batch) * p.ngroups;
-    tc_qimage_kernel<NCOL, INTP, IMMA><<<dim3(static_cast<unsigned>(groups)), dim3(128), 0, stream>>>(p);
+    const SchedArgs sa = sched ? *sched : SchedArgs{};
+    const int extra = sched ? 1 : 0;
+    tc_qimage_kernel<NCOL, INTP, IMMA>
+        <<<dim3(static_cast<unsigned>(groups + extra)), dim3(128), 0, stream>>>(p, sa, extra);
+  } else if (sched) {
+    launch_schedule(sched->seq_lens, sched->batch, sched->P, sched->max_pages, sched->target,
+                    sched->sink, sched->window, sched->nq, sched->split_off, sched->splits,
+                    sched->max_splits, sched->num_splits, sched->item_ctr, sched->err, stream);
   }
   // a plain launch: overlapping this kernel's start with the previous kernel
   // (programmatic dependent launch) measured slower for this kernel
@@ -1816,26 +1841,28 @@ static bool tc_imma(const DecodeParams &p, bool page_fmt_given) {
 }
 
 template <int FEAT>
-static cudaError_t tc_launch_f(const DecodeParams &p, int grid, cudaStream_t stream) {
+static cudaError_t tc_launch_f(const DecodeParams &p, int grid, cudaStream_t stream,
+                               const SchedArgs *sched) {
   const bool ints = tc_int_pools(p, p.page_fmt != nullptr);
   // quantised pages under 128 tokens (uniform format, at most 8 rows per group)
   const bool small = ints && p.P < TC_T;
   if (ints && tc_imma(p, p.page_fmt != nullptr))
-    return small ? tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, true>(p, grid, stream)
-                 : tc_launch_t<16, true, FEAT, true>(p, grid, stream);
-  if (small) return tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, false>(p, grid, stream);
+    return small ? tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, true>(p, grid, stream, sched)
+                 : tc_launch_t<16, true, FEAT, true>(p, grid, stream, sched);
+  if (small) return tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, false>(p, grid, stream, sched);
   if (p.gmax <= 8)
-    return ints ? tc_launch_t<16, true, FEAT, false>(p, grid, stream)
-                : tc_launch_t<16, false, FEAT, false>(p, grid, stream);
-  return ints ? tc_launch_t<32, true, FEAT, false>(p, grid, stream)
-              : tc_launch_t<32, false, FEAT, false>(p, grid, stream);
+    return ints ? tc_launch_t<16, true, FEAT, false>(p, grid, stream, sched)
+                : tc_launch_t<16, false, FEAT, false>(p, grid, stream, sched);
+  return ints ? tc_launch_t<32, true, FEAT, false>(p, grid, stream, sched)
+              : tc_launch_t<32, false, FEAT, false>(p, grid, stream, sched);
 }
 
-cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream) {
+cudaError_t launch_decode_tc(const DecodeParams &p, int grid, cudaStream_t stream,
+                             const SchedArgs *sched) {
   // plain decode runs neither the per-row causal masks nor the subset masks
-  if (p.nq > 1) return tc_launch_f<TC_FEAT_MULTI>(p, grid, stream);
-  if (p.window > 0) return tc_launch_f<TC_FEAT_SUBSET>(p, grid, stream);
-  return tc_launch_f<TC_FEAT_PLAIN>(p, grid, stream);
+  if (p.nq > 1) return tc_launch_f<TC_FEAT_MULTI>(p, grid, stream, sched);
+  if (p.window > 0) return tc_launch_f<TC_FEAT_SUBSET>(p, grid, stream, sched);
+  return tc_launch_f<TC_FEAT_PLAIN>(p, grid, stream, sched);
 }
 
 }  // namespace cfr
