@@ -117,6 +117,9 @@ constexpr int TC_FEAT_PLAIN = 0, TC_FEAT_MULTI = 1, TC_FEAT_SUBSET = 2;
 // cache (a tile holds several pages, each with its own scales); its own
 // instantiations, so that the variants for larger pages carry none of it
 constexpr int TC_FEAT_SMALL_PAGES = 4;
+// OR'ed into the feature of int8-MMA variants: a uniform int8 cache, whose tiles
+// (int8 codes only: 16 KiB of K and 16 KiB of V) fit six 32 KiB stages
+constexpr int TC_FEAT_COMPACT_I8 = 8;
 __host__ __device__ constexpr int tc_feat(int feat) { return feat & 3; }
 
 // one work item as producer warp 0 publishes it (see tc_publish_item)
@@ -354,21 +357,22 @@ struct TcCtx {
   uint8_t *op, *qop, *pop;
   long long nitems;
   int nsplit;
-  // head_dim 64 in a 16-column variant other than int8-MMA: six stages of 32 KiB
-  // (K half, V half) instead of three of 64 KiB
+  // six stages of 32 KiB (K, V) instead of three of 64 KiB: head_dim 64 in a
+  // 16-column variant other than int8-MMA (compact, set at run time), and the
+  // int8-MMA variants of uniform int8 caches (always)
   bool compact;
   // stage geometry: nst() stages of sbytes() bytes; the V operand (and the raw
   // codes of quantised tiles) at voff() in a stage, the raw V codes rawv() bytes
-  // after the raw K codes.  Compile-time constants where compact cannot hold.
+  // after the raw K codes.  Compile-time constants where the choice is.
   static constexpr bool kMayCompact = NCOL == 16 && !IMMA;
+  static constexpr bool kAlwaysCompact = IMMA && (FEAT & TC_FEAT_COMPACT_I8) != 0;
+  __device__ __forceinline__ bool is_compact() const { return kAlwaysCompact || (kMayCompact && compact); }
   __device__ __forceinline__ int nst() const {
-    return kMayCompact && compact ? 2 * TcCfg<NCOL, INTP>::STAGES : TcCfg<NCOL, INTP>::STAGES;
+    return is_compact() ? 2 * TcCfg<NCOL, INTP>::STAGES : TcCfg<NCOL, INTP>::STAGES;
   }
-  __device__ __forceinline__ int sbytes() const {
-    return kMayCompact && compact ? TC_OP_BYTES / 2 : TC_OP_BYTES;
-  }
-  __device__ __forceinline__ int voff() const { return kMayCompact && compact ? TC_HALF : 2 * TC_HALF; }
-  __device__ __forceinline__ int rawv() const { return kMayCompact && compact ? TC_RAW_K / 2 : TC_RAW_K; }
+  __device__ __forceinline__ int sbytes() const { return is_compact() ? TC_OP_BYTES / 2 : TC_OP_BYTES; }
+  __device__ __forceinline__ int voff() const { return is_compact() ? TC_HALF : 2 * TC_HALF; }
+  __device__ __forceinline__ int rawv() const { return is_compact() ? TC_RAW_K / 2 : TC_RAW_K; }
 };
 
 // query rows one tile holds: 4 in IMMA variants (their int8 digit columns are 4
@@ -663,7 +667,12 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
                     : fmt == CFR_FMT_I4    ? KIND_I4
                     : fmt == CFR_FMT_FP8   ? KIND_FP8
                                            : KIND_BF16;
-  const int kind = __shfl_sync(0xffffffffu, kind0, vb ? __ffs(vb) - 1 : 0);
+  // (a tile with no valid piece in a uniform int8 cache keeps the int8 kind: its
+  // stage has no room for a bf16 V, and its stale int8 codes meet zero
+  // probabilities)
+  const int kind = !vb && TcCtx<NCOL, INTP, FEAT, IMMA>::kAlwaysCompact
+                       ? KIND_I8
+                       : __shfl_sync(0xffffffffu, kind0, vb ? __ffs(vb) - 1 : 0);
   // a bf16 tile whose 128 rows all hold tokens goes straight to the MMA, and so
   // does every int8 tile of an IMMA variant (its codes are the operand; rows
   // that hold no token carry finite codes that meet a zero probability); every
@@ -676,7 +685,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
   constexpr bool pieces = tc_pieces<NCOL, INTP, FEAT>();
   if (!pieces) {
     // one piece per quantised tile (pages of 128 tokens or more): lane 0's scales
-    if (lane == 0 && kind != KIND_BF16) {
+    if (lane == 0 && kind != KIND_BF16 && pvalid) {
       const float2 sc = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
       ks = sc.x;
       vs = vs_max = sc.y;
@@ -700,7 +709,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
     } else if (IMMA && kind == KIND_I8) {
       // a full box of K and of V per valid piece (one 128-row box with pages of
       // 128 tokens or more)
-      bytes = static_cast<uint32_t>(p.P >= TC_T ? 1 : __popc(vb)) * 2u * box_rows * 128u;
+      bytes = static_cast<uint32_t>(__popc(vb)) * 2u * box_rows * 128u;
     } else if (p.P >= TC_T) {
       bytes = 2u * rows * static_cast<uint32_t>(row_bytes(fmt, p.D));  // the tile's rows of one page
     } else {
@@ -752,7 +761,7 @@ __device__ __forceinline__ bool tc_produce_tile(TcCtx<NCOL, INTP, FEAT, IMMA> &c
       // `lane` at row r (boxes of min(P, 128) rows)
       const int y = static_cast<int>((id * p.Hkv + p.grp_kv[g]) * p.P + tin0);
       tma_load_2d(op + r * 128, &c.maps.k8, 0, y, done);
-      tma_load_2d(op + 2 * TC_HALF + r * 128, &c.maps.v8, 0, y, done);
+      tma_load_2d(op + c.voff() + r * 128, &c.maps.v8, 0, y, done);
     } else if (IMMA && kind == KIND_I4) {
       // raw codes above the int8 operands the staging warps write (K at TC_HALF,
       // V at 3 * TC_HALF), piece `lane` at row r
@@ -965,7 +974,7 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
               *reinterpret_cast<uint4 *>(op + c.voff() + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
-              if (IMMA || p.D == TC_D)
+              if ((IMMA || p.D == TC_D) && !c.is_compact())
                 *reinterpret_cast<uint4 *>(op + 3 * TC_HALF + sw128(r, ch)) = make_uint4(0, 0, 0, 0);
             }
           }
@@ -1846,9 +1855,14 @@ static cudaError_t tc_launch_f(const DecodeParams &p, int grid, cudaStream_t str
   const bool ints = tc_int_pools(p, p.page_fmt != nullptr);
   // quantised pages under 128 tokens (uniform format, at most 8 rows per group)
   const bool small = ints && p.P < TC_T;
-  if (ints && tc_imma(p, p.page_fmt != nullptr))
-    return small ? tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, true>(p, grid, stream, sched)
+  if (ints && tc_imma(p, p.page_fmt != nullptr)) {
+    constexpr int S = TC_FEAT_SMALL_PAGES, C = TC_FEAT_COMPACT_I8;
+    if (!p.page_fmt && p.uniform_fmt == CFR_FMT_I8)  // int8 tiles only: six 32 KiB stages
+      return small ? tc_launch_t<16, true, FEAT | S | C, true>(p, grid, stream, sched)
+                   : tc_launch_t<16, true, FEAT | C, true>(p, grid, stream, sched);
+    return small ? tc_launch_t<16, true, FEAT | S, true>(p, grid, stream, sched)
                  : tc_launch_t<16, true, FEAT, true>(p, grid, stream, sched);
+  }
   if (small) return tc_launch_t<16, true, FEAT | TC_FEAT_SMALL_PAGES, false>(p, grid, stream, sched);
   if (p.gmax <= 8)
     return ints ? tc_launch_t<16, true, FEAT, false>(p, grid, stream, sched)
