@@ -361,3 +361,36 @@ def test_small_quantised_pages_on_the_tensor_core_kernel(fmt, P, d):
     out, lse, err = run(case)
     assert err == 0
     check(case, out, lse)
+
+
+BAD_PAGE_SHAPES = {
+    # uniform int8, one page per tile: the int8-MMA variant with six 32 KiB stages
+    "i8_p128": dict(d=128, P=128, fmt="i8"),
+    # uniform int8, eight pages per tile (one of them bad)
+    "i8_p16": dict(d=128, P=16, fmt="i8"),
+    # uniform int4, one page per tile: the int8-MMA variant with three stages
+    "i4_p128": dict(d=128, P=128, fmt="i4"),
+    # bf16, eight pages per tile
+    "bf16_p16": dict(d=128, P=16, fmt="bf16"),
+    # int8 at head_dim 64 (fp16 staging, six 32 KiB stages), two pages per tile
+    "i8_d64_p64": dict(d=64, P=64, fmt="i8"),
+}
+
+
+@pytest.mark.parametrize("shape", list(BAD_PAGE_SHAPES))
+@pytest.mark.parametrize("how", ["id_too_big", "id_negative"])
+def test_bad_page_on_the_tensor_core_kernel(shape, how):
+    # a tile whose only page (or one of whose pages) has a bad id: its tokens
+    # are skipped and reported, the rest equals attention without them
+    kw = BAD_PAGE_SHAPES[shape]
+    P = kw["P"]
+    case = small_case(B=2, Hq=8, Hkv=2, lens=(5 * P + 3, 2 * P + 1), q_fmt="bf16", alibi=True,
+                      seed=P, **kw)
+    assert binding.decode_path(case) == binding.PATH_TENSOR_CORE
+    case.page_table[0, 1] = (1 << 20) if how == "id_too_big" else -3
+    out, lse, err = run(case)
+    assert err & binding.DEVERR_PAGE_ID
+    hc = case.to("cpu")
+    ref_o, _ = oracle.attend(hc, mode=0, skip_invalid=True)
+    ref_o = ref_o.reshape(2, 8, kw["d"])
+    np.testing.assert_allclose(out.double().numpy(), ref_o, atol=2e-3 * pool_vmax(hc), rtol=0)
