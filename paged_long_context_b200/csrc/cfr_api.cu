@@ -9,7 +9,7 @@
 namespace cfr {
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
-                     int sink, int window, int nq, int32_t *split_off, int32_t *splits,
+                     int sink, int window, int nq, int unit, int32_t *split_off, int32_t *splits,
                      int max_splits, int32_t *num_splits, uint32_t *item_ctr, uint32_t *err,
                      cudaStream_t stream);
 void launch_merge(const float *part_acc, const float *part_m, const float *part_l,
@@ -101,7 +101,17 @@ int target_splits(int sms, int hkv, int per_sm = kItemsPerSmMixed) {
   return static_cast<int>(t);
 }
 
-// workspace header: [0] split count, [1] split length in pages; at byte
+// The decode schedule's unit (tokens): the page, or 128 tokens (every kernel's
+// tile divides 128) when pages are a larger multiple of 128 and the page tables
+// hold fewer pages than the GPU has SMs, so that a short batch of long pages
+// still spreads over the SMs.  (Splitting pages of larger batches measured
+// slower: the mixed-format cache took 27 % longer.)
+int schedule_unit(int page_tokens, int batch, int max_pages, int sms) {
+  const bool few_pages = static_cast<long long>(batch) * max_pages < sms;
+  return page_tokens > 128 && page_tokens % 128 == 0 && few_pages ? 128 : page_tokens;
+}
+
+// workspace header: [0] split count, [1] split length in schedule units; at byte
 // kItemCtrOffset the decode kernel's work-item claim counter and finished-CTA count
 constexpr size_t kItemCtrOffset = 64;
 
@@ -110,10 +120,11 @@ struct WsLayout {
   int max_splits;
 };
 
-bool ws_layout(int batch, int hq, int hkv, int d, int max_pages, int target, WsLayout *w) {
-  // ceil(len / chunk) summed over at most two page ranges per sequence
+bool ws_layout(int batch, int hq, int hkv, int d, int max_pages, int page_tokens, int unit,
+               int target, WsLayout *w) {
+  // ceil(len / chunk) summed over at most two unit ranges per sequence
   long long ms = static_cast<long long>(target) + 2LL * batch;
-  const long long cap = static_cast<long long>(batch) * max_pages;
+  const long long cap = static_cast<long long>(batch) * max_pages * (page_tokens / unit);
   if (cap < ms) ms = cap;
   if (ms < 1) ms = 1;
   if (ms > INT_MAX / 4) return false;
@@ -286,7 +297,8 @@ size_t cfr_paged_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
   DeviceInfo di;
   if (!device_info(&di)) return 0;
   WsLayout w;
-  if (!ws_layout(batch, num_q_heads, num_kv_heads, head_dim, max_pages,
+  if (!ws_layout(batch, num_q_heads, num_kv_heads, head_dim, max_pages, page_tokens,
+                 schedule_unit(page_tokens, batch, max_pages, di.sms),
                  target_splits(di.sms, num_kv_heads), &w))
     return 0;
   return w.total;
@@ -368,7 +380,9 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   const int per_sm = claimed ? kItemsPerSmClaimed : page_fmt ? kItemsPerSmMixed : kItemsPerSm;
   const int target = target_splits(di.sms, p.ngroups, per_sm);
   WsLayout w;
-  if (!ws_layout(batch, rows, kv->num_kv_heads, kv->head_dim, max_pages, target, &w))
+  const int unit = schedule_unit(kv->page_tokens, batch, max_pages, di.sms);
+  if (!ws_layout(batch, rows, kv->num_kv_heads, kv->head_dim, max_pages, kv->page_tokens, unit,
+                 target, &w))
     return CFR_ERR_OVERFLOW;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return CFR_ERR_WORKSPACE;
 
@@ -386,6 +400,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
   p.splits = splits;
   p.num_splits = num_splits;
   p.max_splits = w.max_splits;
+  p.split_unit = unit;
+  p.max_units = static_cast<int>(static_cast<long long>(max_pages) * kv->page_tokens / p.split_unit);
   // mixed-format caches with quantised pages share their items out in a fixed
   // pattern (no claim counter); see tc_claimed_items
   p.item_ctr = (page_fmt && quantised_pools(p, true)) ? nullptr : item_ctr;
@@ -407,12 +423,13 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
     if (p.stages < 2) return CFR_ERR_UNSUPPORTED;
   }
   const SchedArgs sched{seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, nq,
-                        split_off, splits, w.max_splits, num_splits, item_ctr, err_word};
+                        p.split_unit, split_off, splits, w.max_splits, num_splits, item_ctr,
+                        err_word};
   // the tensor-core path runs a call's schedule inside its own first launch
   const bool sched_in_decode = use_tc && (phases & CFR_PHASE_SCHEDULE) && (phases & CFR_PHASE_DECODE);
   if ((phases & CFR_PHASE_SCHEDULE) && !sched_in_decode) {
     launch_schedule(seq_lens, batch, kv->page_tokens, max_pages, target, sink, window, nq,
-                    split_off, splits, w.max_splits, num_splits, item_ctr, err_word, s);
+                    p.split_unit, split_off, splits, w.max_splits, num_splits, item_ctr, err_word, s);
     if (cudaGetLastError() != cudaSuccess) return CFR_ERR_CUDA;
   }
   if (phases & CFR_PHASE_DECODE) {
@@ -499,8 +516,9 @@ cfr_status cfr_schedule_splits(const int32_t *seq_lens, int32_t batch, int32_t p
   if (batch <= 0 || page_tokens <= 0 || max_pages <= 0 || target_splits <= 0 || max_splits <= 0)
     return CFR_ERR_INVALID_ARG;
   if (static_cast<long long>(max_pages) * page_tokens > INT_MAX) return CFR_ERR_OVERFLOW;
-  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, 0, 0, 1, split_off,
-                  splits, max_splits, num_splits, nullptr, err_word,
+  // (in pages: the schedule unit of this entry point is the page)
+  launch_schedule(seq_lens, batch, page_tokens, max_pages, target_splits, 0, 0, 1, page_tokens,
+                  split_off, splits, max_splits, num_splits, nullptr, err_word,
                   static_cast<cudaStream_t>(stream));
   return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
 }

@@ -51,6 +51,9 @@ struct DecodeParams {
   uint32_t *err;
   int q_fmt, uniform_fmt;
   int batch, max_pages, Hq, Hkv, D, P;
+  // the split table's unit: splits are ranges [pb, pe) of split_unit tokens (P,
+  // or 128 when P is a larger multiple of 128); max_units = max_pages * P / split_unit
+  int split_unit, max_units;
   int pitch;            // shared-memory row pitch (bytes) of the CUDA-core kernel's stages
   int stages;
   float sigma_log2e;    // softmax scale times log2(e)
@@ -339,7 +342,7 @@ struct SplitRange {
 };
 __device__ __forceinline__ SplitRange split_at(const DecodeParams &p, int slot) {
   SplitRange r{p.splits[3 * slot], p.splits[3 * slot + 1], p.splits[3 * slot + 2]};
-  if (r.b < 0 || r.b >= p.batch || r.pb < 0 || r.pe < r.pb || r.pe > p.max_pages) {
+  if (r.b < 0 || r.b >= p.batch || r.pb < 0 || r.pe < r.pb || r.pe > p.max_units) {
     set_err(p.err, CFR_DEVERR_SCHEDULE);
     r.b = 0;
     r.pb = 0;

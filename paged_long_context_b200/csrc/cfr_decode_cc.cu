@@ -224,8 +224,8 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
-    const int tok_end = min(n, pe * P);
-    for (int t0 = pb * P; t0 < tok_end; t0 += CC_T) {
+    const int tok_end = min(n, pe * p.split_unit);
+    for (int t0 = pb * p.split_unit; t0 < tok_end; t0 += CC_T) {
       if (!mbar_wait(&L.empty[stage], phase ^ 1u, p.err, timed_out)) return;
       CcStageMeta &m = L.meta[stage];
       uint8_t *kst = L.ring + static_cast<size_t>(stage) * 2 * CC_T * p.pitch;
@@ -318,7 +318,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
-    const int tok_end = min(n, pe * P);
+    const int tok_end = min(n, pe * p.split_unit);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
 
     // the group's queries (fp32) and ALiBi slopes
@@ -347,7 +347,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
       for (int i = 0; i < DPL; ++i) acc[h][i] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
-    for (int t0 = pb * P; t0 < tok_end; t0 += CC_T) {
+    for (int t0 = pb * p.split_unit; t0 < tok_end; t0 += CC_T) {
       // one thread waits (bounded); the outcome is broadcast so all warps agree
       if (tid == 0) *L.flag = mbar_wait(&L.full[stage], phase, p.err, timed_out) ? 1 : 0;
       consumers_sync();

@@ -165,9 +165,11 @@ __device__ void f32_producer(const DecodeParams &p, const F32Maps &maps, uint64_
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
-    const int tok_end = min(n, pe * P);
-    for (int t0 = pb * P; t0 < tok_end; t0 += C::T) {
-      page_cache_ensure(pc, p, b, t0 / P, (min(t0 + C::T, tok_end) - 1) / P, pe, lane);
+    const int U = p.split_unit;
+    const int tok_end = min(n, pe * U);
+    const int pg_end = U == P ? pe : (pe * U + P - 1) / P;  // pages the split reaches into
+    for (int t0 = pb * U; t0 < tok_end; t0 += C::T) {
+      page_cache_ensure(pc, p, b, t0 / P, (min(t0 + C::T, tok_end) - 1) / P, pg_end, lane);
       if (!f32_produce_tile<D>(p, maps, full, empty, meta, ring, pc, g, n, t0, tok_end, box_rows,
                                stage, phase, timed_out, lane))
         return;
@@ -201,7 +203,7 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
     const SplitRange sr = split_at(p, slot);
     const int b = sr.b, pb = sr.pb, pe = sr.pe;
     const int n = p.seq_lens[b];
-    const int tok_end = min(n, pe * P);
+    const int tok_end = min(n, pe * p.split_unit);
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
 
     float q[GT][32];
@@ -249,7 +251,7 @@ __device__ void f32_consumer(const DecodeParams &p, F32Smem<D, GT> &S, uint8_t *
       for (int i = 0; i < 4; ++i) acc[h][i] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;  // of head `warp` (warps < GT)
 
-    for (int t0 = pb * P; t0 < tok_end; t0 += C::T) {
+    for (int t0 = pb * p.split_unit; t0 < tok_end; t0 += C::T) {
       if (tid == 0) S.flag = mbar_wait(&S.full[stage], phase, p.err, timed_out) ? 1 : 0;
       f_sync();
       if (S.flag == 0) {

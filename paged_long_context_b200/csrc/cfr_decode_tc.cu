@@ -126,8 +126,8 @@ __host__ __device__ constexpr int tc_feat(int feat) { return feat & 3; }
 struct TcItem {
   int item;        // -1: past the CTA's last item, or a wait gave up
   int slot, g, b;  // split slot, kv head, sequence
-  int pb, pe;      // the split's logical pages [pb, pe)
-  int n, t_end;    // sequence length; the split's tokens are [pb * P, t_end)
+  int tb, pg_end;  // the split's first token; the end of its logical pages
+  int n, t_end;    // sequence length; the split's tokens are [tb, t_end)
 };
 
 template <int NP>
@@ -490,7 +490,7 @@ __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> 
   const int s = k & (TC_ITEM_RING - 1);
   TcItem d;
   d.item = -1;
-  d.slot = d.g = d.b = d.pb = d.pe = d.n = d.t_end = 0;
+  d.slot = d.g = d.b = d.tb = d.pg_end = d.n = d.t_end = 0;
   int ok = 1;
   if (lane == 0)
     ok = mbar_wait(&c.S.item_empty[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1) ^ 1u, p.err,
@@ -508,15 +508,16 @@ __device__ __forceinline__ TcItem tc_publish_item(TcCtx<NCOL, INTP, FEAT, IMMA> 
     item_coords(it, c.nsplit, p.gsub, d.slot, d.g);
     const SplitRange sr = split_at(p, d.slot);
     d.b = sr.b;
-    d.pb = sr.pb;
-    d.pe = sr.pe;
+    // the split's range of schedule units, in tokens and in pages
+    d.tb = sr.pb * p.split_unit;
+    d.pg_end = p.split_unit == p.P ? sr.pe : (sr.pe * p.split_unit + p.P - 1) / p.P;
     d.n = p.seq_lens[d.b];
-    d.t_end = min(d.n, d.pe * p.P);
+    d.t_end = min(d.n, sr.pe * p.split_unit);
     const int h0 = p.grp_off[d.g], cnt = p.grp_off[d.g + 1] - h0;
     if (tc_qimg<NCOL>() && lane < NCOL / 2)
       c.S.ring_slope[s][lane] =
           (p.slopes && lane < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + lane])] * kLog2e : 0.f;
-    if (tc_qimg<NCOL>() && d.pb * p.P < d.t_end) {
+    if (tc_qimg<NCOL>() && d.tb < d.t_end) {
       const int buf = kq & 1;
       const long long grp = static_cast<long long>(d.b) * p.ngroups + d.g;
       constexpr uint32_t bytes = static_cast<uint32_t>(TcCfg<NCOL, INTP>::QSTRIDE);
@@ -550,7 +551,7 @@ __device__ __forceinline__ TcItem tc_read_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c,
   const int s = k & (TC_ITEM_RING - 1);
   TcItem d;
   d.item = -1;
-  d.slot = d.g = d.b = d.pb = d.pe = d.n = d.t_end = 0;
+  d.slot = d.g = d.b = d.tb = d.pg_end = d.n = d.t_end = 0;
   if (!warp_wide || (threadIdx.x & 31) == 0) {
     if (mbar_wait(&c.S.item_full[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1), c.p.err,
                   timed_out)) {
@@ -563,8 +564,8 @@ __device__ __forceinline__ TcItem tc_read_item(TcCtx<NCOL, INTP, FEAT, IMMA> &c,
     d.slot = __shfl_sync(0xffffffffu, d.slot, 0);
     d.g = __shfl_sync(0xffffffffu, d.g, 0);
     d.b = __shfl_sync(0xffffffffu, d.b, 0);
-    d.pb = __shfl_sync(0xffffffffu, d.pb, 0);
-    d.pe = __shfl_sync(0xffffffffu, d.pe, 0);
+    d.tb = __shfl_sync(0xffffffffu, d.tb, 0);
+    d.pg_end = __shfl_sync(0xffffffffu, d.pg_end, 0);
     d.n = __shfl_sync(0xffffffffu, d.n, 0);
     d.t_end = __shfl_sync(0xffffffffu, d.t_end, 0);
   }
@@ -584,7 +585,7 @@ __device__ __forceinline__ TcItem tc_read_item_wg(TcCtx<NCOL, INTP, FEAT, IMMA> 
     const int s = k & (TC_ITEM_RING - 1);
     TcItem d;
     d.item = -1;
-    d.slot = d.g = d.b = d.pb = d.pe = d.n = d.t_end = 0;
+    d.slot = d.g = d.b = d.tb = d.pg_end = d.n = d.t_end = 0;
     if (mbar_wait(&c.S.item_full[s], static_cast<uint32_t>((k / TC_ITEM_RING) & 1), c.p.err,
                   timed_out)) {
       d = c.S.ring[s];
@@ -822,9 +823,11 @@ __device__ void tc_producer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out, i
     const TcItem it = pk == 0 ? tc_publish_item(c, k, kq, timed_out, lane)
                               : tc_read_item(c, k, timed_out, true);
     if (it.item < 0) break;
-    const int b = it.b, g = it.g, pb = it.pb, pe = it.pe, n = it.n, tok_end = it.t_end;
-    int pg0 = pb, tin0 = 0;
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T, ++tile) {
+    const int b = it.b, g = it.g, pe = it.pg_end, n = it.n, tok_end = it.t_end;
+    // the first tile's page and row in it (a split starts on a page boundary, or
+    // on a 128-token boundary inside pages that are multiples of 128 tokens)
+    int pg0 = it.tb / P, tin0 = it.tb - pg0 * P;
+    for (int t0 = it.tb; t0 < tok_end; t0 += TC_T, ++tile) {
       if ((tile & (TC_PRODUCERS - 1)) == pk) {
         const int rows = min(TC_T, tok_end - t0);
         const int npiece = (rows + geo.box_rows - 1) >> geo.box_shift;  // <= 16
@@ -953,8 +956,8 @@ __device__ void tc_staging(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   for (int k = 0;; ++k) {
     const TcItem it = tc_read_item_wg(c, k, 3, r, timed_out);
     if (it.item < 0) break;
-    const int pb = it.pb, tok_end = it.t_end;
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+    const int tok_end = it.t_end;
+    for (int t0 = it.tb; t0 < tok_end; t0 += TC_T) {
       // elected bounded wait; the outcome slot is per stage, so a slow reader can
       // never see the next use of the slot (that needs every thread's barrier)
       if (r == 0) c.S.flag_st[stage] = mbar_wait(&c.S.raw_full[stage], phase, p.err, timed_out) ? 1 : 0;
@@ -1045,8 +1048,8 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
   for (int item_k = 0; !*timed_out; ++item_k) {
     const TcItem it = tc_read_item(c, item_k, timed_out, false);
     if (it.item < 0) break;
-    const int pb = it.pb, tok_end = it.t_end;
-    if (pb * P >= tok_end) continue;
+    const int tok_end = it.t_end;
+    if (it.tb >= tok_end) continue;
     // the item's query operand: buffer q_items & 1 filled by producer warp 0
     // (16 columns), or the one buffer the softmax warpgroup wrote (32 columns)
     const int qb = tc_qimg<NCOL>() ? (q_items & 1) : 0;
@@ -1058,7 +1061,7 @@ __device__ void tc_qk_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
     }
     ++q_items;
     const uint32_t qop = q0 + static_cast<uint32_t>(qb * Cfg::QSTRIDE);
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+    for (int t0 = it.tb; t0 < tok_end; t0 += TC_T) {
       if (!mbar_wait(&c.S.op_full[stage], phase, p.err, timed_out)) break;
       if (!mbar_wait(&c.S.s_empty[tc & 1], static_cast<uint32_t>((tc >> 1) & 1) ^ 1u, p.err,
                      timed_out))
@@ -1118,8 +1121,8 @@ __device__ void tc_pv_issuer(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) 
   for (int k = 0; !*timed_out; ++k) {
     const TcItem it = tc_read_item(c, k, timed_out, false);
     if (it.item < 0) break;
-    const int pb = it.pb, tok_end = it.t_end;
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+    const int tok_end = it.t_end;
+    for (int t0 = it.tb; t0 < tok_end; t0 += TC_T) {
       const int ob = static_cast<int>(tc % Cfg::O_BUFS);
       if (!mbar_wait(&c.S.p_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), p.err, timed_out))
         break;
@@ -1396,10 +1399,10 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
   bool nxt_read = false;
 
   for (TcItem it = tc_read_item_wg(c, 0, 2, tsm, timed_out); it.item >= 0; ++k) {
-    const int slot = it.slot, g = it.g, pb = it.pb, n = it.n, tok_end = it.t_end;
+    const int slot = it.slot, g = it.g, n = it.n, tok_end = it.t_end;
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
     if constexpr (!tc_qimg<NCOL>())
-      if (!q_ready && pb * P < tok_end) tc_write_q(c, it, tsm, lane);
+      if (!q_ready && it.tb < tok_end) tc_write_q(c, it, tsm, lane);
     q_ready = false;
     nxt_read = false;
     float qs[4] = {0.f, 0.f, 0.f, 0.f};  // this item's int8 digit scales (max|q_h| / 127)
@@ -1432,7 +1435,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
     bool oi1 = false, oi2 = false;  // the pending P.V products are int32 digit columns
     long long prev1 = -1, prev2 = -1;
 
-    for (int t0 = pb * P; t0 < tok_end; t0 += TC_T) {
+    for (int t0 = it.tb; t0 < tok_end; t0 += TC_T) {
       // ---- scores of tile tc ----
       (void)mbar_wait(&c.S.s_full[tc & 1], static_cast<uint32_t>((tc >> 1) & 1), p.err, timed_out);
       tc_fence_after();
@@ -1574,7 +1577,7 @@ __device__ void tc_softmax(TcCtx<NCOL, INTP, FEAT, IMMA> &c, bool *timed_out) {
         // last QK product has been read
         nxt = tc_read_item_wg(c, k + 1, 2, tsm, timed_out);
         nxt_read = true;
-        if (nxt.item >= 0 && nxt.pb * P < nxt.t_end) {
+        if (nxt.item >= 0 && nxt.tb < nxt.t_end) {
           tc_write_q(c, nxt, tsm, lane);
           q_ready = true;
         }
@@ -1775,7 +1778,7 @@ bool tc_supported(const DecodeParams &p, bool page_fmt_given) {
 }
 
 void launch_schedule(const int32_t *seq_lens, int batch, int P, int max_pages, int target,
-                     int sink, int window, int nq, int32_t *split_off, int32_t *splits,
+                     int sink, int window, int nq, int unit, int32_t *split_off, int32_t *splits,
                      int max_splits, int32_t *num_splits, uint32_t *item_ctr, uint32_t *err,
                      cudaStream_t stream);
 
@@ -1830,7 +1833,7 @@ static cudaError_t tc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
         <<<dim3(static_cast<unsigned>(groups + extra)), dim3(128), 0, stream>>>(p, sa, extra);
   } else if (sched) {
     launch_schedule(sched->seq_lens, sched->batch, sched->P, sched->max_pages, sched->target,
-                    sched->sink, sched->window, sched->nq, sched->split_off, sched->splits,
+                    sched->sink, sched->window, sched->nq, sched->unit, sched->split_off, sched->splits,
                     sched->max_splits, sched->num_splits, sched->item_ctr, sched->err, stream);
   }
   // a plain launch: overlapping this kernel's start with the previous kernel

@@ -23,6 +23,10 @@ namespace cfr {
 struct SchedArgs {
   const int32_t *seq_lens;
   int batch, P, max_pages, target, sink, window, nq;
+  // tokens per schedule unit: splits are ranges of whole units (P, i.e. pages,
+  // or a divisor of P that is a multiple of every kernel's tile, so that a
+  // short sequence of long pages still spreads over many splits)
+  int unit;
   int32_t *split_off;   // [batch + 1]
   int32_t *splits;      // [max_splits][3]
   int max_splits;
@@ -79,7 +83,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *red, int *total)
   return r;
 }
 
-// pages of a sequence of n tokens; -1 when n is outside [min_len, max_pages * P]
+// units of P tokens (pages, or the schedule's smaller unit) of a sequence of n
+// tokens; -1 when n is outside [min_len, max_pages * P]
 __device__ __forceinline__ int valid_pages(int n, int P, int max_pages, int min_len) {
   if (n <= 0 || n < min_len || n > max_pages * P) return -1;
   return (n + P - 1) / P;
@@ -104,7 +109,10 @@ __device__ __forceinline__ void page_ranges(int n, int np, int P, int sink, int 
 // multiple of 32, up to 1024 threads).
 __device__ __forceinline__ void schedule_block(const SchedArgs &a) {
   const int32_t *__restrict__ seq_lens = a.seq_lens;
-  const int batch = a.batch, P = a.P, max_pages = a.max_pages, target = a.target;
+  const int batch = a.batch, max_pages = a.max_pages, target = a.target;
+  // units of U tokens: a sequence of n tokens is valid when 1 <= n <= max_pages * P
+  // (and n >= nq), and spans ceil(n / U) units
+  const int U = a.unit, max_units = static_cast<int>(static_cast<long long>(max_pages) * a.P / U);
   const int sink = a.sink, window = a.window, nq = a.nq, max_splits = a.max_splits;
   int32_t *__restrict__ split_off = a.split_off;
   int32_t *__restrict__ splits = a.splits;
@@ -121,12 +129,12 @@ __device__ __forceinline__ void schedule_block(const SchedArgs &a) {
   long long local = 0;
   for (int b = threadIdx.x; b < batch; b += blockDim.x) {
     const int n = seq_lens[b];
-    const int np = valid_pages(n, P, max_pages, nq);
+    const int np = valid_pages(n, U, max_units, nq);
     if (np < 0) {
       set_err(err, CFR_DEVERR_SEQ_LEN);
     } else {
       int a_end, b_begin;
-      page_ranges(n, np, P, sink, window, &a_end, &b_begin);
+      page_ranges(n, np, U, sink, window, &a_end, &b_begin);
       local += a_end + (np - b_begin);
     }
   }
@@ -140,10 +148,10 @@ __device__ __forceinline__ void schedule_block(const SchedArgs &a) {
   for (int base = 0; base < batch; base += blockDim.x) {
     const int b = base + threadIdx.x;
     const int n = b < batch ? seq_lens[b] : 0;
-    int np = b < batch ? valid_pages(n, P, max_pages, nq) : -1;
+    int np = b < batch ? valid_pages(n, U, max_units, nq) : -1;
     if (np < 0) np = 0;
     int a_end, b_begin;
-    page_ranges(n, np, P, sink, window, &a_end, &b_begin);
+    page_ranges(n, np, U, sink, window, &a_end, &b_begin);
     const int cnt_a = (a_end + chunk - 1) / chunk;
     const int cnt = cnt_a + (np - b_begin + chunk - 1) / chunk;
     int tot = 0;
