@@ -132,7 +132,8 @@ size_t cfr_paged_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32
  *              page, "MHA/MQA/GQA head mapping").  The query heads of a kv head
  *              are decoded together, reading its pages once, in groups of at
  *              most 16: a kv head serving more (MQA, wide GQA) has its pages
- *              read once per group of 16.
+ *              read once per group of 16 (the groups of one split are taken
+ *              side by side, so the later reads usually come from L2).
  *  alibi_slopes device, float [num_q_heads] or NULL: bias -slope_h * (n_b - 1 - j) is
  *              added to the score of token j (CFR-Atlas page, "RoPE/ALiBi
  *              positional policy").
@@ -163,9 +164,12 @@ cfr_status cfr_paged_decode(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
 #define CFR_PHASE_ALL 0x7u
 
 /*
- * cfr_paged_decode split into its three stream-ordered launches, for timing
- * one launch at a time (CUDA events between calls).  Same arguments and checks
- * as cfr_paged_decode; `phases` selects which launches are enqueued.  A call
+ * cfr_paged_decode split into its phases, for timing one at a time (CUDA
+ * events between calls): the split schedule, the decode (on the tensor-core
+ * path with a small launch before it that builds the query operands; a call
+ * with both the schedule and the decode phase runs the schedule inside that
+ * launch) and the merge.  Same arguments and checks as cfr_paged_decode;
+ * `phases` selects which phases are enqueued.  A call
  * without CFR_PHASE_SCHEDULE relies on the workspace still holding what an
  * earlier call with the same arguments (all but q, out and lse) left there: the
  * split schedule, and the work-item counter that the schedule launch zeroes and
