@@ -181,12 +181,19 @@ __device__ __forceinline__ float qmax_of(int fmt) {
   return fmt == CFR_FMT_I8 ? 127.f : fmt == CFR_FMT_I4 ? 7.f : 448.f;
 }
 
-// block (page k, kv head g, K or V) = blockIdx.x
-template <int SRC>
-__global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) {
-  constexpr int R = resident_vectors<SRC>();
-  constexpr int T = kDemoteThreads;
-  __shared__ float red[T / 32];
+// One (page k, kv head g, K or V) block, resolved from blockIdx.x.
+struct DemoteBlock {
+  const uint8_t *src;
+  uint8_t *dst;
+  float *dst_scale;      // null for unquantised destinations
+  float src_scale;       // 1 for unquantised sources
+  long long nvec_valid;  // vectors of kVec elements in the valid rows
+  long long nvec;        // vectors in the whole block
+};
+
+// resolves the CTA's block; false (after reporting) when its slots or valid
+// count are out of range, in which case nothing is written
+__device__ __forceinline__ bool resolve_block(const DemoteParams &p, int src_fmt, DemoteBlock &b) {
   const long long blk_id = blockIdx.x;
   const int kv = static_cast<int>(blk_id & 1);
   const int g = static_cast<int>((blk_id >> 1) % p.Hkv);
@@ -195,17 +202,32 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
   const int valid = p.valid_tokens ? p.valid_tokens[k] : p.P;
   if (s < 0 || s >= p.src_pages || t < 0 || t >= p.dst_pages) {
     if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_PAGE_ID);
-    return;
+    return false;
   }
   if (valid < 1 || valid > p.P) {
     if (threadIdx.x == 0) set_err(p.err, CFR_DEVERR_SEQ_LEN);
-    return;
+    return false;
   }
-  const uint8_t *src = (kv ? p.src_v : p.src_k) + (s * p.Hkv + g) * p.P * row_bytes(SRC, p.D);
-  uint8_t *dst = (kv ? p.dst_v : p.dst_k) + (t * p.Hkv + g) * p.P * row_bytes(p.dst_fmt, p.D);
-  const float src_scale = is_quantised(SRC) ? p.src_scales[(s * p.Hkv + g) * 2 + kv] : 1.f;
-  const long long nvec_valid = static_cast<long long>(valid) * p.D / kVec;
-  const long long nvec = static_cast<long long>(p.P) * p.D / kVec;
+  b.src = (kv ? p.src_v : p.src_k) + (s * p.Hkv + g) * p.P * row_bytes(src_fmt, p.D);
+  b.dst = (kv ? p.dst_v : p.dst_k) + (t * p.Hkv + g) * p.P * row_bytes(p.dst_fmt, p.D);
+  b.dst_scale = is_quantised(p.dst_fmt) ? p.dst_scales + (t * p.Hkv + g) * 2 + kv : nullptr;
+  b.src_scale = is_quantised(src_fmt) ? p.src_scales[(s * p.Hkv + g) * 2 + kv] : 1.f;
+  b.nvec_valid = static_cast<long long>(valid) * p.D / kVec;
+  b.nvec = static_cast<long long>(p.P) * p.D / kVec;
+  return true;
+}
+
+// The block with every decision taken as written above (IEEE division per
+// element).  Called by all CTAs of the block together (it holds __syncthreads).
+template <int SRC>
+__device__ __forceinline__ void demote_block_exact(const DemoteParams &p, const DemoteBlock &b,
+                                                   float *red) {
+  constexpr int R = resident_vectors<SRC>();
+  constexpr int T = kDemoteThreads;
+  const uint8_t *src = b.src;
+  uint8_t *dst = b.dst;
+  const float src_scale = b.src_scale;
+  const long long nvec_valid = b.nvec_valid;
   const int tid = threadIdx.x;
   // the whole valid part of the block fits the registers of the CTA
   const bool resident = nvec_valid <= static_cast<long long>(R) * T;
@@ -240,7 +262,7 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
 #pragma unroll
     for (int w = 1; w < T / 32; ++w) amax = fmaxf(amax, red[w]);
     scale = __fdiv_rn(amax, qmax_of(p.dst_fmt));
-    if (tid == 0) p.dst_scales[(t * p.Hkv + g) * 2 + kv] = scale;
+    if (tid == 0) *b.dst_scale = scale;
   } else if (resident) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -278,7 +300,181 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
       }
     }
   }
-  for (long long v = nvec_valid + tid; v < nvec; v += T) store_zero8(p.dst_fmt, dst, v * kVec);
+  for (long long v = nvec_valid + tid; v < b.nvec; v += T) store_zero8(p.dst_fmt, dst, v * kVec);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) {
+  __shared__ float red[kDemoteThreads / 32];
+  DemoteBlock b;
+  if (!resolve_block(p, SRC, b)) return;
+  demote_block_exact<SRC>(p, b, red);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 -> int8 / int4, the hot-to-cold step of the cascade.
+//
+// The codes are the ones defined above, code = rint(fl(x / scale)), reached
+// without a division per element.  Let q = x / scale (exact) and f = fl(q).
+// With a normal, finite scale and r = fl(1 / scale) (one correctly rounded
+// reciprocal per block), take r- = fl(r * (1 - 2^-20)) and r+ = fl(r * (1 + 2^-20)).
+// Each of r, r-, r+ and f carries a relative rounding error of at most 2^-24,
+// so x*r- and x*r+ (exact products) lie on either side of f:
+//   |x*r-| <= |q| (1 - 2^-20 + 2^-23) < |f|,   |x*r+| >= |q| (1 + 2^-20 - 2^-23) > |f|
+// (for tiny |q| all three round to 0).  One fused multiply-add of each into
+// the magic constant 1.5 * 2^23, whose unit in the last place is 1, rounds
+// the exact product to the nearest integer (ties to even) and leaves it in
+// the low bits of the sum.  Rounding to nearest is monotone, so when both
+// sums agree they equal rint(f): that is the code, and |code| <= Q (the clamp
+// cannot bind: |x| <= max|x| and scale >= max|x| / Q to within 2^-24).  When
+// they differ (a half-integer within about |q| * 2^-20 of the product: about
+// one element in 15,000 for random data, and every NaN), the eight elements
+// of the vector are encoded again with the IEEE division.  A block whose
+// maximum is infinite or whose scale is zero or subnormal (where the bounds
+// above fail) is encoded with the division throughout.
+// max|x| is taken on the bf16 pairs (|a| vs |b| maxima, which ignore NaN as
+// fmaxf does), equal to the fp32 maximum of the decoded values.
+// ---------------------------------------------------------------------------
+
+constexpr float kRintMagic = 12582912.0f;         // 1.5 * 2^23
+constexpr uint32_t kRintMagicBits = 0x4B400000u;  // its bit pattern
+
+// Running max|x| of bf16 pairs: per half, max(|m|, |w|) (its sign bit left
+// arbitrary).  The bf16 max returns the other operand when one is NaN, as
+// fmaxf does.
+__device__ __forceinline__ uint32_t absmax_acc(uint32_t m, uint32_t w) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(w));
+  return d;
+}
+
+__device__ __forceinline__ float absmax_value(uint32_t m) {
+  return fmaxf(bf16_lo(m & 0x7FFF7FFFu), bf16_hi(m & 0x7FFF7FFFu));
+}
+
+__device__ __forceinline__ void bf16_decode8(const uint4 &w, float (&x)[kVec]) {
+  const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    x[2 * k] = bf16_lo(a[k]);
+    x[2 * k + 1] = bf16_hi(a[k]);
+  }
+}
+
+// the eight codes of one vector (8 bf16 in w), each as 0x4B400000 + code, from
+// the two bracketing products; true when they disagree somewhere (the vector
+// is then encoded again by bf16_codes8_exact)
+__device__ __forceinline__ bool bf16_codes8_fast(const uint4 &w, float r_lo, float r_hi,
+                                                 uint32_t (&tb)[kVec]) {
+  float x[kVec];
+  bf16_decode8(w, x);
+  bool near = false;
+#pragma unroll
+  for (int k = 0; k < kVec; ++k) {
+    const float lo = __fmaf_rn(x[k], r_lo, kRintMagic);
+    const float hi = __fmaf_rn(x[k], r_hi, kRintMagic);
+    near |= lo != hi;
+    tb[k] = __float_as_uint(lo);
+  }
+  return near;
+}
+
+// the same codes with the IEEE division
+template <int Q>
+__device__ __forceinline__ void bf16_codes8_exact(const uint4 &w, float scale, uint32_t (&tb)[kVec]) {
+  float x[kVec];
+  bf16_decode8(w, x);
+#pragma unroll
+  for (int k = 0; k < kVec; ++k) tb[k] = kRintMagicBits + static_cast<uint32_t>(int_code(x[k], scale, Q));
+}
+
+// stores eight codes (low byte / nibble of each tb) as vector v of the block
+template <int DST>
+__device__ __forceinline__ void store_codes8(uint8_t *dst, int v, const uint32_t (&tb)[kVec]) {
+  if constexpr (DST == CFR_FMT_I8) {
+    const uint32_t lo = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040), 0x5410);
+    reinterpret_cast<uint2 *>(dst)[v] = make_uint2(lo, hi);
+  } else {  // element 2i in the low nibble of byte i
+    uint32_t n[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) n[k] = (tb[2 * k] & 0x0Fu) | (tb[2 * k + 1] << 4);
+    reinterpret_cast<uint32_t *>(dst)[v] =
+        __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
+  }
+}
+
+// The block is staged in shared memory by one bulk copy (all of it in flight
+// at once), with three 256-thread CTAs per SM; the max pass and the encode
+// pass read it there.  Blocks of up to 64 KiB (page_tokens x head_dim <= 32768).
+constexpr int kSmemThreads = 256;
+constexpr int kSmemBlockBytes = 65536;
+
+template <int DST>
+__global__ void __launch_bounds__(kSmemThreads, 3) demote_bf16_int_kernel(DemoteParams p) {
+  constexpr int T = kSmemThreads;
+  constexpr int Q = DST == CFR_FMT_I8 ? 127 : 7;
+  extern __shared__ __align__(128) uint4 stage[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t redw[T / 32];
+  DemoteBlock b;
+  if (!resolve_block(p, CFR_FMT_BF16, b)) return;
+  const int tid = threadIdx.x;
+  const int nv = static_cast<int>(b.nvec_valid);
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nv) * 16u);
+    bulk_g2s(stage, b.src, static_cast<uint32_t>(nv) * 16u, &bar);
+  }
+  __syncthreads();
+  bool timed_out = false;
+  if (!mbar_wait(&bar, 0, p.err, &timed_out)) return;
+  uint32_t m = 0u;
+#pragma unroll 4
+  for (int v = tid; v < nv; v += T) {
+    const uint4 w = stage[v];
+    m = absmax_acc(absmax_acc(absmax_acc(absmax_acc(m, w.x), w.y), w.z), w.w);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = absmax_acc(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((tid & 31) == 0) redw[tid >> 5] = m;
+  __syncthreads();
+  m = redw[0];
+#pragma unroll
+  for (int w = 1; w < T / 32; ++w) m = absmax_acc(m, redw[w]);
+  const float amax = absmax_value(m);
+  const float scale = __fdiv_rn(amax, static_cast<float>(Q));
+  const bool fast = scale >= 1.17549435e-38f && scale <= 3.40282347e+38f;  // normal and finite
+  if (tid == 0) *b.dst_scale = scale;
+  // encode: vectors near a tie are marked in `redo` and encoded again after
+  // the loop, which keeps the division out of the loop body
+  static_assert(kSmemBlockBytes / 16 / T <= 32, "one bit per vector of a thread");
+  uint32_t redo = 0u;
+  if (fast) {
+    const float r = __frcp_rn(scale);
+    const float r_lo = __fmul_rn(r, 1.f - 0x1p-20f), r_hi = __fmul_rn(r, 1.f + 0x1p-20f);
+#pragma unroll 4
+    for (int i = 0; i < kSmemBlockBytes / 16 / T; ++i) {
+      const int v = i * T + tid;
+      if (v < nv) {
+        uint32_t tb[kVec];
+        redo |= static_cast<uint32_t>(bf16_codes8_fast(stage[v], r_lo, r_hi, tb)) << i;
+        store_codes8<DST>(b.dst, v, tb);
+      }
+    }
+  } else {
+    for (int i = 0; i * T + tid < nv; ++i) redo |= 1u << i;
+  }
+  while (redo) {
+    const int i = __ffs(redo) - 1;
+    redo &= redo - 1;
+    const int v = i * T + tid;
+    uint32_t tb[kVec];
+    bf16_codes8_exact<Q>(stage[v], scale, tb);
+    store_codes8<DST>(b.dst, v, tb);
+  }
+  for (long long v = b.nvec_valid + tid; v < b.nvec; v += T) store_zero8(DST, b.dst, v * kVec);
 }
 
 struct AppendParams {
@@ -402,6 +598,18 @@ cfr_status cfr_demote_pages(const cfr_kv_pool *kv, int32_t src_fmt, int32_t dst_
   p.P = kv->page_tokens;
   const unsigned blocks = static_cast<unsigned>(num_pages) * kv->num_kv_heads * 2u;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the bf16 -> int kernel stages a whole block in shared memory
+  const bool fits = static_cast<long long>(kv->page_tokens) * row_bytes(CFR_FMT_BF16, kv->head_dim) <=
+                    kSmemBlockBytes;
+  if (fits && src_fmt == CFR_FMT_BF16 && (dst_fmt == CFR_FMT_I8 || dst_fmt == CFR_FMT_I4)) {
+    auto kern = dst_fmt == CFR_FMT_I8 ? demote_bf16_int_kernel<CFR_FMT_I8>
+                                      : demote_bf16_int_kernel<CFR_FMT_I4>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBlockBytes) !=
+        cudaSuccess)
+      return CFR_ERR_CUDA;
+    kern<<<blocks, kSmemThreads, kSmemBlockBytes, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
+  }
   switch (src_fmt) {
     case CFR_FMT_F32: demote_kernel<CFR_FMT_F32><<<blocks, kDemoteThreads, 0, s>>>(p); break;
     case CFR_FMT_BF16: demote_kernel<CFR_FMT_BF16><<<blocks, kDemoteThreads, 0, s>>>(p); break;

@@ -105,6 +105,114 @@ def test_demote_reports_and_skips_bad_pages():
     assert int((hk[len(pages):] != 0xAB).sum()) == 0            # skipped pages untouched
 
 
+# ---------------------------------------------------------------------------
+# bf16 -> int8 / int4 over every bf16 input, and the blocks at the edges of the
+# encoder (ties, NaN, infinities, zero and subnormal scales)
+# ---------------------------------------------------------------------------
+
+def _bf16_blocks_case(blocks, seed=11):
+    """A bf16 cache (head_dim 128, 16-token pages, 2 kv heads) whose first
+    len(blocks) (page, kv head, K-or-V) blocks hold the given bf16 bit patterns
+    (2048 each, in the order the demotion numbers its blocks); the rest keep the
+    generator's values."""
+    Hkv, P, d = 2, 16, 128
+    per_page = 2 * Hkv
+    npages = -(-len(blocks) // per_page)
+    case = _src_case(BF16, d, P, lens=(P * npages,), seed=seed)
+    pages = _pages_of(case)
+    k = case.k_pool[BF16].view(torch.int16)
+    v = case.v_pool[BF16].view(torch.int16)
+    for i, bits in enumerate(blocks):
+        j, rest = divmod(i, per_page)
+        g, kv = divmod(rest, 2)
+        t = torch.from_numpy(np.asarray(bits, dtype=np.uint16).view(np.int16).reshape(P, d))
+        (v if kv else k)[pages[j][0], g] = t.to(k.device)
+    return case, pages
+
+
+def _demote_blocks_exact(blocks, dst):
+    case, pages = _bf16_blocks_case(blocks)
+    n = len(pages)
+    (hk, hv, hsc, err), (ok, ov, osc, oerr) = _demote_both(
+        case, BF16, dst, [s for s, _ in pages], list(range(n)), [v for _, v in pages], n)
+    assert err == 0 and oerr == 0
+    assert torch.equal(hsc, osc)
+    assert torch.equal(hk, ok) and torch.equal(hv, ov)
+    return hsc
+
+
+@pytest.mark.parametrize("dst", [I8, I4], ids=["int8", "int4"])
+@pytest.mark.parametrize("amax_bits", [0x3F80, 0x3F4A, 0x4040, 0x3FFE, 0x7F00, 0x0D80, 0x0400, 0x0300],
+                         ids=lambda b: f"amax{b:04x}")
+def test_demote_bf16_to_int_every_input(dst, amax_bits):
+    # every bf16 value of magnitude up to max|x| (both signs, zeros and
+    # subnormals included), shuffled over blocks that each also hold max|x|,
+    # so every block has the same scale: each possible input of that scale is
+    # encoded once and compared byte for byte with the oracle.  0x0400 gives
+    # the smallest normal scales (2^-119 / Q); 0x0300 a subnormal scale.
+    rng = np.random.default_rng(amax_bits)
+    mags = np.arange(0, amax_bits + 1, dtype=np.uint32)
+    vals = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)
+    rng.shuffle(vals)
+    chunk = 2047
+    blocks = []
+    for c0 in range(0, len(vals), chunk):
+        part = vals[c0:c0 + chunk]
+        part = np.concatenate([part, np.full(chunk - len(part), amax_bits, np.uint16)])
+        blk = np.concatenate([[amax_bits], part]).astype(np.uint16)
+        rng.shuffle(blk)
+        blocks.append(blk)
+    sc = _demote_blocks_exact(blocks, dst)
+    assert bool((sc.view(-1)[: len(blocks)] > 0).all())
+
+
+@pytest.mark.parametrize("dst", [I8, I4], ids=["int8", "int4"])
+def test_demote_bf16_to_int_edge_blocks(dst):
+    rng = np.random.default_rng(3)
+    n = 2048
+
+    def finite(lo_bits=0x3000, hi_bits=0x3F80):
+        m = rng.integers(lo_bits, hi_bits, size=n, dtype=np.uint32)
+        return (m | (rng.integers(0, 2, size=n, dtype=np.uint32) << 15)).astype(np.uint16)
+
+    q = 127 if dst == I8 else 7
+    blocks = []
+    # exact ties: scale = 2^-6 (int8) or 2^-2 (int4), values (k + 1/2) * scale
+    unit = 64 if dst == I8 else 4
+    amax = torch.tensor([q / unit], dtype=torch.bfloat16).view(torch.int16).item() & 0xFFFF
+    ks = rng.integers(-q, q, size=n)
+    ties = torch.tensor((ks + 0.5) / unit, dtype=torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ties[0] = amax
+    blocks.append(ties)
+    # NaNs (with payloads and signs) among finite values: max|x| ignores them, their codes are 0
+    b = finite()
+    b[rng.choice(n, 40, replace=False)] = np.array([0x7FC0, 0x7FC1, 0xFFC0, 0x7F81] * 10, np.uint16)
+    blocks.append(b)
+    # an infinity: scale is infinite and every code 0
+    b = finite()
+    b[5] = 0x7F80
+    blocks.append(b)
+    b = np.zeros(n, np.uint16)
+    b[100] = 0xFF80
+    blocks.append(b)
+    # all zeros of both signs: scale 0
+    blocks.append((rng.integers(0, 2, size=n, dtype=np.uint32) << 15).astype(np.uint16))
+    # subnormals only (scale subnormal)
+    blocks.append(finite(0x0001, 0x0080))
+    # a subnormal maximum among zeros
+    b = np.zeros(n, np.uint16)
+    b[7] = 0x0001
+    blocks.append(b)
+    # large magnitudes next to the largest finite bf16
+    blocks.append(finite(0x7E00, 0x7F80))
+    # tiny values under a normal maximum (codes 0 and +-1)
+    b = finite(0x0001, 0x0400)
+    b[9] = 0x0C00
+    blocks.append(b)
+    sc = _demote_blocks_exact(blocks, dst)
+    assert float(sc.view(-1)[0]) == 1.0 / unit
+
+
 @pytest.mark.parametrize("P", [16, 256])
 def test_demoted_cache_decodes(P):
     # a bf16 cache whose oldest pages are demoted on the GPU to int4 / int8 / FP8
