@@ -453,8 +453,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 // builds query operands inside the pipeline.  Two ways of choosing the items,
 // by measurement:
 //  - fixed: CTA x takes items x, x + grid, x + 2 grid, ...
-//  - claimed (plain and multi-query decode over bf16 pools, or over int8 / int4
-//    pools of one format in the IMMA variants): CTA x starts with item x and
+//  - claimed (plain, multi-query and sink + window decode over bf16 pools, or
+//    over int8 / int4 pools of one format in the IMMA variants): CTA x starts with item x and
 //    claims every further item from a global counter when producer warp 0
 //    reaches it, so SMs that the memory system serves faster take more items and
 //    all CTAs finish together.  Over pools of mixed formats the items differ in
@@ -462,7 +462,7 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 //    no counter (item_ctr = null), which selects the fixed share.
 template <bool INTP, int FEAT, bool IMMA>
 __host__ __device__ constexpr bool tc_claimed_items() {
-  return (!INTP || IMMA) && tc_feat(FEAT) != TC_FEAT_SUBSET;
+  return !INTP || IMMA;
 }
 
 // quantised pages shorter than a tile (several pages, each with its scales, in
