@@ -6,11 +6,12 @@
 // "MHA/MQA/GQA head mapping").
 //
 // Warp roles:
-//  - warp 8 (one elected lane) is the producer: it resolves every page of the
-//    item through the page table, checks slot, format and pool, and streams
-//    each 64-token tile of K and V into a shared-memory ring with 1-D bulk
-//    copies (TMA engine, completion on an mbarrier).  Pages that do not
-//    resolve are skipped and reported in the error word, never dereferenced.
+//  - warp 8 is the producer: lane i resolves page piece i of a tile (the
+//    tile's rows of one page) through the page table, checks slot, format and
+//    pool, and copies its K and V rows into a shared-memory ring with one 1-D
+//    bulk copy each (TMA engine, completion on an mbarrier), packed at the
+//    piece's own row size.  Pages that do not resolve are skipped and reported
+//    in the error word, never dereferenced.
 //  - warps 0-7 consume tiles.  Per tile: (1) scores s = sigma*(q.k)*scale_k +
 //    ALiBi, in base 2, eight lanes per token row; (2) per head, the tile max,
 //    the rescale factor 2^(m_old - m_new), p = 2^(s - m_new) and the running
@@ -35,10 +36,14 @@ constexpr int CC_WARPS = 8;    // consumer warps
 constexpr int CC_THREADS = (CC_WARPS + 1) * 32;
 constexpr int CC_MAXF = 16;    // fragments (page pieces) per tile; page_tokens >= 8 gives <= 9
 
+// A page piece of a tile: tile rows [r0, r0 + rows of the piece) of one page.
+// Its K rows sit packed at their own row size rb from byte `off` of the
+// stage's K region (V rows likewise in the V region).
 struct CcFrag {
   int fmt;
   int ok;
   float ks, vs;
+  int off, rb, r0;
 };
 
 struct CcStageMeta {
@@ -211,10 +216,12 @@ __device__ inline CcLayout cc_layout(uint8_t *smem, int stages, int pitch) {
   return L;
 }
 
-// Producer: one lane streams every tile of every item of this CTA.
+// Producer (warp 8): every tile of every item of this CTA.  Lane i resolves
+// piece i of the tile, so a tile's page-table reads are one round trip.
 template <int D>
 __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long nitems,
                             bool *timed_out) {
+  const int lane = threadIdx.x & 31;
   int stage = 0;
   uint32_t phase = 0;
   const int P = p.P;
@@ -226,71 +233,71 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
     const int n = p.seq_lens[b];
     const int tok_end = min(n, pe * p.split_unit);
     for (int t0 = pb * p.split_unit; t0 < tok_end; t0 += CC_T) {
-      if (!mbar_wait(&L.empty[stage], phase ^ 1u, p.err, timed_out)) return;
-      CcStageMeta &m = L.meta[stage];
-      uint8_t *kst = L.ring + static_cast<size_t>(stage) * 2 * CC_T * p.pitch;
-      uint8_t *vst = kst + CC_T * p.pitch;
       const int rows = min(CC_T, tok_end - t0);
-      m.rows = rows;
-      m.t0 = t0;
-      // resolve the page pieces of this tile
-      int nf = 0;
-      uint32_t bytes = 0;
-      for (int r = 0; r < rows;) {
-        const int j = t0 + r, pg = j / P, tin = j - pg * P;
-        const int fr = min(rows - r, P - tin);
+      // piece `lane`: tile rows [r0, r1) of page pg
+      const int pg = t0 / P + lane;
+      const int r0 = max(t0, pg * P) - t0;
+      const int r1 = min(t0 + rows, (pg + 1) * P) - t0;
+      const bool have = lane < CC_MAXF && r0 < r1;
+      CcFrag f;
+      f.fmt = -1;
+      f.ok = 0;
+      f.ks = f.vs = 1.f;
+      f.rb = 0;
+      f.r0 = r0;
+      long long id = -1;
+      if (have) {
         const long long cell = static_cast<long long>(b) * p.max_pages + pg;
-        const int fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
-        const long long id = p.page_table[cell];
-        CcFrag f;
-        f.fmt = fmt;
-        f.ok = 0;
-        f.ks = f.vs = 1.f;
-        if (fmt < 0 || fmt >= kFmtCount) {
+        f.fmt = p.page_fmt ? static_cast<int>(p.page_fmt[cell]) : p.uniform_fmt;
+        id = p.page_table[cell];
+        if (f.fmt < 0 || f.fmt >= kFmtCount) {
           set_err(p.err, CFR_DEVERR_PAGE_FMT);
-        } else if (!p.k_pool[fmt] || !p.v_pool[fmt] || (is_quantised(fmt) && !p.scales[fmt])) {
+        } else if (!p.k_pool[f.fmt] || !p.v_pool[f.fmt] || (is_quantised(f.fmt) && !p.scales[f.fmt])) {
           set_err(p.err, CFR_DEVERR_POOL);
-        } else if (id < 0 || id >= p.pool_pages[fmt]) {
+        } else if (id < 0 || id >= p.pool_pages[f.fmt]) {
           set_err(p.err, CFR_DEVERR_PAGE_ID);
         } else {
           f.ok = 1;
-          if (is_quantised(fmt)) {
-            const float2 s = *reinterpret_cast<const float2 *>(p.scales[fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
+          f.rb = row_bytes(f.fmt, D);
+          if (is_quantised(f.fmt)) {
+            const float2 s = *reinterpret_cast<const float2 *>(p.scales[f.fmt] + (id * p.Hkv + p.grp_kv[g]) * 2);
             f.ks = s.x;
             f.vs = s.y;
           }
-          bytes += 2u * fr * row_bytes(fmt, D);
         }
-        m.frag[nf] = f;
-        for (int rr = r; rr < r + fr; ++rr) m.row_frag[rr] = static_cast<int8_t>(nf);
-        ++nf;
-        r += fr;
       }
-      mbar_arrive_expect_tx(&L.full[stage], bytes);
-      // issue the copies
-      int fi = 0;
-      for (int r = 0; r < rows; ++fi) {
-        const int j = t0 + r, pg = j / P, tin = j - pg * P;
-        const int fr = min(rows - r, P - tin);
-        const CcFrag &f = m.frag[fi];
-        if (f.ok) {
-          const long long cell = static_cast<long long>(b) * p.max_pages + pg;
-          const long long id = p.page_table[cell];
-          const int rb = row_bytes(f.fmt, D);
-          const long long off = ((id * p.Hkv + p.grp_kv[g]) * P + tin) * rb;
-          const uint8_t *ks = p.k_pool[f.fmt] + off;
-          const uint8_t *vs = p.v_pool[f.fmt] + off;
-          if (rb == p.pitch) {
-            bulk_g2s(kst + r * p.pitch, ks, fr * rb, &L.full[stage]);
-            bulk_g2s(vst + r * p.pitch, vs, fr * rb, &L.full[stage]);
-          } else {
-            for (int rr = 0; rr < fr; ++rr) {
-              bulk_g2s(kst + (r + rr) * p.pitch, ks + rr * rb, rb, &L.full[stage]);
-              bulk_g2s(vst + (r + rr) * p.pitch, vs + rr * rb, rb, &L.full[stage]);
-            }
-          }
-        }
-        r += fr;
+      // packed byte offsets of the pieces in the K (and V) region: an
+      // exclusive prefix sum over the lanes (every row size is a multiple of 16)
+      const uint32_t pbytes = f.ok ? static_cast<uint32_t>((r1 - r0) * f.rb) : 0u;
+      uint32_t incl = pbytes;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      f.off = static_cast<int>(incl - pbytes);
+      const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+      // the stage must be free before its description and bytes are replaced
+      const bool waited = mbar_wait(&L.empty[stage], phase ^ 1u, p.err, timed_out);
+      if (!__all_sync(0xffffffffu, waited)) return;
+      CcStageMeta &m = L.meta[stage];
+      uint8_t *kst = L.ring + static_cast<size_t>(stage) * 2 * CC_T * p.pitch;
+      uint8_t *vst = kst + CC_T * p.pitch;
+      if (have) {
+        m.frag[lane] = f;
+        for (int r = r0; r < r1; ++r) m.row_frag[r] = static_cast<int8_t>(lane);
+      }
+      if (lane == 0) {
+        m.rows = rows;
+        m.t0 = t0;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&L.full[stage], 2u * total);
+      __syncwarp();
+      if (f.ok) {
+        const long long off = ((id * p.Hkv + p.grp_kv[g]) * P + (t0 + r0 - pg * P)) * f.rb;
+        bulk_g2s(kst + f.off, p.k_pool[f.fmt] + off, pbytes, &L.full[stage]);
+        bulk_g2s(vst + f.off, p.v_pool[f.fmt] + off, pbytes, &L.full[stage]);
       }
       if (++stage == p.stages) {
         stage = 0;
@@ -307,7 +314,6 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
   constexpr int DPL = D / 32;   // dims per lane in the P.V step
   constexpr int HC = GT < 4 ? GT : 4;  // heads per reduction round
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int P = p.P;
   int stage = 0;
   uint32_t phase = 0;
   int tile_ctr = 0;
@@ -378,7 +384,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
             valid = true;
             ks = f.ks;
             float x[EPT];
-            load_elems<EPT>(f.fmt, kst + r * p.pitch, j8 * EPT, x);
+            load_elems<EPT>(f.fmt, kst + f.off + (r - f.r0) * f.rb, j8 * EPT, x);
 #pragma unroll
             for (int h = 0; h < GT; ++h) {
               const float4 *qq = reinterpret_cast<const float4 *>(L.q_s + h * D + j8 * EPT);
@@ -457,7 +463,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
         const CcFrag f = m.frag[m.row_frag[r]];
         if (!f.ok || !in_token_set(p, n, m.t0 + r)) continue;
         float v[DPL];
-        load_elems<DPL>(f.fmt, vst + r * p.pitch, lane * DPL, v);
+        load_elems<DPL>(f.fmt, vst + f.off + (r - f.r0) * f.rb, lane * DPL, v);
 #pragma unroll
         for (int h = 0; h < GT; ++h) {
           const float pw = sc[h * CC_T + r] * f.vs;
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_c
       static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.ngroups;
   bool timed_out = false;
   if (threadIdx.x >= CC_WARPS * 32) {
-    if (threadIdx.x == CC_WARPS * 32) cc_producer<D>(p, L, nitems, &timed_out);
+    cc_producer<D>(p, L, nitems, &timed_out);
   } else {
     cc_consumer<D, GT>(p, L, nitems, &timed_out);
   }
