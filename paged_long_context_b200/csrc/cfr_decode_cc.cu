@@ -5,23 +5,24 @@
 // share kv head g (GQA: one K/V read serves the whole group; CFR-Atlas page,
 // "MHA/MQA/GQA head mapping").
 //
-// Warp roles:
-//  - warp 8 is the producer: lane i resolves page piece i of a tile (the
+// Warp roles (W = 16 consumer warps, or 8 when GT x D > 512 leaves too few
+// registers for 16):
+//  - warp W is the producer: lane i resolves page piece i of a tile (the
 //    tile's rows of one page) through the page table, checks slot, format and
 //    pool, and copies its K and V rows into a shared-memory ring with one 1-D
 //    bulk copy each (TMA engine, completion on an mbarrier), packed at the
 //    piece's own row size.  Pages that do not resolve are skipped and reported
 //    in the error word, never dereferenced.
-//  - warps 0-7 consume tiles.  Per tile: (1) scores s = sigma*(q.k)*scale_k +
+//  - warps 0..W-1 consume tiles.  Per tile: (1) scores s = sigma*(q.k)*scale_k +
 //    ALiBi, in base 2, eight lanes per token row; (2) per head, the tile max,
 //    the rescale factor 2^(m_old - m_new), p = 2^(s - m_new) and the running
 //    normaliser -- the exact fold of online softmax (CFR-Atlas page, "exact
 //    folded online-softmax attention pass"; ARGUS page, "page-by-page online
-//    softmax"); (3) acc = acc*alpha + sum_t p_t*scale_v*v_t, one warp per eight
+//    softmax"); (3) acc = acc*alpha + sum_t p_t*scale_v*v_t, one warp per 64 / W
 //    tokens, lanes across head_dim.  Quantised rows are expanded to fp32 in
 //    registers only (ARGUS page, "Transient FP16 Reconstruction ... in GPU
 //    SRAM"); scales multiply the dot product and p, never the stored codes.
-//  - At the end of an item the eight warps' accumulators are summed in a fixed
+//  - At the end of an item the W warps' accumulators are summed in a fixed
 //    order and (m, l, acc) is written as the split's partial for the merge.
 //
 // Tokens past the sequence length, tokens outside a sink + recent-window subset
@@ -32,8 +33,11 @@
 namespace cfr {
 
 constexpr int CC_T = 64;       // tokens per tile
-constexpr int CC_WARPS = 8;    // consumer warps
-constexpr int CC_THREADS = (CC_WARPS + 1) * 32;
+// consumer warps W: 16 while the accumulators (GT x D / 32 floats per lane)
+// leave room for them in the register file, else 8; one producer warp more
+__host__ __device__ constexpr int cc_warps(int D, int GT) { return GT * D <= 512 ? 16 : 8; }
+template <int W>
+__host__ __device__ constexpr int cc_threads() { return (W + 1) * 32; }
 constexpr int CC_MAXF = 16;    // fragments (page pieces) per tile; page_tokens >= 8 gives <= 9
 
 // A page piece of a tile: tile rows [r0, r0 + rows of the piece) of one page.
@@ -53,8 +57,9 @@ struct CcStageMeta {
   int t0;
 };
 
+template <int W>
 __device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(CC_WARPS * 32) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
 }
 
 // N consecutive elements starting at element e0 of a stored row, widened to fp32
@@ -168,25 +173,27 @@ struct CcLayout {
   float *alpha;    // [2][GT]
   float *slope2;   // [GT] slope * log2(e)
   int *qoff;       // [GT] causal offset of each query row
-  float *red;      // [CC_WARPS][4][D]
+  float *red;      // [W][4][D]
   int *flag;       // [1] wait outcome broadcast
   uint8_t *ring;   // [stages][2][T][pitch]
 };
 
 template <int D, int GT>
 __host__ __device__ inline size_t cc_fixed_bytes(int stages) {
+  constexpr int W = cc_warps(D, GT);
   size_t o = 0;
   o += 2 * stages * sizeof(uint64_t);
   o = (o + 15) & ~size_t(15);
   o += stages * sizeof(CcStageMeta);
   o = (o + 15) & ~size_t(15);
-  o += GT * D * 4 + 2 * GT * CC_T * 4 + 2 * GT * 4 + GT * 4 + GT * 4 + CC_WARPS * 4 * D * 4 + 16;
+  o += GT * D * 4 + 2 * GT * CC_T * 4 + 2 * GT * 4 + GT * 4 + GT * 4 + W * 4 * D * 4 + 16;
   o = (o + 127) & ~size_t(127);
   return o;
 }
 
 template <int D, int GT>
 __device__ inline CcLayout cc_layout(uint8_t *smem, int stages, int pitch) {
+  constexpr int W = cc_warps(D, GT);
   CcLayout L;
   size_t o = 0;
   L.full = reinterpret_cast<uint64_t *>(smem);
@@ -207,7 +214,7 @@ __device__ inline CcLayout cc_layout(uint8_t *smem, int stages, int pitch) {
   L.qoff = reinterpret_cast<int *>(smem + o);
   o += GT * 4;
   L.red = reinterpret_cast<float *>(smem + o);
-  o += CC_WARPS * 4 * D * 4;
+  o += W * 4 * D * 4;
   L.flag = reinterpret_cast<int *>(smem + o);
   o += 16;
   o = (o + 127) & ~size_t(127);
@@ -310,6 +317,8 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
 template <int D, int GT>
 __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long nitems,
                             bool *timed_out) {
+  constexpr int W = cc_warps(D, GT);      // consumer warps
+  constexpr int HK = (16 + W - 1) / W;    // query rows per warp in the fold
   constexpr int EPT = D / 8;    // elements per thread in the score step (8 lanes per row)
   constexpr int DPL = D / 32;   // dims per lane in the P.V step
   constexpr int HC = GT < 4 ? GT : 4;  // heads per reduction round
@@ -328,7 +337,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
     const int h0 = p.grp_off[g], cnt = p.grp_off[g + 1] - h0;
 
     // the group's queries (fp32) and ALiBi slopes
-    for (int i = tid; i < GT * D; i += CC_WARPS * 32) {
+    for (int i = tid; i < GT * D; i += W * 32) {
       const int hh = i / D, e = i - hh * D;
       float v = 0.f;
       if (hh < cnt) {
@@ -344,19 +353,24 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
           (p.slopes && tid < cnt) ? p.slopes[row_head(p, p.grp_heads[h0 + tid])] * kLog2e : 0.f;
       L.qoff[tid] = tid < cnt ? row_offset(p, p.grp_heads[h0 + tid]) : 0;
     }
-    consumers_sync();
+    consumers_sync<W>();
 
     float acc[GT][DPL];
 #pragma unroll
     for (int h = 0; h < GT; ++h)
 #pragma unroll
       for (int i = 0; i < DPL; ++i) acc[h][i] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float m_run[HK], l_run[HK];
+#pragma unroll
+    for (int k = 0; k < HK; ++k) {
+      m_run[k] = -INFINITY;
+      l_run[k] = 0.f;
+    }
 
     for (int t0 = pb * p.split_unit; t0 < tok_end; t0 += CC_T) {
       // one thread waits (bounded); the outcome is broadcast so all warps agree
       if (tid == 0) *L.flag = mbar_wait(&L.full[stage], phase, p.err, timed_out) ? 1 : 0;
-      consumers_sync();
+      consumers_sync<W>();
       if (*L.flag == 0) {
         *timed_out = true;
         return;
@@ -371,8 +385,8 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
 
       // (1) scores, base 2
 #pragma unroll
-      for (int pass = 0; pass < CC_T / 32; ++pass) {
-        const int r = pass * 32 + warp * 4 + (lane >> 3), j8 = lane & 7;
+      for (int pass = 0; pass < CC_T / (4 * W); ++pass) {
+        const int r = pass * 4 * W + warp * 4 + (lane >> 3), j8 = lane & 7;
         float dot[GT];
 #pragma unroll
         for (int h = 0; h < GT; ++h) dot[h] = 0.f;
@@ -417,12 +431,12 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
             }
         }
       }
-      consumers_sync();
+      consumers_sync<W>();
 
       // (2) fold: tile max, rescale factor, probabilities, running normaliser
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int hh = warp + 8 * k;
+      for (int k = 0; k < HK; ++k) {
+        const int hh = warp + W * k;
         if (hh < GT) {
           const float v0 = sc[hh * CC_T + lane], v1 = sc[hh * CC_T + lane + 32];
           float mt = fmaxf(v0, v1);
@@ -445,7 +459,7 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
           if (lane == 0) al[hh] = alpha;
         }
       }
-      consumers_sync();
+      consumers_sync<W>();
 
       // (3) acc = acc*alpha + sum_t p_t * scale_v * v_t over this warp's 8 tokens
 #pragma unroll
@@ -457,8 +471,8 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
         }
       }
 #pragma unroll 2
-      for (int rr = 0; rr < CC_T / CC_WARPS; ++rr) {
-        const int r = warp * (CC_T / CC_WARPS) + rr;
+      for (int rr = 0; rr < CC_T / W; ++rr) {
+        const int r = warp * (CC_T / W) + rr;
         if (r >= rows) break;
         const CcFrag f = m.frag[m.row_frag[r]];
         if (!f.ok || !in_token_set(p, n, m.t0 + r)) continue;
@@ -484,41 +498,43 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
     float *pa = p.part_acc + static_cast<long long>(slot) * p.Hq * D;
 #pragma unroll
     for (int c0 = 0; c0 < GT; c0 += HC) {
-      consumers_sync();
+      consumers_sync<W>();
 #pragma unroll
       for (int hh = 0; hh < HC; ++hh)
 #pragma unroll
         for (int i = 0; i < DPL; ++i) L.red[(warp * HC + hh) * D + lane * DPL + i] = acc[c0 + hh][i];
-      consumers_sync();
-      for (int e = tid; e < HC * D; e += CC_WARPS * 32) {
+      consumers_sync<W>();
+      for (int e = tid; e < HC * D; e += W * 32) {
         const int hh = e / D, i = e - hh * D;
         float s = 0.f;
 #pragma unroll
-        for (int w = 0; w < CC_WARPS; ++w) s += L.red[(w * HC + hh) * D + i];
+        for (int w = 0; w < W; ++w) s += L.red[(w * HC + hh) * D + i];
         if (c0 + hh < cnt) pa[static_cast<long long>(p.grp_heads[h0 + c0 + hh]) * D + i] = s;
       }
     }
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int hh = warp + 8 * k;
+    for (int k = 0; k < HK; ++k) {
+      const int hh = warp + W * k;
       if (hh < GT && hh < cnt && lane == 0) {
         const long long c = static_cast<long long>(slot) * p.Hq + p.grp_heads[h0 + hh];
         p.part_m[c] = m_run[k];
         p.part_l[c] = l_run[k];
       }
     }
-    consumers_sync();
+    consumers_sync<W>();
   }
 }
 
 template <int D, int GT>
-__global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(cc_threads<cc_warps(D, GT)>(), 1)
+    cc_decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int W = cc_warps(D, GT);
   extern __shared__ __align__(128) uint8_t smem[];
   const CcLayout L = cc_layout<D, GT>(smem, p.stages, p.pitch);
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&L.full[s], 1);
-      mbar_init(&L.empty[s], CC_WARPS);
+      mbar_init(&L.empty[s], W);
     }
     fence_mbar_init();
   }
@@ -528,7 +544,7 @@ __global__ void __launch_bounds__(CC_THREADS, 1) cc_decode_kernel(const __grid_c
   const long long nitems =
       static_cast<long long>(schedule_split_count(p, threadIdx.x == 0 && blockIdx.x == 0)) * p.ngroups;
   bool timed_out = false;
-  if (threadIdx.x >= CC_WARPS * 32) {
+  if (threadIdx.x >= W * 32) {
     cc_producer<D>(p, L, nitems, &timed_out);
   } else {
     cc_consumer<D, GT>(p, L, nitems, &timed_out);
@@ -543,7 +559,8 @@ static cudaError_t cc_launch_t(const DecodeParams &p, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_after_previous(cc_decode_kernel<D, GT>, dim3(grid), dim3(CC_THREADS), smem, stream, p);
+  e = launch_after_previous(cc_decode_kernel<D, GT>, dim3(grid), dim3(cc_threads<cc_warps(D, GT)>()), smem,
+                            stream, p);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
