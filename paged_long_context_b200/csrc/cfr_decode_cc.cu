@@ -40,9 +40,9 @@ template <int W>
 __host__ __device__ constexpr int cc_threads() { return (W + 1) * 32; }
 constexpr int CC_MAXF = 16;    // fragments (page pieces) per tile; page_tokens >= 8 gives <= 9
 
-// A page piece of a tile: tile rows [r0, r0 + rows of the piece) of one page.
-// Its K rows sit packed at their own row size rb from byte `off` of the
-// stage's K region (V rows likewise in the V region).
+// A page piece of a tile (the producer's view): tile rows [r0, r0 + rows of
+// the piece) of one page, whose K rows sit packed at their own row size rb
+// from byte `off` of the stage's K region (V rows likewise in the V region).
 struct CcFrag {
   int fmt;
   int ok;
@@ -50,9 +50,16 @@ struct CcFrag {
   int off, rb, r0;
 };
 
+// Tile row r of a stage: its K row at byte `off` of the stage's K region (its
+// V row at the same offset of the V region), format and readability, scales.
+struct __align__(16) CcRow {
+  int off;
+  int fmt_ok;  // format | 256 when the row's page resolved (else the row is not read)
+  float ks, vs;
+};
+
 struct CcStageMeta {
-  CcFrag frag[CC_MAXF];
-  int8_t row_frag[CC_T];
+  CcRow row[CC_T];
   int rows;
   int t0;
 };
@@ -291,8 +298,14 @@ __device__ void cc_producer(const DecodeParams &p, const CcLayout &L, long long 
       uint8_t *kst = L.ring + static_cast<size_t>(stage) * 2 * CC_T * p.pitch;
       uint8_t *vst = kst + CC_T * p.pitch;
       if (have) {
-        m.frag[lane] = f;
-        for (int r = r0; r < r1; ++r) m.row_frag[r] = static_cast<int8_t>(lane);
+        CcRow rw;
+        rw.fmt_ok = f.ok ? (f.fmt | 256) : 0;
+        rw.ks = f.ks;
+        rw.vs = f.vs;
+        for (int r = r0; r < r1; ++r) {
+          rw.off = f.off + (r - r0) * f.rb;
+          m.row[r] = rw;
+        }
       }
       if (lane == 0) {
         m.rows = rows;
@@ -354,6 +367,16 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
       L.qoff[tid] = tid < cnt ? row_offset(p, p.grp_heads[h0 + tid]) : 0;
     }
     consumers_sync<W>();
+    // this lane's query elements of the score step (8 lanes per token row,
+    // EPT dims each), in registers while they fit beside the accumulators
+    constexpr bool kQRegs = GT * EPT * (D / 64) <= 32;
+    float qr[kQRegs ? GT : 1][kQRegs ? EPT : 1];
+    if constexpr (kQRegs) {
+#pragma unroll
+      for (int h = 0; h < GT; ++h)
+#pragma unroll
+        for (int i = 0; i < EPT; ++i) qr[h][i] = L.q_s[h * D + (lane & 7) * EPT + i];
+    }
 
     float acc[GT][DPL];
 #pragma unroll
@@ -393,22 +416,27 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
         bool valid = false;
         float ks = 1.f;
         if (r < rows) {
-          const CcFrag f = m.frag[m.row_frag[r]];
-          if (f.ok && in_token_set(p, n, m.t0 + r)) {
+          const CcRow rw = m.row[r];
+          if ((rw.fmt_ok & 256) && in_token_set(p, n, m.t0 + r)) {
             valid = true;
-            ks = f.ks;
+            ks = rw.ks;
             float x[EPT];
-            load_elems<EPT>(f.fmt, kst + f.off + (r - f.r0) * f.rb, j8 * EPT, x);
+            load_elems<EPT>(rw.fmt_ok & 255, kst + rw.off, j8 * EPT, x);
 #pragma unroll
             for (int h = 0; h < GT; ++h) {
-              const float4 *qq = reinterpret_cast<const float4 *>(L.q_s + h * D + j8 * EPT);
+              if constexpr (kQRegs) {
 #pragma unroll
-              for (int i = 0; i < EPT / 4; ++i) {
-                const float4 q4 = qq[i];
-                dot[h] = fmaf(q4.x, x[4 * i], dot[h]);
-                dot[h] = fmaf(q4.y, x[4 * i + 1], dot[h]);
-                dot[h] = fmaf(q4.z, x[4 * i + 2], dot[h]);
-                dot[h] = fmaf(q4.w, x[4 * i + 3], dot[h]);
+                for (int i = 0; i < EPT; ++i) dot[h] = fmaf(qr[h][i], x[i], dot[h]);
+              } else {
+                const float4 *qq = reinterpret_cast<const float4 *>(L.q_s + h * D + j8 * EPT);
+#pragma unroll
+                for (int i = 0; i < EPT / 4; ++i) {
+                  const float4 q4 = qq[i];
+                  dot[h] = fmaf(q4.x, x[4 * i], dot[h]);
+                  dot[h] = fmaf(q4.y, x[4 * i + 1], dot[h]);
+                  dot[h] = fmaf(q4.z, x[4 * i + 2], dot[h]);
+                  dot[h] = fmaf(q4.w, x[4 * i + 3], dot[h]);
+                }
               }
             }
           }
@@ -474,13 +502,13 @@ __device__ void cc_consumer(const DecodeParams &p, const CcLayout &L, long long 
       for (int rr = 0; rr < CC_T / W; ++rr) {
         const int r = warp * (CC_T / W) + rr;
         if (r >= rows) break;
-        const CcFrag f = m.frag[m.row_frag[r]];
-        if (!f.ok || !in_token_set(p, n, m.t0 + r)) continue;
+        const CcRow rw = m.row[r];
+        if (!(rw.fmt_ok & 256) || !in_token_set(p, n, m.t0 + r)) continue;
         float v[DPL];
-        load_elems<DPL>(f.fmt, vst + f.off + (r - f.r0) * f.rb, lane * DPL, v);
+        load_elems<DPL>(rw.fmt_ok & 255, vst + rw.off, lane * DPL, v);
 #pragma unroll
         for (int h = 0; h < GT; ++h) {
-          const float pw = sc[h * CC_T + r] * f.vs;
+          const float pw = sc[h * CC_T + r] * rw.vs;
 #pragma unroll
           for (int i = 0; i < DPL; ++i) acc[h][i] = fmaf(pw, v[i], acc[h][i]);
         }
