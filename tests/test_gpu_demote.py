@@ -91,6 +91,21 @@ def test_demote_bit_exact(src, dst, d, P):
         assert torch.equal(hsc, osc)
 
 
+@pytest.mark.parametrize("dst", [I8, I4], ids=["int8", "int4"])
+@pytest.mark.parametrize("d,P", [(64, 512), (128, 512), (128, 264)])
+def test_demote_bf16_block_size_boundary(dst, d, P):
+    # bf16 blocks of exactly 64 KiB (d 64, 512-token pages) take the shared-memory
+    # kernel; larger ones (d 128 at 512 or 264 tokens) the general one: both
+    # bit-exact, including a partial last page
+    case = _src_case(BF16, d, P, lens=(2 * P - 5, P))
+    pages = _pages_of(case)
+    n = len(pages)
+    (hk, hv, hsc, err), (ok, ov, osc, oerr) = _demote_both(
+        case, BF16, dst, [s for s, _ in pages], list(range(n)), [v for _, v in pages], n)
+    assert err == 0 and oerr == 0
+    assert torch.equal(hk, ok) and torch.equal(hv, ov) and torch.equal(hsc, osc)
+
+
 def test_demote_reports_and_skips_bad_pages():
     case = _src_case(BF16, 128, 16, lens=(64,))
     pages = _pages_of(case)
