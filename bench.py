@@ -262,7 +262,7 @@ def record_traffic(args):
     to the full workload by the K/V bytes (DRAM traffic of these kernels grows in
     proportion to the tokens read)."""
     demote = args.workload == "demote"
-    regex = r"demote_(bf16_int_)?kernel" if demote else r"decode_kernel"
+    regex = r"demote_(staged_)?kernel" if demote else r"decode_kernel"
     rows = ncu_csv_metrics(args.record_traffic, regex)
     if not rows:
         raise SystemExit(f"no {regex} launch in {args.record_traffic}")
@@ -564,7 +564,7 @@ def run_ours(args, dist):
     return case, res
 
 
-OUR_KERNELS = re.compile(r"(schedule|qimage|decode|merge|demote|demote_bf16_int)_kernel")
+OUR_KERNELS = re.compile(r"(schedule|qimage|decode|merge|demote|demote_staged)_kernel")
 
 
 def count_launches(step):
@@ -781,7 +781,7 @@ def run_demote(args, dist):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "us_per_step": round(e2e_ms * 1e3, 2)},
         "gpu_launches": len(jobs) * K,
-        "gpu_launches_note": f"{len(jobs)} demote_bf16_int_kernel launches per step (one per destination format)",
+        "gpu_launches_note": f"{len(jobs)} demote_staged_kernel launches per step (one per destination format)",
         "clocks": clk.summary(),
         "device_err_word": int(err.item()),
     }

@@ -364,8 +364,8 @@ cfr_status cfr_gather_pages(const cfr_kv_pool *kv, const int32_t *page_table,
  * A block of zeros gets scale 0 and zero codes.  Rows at or past the valid
  * count are written as zero bytes.  Codes and scales are bit-exact functions
  * of the stored source bytes.  NaN values are left out of max|x| and get
- * integer code 0 (checked for bf16 sources into int8 and int4); other NaN
- * codes are unspecified.
+ * integer code 0 and E4M3 code 0x7F; NaN bf16 and fp32 destination values are
+ * unspecified NaNs.
  *
  *  kv           host; geometry (num_kv_heads, head_dim 64 or 128, page_tokens >= 8)
  *               and the source pool k_pool/v_pool/scales/pool_pages[src_fmt].

@@ -125,7 +125,9 @@ __device__ __forceinline__ int int_code(float x, float scale, int q) {
 
 __device__ __forceinline__ uint32_t fp8_code(float x, float scale) {
   if (!(scale > 0.f)) return 0u;
-  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(x, scale), __NV_SATFINITE, __NV_E4M3));
+  const float q = __fdiv_rn(x, scale);
+  if (q != q) return 0x7Fu;  // NaN: the positive E4M3 NaN code
+  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3));
 }
 
 // encodes eight values and stores them at element e of the destination block
@@ -312,10 +314,11 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
 }
 
 // ---------------------------------------------------------------------------
-// bf16 -> int8 / int4, the hot-to-cold step of the cascade.
+// The cascade's steps (bf16 -> E4M3 / int8 / int4, int8 -> int4 or E4M3,
+// E4M3 -> int8 or int4) on blocks staged in shared memory.
 //
-// The codes are the ones defined above, code = rint(fl(x / scale)), reached
-// without a division per element.  Let q = x / scale (exact) and f = fl(q).
+// The codes are the ones defined above, code = rint(fl(x / scale)) (or the
+// E4M3 code of fl(x / scale)), reached without a division per element.  Let q = x / scale (exact) and f = fl(q).
 // With a normal, finite scale and r = fl(1 / scale) (one correctly rounded
 // reciprocal per block), take r- = fl(r * (1 - 2^-20)) and r+ = fl(r * (1 + 2^-20)).
 // Each of r, r-, r+ and f carries a relative rounding error of at most 2^-24,
@@ -329,11 +332,13 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
 // cannot bind: |x| <= max|x| and scale >= max|x| / Q to within 2^-24).  When
 // they differ (a half-integer within about |q| * 2^-20 of the product: about
 // one element in 15,000 for random data, and every NaN), the eight elements
-// of the vector are encoded again with the IEEE division.  A block whose
-// maximum is infinite or whose scale is zero or subnormal (where the bounds
-// above fail) is encoded with the division throughout.
-// max|x| is taken on the bf16 pairs (|a| vs |b| maxima, which ignore NaN as
-// fmaxf does), equal to the fp32 maximum of the decoded values.
+// of the vector are encoded again with the IEEE division.  E4M3 destinations
+// round the two products to fp32 and then to E4M3, both monotone, so equal
+// codes of the two are the code of f.  A block whose maximum is infinite or
+// whose scale is zero or subnormal (where the bounds above fail) is encoded
+// with the division throughout.
+// max|x| is taken on the codes (src_absmax_acc), equal to the fp32 maximum of
+// the decoded values.
 // ---------------------------------------------------------------------------
 
 constexpr float kRintMagic = 12582912.0f;         // 1.5 * 2^23
@@ -352,114 +357,194 @@ __device__ __forceinline__ float absmax_value(uint32_t m) {
   return fmaxf(bf16_lo(m & 0x7FFF7FFFu), bf16_hi(m & 0x7FFF7FFFu));
 }
 
-__device__ __forceinline__ void bf16_decode8(const uint4 &w, float (&x)[kVec]) {
-  const uint32_t a[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    x[2 * k] = bf16_lo(a[k]);
-    x[2 * k + 1] = bf16_hi(a[k]);
-  }
-}
-
-// the eight codes of one vector (8 bf16 in w), each as 0x4B400000 + code, from
-// the two bracketing products; true when they disagree somewhere (the vector
-// is then encoded again by bf16_codes8_exact)
-__device__ __forceinline__ bool bf16_codes8_fast(const uint4 &w, float r_lo, float r_hi,
-                                                 uint32_t (&tb)[kVec]) {
-  float x[kVec];
-  bf16_decode8(w, x);
-  bool near = false;
-#pragma unroll
-  for (int k = 0; k < kVec; ++k) {
-    const float lo = __fmaf_rn(x[k], r_lo, kRintMagic);
-    const float hi = __fmaf_rn(x[k], r_hi, kRintMagic);
-    near |= lo != hi;
-    tb[k] = __float_as_uint(lo);
-  }
-  return near;
-}
-
-// the same codes with the IEEE division
-template <int Q>
-__device__ __forceinline__ void bf16_codes8_exact(const uint4 &w, float scale, uint32_t (&tb)[kVec]) {
-  float x[kVec];
-  bf16_decode8(w, x);
-#pragma unroll
-  for (int k = 0; k < kVec; ++k) tb[k] = kRintMagicBits + static_cast<uint32_t>(int_code(x[k], scale, Q));
-}
-
-// stores eight codes (low byte / nibble of each tb) as vector v of the block
+// stores eight codes (the low byte, or for int4 the low nibble, of each tb)
+// as vector v of the block
 template <int DST>
 __device__ __forceinline__ void store_codes8(uint8_t *dst, int v, const uint32_t (&tb)[kVec]) {
-  if constexpr (DST == CFR_FMT_I8) {
-    const uint32_t lo = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
-    const uint32_t hi = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040), 0x5410);
-    reinterpret_cast<uint2 *>(dst)[v] = make_uint2(lo, hi);
-  } else {  // element 2i in the low nibble of byte i
+  if constexpr (DST == CFR_FMT_I4) {  // element 2i in the low nibble of byte i
     uint32_t n[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) n[k] = (tb[2 * k] & 0x0Fu) | (tb[2 * k + 1] << 4);
     reinterpret_cast<uint32_t *>(dst)[v] =
         __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
+  } else {  // int8 and E4M3: one byte each
+    const uint32_t lo = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(tb[4], tb[5], 0x0040), __byte_perm(tb[6], tb[7], 0x0040), 0x5410);
+    reinterpret_cast<uint2 *>(dst)[v] = make_uint2(lo, hi);
   }
+}
+
+// The eight codes of one vector of decoded values x, from the two bracketing
+// products x * r_lo and x * r_hi; true when they disagree somewhere (or a
+// value is NaN), and the vector must be encoded again with the division.
+//  - int8 / int4: each as 0x4B400000 + code (the rounded sum with 1.5 * 2^23);
+//  - E4M3: the code of each rounded product (rounding to fp32 and then to E4M3
+//    are both monotone, so equal codes of the two products are the code of
+//    fl(x / scale), which lies between them).
+template <int DST>
+__device__ __forceinline__ bool codes8_fast(const float (&x)[kVec], float r_lo, float r_hi,
+                                            uint32_t (&tb)[kVec]) {
+  bool near = false;
+#pragma unroll
+  for (int k = 0; k < kVec; ++k) {
+    if constexpr (DST == CFR_FMT_FP8) {
+      const uint32_t lo = __nv_cvt_float_to_fp8(__fmul_rn(x[k], r_lo), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float_to_fp8(__fmul_rn(x[k], r_hi), __NV_SATFINITE, __NV_E4M3);
+      near |= (lo != hi) || (x[k] != x[k]);
+      tb[k] = lo;
+    } else {
+      const float lo = __fmaf_rn(x[k], r_lo, kRintMagic);
+      const float hi = __fmaf_rn(x[k], r_hi, kRintMagic);
+      near |= lo != hi;
+      tb[k] = __float_as_uint(lo);
+    }
+  }
+  return near;
+}
+
+// the same codes with the IEEE division
+template <int DST>
+__device__ __forceinline__ void codes8_exact(const float (&x)[kVec], float scale, uint32_t (&tb)[kVec]) {
+#pragma unroll
+  for (int k = 0; k < kVec; ++k) {
+    if constexpr (DST == CFR_FMT_FP8)
+      tb[k] = fp8_code(x[k], scale);
+    else
+      tb[k] = kRintMagicBits + static_cast<uint32_t>(int_code(x[k], scale, DST == CFR_FMT_I8 ? 127 : 7));
+  }
+}
+
+// Running max|code| of one source vector, in the source's own terms:
+//  - bf16: per half of m, max(|m|, |w|) of the bf16 pairs (NaN left out);
+//  - int8: the largest |code| (0..128);
+//  - E4M3: the largest magnitude byte (0..0x7E), NaN codes (0x7F) left out.
+// For quantised sources max|x| = fl(max value * scale) for a non-negative
+// finite scale, since x = fl(code * scale) is monotone in |code|.
+template <int SRC>
+__device__ __forceinline__ uint32_t src_absmax_acc(uint32_t m, const RawVec<SRC> &r) {
+  if constexpr (SRC == CFR_FMT_BF16) {
+    return absmax_acc(absmax_acc(absmax_acc(absmax_acc(m, r.a.x), r.a.y), r.a.z), r.a.w);
+  } else {
+    const uint32_t w[2] = {r.w.x, r.w.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if constexpr (SRC == CFR_FMT_I8) {
+          const int c = static_cast<int8_t>((w[i] >> (8 * k)) & 0xFFu);
+          m = max(m, static_cast<uint32_t>(abs(c)));
+        } else {  // CFR_FMT_FP8
+          const uint32_t mag = (w[i] >> (8 * k)) & 0x7Fu;
+          m = mag == 0x7Fu ? m : max(m, mag);
+        }
+      }
+    return m;
+  }
+}
+
+template <int SRC>
+__device__ __forceinline__ uint32_t src_absmax_combine(uint32_t a, uint32_t b) {
+  if constexpr (SRC == CFR_FMT_BF16)
+    return absmax_acc(a, b);
+  else
+    return max(a, b);
+}
+
+template <int SRC>
+__device__ __forceinline__ float src_absmax_value(uint32_t m, float src_scale) {
+  if constexpr (SRC == CFR_FMT_BF16)
+    return absmax_value(m);
+  else if constexpr (SRC == CFR_FMT_I8)
+    return __fmul_rn(static_cast<float>(m), src_scale);
+  else
+    return __fmul_rn(e4m3_at(m, 0), src_scale);
 }
 
 // The block is staged in shared memory by one bulk copy (all of it in flight
 // at once), with three 256-thread CTAs per SM; the max pass and the encode
-// pass read it there.  Blocks of up to 64 KiB (page_tokens x head_dim <= 32768).
+// pass read it there.  Blocks of up to 64 KiB and 8192 vectors of 8 elements.
+// Pairs: bf16 -> int8 / int4 / E4M3, int8 -> int4 / E4M3, E4M3 -> int8 (E4M3
+// -> int4 measured faster on the general kernel).
 constexpr int kSmemThreads = 256;
 constexpr int kSmemBlockBytes = 65536;
+constexpr int kSmemMaxVecs = 32 * kSmemThreads;  // one bit per vector of a thread in `redo`
 
-template <int DST>
-__global__ void __launch_bounds__(kSmemThreads, 3) demote_bf16_int_kernel(DemoteParams p) {
+template <int SRC, int DST>
+__global__ void __launch_bounds__(kSmemThreads, 3) demote_staged_kernel(DemoteParams p) {
   constexpr int T = kSmemThreads;
-  constexpr int Q = DST == CFR_FMT_I8 ? 127 : 7;
-  extern __shared__ __align__(128) uint4 stage[];
+  // vectors of a thread: as many as a 64 KiB block holds, at most 32
+  constexpr int ITERS = kSmemBlockBytes / static_cast<int>(sizeof(RawVec<SRC>)) / T < kSmemMaxVecs / T
+                            ? kSmemBlockBytes / static_cast<int>(sizeof(RawVec<SRC>)) / T
+                            : kSmemMaxVecs / T;
+  extern __shared__ __align__(128) uint8_t stage_bytes[];
+  const RawVec<SRC> *stage = reinterpret_cast<const RawVec<SRC> *>(stage_bytes);
   __shared__ uint64_t bar;
   __shared__ uint32_t redw[T / 32];
+  __shared__ float redf[T / 32];
   DemoteBlock b;
-  if (!resolve_block(p, CFR_FMT_BF16, b)) return;
+  if (!resolve_block(p, SRC, b)) return;
   const int tid = threadIdx.x;
   const int nv = static_cast<int>(b.nvec_valid);
+  const float s_src = b.src_scale;
   if (tid == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nv) * 16u);
-    bulk_g2s(stage, b.src, static_cast<uint32_t>(nv) * 16u, &bar);
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nv * sizeof(RawVec<SRC>)));
+    bulk_g2s(stage_bytes, b.src, static_cast<uint32_t>(nv * sizeof(RawVec<SRC>)), &bar);
   }
   __syncthreads();
   bool timed_out = false;
   if (!mbar_wait(&bar, 0, p.err, &timed_out)) return;
-  uint32_t m = 0u;
+  // max|x|: from the codes while the source scale is finite and non-negative,
+  // else over the decoded values as written (fmaxf, NaN left out)
+  const bool src_ok = SRC == CFR_FMT_BF16 || (s_src >= 0.f && s_src <= 3.40282347e+38f);
+  float amax;
+  if (src_ok) {
+    uint32_t m = 0u;
 #pragma unroll 4
-  for (int v = tid; v < nv; v += T) {
-    const uint4 w = stage[v];
-    m = absmax_acc(absmax_acc(absmax_acc(absmax_acc(m, w.x), w.y), w.z), w.w);
+    for (int v = tid; v < nv; v += T) m = src_absmax_acc<SRC>(m, stage[v]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = src_absmax_combine<SRC>(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) redw[tid >> 5] = m;
+    __syncthreads();
+    m = redw[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) m = src_absmax_combine<SRC>(m, redw[w]);
+    amax = src_absmax_value<SRC>(m, s_src);
+  } else {
+    float a = 0.f;
+    for (int v = tid; v < nv; v += T) {
+      float x[kVec];
+      decode_raw<SRC>(stage[v], s_src, x);
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) a = fmaxf(a, fabsf(x[k]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((tid & 31) == 0) redf[tid >> 5] = a;
+    __syncthreads();
+    a = redf[0];
+#pragma unroll
+    for (int w = 1; w < T / 32; ++w) a = fmaxf(a, redf[w]);
+    amax = a;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = absmax_acc(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((tid & 31) == 0) redw[tid >> 5] = m;
-  __syncthreads();
-  m = redw[0];
-#pragma unroll
-  for (int w = 1; w < T / 32; ++w) m = absmax_acc(m, redw[w]);
-  const float amax = absmax_value(m);
-  const float scale = __fdiv_rn(amax, static_cast<float>(Q));
+  const float scale = __fdiv_rn(amax, qmax_of(DST));
   const bool fast = scale >= 1.17549435e-38f && scale <= 3.40282347e+38f;  // normal and finite
   if (tid == 0) *b.dst_scale = scale;
   // encode: vectors near a tie are marked in `redo` and encoded again after
   // the loop, which keeps the division out of the loop body
-  static_assert(kSmemBlockBytes / 16 / T <= 32, "one bit per vector of a thread");
   uint32_t redo = 0u;
   if (fast) {
     const float r = __frcp_rn(scale);
     const float r_lo = __fmul_rn(r, 1.f - 0x1p-20f), r_hi = __fmul_rn(r, 1.f + 0x1p-20f);
 #pragma unroll 4
-    for (int i = 0; i < kSmemBlockBytes / 16 / T; ++i) {
+    for (int i = 0; i < ITERS; ++i) {
       const int v = i * T + tid;
       if (v < nv) {
+        float x[kVec];
+        decode_raw<SRC>(stage[v], s_src, x);
         uint32_t tb[kVec];
-        redo |= static_cast<uint32_t>(bf16_codes8_fast(stage[v], r_lo, r_hi, tb)) << i;
+        redo |= static_cast<uint32_t>(codes8_fast<DST>(x, r_lo, r_hi, tb)) << i;
         store_codes8<DST>(b.dst, v, tb);
       }
     }
@@ -470,11 +555,37 @@ __global__ void __launch_bounds__(kSmemThreads, 3) demote_bf16_int_kernel(Demote
     const int i = __ffs(redo) - 1;
     redo &= redo - 1;
     const int v = i * T + tid;
+    float x[kVec];
+    decode_raw<SRC>(stage[v], s_src, x);
     uint32_t tb[kVec];
-    bf16_codes8_exact<Q>(stage[v], scale, tb);
+    codes8_exact<DST>(x, scale, tb);
     store_codes8<DST>(b.dst, v, tb);
   }
   for (long long v = b.nvec_valid + tid; v < b.nvec; v += T) store_zero8(DST, b.dst, v * kVec);
+}
+
+template <int SRC, int DST>
+cudaError_t launch_staged(const DemoteParams &p, unsigned blocks, cudaStream_t s) {
+  auto kern = demote_staged_kernel<SRC, DST>;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBlockBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<blocks, kSmemThreads, kSmemBlockBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+// the staged kernel for (src, dst) when it serves the pair and the block fits;
+// cudaErrorNotSupported otherwise
+cudaError_t try_launch_staged(const DemoteParams &p, int src, int dst, unsigned blocks, cudaStream_t s) {
+  const long long vecs = static_cast<long long>(p.P) * p.D / kVec;
+  const long long bytes = static_cast<long long>(p.P) * row_bytes(src, p.D);
+  if (vecs > kSmemMaxVecs || bytes > kSmemBlockBytes) return cudaErrorNotSupported;
+#define CFR_STAGED(S, D) \
+  if (src == S && dst == D) return launch_staged<S, D>(p, blocks, s);
+  CFR_STAGED(CFR_FMT_BF16, CFR_FMT_I8) CFR_STAGED(CFR_FMT_BF16, CFR_FMT_I4) CFR_STAGED(CFR_FMT_BF16, CFR_FMT_FP8)
+  CFR_STAGED(CFR_FMT_I8, CFR_FMT_I4) CFR_STAGED(CFR_FMT_I8, CFR_FMT_FP8) CFR_STAGED(CFR_FMT_FP8, CFR_FMT_I8)
+#undef CFR_STAGED
+  return cudaErrorNotSupported;
 }
 
 struct AppendParams {
@@ -598,18 +709,8 @@ cfr_status cfr_demote_pages(const cfr_kv_pool *kv, int32_t src_fmt, int32_t dst_
   p.P = kv->page_tokens;
   const unsigned blocks = static_cast<unsigned>(num_pages) * kv->num_kv_heads * 2u;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the bf16 -> int kernel stages a whole block in shared memory
-  const bool fits = static_cast<long long>(kv->page_tokens) * row_bytes(CFR_FMT_BF16, kv->head_dim) <=
-                    kSmemBlockBytes;
-  if (fits && src_fmt == CFR_FMT_BF16 && (dst_fmt == CFR_FMT_I8 || dst_fmt == CFR_FMT_I4)) {
-    auto kern = dst_fmt == CFR_FMT_I8 ? demote_bf16_int_kernel<CFR_FMT_I8>
-                                      : demote_bf16_int_kernel<CFR_FMT_I4>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBlockBytes) !=
-        cudaSuccess)
-      return CFR_ERR_CUDA;
-    kern<<<blocks, kSmemThreads, kSmemBlockBytes, s>>>(p);
-    return cudaGetLastError() == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
-  }
+  const cudaError_t staged = try_launch_staged(p, src_fmt, dst_fmt, blocks, s);
+  if (staged != cudaErrorNotSupported) return staged == cudaSuccess ? CFR_OK : CFR_ERR_CUDA;
   switch (src_fmt) {
     case CFR_FMT_F32: demote_kernel<CFR_FMT_F32><<<blocks, kDemoteThreads, 0, s>>>(p); break;
     case CFR_FMT_BF16: demote_kernel<CFR_FMT_BF16><<<blocks, kDemoteThreads, 0, s>>>(p); break;

@@ -106,6 +106,37 @@ def test_demote_bf16_block_size_boundary(dst, d, P):
     assert torch.equal(hk, ok) and torch.equal(hv, ov) and torch.equal(hsc, osc)
 
 
+@pytest.mark.parametrize("src,dst", [(I8, I4), (I8, FP8), (FP8, I8), (FP8, I4)],
+                         ids=["int8-int4", "int8-fp8", "fp8-int8", "fp8-int4"])
+def test_demote_quantised_source_every_code(src, dst):
+    # every one of the 256 source codes in each block, under K/V scales that
+    # include zero, a subnormal, a negative, an infinite and a NaN scale; codes
+    # and scales byte for byte against the oracle
+    Hkv, P, d = 2, 16, 128
+    scales = [1.0, 0.0123, 3.7e-3, 1e-39, 0.0, -0.5, float("inf"), float("nan")]
+    nblk = len(scales)
+    npages = -(-nblk // (2 * Hkv))
+    case = _src_case(src, d, P, lens=(P * npages,), seed=17)
+    pages = _pages_of(case)
+    rng = np.random.default_rng(src * 7 + dst)
+    k = case.k_pool[src]
+    v = case.v_pool[src]
+    sc = case.scales[src]
+    for i, s_ in enumerate(scales):
+        j, rest = divmod(i, 2 * Hkv)
+        g, kv = divmod(rest, 2)
+        codes = np.resize(np.arange(256, dtype=np.uint8), P * d)
+        rng.shuffle(codes)
+        (v if kv else k)[pages[j][0], g] = torch.from_numpy(codes.reshape(P, d)).to(k.device)
+        sc[pages[j][0], g, kv] = s_
+    n = len(pages)
+    (hk, hv, hsc, err), (ok, ov, osc, oerr) = _demote_both(
+        case, src, dst, [s for s, _ in pages], list(range(n)), [v_ for _, v_ in pages], n)
+    assert err == 0 and oerr == 0
+    assert torch.equal(hk, ok) and torch.equal(hv, ov)
+    assert torch.equal(hsc.view(torch.int32), osc.view(torch.int32))
+
+
 def test_demote_reports_and_skips_bad_pages():
     case = _src_case(BF16, 128, 16, lens=(64,))
     pages = _pages_of(case)
@@ -156,7 +187,7 @@ def _demote_blocks_exact(blocks, dst):
     return hsc
 
 
-@pytest.mark.parametrize("dst", [I8, I4], ids=["int8", "int4"])
+@pytest.mark.parametrize("dst", [I8, I4, FP8], ids=["int8", "int4", "fp8"])
 @pytest.mark.parametrize("amax_bits", [0x3F80, 0x3F4A, 0x4040, 0x3FFE, 0x7F00, 0x0D80, 0x0400, 0x0300],
                          ids=lambda b: f"amax{b:04x}")
 def test_demote_bf16_to_int_every_input(dst, amax_bits):
@@ -181,7 +212,7 @@ def test_demote_bf16_to_int_every_input(dst, amax_bits):
     assert bool((sc.view(-1)[: len(blocks)] > 0).all())
 
 
-@pytest.mark.parametrize("dst", [I8, I4], ids=["int8", "int4"])
+@pytest.mark.parametrize("dst", [I8, I4, FP8], ids=["int8", "int4", "fp8"])
 def test_demote_bf16_to_int_edge_blocks(dst):
     rng = np.random.default_rng(3)
     n = 2048
@@ -190,15 +221,26 @@ def test_demote_bf16_to_int_edge_blocks(dst):
         m = rng.integers(lo_bits, hi_bits, size=n, dtype=np.uint32)
         return (m | (rng.integers(0, 2, size=n, dtype=np.uint32) << 15)).astype(np.uint16)
 
-    q = 127 if dst == I8 else 7
     blocks = []
-    # exact ties: scale = 2^-6 (int8) or 2^-2 (int4), values (k + 1/2) * scale
-    unit = 64 if dst == I8 else 4
-    amax = torch.tensor([q / unit], dtype=torch.bfloat16).view(torch.int16).item() & 0xFFFF
-    ks = rng.integers(-q, q, size=n)
-    ties = torch.tensor((ks + 0.5) / unit, dtype=torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
-    ties[0] = amax
-    blocks.append(ties)
+    if dst == FP8:
+        # scale 1 (max|x| = 448): every midpoint between neighbouring E4M3 values,
+        # both signs, each an exact tie of the E4M3 rounding
+        vals = np.array([float(torch.tensor([c], dtype=torch.uint8).view(torch.float8_e4m3fn).float())
+                         for c in range(0x7F)])
+        mids = (vals[:-1] + vals[1:]) / 2
+        mids = np.concatenate([mids, -mids])
+        ties = np.resize(mids, n)
+        rng.shuffle(ties)
+        ties[0] = 448.0
+        unit = 1.0
+    else:
+        # exact ties: scale = 2^-6 (int8) or 2^-2 (int4), values (k + 1/2) * scale
+        q = 127 if dst == I8 else 7
+        unit = 64 if dst == I8 else 4
+        ks = rng.integers(-q, q, size=n)
+        ties = (ks + 0.5) / unit
+        ties[0] = q / unit
+    blocks.append(torch.tensor(ties, dtype=torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
     # NaNs (with payloads and signs) among finite values: max|x| ignores them, their codes are 0
     b = finite()
     b[rng.choice(n, 40, replace=False)] = np.array([0x7FC0, 0x7FC1, 0xFFC0, 0x7F81] * 10, np.uint16)
