@@ -79,12 +79,13 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 //  - The tcgen05 path over bf16-only pools, and over uniform int8 / int4 pools
 //    in its int8-MMA variant, balances at run time (its CTAs claim items from a
 //    counter), so it takes the fewest, longest items: 4 per SM measured faster
-//    than 8 or 16.
+//    than 8 or 16, and 2 per SM for sink + window subsets and for groups of
+//    more than 8 rows (the 32-column variants), whose tiles cost more.
 //  - Other uniform caches are shared out in a fixed pattern: 8 per SM.
 //  - A cache of mixed storage formats has items of unequal cost (a page of
 //    int4 codes is a quarter of the bytes of a bf16 page, but takes longer to
 //    expand), so its fixed share is cut finer: 16 per SM.
-constexpr int kItemsPerSmClaimed = 4, kItemsPerSm = 8, kItemsPerSmMixed = 16;
+constexpr int kItemsPerSmClaimed = 4, kItemsPerSmClaimedLong = 2, kItemsPerSm = 8, kItemsPerSmMixed = 16;
 
 // true when a decode over these pools expands quantised codes on chip
 bool quantised_pools(const DecodeParams &p, bool page_fmt_given) {
@@ -377,7 +378,8 @@ cfr_status decode_impl(const void *q, int32_t q_fmt, const cfr_kv_pool *kv,
       use_tc && (!quantised_pools(p, page_fmt != nullptr) ||
                  (!page_fmt && p.gmax <= 4 && kv->head_dim == 128 &&
                   (uniform_fmt == CFR_FMT_I8 || uniform_fmt == CFR_FMT_I4)));
-  const int per_sm = claimed ? kItemsPerSmClaimed : page_fmt ? kItemsPerSmMixed : kItemsPerSm;
+  const int per_sm = claimed ? ((window > 0 || p.gmax > 8) ? kItemsPerSmClaimedLong : kItemsPerSmClaimed)
+                     : page_fmt ? kItemsPerSmMixed : kItemsPerSm;
   const int target = target_splits(di.sms, p.ngroups, per_sm);
   WsLayout w;
   const int unit = schedule_unit(kv->page_tokens, batch, max_pages, di.sms);
