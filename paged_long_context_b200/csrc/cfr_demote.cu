@@ -330,9 +330,11 @@ __global__ void __launch_bounds__(kDemoteThreads) demote_kernel(DemoteParams p) 
 // the low bits of the sum.  Rounding to nearest is monotone, so when both
 // sums agree they equal rint(f): that is the code, and |code| <= Q (the clamp
 // cannot bind: |x| <= max|x| and scale >= max|x| / Q to within 2^-24).  When
-// they differ (a half-integer within about |q| * 2^-20 of the product: about
-// one element in 15,000 for random data, and every NaN), the eight elements
-// of the vector are encoded again with the IEEE division.  E4M3 destinations
+// they differ (a half-integer within about |q| * 2^-20 of the product, and
+// every NaN), the eight elements of the vector are encoded again with the
+// IEEE division.  On bf16 blocks of N(0,1) values that is about one element in
+// 600: a value that is a simple fraction of max|x| (max|x| / 2, say) puts
+// x / scale within an ulp of a half-integer.  E4M3 destinations
 // round the two products to fp32 and then to E4M3, both monotone, so equal
 // codes of the two are the code of f.  A block whose maximum is infinite or
 // whose scale is zero or subnormal (where the bounds above fail) is encoded
